@@ -1,0 +1,150 @@
+"""fp64 CPU oracle for the Kimi Delta Attention (KDA) token mixer.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+``bench.py``'s CPU-baseline leg / ``--impl reference`` arm may import this
+package.  The product package ``gated_delta_rule_88_b200`` never imports it, and
+this package imports nothing from the product package: the two share no code.
+
+The arithmetic lives in ``kda_oracle.c`` (plain C, fp64, token by token; see its
+header for the cited recurrence).  This module only marshals arguments: it
+slices each (sequence, head) out of the caller's tensors, widens them exactly to
+fp64, calls the C routine, and scatters the results.  Independent
+(sequence, head) recurrences run on a thread pool (ctypes releases the GIL).
+
+Layouts follow the library's C ABI:
+  dense : q,k,g [B,T,H,dk]; v [B,T,H,dv]; beta [B,T,H]; states [B,H,dk,dv]
+  varlen: B == 1, cu_seqlens [N+1] int; states [N,H,dk,dv]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libkda_oracle.so")
+_lib = None
+_lib_lock = threading.Lock()
+
+
+def build(force: bool = False) -> str:
+    """Compile kda_oracle.c into libkda_oracle.so next to it (gcc, -O2)."""
+    if force or not os.path.exists(_LIB_PATH) or (
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c99", "-shared", "-fPIC",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lib_lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            f = lib.kda_oracle_recurrence
+            dp = ctypes.POINTER(ctypes.c_double)
+            L = ctypes.c_long
+            f.argtypes = [L, ctypes.c_int, ctypes.c_int,
+                          dp, L, dp, L, dp, L, dp, L, dp, L, dp, dp, L]
+            f.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def recurrence(q, k, v, g, beta, S0=None):
+    """One (sequence, head): q,k,g [T,dk]; v [T,dv]; beta [T]; S0 [dk,dv].
+
+    Inputs are any real arrays/tensors; they are widened to fp64.
+    Returns (o [T,dv] fp64, S_T [dk,dv] fp64) as numpy arrays.
+    """
+    lib = _load()
+    q = _f64(q); k = _f64(k); v = _f64(v); g = _f64(g); beta = _f64(beta)
+    T, dk = q.shape
+    dv = v.shape[1]
+    assert k.shape == (T, dk) and g.shape == (T, dk) and v.shape == (T, dv)
+    assert beta.shape == (T,)
+    S = np.zeros((dk, dv)) if S0 is None else _f64(S0).copy()
+    assert S.shape == (dk, dv)
+    o = np.zeros((T, dv))
+    rc = lib.kda_oracle_recurrence(T, dk, dv, _ptr(q), dk, _ptr(k), dk,
+                                   _ptr(v), dv, _ptr(g), dk, _ptr(beta), 1,
+                                   _ptr(S), _ptr(o), dv)
+    if rc != 0:
+        raise RuntimeError("kda_oracle_recurrence failed")
+    return o, S
+
+
+def _f64(x) -> np.ndarray:
+    if isinstance(x, torch.Tensor):
+        return np.ascontiguousarray(x.detach().cpu().to(torch.float64).numpy())
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _threads(n_tasks: int, threads: int | None) -> int:
+    if threads is None:
+        threads = os.cpu_count() or 1
+    return max(1, min(threads, n_tasks))
+
+
+def forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None,
+            threads: int | None = None, heads=None, seqs=None,
+            want_output: bool = True):
+    """Full KDA forward over all (sequence, head) pairs, fp64.
+
+    q,k,g: [B,T,H,dk]; v: [B,T,H,dv]; beta: [B,T,H] (CPU tensors, any dtype).
+    initial_state: None (zeros) or [N,H,dk,dv].  cu_seqlens: None (dense, N=B)
+    or [N+1] offsets into T with B == 1.
+    heads / seqs: optional subsets to evaluate (others left as NaN).
+    Returns (o [B,T,H,dv] float64 tensor, final_state [N,H,dk,dv] float64).
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is None:
+        N = B
+        ranges = [(b, 0, T) for b in range(B)]
+    else:
+        assert B == 1
+        cu = [int(x) for x in torch.as_tensor(cu_seqlens).tolist()]
+        N = len(cu) - 1
+        ranges = [(0, cu[n], cu[n + 1]) for n in range(N)]
+    heads = list(range(H)) if heads is None else list(heads)
+    seqs = list(range(N)) if seqs is None else list(seqs)
+    o = torch.full((B, T, H, dv), float("nan"), dtype=torch.float64)
+    sT = torch.full((N, H, dk, dv), float("nan"), dtype=torch.float64)
+
+    def task(n, h):
+        b, s, e = ranges[n]
+        S0 = None if initial_state is None else initial_state[n, h]
+        on, Sn = recurrence(q[b, s:e, h], k[b, s:e, h], v[b, s:e, h],
+                            g[b, s:e, h], beta[b, s:e, h], S0)
+        if want_output:
+            o[b, s:e, h] = torch.from_numpy(on)
+        sT[n, h] = torch.from_numpy(Sn)
+
+    jobs = [(n, h) for n in seqs for h in heads]
+    with ThreadPoolExecutor(_threads(len(jobs), threads)) as ex:
+        for f in [ex.submit(task, n, h) for n, h in jobs]:
+            f.result()
+    return o, sT
+
+
+def decode_step(q, k, v, g, beta, state, threads: int | None = None):
+    """One recurrent step for N sequences: q,k,g [N,H,dk]; v [N,H,dv];
+    beta [N,H]; state [N,H,dk,dv].  Returns (o [N,H,dv], new state), fp64."""
+    o, sT = forward(q.unsqueeze(1), k.unsqueeze(1), v.unsqueeze(1),
+                    g.unsqueeze(1), beta.unsqueeze(1), initial_state=state,
+                    threads=threads)
+    return o[:, 0], sT

@@ -1,0 +1,183 @@
+"""Kimi Delta Attention (KDA) token mixer for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/kda.h`` (``libkda_b200.so``):
+argument marshalling only.  Tensors must be CUDA tensors; every step of the
+computation runs in the library's kernels.  There is no CPU path: if the
+shared library is missing or cannot be loaded, calls raise.
+
+Entry points (same names as the C ABI):
+    kda_chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None,
+                  out=None, final_state=None, output_final_state=True)
+        -> (out, final_state or None)
+    kda_recurrent_step(q, k, v, g, beta, state, out=None) -> out
+    kda_get_device_error(stream=None) -> int
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = ["kda_chunk_fwd", "kda_recurrent_step", "kda_get_device_error", "KDAError",
+           "library_path", "load_library"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_PKG, "libkda_b200.so")
+_lib = None
+_lock = threading.Lock()
+
+KDA_F32, KDA_BF16 = 0, 1
+_STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
+           3: "KDA_ERR_CUDA", 4: "KDA_ERR_DEVICE"}
+
+
+class KDAError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def load_library():
+    """Load libkda_b200.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(library_path):
+            raise RuntimeError(
+                f"{library_path} not found: build it with "
+                "`python -m gated_delta_rule_88_b200.build` (no CPU fallback exists)")
+        lib = ctypes.CDLL(library_path)
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        lib.kda_chunk_fwd.argtypes = [vp] * 9 + [i] * 7 + [vp]
+        lib.kda_chunk_fwd.restype = i
+        lib.kda_recurrent_step.argtypes = [vp] * 7 + [i] * 5 + [vp]
+        lib.kda_recurrent_step.restype = i
+        lib.kda_get_device_error.argtypes = [vp, ctypes.POINTER(i)]
+        lib.kda_get_device_error.restype = i
+        lib.kda_last_error_message.restype = ctypes.c_char_p
+        lib.kda_status_string.restype = ctypes.c_char_p
+        lib.kda_status_string.argtypes = [i]
+        lib.kda_version.restype = ctypes.c_char_p
+        _lib = lib
+        return lib
+
+
+def _check(rc: int):
+    if rc != 0:
+        msg = load_library().kda_last_error_message().decode(errors="replace")
+        raise KDAError(rc, msg)
+
+
+def _dptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    if t.dtype == torch.float32:
+        return KDA_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _need(t: torch.Tensor, name: str, device, dtype=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def kda_chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, out=None,
+                  final_state=None, output_final_state: bool = True):
+    """Chunkwise KDA prefill.  q,k,g [B,T,H,dk]; v [B,T,H,dv]; beta [B,T,H];
+    states [N,H,dk,dv] fp32 (N = B, or len(cu_seqlens)-1 in varlen mode)."""
+    lib = load_library()
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("kda_chunk_fwd needs CUDA tensors (no CPU path)")
+    dt = q.dtype
+    _dtype_code(q)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dev, dt)
+    _need(g, "g", dev, torch.float32)
+    _need(beta, "beta", dev, torch.float32)
+    if k.shape != q.shape or g.shape != q.shape or v.shape[:3] != q.shape[:3] or beta.shape != q.shape[:3]:
+        raise ValueError("shape mismatch among q, k, v, g, beta")
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", dev, torch.int32)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    if initial_state is not None:
+        _need(initial_state, "initial_state", dev, torch.float32)
+        if tuple(initial_state.shape) != (N, H, dk, dv):
+            raise ValueError(f"initial_state must be [{N},{H},{dk},{dv}]")
+    if out is None:
+        out = torch.empty(B, T, H, dv, dtype=dt, device=dev)
+    else:
+        _need(out, "out", dev, dt)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    elif final_state is not None:
+        _need(final_state, "final_state", dev, torch.float32)
+    with torch.cuda.device(dev):
+        rc = lib.kda_chunk_fwd(_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta),
+                               _dptr(initial_state), _dptr(cu_seqlens), _dptr(out),
+                               _dptr(final_state), B, T, H, dk, dv, N, _dtype_code(q),
+                               _stream_handle(dev))
+    _check(rc)
+    return out, final_state
+
+
+def kda_recurrent_step(q, k, v, g, beta, state, out=None):
+    """One decode token per sequence.  q,k,g [N,H,dk]; v [N,H,dv]; beta [N,H];
+    state [N,H,dk,dv] fp32 updated in place.  Returns out [N,H,dv]."""
+    lib = load_library()
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("kda_recurrent_step needs CUDA tensors (no CPU path)")
+    dt = q.dtype
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dev, dt)
+    _need(g, "g", dev, torch.float32)
+    _need(beta, "beta", dev, torch.float32)
+    _need(state, "state", dev, torch.float32)
+    if tuple(state.shape) != (N, H, dk, dv):
+        raise ValueError(f"state must be [{N},{H},{dk},{dv}]")
+    if out is None:
+        out = torch.empty(N, H, dv, dtype=dt, device=dev)
+    else:
+        _need(out, "out", dev, dt)
+    with torch.cuda.device(dev):
+        rc = lib.kda_recurrent_step(_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta),
+                                    _dptr(state), _dptr(out), N, H, dk, dv, _dtype_code(q),
+                                    _stream_handle(dev))
+    _check(rc)
+    return out
+
+
+def kda_get_device_error(stream=None) -> int:
+    """Synchronise the stream and read-and-clear the device error word."""
+    lib = load_library()
+    code = ctypes.c_int(0)
+    handle = ctypes.c_void_p(stream.cuda_stream if stream is not None
+                             else torch.cuda.current_stream().cuda_stream)
+    rc = lib.kda_get_device_error(handle, ctypes.byref(code))
+    if rc not in (0, 4):
+        _check(rc)
+    return code.value

@@ -1,0 +1,138 @@
+// decode.cu -- the KDA recurrent decode step (one token per sequence).
+//
+// Kimi Linear paper notes (paper-notes-site): section 2 gives the recurrence,
+// section 3 the fused recurrent mode for short queries, which keeps only the
+// recurrent state.  Per (sequence, head):
+//     a = exp(g);  S' = Diag(a) S;  u = beta (v - S'^T k);
+//     S = S' + k u^T;  o = S^T q = S'^T q + (q.k) u
+// The state (dk x dv fp32, 64 KiB at d = 128) is read once and written once;
+// everything else is small.  The kernel is HBM-bound: one CTA streams one
+// state with 128-bit loads/stores, keeps it in registers while two column
+// reductions (k^T S', q^T S') run, and writes it back.
+//
+// Mapping (NT = 256 threads): thread t owns the float4 column group
+// t % (DV/4) of rows [rg*RPT, rg*RPT + RPT), rg = t / (DV/4).  At
+// DK = DV = 128 a warp covers one full 512-byte row per load instruction.
+// Column sums over rows: in-thread over RPT rows, then across row groups
+// through shared memory.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace kda {
+
+template <int DK, int DV, typename Tin>
+__global__ void __launch_bounds__(256, 2)
+decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
+                   const Tin *__restrict__ v, const float *__restrict__ g,
+                   const float *__restrict__ beta, float *__restrict__ state,
+                   Tin *__restrict__ out)
+{
+    constexpr int NT = 256;
+    constexpr int C4 = DV / 4;       // float4 groups per row
+    constexpr int RG = NT / C4;      // row groups
+    constexpr int RPT = DK / RG;     // rows per thread
+    static_assert(NT % C4 == 0 && DK % RG == 0, "bad decode tiling");
+
+    const size_t nh = blockIdx.x;    // flattened (sequence, head)
+    const int tid = threadIdx.x;
+    const int c4 = tid % C4;
+    const int rg = tid / C4;
+
+    __shared__ float ks[DK], qs[DK], as_[DK];
+    __shared__ __align__(16) float red_k[RG][DV + 4];
+    __shared__ __align__(16) float red_q[RG][DV + 4];
+    __shared__ __align__(16) float us[DV];
+    __shared__ float qk_part[NT / 32];
+
+    // 1. Issue every state load first (64 KiB in flight per CTA at d=128).
+    float4 *Sp = reinterpret_cast<float4 *>(state + nh * (size_t)(DK * DV));
+    float4 s[RPT];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) s[r] = ld_stream(Sp + (size_t)(rg * RPT + r) * C4 + c4);
+
+    // 2. Token vectors; alpha = exp(g).
+    float qk = 0.f;
+    if (tid < DK) {
+        const float kv = to_f(k[nh * DK + tid]);
+        const float qv = to_f(q[nh * DK + tid]);
+        ks[tid] = kv;
+        qs[tid] = qv;
+        as_[tid] = expf(g[nh * DK + tid]);
+        qk = kv * qv;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, o);
+    if ((tid & 31) == 0) qk_part[tid >> 5] = qk;
+    __syncthreads();
+
+    // 3. S' = Diag(a) S and the per-thread partial column sums.
+    float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+        const int row = rg * RPT + r;
+        const float a = as_[row], kr = ks[row], qr = qs[row];
+        s[r].x *= a; s[r].y *= a; s[r].z *= a; s[r].w *= a;
+        pk[0] += kr * s[r].x; pk[1] += kr * s[r].y; pk[2] += kr * s[r].z; pk[3] += kr * s[r].w;
+        pq[0] += qr * s[r].x; pq[1] += qr * s[r].y; pq[2] += qr * s[r].z; pq[3] += qr * s[r].w;
+    }
+    reinterpret_cast<float4 *>(&red_k[rg][0])[c4] = make_float4(pk[0], pk[1], pk[2], pk[3]);
+    reinterpret_cast<float4 *>(&red_q[rg][0])[c4] = make_float4(pq[0], pq[1], pq[2], pq[3]);
+    __syncthreads();
+
+    // 4. Finish the column sums; u = beta (v - S'^T k); o = S'^T q + (q.k) u.
+    if (tid < DV) {
+        float kS = 0.f, qS = 0.f;
+#pragma unroll
+        for (int i = 0; i < RG; ++i) { kS += red_k[i][tid]; qS += red_q[i][tid]; }
+        float qk_all = 0.f;
+#pragma unroll
+        for (int w = 0; w < NT / 32; ++w) qk_all += qk_part[w];
+        const float b = beta[nh];
+        const float u = b * (to_f(v[nh * DV + tid]) - kS);
+        us[tid] = u;
+        out[nh * DV + tid] = from_f<Tin>(qS + qk_all * u);
+    }
+    __syncthreads();
+
+    // 5. S = S' + k u^T, written once.
+    const float4 u4 = reinterpret_cast<const float4 *>(us)[c4];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+        const float kr = ks[rg * RPT + r];
+        float4 o4 = s[r];
+        o4.x += kr * u4.x; o4.y += kr * u4.y; o4.z += kr * u4.z; o4.w += kr * u4.w;
+        st_stream(Sp + (size_t)(rg * RPT + r) * C4 + c4, o4);
+    }
+}
+
+template <int DK, int DV, typename Tin>
+static cudaError_t launch_decode_t(const void *q, const void *k, const void *v,
+                                   const float *g, const float *beta, float *state,
+                                   void *out, int NH, cudaStream_t st)
+{
+    decode_step_kernel<DK, DV, Tin><<<NH, 256, 0, st>>>(
+        (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, state, (Tin *)out);
+    return cudaGetLastError();
+}
+
+template <typename Tin>
+static cudaError_t launch_decode_d(const void *q, const void *k, const void *v,
+                                   const float *g, const float *beta, float *state,
+                                   void *out, int NH, int dk, int dv, cudaStream_t st)
+{
+    if (dk == 128 && dv == 128) return launch_decode_t<128, 128, Tin>(q, k, v, g, beta, state, out, NH, st);
+    if (dk == 64 && dv == 64) return launch_decode_t<64, 64, Tin>(q, k, v, g, beta, state, out, NH, st);
+    if (dk == 128 && dv == 64) return launch_decode_t<128, 64, Tin>(q, k, v, g, beta, state, out, NH, st);
+    if (dk == 64 && dv == 128) return launch_decode_t<64, 128, Tin>(q, k, v, g, beta, state, out, NH, st);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, float *state, void *out, int NH, int dk,
+                          int dv, bool bf16, cudaStream_t st)
+{
+    if (bf16) return launch_decode_d<__nv_bfloat16>(q, k, v, g, beta, state, out, NH, dk, dv, st);
+    return launch_decode_d<float>(q, k, v, g, beta, state, out, NH, dk, dv, st);
+}
+
+}  // namespace kda

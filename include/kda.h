@@ -1,0 +1,143 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention (KDA) library.
+ *
+ * The token mixer (Kimi Linear paper notes, paper-notes-site, section 2,
+ * KDA recurrence equation; the bullet between the terms read as "+"):
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ *
+ * per (sequence, head), with an fp32 state S of shape dk x dv (row c = key
+ * channel c) and a per-channel decay alpha_t = exp(g_t).  Two entry points:
+ *
+ *   kda_chunk_fwd       prefill: the chunkwise-parallel form (chunk C = 64)
+ *                       of the paper notes, section 3 (old-state contribution
+ *                       through the chunk's transitions plus the intra-chunk
+ *                       writes, via a WY-like W,U representation);
+ *   kda_recurrent_step  decode: one token per sequence, the fused recurrent
+ *                       form the same section names for short queries.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers (cudaMalloc'd or any memory the
+ *     device can address), contiguous, row-major, 16-byte aligned (beta and
+ *     cu_seqlens: 4-byte aligned).  The
+ *     caller allocates and owns every buffer; the library keeps no pointer
+ *     after a call returns.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *     enqueued on it and the call returns without synchronising.
+ *   - g is log(alpha) (fp32, any finite value <= 0 is a decay; see the
+ *     per-function numerical range), beta is fp32.  q is used as given: no
+ *     scale, L2 norm, gate or sigmoid is applied inside.
+ *   - Argument errors return synchronously and enqueue nothing.  A failed
+ *     launch returns KDA_ERR_CUDA.  Conditions detected on the device (a
+ *     bounded wait that ran out) set a per-device error word that
+ *     kda_get_device_error() reports; no kernel traps.
+ *   - kda_last_error_message() gives a human-readable detail of the calling
+ *     thread's last failing call.
+ */
+#ifndef KDA_B200_H
+#define KDA_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, bad offsets */
+    KDA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (dk, dv, dtype) */
+    KDA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+    KDA_ERR_DEVICE = 4        /* the device error word was set */
+} kda_status;
+
+typedef enum {
+    KDA_F32 = 0,   /* q, k, v, out are float32 */
+    KDA_BF16 = 1   /* q, k, v, out are bfloat16 */
+} kda_dtype;
+
+/*
+ * kda_chunk_fwd -- prefill forward over whole sequences.
+ *
+ * Source: Kimi Linear paper notes (paper-notes-site), section 2 (recurrence)
+ * and section 3 (chunkwise parallel form; the layer passes initial_state and
+ * receives the final recurrent state); the whoami-wesleyyou blog, "context
+ * modification and checkpoint" section (a state is the checkpoint of its
+ * prefix: resuming from it continues the recurrence exactly).
+ *
+ * Layout (dense mode, cu_seqlens == NULL; N = B sequences of length T):
+ *   q, k   [B, T, H, dk]  dtype        v    [B, T, H, dv]  dtype
+ *   g      [B, T, H, dk]  float32      beta [B, T, H]      float32
+ *   out    [B, T, H, dv]  dtype (written, rounded to nearest even for bf16)
+ *   initial_state [N, H, dk, dv] float32, or NULL for zeros
+ *   final_state   [N, H, dk, dv] float32, or NULL to skip; it may equal
+ *                 initial_state (in-place resume)
+ * Varlen mode (cu_seqlens != NULL): B must be 1; cu_seqlens is a device
+ *   int32 array [num_seqs + 1] with cu[0] = 0, non-decreasing, cu[num_seqs] =
+ *   T; sequence n is tokens [cu[n], cu[n+1]).  Zero-length sequences are
+ *   allowed (final = initial).  The offsets are read on the device; they are
+ *   not validated there beyond clamping to [0, T].
+ *   In dense mode num_seqs is ignored (N = B).
+ *
+ * Supported: dtype KDA_BF16 with dk = dv = 128 (tensor-core path), and
+ *   KDA_F32 with dk, dv in {64, 128} (exact fp32 path).  Others return
+ *   KDA_ERR_UNSUPPORTED.
+ * Numerical range (bf16 path): per-token g >= -5 keeps every exponent the
+ *   chunk form takes within fp32 range (sub-chunks of 16 tokens).
+ * Aliasing: out must not overlap any input.
+ * Memory: the bf16 path takes a stream-ordered scratch buffer from a
+ *   library-private pool on the current device (cudaMallocFromPoolAsync on
+ *   `stream`), freed stream-ordered before the call returns; the pool keeps
+ *   the memory for reuse by later calls.
+ */
+kda_status kda_chunk_fwd(const void *q, const void *k, const void *v,
+                         const float *g, const float *beta,
+                         const float *initial_state, const int32_t *cu_seqlens,
+                         void *out, float *final_state,
+                         int B, int T, int H, int dk, int dv, int num_seqs,
+                         kda_dtype dtype, void *stream);
+
+/*
+ * kda_recurrent_step -- one decode token for each of N sequences.
+ *
+ * Source: Kimi Linear paper notes (paper-notes-site), section 2 (recurrence)
+ * and section 3 (the fused recurrent mode used for short queries outside
+ * training: only the recurrent state is kept).
+ *
+ * Layout: q, k [N, H, dk] dtype; v [N, H, dv] dtype; g [N, H, dk] float32;
+ *   beta [N, H] float32; state_inout [N, H, dk, dv] float32, read and
+ *   overwritten in place with S_t; out [N, H, dv] dtype.
+ * Computes a = exp(g); S' = Diag(a) S; u = beta (v - S'^T k);
+ *   S = S' + k u^T; o = S^T q, reading and writing each state once.
+ * Supported: dk, dv in {64, 128}, dtype KDA_BF16 or KDA_F32.  Any finite g.
+ * Aliasing: out must not overlap any input; state_inout must not overlap
+ *   the token inputs.
+ */
+kda_status kda_recurrent_step(const void *q, const void *k, const void *v,
+                              const float *g, const float *beta,
+                              float *state_inout, void *out,
+                              int N, int H, int dk, int dv,
+                              kda_dtype dtype, void *stream);
+
+/* Static string for a status code. */
+const char *kda_status_string(kda_status s);
+
+/* Detail of the calling thread's last failing call ("" if none). */
+const char *kda_last_error_message(void);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's error
+ * word.  *code_out (may be NULL) receives the raw word (0 = clean).
+ * Returns KDA_OK if the word was 0, KDA_ERR_DEVICE if it was set, or
+ * KDA_ERR_CUDA if the synchronisation failed.
+ */
+kda_status kda_get_device_error(void *stream, int *code_out);
+
+/* Library version, "major.minor.patch". */
+const char *kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KDA_B200_H */

@@ -1,0 +1,119 @@
+"""Host-side checks of the C-ABI library (no GPU needed).
+
+The library must load, export every function include/kda.h declares, and
+reject bad arguments synchronously (before any CUDA call) with the status the
+header documents.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_88_b200 as kda
+from gated_delta_rule_88_b200 import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return kda.load_library()
+
+
+def declared_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not h.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", h)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(kda_\w+)\s*\(", src, flags=re.M)
+    return names
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ("kda_chunk_fwd", "kda_recurrent_step", "kda_status_string",
+              "kda_get_device_error", "kda_last_error_message", "kda_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_status_strings(lib):
+    assert lib.kda_status_string(0) == b"KDA_OK"
+    assert lib.kda_status_string(1) == b"KDA_ERR_INVALID_ARG"
+    assert lib.kda_status_string(2) == b"KDA_ERR_UNSUPPORTED"
+    assert lib.kda_version().decode().count(".") == 2
+
+
+FAKE = 0x10000  # a 16-byte aligned fake device address; never dereferenced
+
+
+def chunk(lib, *, q=FAKE, k=FAKE, v=FAKE, g=FAKE, b=FAKE, s0=None, cu=None, out=FAKE,
+          sT=None, B=1, T=64, H=1, dk=128, dv=128, N=1, dtype=1):
+    P = ctypes.c_void_p
+    return lib.kda_chunk_fwd(P(q), P(k), P(v), P(g), P(b), P(s0), P(cu), P(out), P(sT),
+                             B, T, H, dk, dv, N, dtype, None)
+
+
+def step(lib, *, q=FAKE, k=FAKE, v=FAKE, g=FAKE, b=FAKE, s=FAKE, out=FAKE, N=1, H=1,
+         dk=128, dv=128, dtype=1):
+    P = ctypes.c_void_p
+    return lib.kda_recurrent_step(P(q), P(k), P(v), P(g), P(b), P(s), P(out), N, H, dk, dv,
+                                  dtype, None)
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "g", "b", "out"])
+def test_chunk_null_pointer_rejected(lib, field):
+    assert chunk(lib, **{field: 0}) == 1
+    assert b"null" in lib.kda_last_error_message()
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(T=-1), dict(H=0), dict(dk=0), dict(dv=-3),
+                                dict(dtype=7), dict(B=2, cu=FAKE, N=2),
+                                dict(cu=FAKE, N=0), dict(q=FAKE + 8), dict(s0=FAKE + 4),
+                                dict(cu=FAKE + 2, N=1), dict(b=FAKE + 2), dict(B=70000),
+                                dict(T=1 << 30, B=4)])
+def test_chunk_bad_arguments_rejected(lib, kw):
+    assert chunk(lib, **kw) == 1
+
+
+@pytest.mark.parametrize("kw", [dict(dk=96, dv=96), dict(dk=128, dv=64), dict(dk=64, dv=64),
+                                dict(dtype=0, dk=32, dv=64), dict(dtype=0, dk=128, dv=256)])
+def test_chunk_unsupported_rejected(lib, kw):
+    assert chunk(lib, **kw) == 2
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "g", "b", "s", "out"])
+def test_step_null_pointer_rejected(lib, field):
+    assert step(lib, **{field: 0}) == 1
+
+
+@pytest.mark.parametrize("kw", [dict(N=-1), dict(H=0), dict(dtype=5), dict(s=FAKE + 8), dict(b=FAKE + 1),
+                                dict(N=1 << 20, H=1 << 12)])
+def test_step_bad_arguments_rejected(lib, kw):
+    assert step(lib, **kw) == 1
+
+
+@pytest.mark.parametrize("kw", [dict(dk=32), dict(dv=96), dict(dk=256, dv=256)])
+def test_step_unsupported_rejected(lib, kw):
+    assert step(lib, **kw) == 2
+
+
+def test_step_empty_batch_is_a_no_op(lib):
+    assert step(lib, N=0) == 0
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 4, 1, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        kda.kda_chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))
+    with pytest.raises(ValueError, match="CUDA"):
+        kda.kda_recurrent_step(x[0], x[0], x[0], x[0], torch.zeros(4, 1), torch.zeros(4, 1, 64, 64))

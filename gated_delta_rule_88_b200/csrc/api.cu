@@ -4,11 +4,14 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <mutex>
+
 #include <cuda_runtime.h>
 
 #include "../../include/kda.h"
 #include "common.cuh"
 #include "kernels.h"
+#include "chunk_ws.h"
 
 namespace kda {
 // The per-device error word (see common.cuh).  Host code reaches it through
@@ -45,6 +48,38 @@ kda_status cuda_fail(cudaError_t e, const char *what) {
 }
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Library-private stream-ordered memory pool per device.  Its release
+// threshold is unbounded, so scratch freed at the end of a call stays
+// reserved for the next one instead of returning to the driver.
+cudaError_t get_pool(cudaMemPool_t *out, int *sm_count) {
+    static std::mutex mu;
+    static cudaMemPool_t pools[64] = {};
+    static int sms[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!pools[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t p;
+        e = cudaMemPoolCreate(&p, &props);
+        if (e != cudaSuccess) return e;
+        uint64_t thr = ~0ull;
+        e = cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &thr);
+        if (e != cudaSuccess) return e;
+        e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        pools[dev] = p;
+    }
+    *out = pools[dev];
+    *sm_count = sms[dev];
+    return cudaSuccess;
+}
 
 }  // namespace
 
@@ -154,7 +189,46 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const floa
         if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd(f32) launch");
         return KDA_OK;
     }
-    return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd(bf16): dk=%d dv=%d not supported", dk, dv);
+    if (dk != 128 || dv != 128)
+        return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd(bf16): dk=%d dv=%d (supported: 128, 128)",
+                    dk, dv);
+    if (N == 0 || total_T == 0) {
+        // nothing to process: final = initial (or zeros)
+        if (final_state) {
+            const size_t bytes = (size_t)N * H * dk * dv * sizeof(float);
+            cudaError_t e = initial_state
+                ? (initial_state == final_state ? cudaSuccess
+                   : cudaMemcpyAsync(final_state, initial_state, bytes, cudaMemcpyDeviceToDevice, st))
+                : cudaMemsetAsync(final_state, 0, bytes, st);
+            if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd(bf16) empty input");
+        }
+        return KDA_OK;
+    }
+    const long long max_chunks = cu_seqlens ? (total_T + 63) / 64 + N : (long long)B * ((T + 63) / 64);
+    const size_t coff_bytes = (((size_t)N + 1) * sizeof(int32_t) + 255) & ~(size_t)255;
+    const size_t bytes = coff_bytes + (size_t)max_chunks * H * kda::ws::RECORD;
+    cudaMemPool_t pool;
+    int sms = 148;
+    cudaError_t e = get_pool(&pool, &sms);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd(bf16) memory pool");
+    void *scratch = nullptr;
+    e = cudaMallocFromPoolAsync(&scratch, bytes, pool, st);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd(bf16) scratch allocation");
+    int32_t *coff = (int32_t *)scratch;
+    unsigned char *records = (unsigned char *)scratch + coff_bytes;
+    const long long units = (long long)N * H;
+    const int dvt = units * 8 <= sms ? 16 : units * 4 <= sms ? 32 : 64;
+    if (cu_seqlens) e = kda::launch_chunk_plan(cu_seqlens, N, (int)total_T, coff, st);
+    if (e == cudaSuccess)
+        e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, coff, N, T, (int)total_T, H,
+                                   (int)max_chunks, records, st);
+    if (e == cudaSuccess)
+        e = kda::launch_chunk_chain(records, cu_seqlens, coff, initial_state, final_state, out, N,
+                                    T, (int)total_T, H, dvt, (int)max_chunks, kda::error_word(), st);
+    cudaError_t e2 = cudaFreeAsync(scratch, st);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd(bf16) launch");
+    if (e2 != cudaSuccess) return cuda_fail(e2, "kda_chunk_fwd(bf16) scratch release");
+    return KDA_OK;
 }
 
 }  // extern "C"

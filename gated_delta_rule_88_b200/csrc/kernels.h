@@ -6,6 +6,9 @@
 
 namespace kda {
 
+// Address of the current device's error word (see common.cuh), or nullptr.
+int *error_word();
+
 // One decode step for NH = N*H (sequence, head) pairs; state updated in place.
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
                           const float *beta, float *state, void *out, int NH, int dk,
@@ -19,5 +22,21 @@ cudaError_t launch_chunk_f32(const float *q, const float *k, const float *v, con
                              const float *beta, const float *s0, const int32_t *cu,
                              float *out, float *sT, int N, int T, int total_T, int H,
                              int dk, int dv, cudaStream_t st);
+
+// bf16 tensor-core prefill (dk = dv = 128) in two launches over a scratch
+// buffer of per-(chunk, head) records (chunk_ws.h):
+//   chunk_plan  (varlen only) chunk offsets per sequence -> coff[N+1]
+//   chunk_prep  parallel over (chunk, head): G, A, P, T, W, U, Qg, Kt, e^{G_C}
+//   chunk_chain sequential over chunks per (sequence, head, dv tile)
+size_t chunk_prep_smem_bytes();
+cudaError_t launch_chunk_plan(const int32_t *cu, int N, int total_T, int32_t *coff,
+                              cudaStream_t st);
+cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, const int32_t *cu, const int32_t *coff,
+                              int N, int T, int total_T, int H, int max_chunks,
+                              unsigned char *wsp, cudaStream_t st);
+cudaError_t launch_chunk_chain(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
+                               const float *s0, float *sT, void *out, int N, int T, int total_T,
+                               int H, int dvt, int max_chunks, int *err, cudaStream_t st);
 
 }  // namespace kda

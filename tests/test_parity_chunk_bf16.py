@@ -1,0 +1,146 @@
+"""GPU parity: kda_chunk_fwd with bf16 inputs (tensor-core chunk path) vs the
+fp64 oracle.  Tolerance: ||x - ref||_inf / ||ref||_inf <= 2e-2 on outputs and
+on each final state (fp32 state)."""
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_88_b200 import kda_chunk_fwd, kda_get_device_error
+from gated_delta_rule_88_b200 import workloads as W
+from helpers import assert_close, rel_inf, rms_rel
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+BF = torch.bfloat16
+
+
+def _run(inp, **kw):
+    d = inp.to(DEV)
+    o, sT = kda_chunk_fwd(d.q, d.k, d.v, d.g, d.beta, d.initial_state, d.cu_seqlens, **kw)
+    torch.cuda.synchronize()
+    assert kda_get_device_error() == 0
+    return o, sT
+
+
+def _check(inp, heads=None):
+    o, sT = _run(inp)
+    o_ref, s_ref = oracle.forward(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.initial_state,
+                                  inp.cu_seqlens, heads=heads)
+    if heads is not None:
+        o, sT = o[:, :, heads], sT[:, heads]
+        o_ref, s_ref = o_ref[:, :, heads], s_ref[:, heads]
+    assert_close(o, o_ref, BF, "o")
+    for n in range(sT.shape[0]):
+        assert_close(sT[n], s_ref[n], BF, f"final state {n}")
+    return o, sT, o_ref, s_ref
+
+
+@pytest.mark.parametrize("T", [1, 16, 63, 64, 65, 127, 200, 333])
+def test_ragged_lengths(T):
+    _check(W.prefill(2, T, 3, 128, 128, BF, seed=100 + T, initial_state_std=0.02))
+
+
+def test_zero_initial_state_null_pointer():
+    _check(W.prefill(1, 300, 4, 128, 128, BF, seed=9))
+
+
+@pytest.mark.parametrize("gate", ["offset16", "zero"])
+def test_gate_variants(gate):
+    _check(W.prefill(1, 257, 3, 128, 128, BF, seed=4, gate=gate, initial_state_std=0.02))
+
+
+def test_strongest_supported_decay():
+    """per-token g at the documented floor (-5) on a third of the channels:
+    every sub-chunk exponent sits at its extreme"""
+    inp = W.prefill(1, 256, 2, 128, 128, BF, seed=12, initial_state_std=0.02)
+    inp.g[..., ::3] = -5.0
+    _check(inp)
+
+
+def test_varlen_with_empty_and_short_sequences():
+    inp = W.prefill(1, 0, 3, 128, 128, BF, seed=21, initial_state_std=0.02,
+                    seq_lens=[70, 0, 1, 128, 0, 200, 64, 65])
+    o, sT, _, _ = _check(inp)
+    assert torch.equal(sT[1].cpu(), inp.initial_state[1])
+    assert torch.equal(sT[4].cpu(), inp.initial_state[4])
+
+
+def test_varlen_equals_separate_runs():
+    lens = [100, 37, 256]
+    inp = W.prefill(1, 0, 2, 128, 128, BF, seed=31, initial_state_std=0.02, seq_lens=lens)
+    o, sT = _run(inp)
+    d = inp.to(DEV)
+    cu = inp.cu_seqlens.tolist()
+    for n in range(len(lens)):
+        s, e = cu[n], cu[n + 1]
+        on, sn = kda_chunk_fwd(d.q[:, s:e].contiguous(), d.k[:, s:e].contiguous(),
+                               d.v[:, s:e].contiguous(), d.g[:, s:e].contiguous(),
+                               d.beta[:, s:e].contiguous(), d.initial_state[n:n + 1].contiguous())
+        # same kernels, same chunk boundaries -> identical results
+        assert torch.equal(on, o[:, s:e])
+        assert torch.equal(sn[0], sT[n])
+
+
+def test_split_resume_matches_unsplit():
+    inp = W.prefill(1, 400, 2, 128, 128, BF, seed=5, initial_state_std=0.02)
+    d = inp.to(DEV)
+    o, s = kda_chunk_fwd(d.q, d.k, d.v, d.g, d.beta, d.initial_state)
+    cut = 150   # not a multiple of the chunk length
+    sl = lambda x, a, b: x[:, a:b].contiguous()
+    oa, sa = kda_chunk_fwd(sl(d.q, 0, cut), sl(d.k, 0, cut), sl(d.v, 0, cut), sl(d.g, 0, cut),
+                           sl(d.beta, 0, cut), d.initial_state)
+    ob, sb = kda_chunk_fwd(sl(d.q, cut, 400), sl(d.k, cut, 400), sl(d.v, cut, 400),
+                           sl(d.g, cut, 400), sl(d.beta, cut, 400), sa)
+    assert_close(torch.cat([oa, ob], 1), o, BF, "o split")
+    assert_close(sb, s, BF, "state split")
+    o_ref, s_ref = oracle.forward(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.initial_state)
+    assert_close(torch.cat([oa, ob], 1), o_ref, BF, "o split vs oracle")
+    assert_close(sb, s_ref, BF, "state split vs oracle")
+
+
+def test_inplace_state_and_no_final_state():
+    inp = W.prefill(1, 130, 2, 128, 128, BF, seed=8, initial_state_std=0.02)
+    d = inp.to(DEV)
+    o_ref, s_ref = oracle.forward(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.initial_state)
+    st = d.initial_state.clone()
+    o, s = kda_chunk_fwd(d.q, d.k, d.v, d.g, d.beta, st, final_state=st)
+    torch.cuda.synchronize()
+    assert_close(st, s_ref, BF, "in-place state")
+    o2, s2 = kda_chunk_fwd(d.q, d.k, d.v, d.g, d.beta, d.initial_state, output_final_state=False)
+    assert s2 is None
+    assert torch.equal(o2, o)
+
+
+def test_prefill_t8192_h32_full():
+    """The T = 8192, H = 32 workload, every head against the oracle."""
+    inp = W.named_prefill("prefill_t8192_h32_d128")
+    o, sT, o_ref, s_ref = _check(inp)
+    print(f"o rel {rel_inf(o, o_ref):.2e} rms {rms_rel(o, o_ref):.2e}; "
+          f"S rel {rel_inf(sT, s_ref):.2e}")
+
+
+def test_prefill_t65536_h32_sampled_heads():
+    """The T = 65536, H = 32 long-memory workload; four heads, full length."""
+    inp = W.named_prefill("prefill_t65536_h32_d128")
+    _check(inp, heads=[0, 9, 22, 31])
+
+
+def test_varlen8_resume_sampled_heads():
+    """8 packed sequences, lengths U[1024, 32768], per-sequence initial states.
+    Each sequence is also split at a non-multiple of 64 and resumed; the
+    resumed run must match the unsplit one and the oracle."""
+    inp = W.named_prefill("varlen8_h32_d128_resume")
+    heads = [0, 13, 31]
+    o, sT, o_ref, s_ref = _check(inp, heads=heads)
+    d = inp.to(DEV)
+    cu = inp.cu_seqlens.tolist()
+    for n in range(8):
+        s, e = cu[n], cu[n + 1]
+        cut = s + (e - s) // 3 + 17
+        sl = lambda x, a, b: x[:, a:b].contiguous()
+        _, sa = kda_chunk_fwd(sl(d.q, s, cut), sl(d.k, s, cut), sl(d.v, s, cut), sl(d.g, s, cut),
+                              sl(d.beta, s, cut), d.initial_state[n:n + 1].contiguous())
+        ob, sb = kda_chunk_fwd(sl(d.q, cut, e), sl(d.k, cut, e), sl(d.v, cut, e), sl(d.g, cut, e),
+                               sl(d.beta, cut, e), sa)
+        assert_close(sb[0][heads], s_ref[n][heads], BF, f"resumed state {n}")
+        assert_close(ob[:, :, heads], o_ref[:, cut:e][:, :, heads], BF, f"resumed o {n}")

@@ -31,9 +31,13 @@ int *error_word() {
 }
 }  // namespace kda
 
-namespace {
-
+namespace kda {
+// Detail of the calling thread's last failing call (kda_last_error_message).
 thread_local char t_msg[512] = "";
+}  // namespace kda
+
+namespace {
+using kda::t_msg;
 
 kda_status fail(kda_status s, const char *fmt, ...) {
     va_list ap;

@@ -120,6 +120,42 @@ kda_status kda_recurrent_step(const void *q, const void *k, const void *v,
                               int N, int H, int dk, int dv,
                               kda_dtype dtype, void *stream);
 
+/*
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate
+ * device memory.  The paper has no counterpart: this is a deployment variant
+ * of the bf16 chunked prefill.
+ *
+ * Who needs it: code running inside a host application that owns all device
+ * memory and forbids its components from allocating (an inference engine that
+ * reserves its whole budget up front, where an extra cudaMalloc fails or
+ * breaks its accounting), and code on paths where an allocation call is not
+ * permitted.  This entry point calls no cudaMalloc, cudaFree or other
+ * allocating routine; its scratch is a fixed 32 MiB device array inside the
+ * library (allocated once on every device that loads the library, kept until
+ * the process exits).
+ *
+ * Arguments, layouts and results are those of kda_chunk_fwd.  Supported:
+ * KDA_BF16 with dk = dv = 128 only (other dtypes/dims: KDA_ERR_UNSUPPORTED).
+ * Size limit: it returns KDA_ERR_INVALID_ARG, with the needed and the
+ * available byte counts in kda_last_error_message(), when
+ *     roundup256(4 * (N + 1)) + slots * H * 74240 > 32 MiB,
+ * where slots = B * ceil(T / 64) in dense mode and ceil(T / 64) + num_seqs in
+ * varlen mode (e.g. 451 (chunk, head) slots: T = 1024 with H <= 28).
+ * First call on a device: it looks up the array's device address there
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture on the device.
+ * Concurrency: every call uses the same array, which keeps the previous
+ * call's contents (nothing in it needs to start cleared).  Calls whose work
+ * overlaps on the GPU -- on different streams, or from different threads --
+ * race on it; serialise them.
+ */
+kda_status kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
+                                 const float *g, const float *beta,
+                                 const float *initial_state, const int32_t *cu_seqlens,
+                                 void *out, float *final_state,
+                                 int B, int T, int H, int dk, int dv, int num_seqs,
+                                 kda_dtype dtype, void *stream);
+
 /* Static string for a status code. */
 const char *kda_status_string(kda_status s);
 

@@ -27,43 +27,33 @@ namespace {
 constexpr int C = ws::C;
 constexpr int D = ws::D;
 constexpr int NT = 256;
-constexpr int PB = D + 8;
-constexpr int PP = C + 8;
 
 template <int DVT>
-struct ChainSmem {
+struct __align__(1024) ChainSmem {
     static constexpr int PV = DVT + 8;
-    __nv_bfloat16 AW[2][2 * C][PB];   // rows 0-63: W, rows 64-127: Qg
-    __nv_bfloat16 KT[2][C][PB];       // Kt
-    __nv_bfloat16 Pm[2][C][PP];       // P
-    __nv_bfloat16 Ut[2][C][PV];       // U tile
+    static constexpr int UT = DVT > 32 ? DVT / 32 : 1;   // U tiles of 32 columns
+    unsigned char AW[2][32768];       // [W; Qg], K-major SW128 image (chunk_ws.h)
+    unsigned char KTT[2][16384];      // Kt^T, K-major SW128 image
+    unsigned char Pm[2][8192];        // P, K-major SW128 image
+    unsigned char Ut[2][UT * 4096];   // U tile(s), plain [64][32]
     float eGC[2][D];
     __nv_bfloat16 Sb[D][PV];          // bf16 copy of the state tile
     __nv_bfloat16 Vn[C][PV];          // V_new (bf16)
 };
 
+// byte offset of 16-byte chunk j (0..7) of row r in a SW128 image
+__device__ __forceinline__ int sw_chunk(int r, int j) { return r * 128 + ((j ^ (r & 7)) << 4); }
+
 template <int DVT>
 __device__ __forceinline__ void load_record(ChainSmem<DVT> &sm, int buf, const unsigned char *rec,
                                             int n0, int tid)
 {
-    // [W; Qg]: 128 rows x 256 B
-    for (int i = tid; i < 2 * C * (D / 8); i += NT) {
-        const int r = i / (D / 8), c8 = (i % (D / 8)) * 8;
-        const size_t off = (r < C ? ws::OFF_W : ws::OFF_QG) + ((size_t)(r & (C - 1)) * D + c8) * 2;
-        cp_async16(&sm.AW[buf][r][c8], rec + off);
-    }
-    for (int i = tid; i < C * (D / 8); i += NT) {
-        const int r = i / (D / 8), c8 = (i % (D / 8)) * 8;
-        cp_async16(&sm.KT[buf][r][c8], rec + ws::OFF_KT + ((size_t)r * D + c8) * 2);
-    }
-    for (int i = tid; i < C * (C / 8); i += NT) {
-        const int r = i / (C / 8), c8 = (i % (C / 8)) * 8;
-        cp_async16(&sm.Pm[buf][r][c8], rec + ws::OFF_P + ((size_t)r * C + c8) * 2);
-    }
-    for (int i = tid; i < C * (DVT / 8); i += NT) {
-        const int r = i / (DVT / 8), c8 = (i % (DVT / 8)) * 8;
-        cp_async16(&sm.Ut[buf][r][c8], rec + ws::OFF_U + ((size_t)r * D + n0 + c8) * 2);
-    }
+    constexpr int UT = ChainSmem<DVT>::UT;
+    for (int i = tid; i < 32768 / 16; i += NT) cp_async16(&sm.AW[buf][i * 16], rec + ws::OFF_AW + i * 16);
+    for (int i = tid; i < 16384 / 16; i += NT) cp_async16(&sm.KTT[buf][i * 16], rec + ws::OFF_KTT + i * 16);
+    for (int i = tid; i < 8192 / 16; i += NT) cp_async16(&sm.Pm[buf][i * 16], rec + ws::OFF_P + i * 16);
+    const unsigned char *u = rec + ws::OFF_U + (size_t)(n0 >> 5) * ws::U_TILE;
+    for (int i = tid; i < UT * 4096 / 16; i += NT) cp_async16(&sm.Ut[buf][i * 16], u + i * 16);
     if (tid < D / 4) cp_async16(&sm.eGC[buf][tid * 4], rec + ws::OFF_EGC + tid * 16);
 }
 
@@ -75,7 +65,7 @@ chunk_chain_kernel(const unsigned char *__restrict__ wsp, const int32_t *__restr
                    int H, int cps, int max_chunks, int *__restrict__ err)
 {
     constexpr int NTN = DVT / 8;      // n-tiles of 8 columns
-    extern __shared__ __align__(16) unsigned char smem_raw[];
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
     ChainSmem<DVT> &sm = *reinterpret_cast<ChainSmem<DVT> *>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tig = lane & 3;
@@ -127,9 +117,8 @@ chunk_chain_kernel(const unsigned char *__restrict__ wsp, const int32_t *__restr
     cp_async_commit();
 
     // ldmatrix lane offsets
-    const int a_row = (lane & 7) + 8 * ((lane >> 3) & 1), a_col = 8 * (lane >> 4);
+    const int a_row = (lane & 7) + 8 * ((lane >> 3) & 1);
     const int bt_k = (lane & 7) + 8 * ((lane >> 3) & 1), bt_n = 8 * (lane >> 4);
-    const int at_k = (lane & 7) + 8 * (lane >> 4), at_m = 8 * ((lane >> 3) & 1);
 
     for (int ci = 0; ci < nchunks; ++ci) {
         const int buf = ci & 1;
@@ -146,7 +135,10 @@ chunk_chain_kernel(const unsigned char *__restrict__ wsp, const int32_t *__restr
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
             uint32_t a[4];
-            ldsm_x4(a, &sm.AW[buf][16 * warp + a_row][16 * ks + a_col]);
+            {
+                const int r = 16 * warp + a_row, jj = 2 * ks + (lane >> 4);
+                ldsm_x4(a, &sm.AW[buf][(jj >> 3) * 16384 + sw_chunk(r, jj & 7)]);
+            }
 #pragma unroll
             for (int np = 0; np < NTN / 2; ++np) {
                 uint32_t b[4];
@@ -161,8 +153,10 @@ chunk_chain_kernel(const unsigned char *__restrict__ wsp, const int32_t *__restr
 #pragma unroll
             for (int nt = 0; nt < NTN; ++nt) {
                 const int c = 8 * nt + 2 * tig;
-                const __nv_bfloat162 u0 = *reinterpret_cast<const __nv_bfloat162 *>(&sm.Ut[buf][r0][c]);
-                const __nv_bfloat162 u1 = *reinterpret_cast<const __nv_bfloat162 *>(&sm.Ut[buf][r0 + 8][c]);
+                const int lc = (n0 & 31) + c;   // column within the loaded U tile(s)
+                const unsigned char *ut = &sm.Ut[buf][(lc >> 5) * 4096 + ((lc & 31) << 1)];
+                const __nv_bfloat162 u0 = *reinterpret_cast<const __nv_bfloat162 *>(ut + r0 * 64);
+                const __nv_bfloat162 u1 = *reinterpret_cast<const __nv_bfloat162 *>(ut + (r0 + 8) * 64);
                 *reinterpret_cast<uint32_t *>(&sm.Vn[r0][c]) =
                     pack_bf16(__low2float(u0) - acc[nt][0], __high2float(u0) - acc[nt][1]);
                 *reinterpret_cast<uint32_t *>(&sm.Vn[r0 + 8][c]) =
@@ -175,7 +169,7 @@ chunk_chain_kernel(const unsigned char *__restrict__ wsp, const int32_t *__restr
             const int I = warp - 4;
             for (int ks = 0; ks <= I; ++ks) {
                 uint32_t a[4];
-                ldsm_x4(a, &sm.Pm[buf][16 * I + a_row][16 * ks + a_col]);
+                ldsm_x4(a, &sm.Pm[buf][sw_chunk(16 * I + a_row, 2 * ks + (lane >> 4))]);
 #pragma unroll
                 for (int np = 0; np < NTN / 2; ++np) {
                     uint32_t b[4];
@@ -207,7 +201,7 @@ chunk_chain_kernel(const unsigned char *__restrict__ wsp, const int32_t *__restr
 #pragma unroll
             for (int ks = 0; ks < C / 16; ++ks) {
                 uint32_t a[4];
-                ldsm_x4_t(a, &sm.KT[buf][16 * ks + at_k][16 * warp + at_m]);
+                ldsm_x4(a, &sm.KTT[buf][sw_chunk(16 * warp + a_row, 2 * ks + (lane >> 4))]);
 #pragma unroll
                 for (int np = 0; np < NTN / 2; ++np) {
                     uint32_t b[4];
@@ -253,9 +247,9 @@ cudaError_t launch_chain_t(const unsigned char *wsp, const int32_t *cu, const in
 
 }  // namespace
 
-cudaError_t launch_chunk_chain(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
-                               const float *s0, float *sT, void *out, int N, int T, int total_T,
-                               int H, int dvt, int max_chunks, int *err, cudaStream_t st)
+cudaError_t launch_chunk_chain_mma(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
+                                   const float *s0, float *sT, void *out, int N, int T, int total_T,
+                                   int H, int dvt, int max_chunks, int *err, cudaStream_t st)
 {
     switch (dvt) {
         case 16: return launch_chain_t<16>(wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st);
@@ -265,4 +259,17 @@ cudaError_t launch_chunk_chain(const unsigned char *wsp, const int32_t *cu, cons
     return cudaErrorInvalidValue;
 }
 
+}  // namespace kda
+
+#include <stdlib.h>
+namespace kda {
+cudaError_t launch_chunk_chain(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
+                               const float *s0, float *sT, void *out, int N, int T, int total_T,
+                               int H, int dvt, int max_chunks, int *err, cudaStream_t st)
+{
+    static const char *mode = getenv("KDA_CHAIN");
+    if (mode && mode[0] == 'm')
+        return launch_chunk_chain_mma(wsp, cu, coff, s0, sT, out, N, T, total_T, H, dvt, max_chunks, err, st);
+    return launch_chunk_chain_tc(wsp, cu, coff, s0, sT, out, N, T, total_T, H, dvt, max_chunks, err, st);
+}
 }  // namespace kda

@@ -1,0 +1,320 @@
+// chunk_chain_tc.cu -- the sequential inter-chunk pass of the bf16 KDA prefill
+// on the Blackwell tensor cores (tcgen05 MMAs, accumulators in TMEM, records
+// streamed by bulk async copies).  dk = dv = 128, C = 64.
+//
+// Kimi Linear paper notes (paper-notes-site), section 3: only the fixed-size
+// state passes between chunks; the output is the inter-chunk part plus the
+// intra-chunk part.  With the per-chunk record of chunk_ws.h, for each chunk in
+// order and one DVT-column tile of the fp32 state S (dk x DVT):
+//     MMA1  D1 = [W; Qg] S            (M = 128: rows 0-63 W S, 64-127 Qg S)
+//           V_new = U - (W S)         (threads 0-63, one token row each)
+//     MMA2  D1 += [* ; P] V_new       (rows 64-127 become O = Qg S + P V_new)
+//     MMA3  D3 = Kt^T V_new           (M = 128 channels)
+//           S <- Diag(e^{G_C}) S + D3 (threads 0-127, one channel row each)
+// The state stays in fp32 registers for the whole sequence; its bf16 copy is
+// the B operand of MMA1.  A operands come straight from the record (K-major,
+// 128-byte swizzle); B operands (S, V_new) are written by the threads in the
+// MN-major interleaved layout.
+//
+// Roles (160 threads): warps 0-3 own TMEM lanes 0-127 (thread t = token row
+// t for D1, channel row t for D3); thread 0 also issues the MMAs.  Warp 4
+// lane 0 streams records into an NS-stage shared-memory ring with
+// cp.async.bulk (plain, no multicast) and mbarrier transaction counts.
+// Every wait is bounded: a wait that runs out sets the device error word and
+// the whole CTA leaves its loop together (OR-reduced barrier), waits (bounded)
+// for copies in flight, frees TMEM and returns.
+#include "chunk_ws.h"
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace kda {
+namespace {
+
+using namespace sm100;
+
+constexpr int C = ws::C;
+constexpr int D = ws::D;
+constexpr int NTHREADS = 160;
+constexpr uint32_t REC_HEAD = 57344;       // [W;Qg] + Kt^T + P, contiguous in the record
+
+template <int DVT, int NS>
+struct TcLayout {
+    static constexpr int UT = DVT > 32 ? 2 : 1;
+    static constexpr uint32_t U_OFF = REC_HEAD;
+    static constexpr uint32_t EGC_OFF = REC_HEAD + UT * 4096;
+    static constexpr uint32_t STAGE = ((EGC_OFF + 512 + 1023) / 1024) * 1024;
+    static constexpr uint32_t TX = REC_HEAD + UT * 4096 + 512;
+    static constexpr uint32_t B1_OFF = NS * STAGE;                 // S^bf16: K=128 x N=DVT
+    static constexpr uint32_t B2_OFF = B1_OFF + 128 * DVT * 2;     // V_new: K=64 x N=DVT
+    static constexpr uint32_t BAR_OFF = B2_OFF + 64 * DVT * 2;
+    static constexpr uint32_t BYTES = BAR_OFF + 8 * (2 * NS + 2) + 16;
+    static constexpr uint32_t NCOLS = 2 * DVT < 32 ? 32 : 2 * DVT;   // TMEM columns (pow2)
+    static constexpr uint32_t B1_SBO = (128 / 8) * 128;             // n-group stride
+    static constexpr uint32_t B2_SBO = (64 / 8) * 128;
+};
+
+// MN-major interleaved core-matrix layout: element (n, k) of a K x N operand
+// at (n / 8) * SBO + (k / 8) * 128 + (k % 8) * 16 + (n % 8) * 2.
+__device__ __forceinline__ uint32_t mn_off(int k, int ng, uint32_t sbo) {
+    return ng * sbo + (k >> 3) * 128 + (k & 7) * 16;
+}
+
+template <int DVT, int NS>
+__global__ void __launch_bounds__(NTHREADS, 1)
+chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__restrict__ cu,
+                      const int32_t *__restrict__ coff, const float *__restrict__ s0,
+                      float *__restrict__ sT, __nv_bfloat16 *__restrict__ out, int T, int total_T,
+                      int H, int cps, int max_chunks, int *__restrict__ err)
+{
+    using L = TcLayout<DVT, NS>;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::BAR_OFF);
+    uint64_t *empty = full + NS;
+    uint64_t *mma1 = empty + NS;
+    uint64_t *mma23 = mma1 + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma23 + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    unsigned char *B1 = sm + L::B1_OFF;
+    unsigned char *B2 = sm + L::B2_OFF;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n0 = blockIdx.x * DVT, h = blockIdx.y, seq = blockIdx.z;
+
+    long long bos, eos;
+    int c_begin;
+    if (cu) {
+        bos = min(max(cu[seq], 0), total_T);
+        eos = min(max(cu[seq + 1], 0), total_T);
+        if (eos < bos) eos = bos;
+        c_begin = coff[seq];
+    } else {
+        bos = (long long)seq * T;
+        eos = bos + T;
+        c_begin = seq * cps;
+    }
+    int nchunks = (int)((eos - bos + C - 1) / C);
+    if (c_begin < 0 || c_begin + nchunks > max_chunks) {
+        if (tid == 0) set_device_error(err, kErrBadOffsets);
+        nchunks = c_begin < 0 ? 0 : max(0, min(nchunks, max_chunks - c_begin));
+    }
+    const unsigned char *rec0 = wsp + ((size_t)max(c_begin, 0) * H + h) * ws::RECORD;
+    const size_t rec_stride = (size_t)H * ws::RECORD;
+
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        mbar_init(mma1, 1);
+        mbar_init(mma23, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) { tmem_alloc(tmem_slot, L::NCOLS); tmem_relinquish(); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // ---------------- loader ----------------
+        if (lane == 0) {
+            int issued = 0;
+            for (int i = 0; i < nchunks; ++i) {
+                const int s = i % NS;
+                if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) {
+                    set_device_error(err, kErrWaitTimeout);
+                    break;
+                }
+                if (*abort_flag) break;
+                const unsigned char *rec = rec0 + (size_t)i * rec_stride;
+                unsigned char *st = sm + (size_t)s * L::STAGE;
+                mbar_arrive_expect_tx(&full[s], L::TX);
+                bulk_g2s(st, rec, REC_HEAD, &full[s]);
+                bulk_g2s(st + L::U_OFF, rec + ws::OFF_U + (size_t)(n0 >> 5) * ws::U_TILE,
+                         L::UT * 4096, &full[s]);
+                bulk_g2s(st + L::EGC_OFF, rec + ws::OFF_EGC, 512, &full[s]);
+                issued = i + 1;
+            }
+            // never leave with copies in flight into this CTA's shared memory
+            for (int j = max(0, issued - NS); j < issued; ++j)
+                mbar_wait(&full[j % NS], (j / NS) & 1, 1u << 20);
+        }
+    } else {
+        // ---------------- math warps: thread t <-> TMEM lane t ----------------
+        const int t = tid;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        constexpr uint32_t IDESC = idesc_bf16(128, DVT, true);
+        float S[DVT];
+        {
+            const size_t sb = (((size_t)seq * H + h) * D + t) * D + n0;
+#pragma unroll
+            for (int j = 0; j < DVT; j += 4) {
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (s0) x = *reinterpret_cast<const float4 *>(s0 + sb + j);
+                S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+            }
+        }
+        auto write_B1 = [&]() {
+#pragma unroll
+            for (int ng = 0; ng < DVT / 8; ++ng) {
+                uint4 pk = make_uint4(pack_bf16(S[8 * ng], S[8 * ng + 1]), pack_bf16(S[8 * ng + 2], S[8 * ng + 3]),
+                                      pack_bf16(S[8 * ng + 4], S[8 * ng + 5]), pack_bf16(S[8 * ng + 6], S[8 * ng + 7]));
+                *reinterpret_cast<uint4 *>(B1 + mn_off(t, ng, L::B1_SBO)) = pk;
+            }
+        };
+        write_B1();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        named_bar(1, 128);
+        tc_fence_after();
+
+        bool failed = false;
+        for (int i = 0; i < nchunks && !failed; ++i) {
+            const int s = i % NS;
+            unsigned char *st = sm + (size_t)s * L::STAGE;
+            const uint32_t st_a = smem_u32(st);
+            const uint32_t b1_a = smem_u32(B1), b2_a = smem_u32(B2);
+            bool ok = true;
+            if (t == 0) {
+                ok = mbar_wait(&full[s], (i / NS) & 1);
+                if (ok) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint64_t ad = smem_desc(st_a + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, 2);
+                        const uint64_t bd = smem_desc(b1_a + kk * 256, 128, L::B1_SBO, 0);
+                        umma_bf16(tmem, ad, bd, IDESC, kk > 0);
+                    }
+                    umma_commit(mma1);
+                    ok = mbar_wait(mma1, i & 1);
+                }
+            }
+            if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+            tc_fence_after();
+            const float eg = reinterpret_cast<const float *>(st + L::EGC_OFF)[t];
+            if (t < 64) {
+                // V_new = U - W S for token row t
+#pragma unroll
+                for (int c16 = 0; c16 < DVT / 16; ++c16) {
+                    float x[16];
+                    tmem_ld16(tmem + lane_base + c16 * 16, x);
+                    tmem_wait_ld();
+                    // column (n0 % 32) + 16 c16 of the loaded U tile(s), row t
+                    const int lc = (n0 & 31) + c16 * 16;
+                    const unsigned char *up = st + L::U_OFF + (lc >> 5) * 4096 + t * 64 + (lc & 31) * 2;
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const __nv_bfloat162 u2 = reinterpret_cast<const __nv_bfloat162 *>(up)[e];
+                        pk[e] = pack_bf16(__low2float(u2) - x[2 * e], __high2float(u2) - x[2 * e + 1]);
+                    }
+                    *reinterpret_cast<uint4 *>(B2 + mn_off(t, 2 * c16, L::B2_SBO)) =
+                        make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4 *>(B2 + mn_off(t, 2 * c16 + 1, L::B2_SBO)) =
+                        make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(1, 128);
+            tc_fence_after();
+            ok = true;
+            if (t == 0) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t bd = smem_desc(b2_a + kk * 256, 128, L::B2_SBO, 0);
+                    const uint64_t ap = smem_desc(st_a + (uint32_t)ws::OFF_P - 8192 + kk * 32, 16, 1024, 2);
+                    umma_bf16(tmem, ap, bd, IDESC, 1);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t bd = smem_desc(b2_a + kk * 256, 128, L::B2_SBO, 0);
+                    const uint64_t ak = smem_desc(st_a + (uint32_t)ws::OFF_KTT + kk * 32, 16, 1024, 2);
+                    umma_bf16(tmem + DVT, ak, bd, IDESC, kk > 0);
+                }
+                umma_commit(mma23);
+                umma_commit(&empty[s]);
+                ok = mbar_wait(mma23, i & 1);
+            }
+            if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+            tc_fence_after();
+            // S <- Diag(e^{G_C}) S + Kt^T V_new   (channel row t)
+#pragma unroll
+            for (int c16 = 0; c16 < DVT / 16; ++c16) {
+                float z[16];
+                tmem_ld16(tmem + lane_base + DVT + c16 * 16, z);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) S[c16 * 16 + e] = eg * S[c16 * 16 + e] + z[e];
+            }
+            write_B1();
+            if (t >= 64) {
+                // O = Qg S + P V_new for token row t - 64
+                const long long tok = bos + (long long)C * i + (t - 64);
+#pragma unroll
+                for (int c16 = 0; c16 < DVT / 16; ++c16) {
+                    float o[16];
+                    tmem_ld16(tmem + lane_base + c16 * 16, o);
+                    tmem_wait_ld();
+                    if (tok < eos) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)tok * H + h) * D + n0 + c16 * 16);
+                        dst[0] = make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]),
+                                            pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
+                        dst[1] = make_uint4(pack_bf16(o[8], o[9]), pack_bf16(o[10], o[11]),
+                                            pack_bf16(o[12], o[13]), pack_bf16(o[14], o[15]));
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(1, 128);
+            tc_fence_after();
+        }
+        if (failed) {
+            if (t == 0) { set_device_error(err, kErrWaitTimeout); *abort_flag = 1; }
+        } else if (sT) {
+            const size_t sb = (((size_t)seq * H + h) * D + t) * D + n0;
+#pragma unroll
+            for (int j = 0; j < DVT; j += 4)
+                *reinterpret_cast<float4 *>(sT + sb + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, L::NCOLS);
+}
+
+template <int DVT, int NS>
+cudaError_t launch_tc(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
+                      const float *s0, float *sT, void *out, int N, int T, int total_T, int H,
+                      int max_chunks, int *err, cudaStream_t st)
+{
+    using L = TcLayout<DVT, NS>;
+    const size_t smem = L::BYTES + 1024;
+    cudaError_t e = cudaFuncSetAttribute(chunk_chain_tc_kernel<DVT, NS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(D / DVT, H, N);
+    chunk_chain_tc_kernel<DVT, NS><<<grid, NTHREADS, smem, st>>>(
+        wsp, cu, coff, s0, sT, (__nv_bfloat16 *)out, T, total_T, H, (T + C - 1) / C, max_chunks, err);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_chain_tc(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
+                                  const float *s0, float *sT, void *out, int N, int T,
+                                  int total_T, int H, int dvt, int max_chunks, int *err,
+                                  cudaStream_t st)
+{
+    switch (dvt) {
+        case 16: return launch_tc<16, 3>(wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st);
+        case 32: return launch_tc<32, 3>(wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st);
+        case 64: return launch_tc<64, 2>(wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace kda

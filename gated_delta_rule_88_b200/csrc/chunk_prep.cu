@@ -4,31 +4,35 @@
 // Kimi Linear paper notes (paper-notes-site), section 3: inside a chunk the
 // intra-chunk writes are gathered by a WY-like representation (W, U) and the
 // output splits into an inter-chunk and an intra-chunk part; section 2 and
-// the constrained-DPLR remark: KDA ties the low-rank factors to k, which saves
-// matrix products and avoids the inverse cumulative-decay (1/Gamma) terms of
-// the general DPLR form.  This kernel produces, for one chunk of one head,
-// the record of chunk_ws.h:
+// the constrained-DPLR remark (with the Figure 2 note): KDA ties the low-rank
+// factors to k, which saves matrix products and avoids the inverse
+// cumulative-decay (1/Gamma) terms of the general DPLR form.  For one chunk of
+// one head this kernel produces the record of chunk_ws.h:
 //     G     = chunk-local inclusive cumsum of g          (per channel)
 //     A_ij  = beta_i sum_c k_ic k_jc e^{G_ic - G_jc}     (j < i)
 //     P_ij  =        sum_c q_ic k_jc e^{G_ic - G_jc}     (j <= i)
 //     T     = (I + A)^-1                                  (unit lower-tri.)
 //     W = T (beta K e^G),  U = T (beta V),  Qg = Q e^G,  Kt = K e^{G_C - G}
 //
-// Exponents (no overflow, no 1/Gamma over the chunk): the chunk is cut into
-// four sub-chunks of 16 tokens, I = 0..3, with block-end cumsums R_I
-// (R_{-1} = 0).  For token i in block I and j in block J <= I,
-//     e^{G_i - G_j} = e^{G_i - R_{I-1}} * e^{R_{I-1} - G_j}
-// The left factor a_i = e^{G_i - R_{I-1}} is <= 1 and depends on i only;
-// the right factor is <= 1 for J < I and spans at most 16 tokens for J = I,
-// so with per-token g >= -5 every factor stays within e^{+-80}.  Row block I
-// therefore needs one right operand Kr^(I)_j = k_j e^{R_{I-1} - G_j}
-// (j < 16(I+1)); the four are stacked in shared memory.
+// Exponents.  The chunk is cut into four sub-chunks of 16 tokens, I = 0..3,
+// with block-end cumsums R_I (R_{-1} = 0).  Per token and channel only
+// alpha = e^g is exponentiated; everything else is a product of alphas:
+//     a_i = e^{G_i - R_{I-1}} (forward product within the block, <= 1)
+//     b_i = e^{R_I - G_i}     (backward product within the block, <= 1)
+//     d_I = e^{R_I - R_{I-1}} (block total)
+// For i in block I and j in block J:
+//     J < I:  e^{G_i - G_j} = a_i * D_JI * b_j,  D_JI = prod_{J<M<I} d_M <= 1
+//     J = I:  e^{G_i - G_j} = a_i * (1 / a_j),   1/a_j <= e^{16 * max|g|}
+// so with per-token g >= -5 no factor leaves e^{+-80}, and no 1/Gamma over the
+// whole chunk is ever formed.
 //
-// Tensor cores: m16n8k16 bf16 MMAs with fp32 accumulation for A, P (left
-// operands (beta k a), (q a); right operand Kr^(I)), and W, U (T rounded to
-// bf16 times (beta K e^G), (beta V)).  T itself is formed in fp32:
-// 16x16 diagonal blocks by forward substitution, off-diagonal blocks by
-// T_IJ = -T_II sum_{M=J}^{I-1} A_IM T_MJ in order of distance I - J.
+// Work split (256 threads, two CTAs per SM): thread (I, channel pair) owns
+// one sub-chunk x two channels for the elementwise forms; A and P are
+// m16n8k16 bf16 MMAs per row block (left operand (beta k a) or (q a), right
+// operand k b scaled by D_JI, or k / a on the diagonal block); T is formed in
+// fp32 (16x16 diagonal blocks by forward substitution, then the 2x2-block
+// recursion T21 = -T22 A21 T11 at 16 and 32 rows); W and U are m16n8k16 MMAs
+// with T rounded once to bf16.
 #include "chunk_ws.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -39,35 +43,40 @@ namespace {
 constexpr int C = ws::C;
 constexpr int D = ws::D;
 constexpr int NT = 256;
-constexpr int PB = D + 8;     // bf16 pitch of 128-wide tiles (conflict-free ldmatrix)
-constexpr int PF = C + 4;     // fp32 pitch of 64x64 tiles
-constexpr int PP = C + 8;     // bf16 pitch of the 64x64 P staging tile
-constexpr int KR_ROWS = 16 + 32 + 48 + 64;
-__host__ __device__ constexpr int kr_base(int I) { return I == 0 ? 0 : I == 1 ? 16 : I == 2 ? 48 : 96; }
+constexpr int TILE = C * D * 2;   // bytes of a 64 x 128 bf16 tile
 
-struct PrepSmem {
-    union {
-        float G[C][D];                        // cumsum of g (phase 1-3)
-        __nv_bfloat16 Pst[C][PP];             // P staging (phase 4-7)
-    };
-    __nv_bfloat16 Xk[C][PB];                  // beta k a      (then W staging)
-    __nv_bfloat16 Xq[C][PB];                  // q a           (then U staging)
-    __nv_bfloat16 KG[C][PB];                  // beta k e^G
-    __nv_bfloat16 Vb[C][PB];                  // beta v
-    __nv_bfloat16 Kr[KR_ROWS][PB];            // k e^{R_{I-1} - G_j}, I = 0..3 stacked
-    float A[C][PF];                           // A (strict lower), fp32
-    float Tm[C][PF];                          // T, fp32
-    float Zs[4][16][17];                      // per-warp 16x16 scratch
-    float R[4][D];                            // block-end cumsums
-    float Eb[4][D];                           // e^{R_{I-1}} (Eb[0] = 1)
-    float F[4][D];                            // e^{R_3 - R_I}
-    float Dm[16][D];                          // e^{R_{I'-1} - R_I}, index I*4+I', I < I'
+// 64 x 128 bf16 tile, 256-byte rows, 16-byte chunk j of row r at j ^ (r & 7)
+__device__ __forceinline__ int toff(int r, int c) {
+    return r * 256 + ((((c >> 3) ^ (r & 7))) << 4) + ((c & 7) << 1);
+}
+__device__ __forceinline__ int toff_chunk(int r, int j) {
+    return r * 256 + (((j ^ (r & 7))) << 4);
+}
+// 64 x 64 fp32 matrix, column groups of 4 XOR-swizzled by row
+__device__ __forceinline__ int fsw(int i, int j) { return i * 64 + (j ^ ((i & 7) << 2)); }
+// index of the (J, I) block pair, J < I
+__device__ __forceinline__ int pair_idx(int J, int I) { return I * (I - 1) / 2 + J; }
+
+struct __align__(16) PrepSmem {
+    unsigned char Xq[TILE];   // q in; then q a          (then A, fp32 64x64)
+    unsigned char Kb[TILE];   // k in; then k b
+    unsigned char Vb[TILE];   // v in; then beta v
+    unsigned char Xk[TILE];   // beta k a                (then T, fp32 64x64)
+    unsigned char Kd[TILE];   // k / a                   (then T-recursion scratch)
+    unsigned char KG[TILE];   // beta k e^G
+    float Dm[6][D];           // D_JI per channel
+    float d[4][D];            // block totals
     float beta[C];
 };
 
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t x, float2 s) {
+    __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162 *>(&x);
+    return pack_bf16(__low2float(v) * s.x, __high2float(v) * s.y);
+}
+
 __device__ __forceinline__ void locate_chunk(int chunk, const int32_t *cu, const int32_t *coff,
-                                             int N, int T, int total_T, int cps, int &seq,
-                                             long long &t0, int &len) {
+                                             int N, int T, int total_T, int cps, long long &t0,
+                                             int &len) {
     long long bos, eos;
     int cidx;
     if (cu) {
@@ -76,13 +85,12 @@ __device__ __forceinline__ void locate_chunk(int chunk, const int32_t *cu, const
             const int mid = (lo + hi) >> 1;
             if (coff[mid] <= chunk) lo = mid; else hi = mid;
         }
-        seq = lo;
-        bos = min(max(cu[seq], 0), total_T);
-        eos = min(max(cu[seq + 1], 0), total_T);
+        bos = min(max(cu[lo], 0), total_T);
+        eos = min(max(cu[lo + 1], 0), total_T);
         if (eos < bos) eos = bos;
-        cidx = chunk - coff[seq];
+        cidx = chunk - coff[lo];
     } else {
-        seq = chunk / cps;
+        const int seq = chunk / cps;
         cidx = chunk - seq * cps;
         bos = (long long)seq * T;
         eos = bos + T;
@@ -91,139 +99,143 @@ __device__ __forceinline__ void locate_chunk(int chunk, const int32_t *cu, const
     len = (int)max(0LL, min((long long)C, eos - t0));
 }
 
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NT, 2)
 chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                   const __nv_bfloat16 *__restrict__ v, const float *__restrict__ g,
                   const float *__restrict__ beta, const int32_t *__restrict__ cu,
                   const int32_t *__restrict__ coff, int N, int T, int total_T, int H, int cps,
                   unsigned char *__restrict__ wsp)
 {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
     PrepSmem &sm = *reinterpret_cast<PrepSmem *>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tig = lane & 3;
     const int chunk = blockIdx.x, h = blockIdx.y;
     if (cu && chunk >= coff[N]) return;
 
-    int seq, len;
+    int len;
     long long t0;
-    locate_chunk(chunk, cu, coff, N, T, total_T, cps, seq, t0, len);
+    locate_chunk(chunk, cu, coff, N, T, total_T, cps, t0, len);
     unsigned char *rec = wsp + ((size_t)chunk * H + h) * ws::RECORD;
+    const size_t row_stride = (size_t)H * D;              // elements between tokens
+    const size_t base = ((size_t)t0 * H + h) * D;         // element offset of (t0, h, 0)
 
-    // ---- phase 1: g -> smem (zero past the end), beta ----
-    for (int i = tid; i < C * (D / 4); i += NT) {
-        const int r = i / (D / 4), c4 = i % (D / 4);
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r < len) x = *reinterpret_cast<const float4 *>(g + ((size_t)(t0 + r) * H + h) * D + c4 * 4);
-        *reinterpret_cast<float4 *>(&sm.G[r][c4 * 4]) = x;
+    // ---- stage q, k, v (zero-filled past the end) ----
+    for (int i = tid; i < 3 * C * (D / 8); i += NT) {
+        const int which = i / (C * (D / 8));
+        const int rem = i - which * (C * (D / 8));
+        const int r = rem >> 4, j = rem & 15;
+        const __nv_bfloat16 *src = which == 0 ? q : which == 1 ? k : v;
+        unsigned char *dst = which == 0 ? sm.Xq : which == 1 ? sm.Kb : sm.Vb;
+        const bool ok = r < len;
+        const __nv_bfloat16 *gp = ok ? src + base + (size_t)r * row_stride + j * 8 : src;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(dst + toff_chunk(r, j))),
+                     "l"(gp), "r"(ok ? 16 : 0));
     }
-    if (tid < C) sm.beta[tid] = (tid < len) ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
-    __syncthreads();
+    cp_async_commit();
 
-    // ---- phase 2: per-channel cumsum and block tables ----
-    if (tid < D) {
-        const int c = tid;
-        float acc = 0.f;
-#pragma unroll 8
-        for (int r = 0; r < C; ++r) { acc += sm.G[r][c]; sm.G[r][c] = acc; }
-        float R[4];
-#pragma unroll
-        for (int I = 0; I < 4; ++I) { R[I] = sm.G[16 * I + 15][c]; sm.R[I][c] = R[I]; }
-        sm.Eb[0][c] = 1.f;
-#pragma unroll
-        for (int I = 1; I < 4; ++I) sm.Eb[I][c] = expf(R[I - 1]);
-#pragma unroll
-        for (int I = 0; I < 3; ++I) sm.F[I][c] = expf(R[3] - R[I]);
-        sm.F[3][c] = 1.f;
-#pragma unroll
-        for (int I = 0; I < 4; ++I)
-#pragma unroll
-            for (int J = I + 1; J < 4; ++J) sm.Dm[I * 4 + J][c] = expf(R[J - 1] - R[I]);
-        reinterpret_cast<float *>(rec + ws::OFF_EGC)[c] = expf(R[3]);
-    }
-    __syncthreads();
-
-    // ---- phase 3: decayed operand forms (8 channels per item) ----
-    for (int it = tid; it < C * (D / 8); it += NT) {
-        const int r = it / (D / 8), c0 = (it % (D / 8)) * 8;
-        const int I = r >> 4;
-        const float br = sm.beta[r];
-        uint4 qraw = make_uint4(0, 0, 0, 0), kraw = make_uint4(0, 0, 0, 0);
-        if (r < len) {
-            const size_t off = ((size_t)(t0 + r) * H + h) * D + c0;
-            qraw = *reinterpret_cast<const uint4 *>(q + off);
-            kraw = *reinterpret_cast<const uint4 *>(k + off);
-        }
-        const __nv_bfloat16 *q8 = reinterpret_cast<const __nv_bfloat16 *>(&qraw);
-        const __nv_bfloat16 *k8 = reinterpret_cast<const __nv_bfloat16 *>(&kraw);
-        uint32_t xk[4], xq[4], kg[4], qg[4], kt[4], krs[4], krv[3][4];
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-            float vxk[2], vxq[2], vkg[2], vqg[2], vkt[2], vkrs[2], vkrv[3][2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int c = c0 + e + u;
-                const float G = sm.G[r][c];
-                const float Rp = I > 0 ? sm.R[I - 1][c] : 0.f;
-                const float a = expf(G - Rp);
-                const float b = expf(sm.R[I][c] - G);
-                const float kv = __bfloat162float(k8[e + u]);
-                const float qv = __bfloat162float(q8[e + u]);
-                const float eG = a * sm.Eb[I][c];
-                vxk[u] = br * kv * a;
-                vxq[u] = qv * a;
-                vkg[u] = br * kv * eG;
-                vqg[u] = qv * eG;
-                vkt[u] = kv * b * sm.F[I][c];
-                vkrs[u] = kv / a;
-#pragma unroll
-                for (int J = 1; J < 4; ++J)
-                    vkrv[J - 1][u] = (I + J < 4) ? kv * b * sm.Dm[I * 4 + I + J][c] : 0.f;
-            }
-            xk[e / 2] = pack_bf16(vxk[0], vxk[1]);
-            xq[e / 2] = pack_bf16(vxq[0], vxq[1]);
-            kg[e / 2] = pack_bf16(vkg[0], vkg[1]);
-            qg[e / 2] = pack_bf16(vqg[0], vqg[1]);
-            kt[e / 2] = pack_bf16(vkt[0], vkt[1]);
-            krs[e / 2] = pack_bf16(vkrs[0], vkrs[1]);
-#pragma unroll
-            for (int J = 0; J < 3; ++J) krv[J][e / 2] = pack_bf16(vkrv[J][0], vkrv[J][1]);
-        }
-        *reinterpret_cast<uint4 *>(&sm.Xk[r][c0]) = make_uint4(xk[0], xk[1], xk[2], xk[3]);
-        *reinterpret_cast<uint4 *>(&sm.Xq[r][c0]) = make_uint4(xq[0], xq[1], xq[2], xq[3]);
-        *reinterpret_cast<uint4 *>(&sm.KG[r][c0]) = make_uint4(kg[0], kg[1], kg[2], kg[3]);
-        // version I holds row r itself (k / a); versions I' > I hold k b Dm
-        *reinterpret_cast<uint4 *>(&sm.Kr[kr_base(I) + r][c0]) = make_uint4(krs[0], krs[1], krs[2], krs[3]);
-#pragma unroll
-        for (int J = 1; J < 4; ++J)
-            if (I + J < 4)
-                *reinterpret_cast<uint4 *>(&sm.Kr[kr_base(I + J) + r][c0]) =
-                    make_uint4(krv[J - 1][0], krv[J - 1][1], krv[J - 1][2], krv[J - 1][3]);
-        *reinterpret_cast<uint4 *>(rec + ws::OFF_QG + ((size_t)r * D + c0) * 2) =
-            make_uint4(qg[0], qg[1], qg[2], qg[3]);
-        *reinterpret_cast<uint4 *>(rec + ws::OFF_KT + ((size_t)r * D + c0) * 2) =
-            make_uint4(kt[0], kt[1], kt[2], kt[3]);
-    }
-    // beta V
-    for (int it = tid; it < C * (D / 8); it += NT) {
-        const int r = it / (D / 8), c0 = (it % (D / 8)) * 8;
-        uint4 vraw = make_uint4(0, 0, 0, 0);
-        if (r < len) vraw = *reinterpret_cast<const uint4 *>(v + ((size_t)(t0 + r) * H + h) * D + c0);
-        const __nv_bfloat16 *v8 = reinterpret_cast<const __nv_bfloat16 *>(&vraw);
-        const float br = sm.beta[r];
-        uint32_t o[4];
-#pragma unroll
-        for (int e = 0; e < 8; e += 2)
-            o[e / 2] = pack_bf16(br * __bfloat162float(v8[e]), br * __bfloat162float(v8[e + 1]));
-        *reinterpret_cast<uint4 *>(&sm.Vb[r][c0]) = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-    __syncthreads();
-
-    // ---- phase 4: A (warps 0-3) and P (warps 4-7), row block I = warp & 3 ----
+    // ---- elementwise ownership: sub-chunk I, channels c0, c0 + 1 ----
+    const int I = tid >> 6, c0 = 2 * (tid & 63);
+    float2 a[16], b[16];
     {
-        const int I = warp & 3;
+        float2 al[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int r = 16 * I + i;
+            float2 gv = make_float2(0.f, 0.f);
+            if (r < len) gv = *reinterpret_cast<const float2 *>(g + base + (size_t)r * row_stride + c0);
+            al[i] = make_float2(expf(gv.x), expf(gv.y));
+        }
+        float2 run = make_float2(1.f, 1.f);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) { run.x *= al[i].x; run.y *= al[i].y; a[i] = run; }
+        run = make_float2(1.f, 1.f);
+#pragma unroll
+        for (int i = 15; i >= 0; --i) { b[i] = run; run.x *= al[i].x; run.y *= al[i].y; }
+    }
+    sm.d[I][c0] = a[15].x;
+    sm.d[I][c0 + 1] = a[15].y;
+    if (tid < C) sm.beta[tid] = (tid < len) ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+    cp_async_wait<0>();
+    __syncthreads();
+
+    float2 E = make_float2(1.f, 1.f), F = make_float2(1.f, 1.f);
+    {
+        float2 dd[4];
+#pragma unroll
+        for (int J = 0; J < 4; ++J) dd[J] = make_float2(sm.d[J][c0], sm.d[J][c0 + 1]);
+#pragma unroll
+        for (int J = 0; J < 4; ++J) {
+            if (J < I) { E.x *= dd[J].x; E.y *= dd[J].y; }
+            if (J > I) { F.x *= dd[J].x; F.y *= dd[J].y; }
+        }
+        if (I == 0) {
+            // e^{G_C} = product of all block totals
+            float2 e = make_float2(dd[0].x * dd[1].x * dd[2].x * dd[3].x,
+                                   dd[0].y * dd[1].y * dd[2].y * dd[3].y);
+            *reinterpret_cast<float2 *>(rec + ws::OFF_EGC + c0 * 4) = e;
+        }
+        // D_JI for the pairs J < I of this thread's block I
+#pragma unroll
+        for (int J = 0; J < 3; ++J) {
+            if (J < I) {
+                float2 m = make_float2(1.f, 1.f);
+#pragma unroll
+                for (int M = 1; M < 3; ++M)
+                    if (M > J && M < I) { m.x *= dd[M].x; m.y *= dd[M].y; }
+                sm.Dm[pair_idx(J, I)][c0] = m.x;
+                sm.Dm[pair_idx(J, I)][c0 + 1] = m.y;
+            }
+        }
+    }
+    {
+        uint32_t kt[2][8];   // Kt for (channel, token pair) -> transposed store
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int r = 16 * I + i;
+            const int o = toff(r, c0);
+            const float br = sm.beta[r];
+            const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(sm.Xq + o);
+            const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(sm.Kb + o);
+            const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162 *>(sm.Vb + o);
+            const float qx = __low2float(q2), qy = __high2float(q2);
+            const float kx = __low2float(k2), ky = __high2float(k2);
+            const float vx = __low2float(v2), vy = __high2float(v2);
+            const float2 ai = a[i], bi = b[i];
+            *reinterpret_cast<uint32_t *>(sm.Xq + o) = pack_bf16(qx * ai.x, qy * ai.y);
+            *reinterpret_cast<uint32_t *>(sm.Xk + o) = pack_bf16(br * kx * ai.x, br * ky * ai.y);
+            *reinterpret_cast<uint32_t *>(sm.KG + o) =
+                pack_bf16(br * kx * ai.x * E.x, br * ky * ai.y * E.y);
+            *reinterpret_cast<uint32_t *>(sm.Kd + o) = pack_bf16(kx / ai.x, ky / ai.y);
+            *reinterpret_cast<uint32_t *>(sm.Kb + o) = pack_bf16(kx * bi.x, ky * bi.y);
+            *reinterpret_cast<uint32_t *>(sm.Vb + o) = pack_bf16(br * vx, br * vy);
+            *reinterpret_cast<uint32_t *>(rec + ws::aw_off(64 + r, c0)) =
+                pack_bf16(qx * ai.x * E.x, qy * ai.y * E.y);
+            const float ktx = kx * bi.x * F.x, kty = ky * bi.y * F.y;
+            if (i & 1) {
+                kt[0][i >> 1] = pack_bf16(__low2float(*reinterpret_cast<__nv_bfloat162 *>(&kt[0][i >> 1])), ktx);
+                kt[1][i >> 1] = pack_bf16(__low2float(*reinterpret_cast<__nv_bfloat162 *>(&kt[1][i >> 1])), kty);
+            } else {
+                kt[0][i >> 1] = pack_bf16(ktx, 0.f);
+                kt[1][i >> 1] = pack_bf16(kty, 0.f);
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int c = c0 + e;
+                *reinterpret_cast<uint4 *>(rec + ws::OFF_KTT + ws::sw128(c, 16 * I + 8 * hh)) =
+                    make_uint4(kt[e][4 * hh], kt[e][4 * hh + 1], kt[e][4 * hh + 2], kt[e][4 * hh + 3]);
+            }
+    }
+    __syncthreads();
+
+    // ---- A (warps 0-3) and P (warps 4-7) for row block Ib = warp & 3 ----
+    {
+        const int Ib = warp & 3;
         const bool isP = warp >= 4;
-        const __nv_bfloat16(*X)[PB] = isP ? sm.Xq : sm.Xk;
+        const unsigned char *X = isP ? sm.Xq : sm.Xk;
         float acc[4][2][4];
 #pragma unroll
         for (int J = 0; J < 4; ++J)
@@ -231,148 +243,188 @@ chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[J][nt][e] = 0.f;
-        const int arow = 16 * I + (lane & 7) + 8 * ((lane >> 3) & 1);
-        const int acol = 8 * (lane >> 4);
+        const int ar = 16 * Ib + (lane & 7) + 8 * ((lane >> 3) & 1);
         const int bn = (lane & 7) + 8 * (lane >> 4);
-        const int bk = 8 * ((lane >> 3) & 1);
+        const int bk = (lane >> 3) & 1;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-            uint32_t a[4];
-            ldsm_x4(a, &X[arow][16 * ks + acol]);
+            uint32_t af[4];
+            ldsm_x4(af, X + toff_chunk(ar, 2 * ks + (lane >> 4)));
 #pragma unroll
             for (int J = 0; J < 4; ++J) {
-                if (J <= I) {
-                    uint32_t b[4];
-                    ldsm_x4(b, &sm.Kr[kr_base(I) + 16 * J + bn][16 * ks + bk]);
-                    mma_bf16(acc[J][0], a, b[0], b[1]);
-                    mma_bf16(acc[J][1], a, b[2], b[3]);
+                if (J <= Ib) {
+                    uint32_t bf[4];
+                    const int br = 16 * J + bn;
+                    ldsm_x4(bf, (J < Ib ? sm.Kb : sm.Kd) + toff_chunk(br, 2 * ks + bk));
+                    if (J < Ib) {
+                        const float *dm = sm.Dm[pair_idx(J, Ib)];
+                        const float2 slo = *reinterpret_cast<const float2 *>(dm + 16 * ks + 2 * tig);
+                        const float2 shi = *reinterpret_cast<const float2 *>(dm + 16 * ks + 8 + 2 * tig);
+                        bf[0] = scale_bf16x2(bf[0], slo);
+                        bf[2] = scale_bf16x2(bf[2], slo);
+                        bf[1] = scale_bf16x2(bf[1], shi);
+                        bf[3] = scale_bf16x2(bf[3], shi);
+                    }
+                    mma_bf16(acc[J][0], af, bf[0], bf[1]);
+                    mma_bf16(acc[J][1], af, bf[2], bf[3]);
                 }
             }
         }
-        __syncthreads();   // G region is now reused as P staging
+        __syncthreads();   // operand tiles are dead: Xq becomes A (fp32)
+        float *Am = reinterpret_cast<float *>(sm.Xq);
 #pragma unroll
         for (int J = 0; J < 4; ++J)
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    const int i = 16 * I + gid + 8 * hh;
+                    const int i = 16 * Ib + gid + 8 * hh;
                     const int j = 16 * J + 8 * nt + 2 * tig;
                     float v0 = acc[J][nt][2 * hh], v1 = acc[J][nt][2 * hh + 1];
                     if (!isP) {
-                        if (J <= I) {
-                            sm.A[i][j] = (j < i) ? v0 : 0.f;
-                            sm.A[i][j + 1] = (j + 1 < i) ? v1 : 0.f;
+                        if (J <= Ib) {
+                            Am[fsw(i, j)] = (j < i) ? v0 : 0.f;
+                            Am[fsw(i, j + 1)] = (j + 1 < i) ? v1 : 0.f;
                         }
                     } else {
-                        v0 = (J <= I && j <= i) ? v0 : 0.f;
-                        v1 = (J <= I && j + 1 <= i) ? v1 : 0.f;
-                        *reinterpret_cast<uint32_t *>(&sm.Pst[i][j]) = pack_bf16(v0, v1);
+                        v0 = (J <= Ib && j <= i) ? v0 : 0.f;
+                        v1 = (J <= Ib && j + 1 <= i) ? v1 : 0.f;
+                        *reinterpret_cast<uint32_t *>(rec + ws::OFF_P + ws::sw128(i, j)) = pack_bf16(v0, v1);
                     }
                 }
     }
     __syncthreads();
 
-    // ---- phase 5: T = (I + A)^-1 ----
-    if (warp < 4 && lane < 16) {
-        const int I = warp, c = lane, o = 16 * I;
+    // ---- T = (I + A)^-1 in fp32 ----
+    const float *Am = reinterpret_cast<const float *>(sm.Xq);
+    float *Tm = reinterpret_cast<float *>(sm.Xk);
+    float *Zs = reinterpret_cast<float *>(sm.Kd);
+    if (warp < 2) {
+        // 16x16 diagonal blocks: lane -> (block, column)
+        const int Bk = 2 * warp + (lane >> 4), c = lane & 15, o = 16 * Bk;
+        float x[16];
+#pragma unroll
         for (int i = 0; i < 16; ++i) {
-            float t;
-            if (i < c) t = 0.f;
-            else if (i == c) t = 1.f;
-            else {
-                float s = 0.f;
-                for (int j = c; j < i; ++j) s += sm.A[o + i][o + j] * sm.Tm[o + j][o + c];
-                t = -s;
-            }
-            sm.Tm[o + i][o + c] = t;
+            float s = 0.f;
+#pragma unroll
+            for (int j = 0; j < i; ++j) s += Am[fsw(o + i, o + j)] * x[j];
+            x[i] = (i < c) ? 0.f : (i == c) ? 1.f : -s;
         }
-    } else if (warp >= 4) {
-        // zero the strictly-upper blocks of T
-        const int I = warp - 4;
-        for (int e = lane; e < 16 * 64; e += 32) {
-            const int i = e / 64, j = e % 64;
-            if (j >= 16 * (I + 1)) sm.Tm[16 * I + i][j] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) Tm[fsw(o + i, o + c)] = x[i];
+    } else {
+        // zero the strictly-upper 16x16 blocks
+        for (int e = tid - 64; e < 6 * 256; e += NT - 64) {
+            const int blk = e >> 8, w = e & 255;
+            const int Ib = blk < 3 ? 0 : blk < 5 ? 1 : 2;
+            const int Jb = blk < 3 ? blk + 1 : blk < 5 ? blk - 1 : 3;
+            Tm[fsw(16 * Ib + (w >> 4), 16 * Jb + (w & 15))] = 0.f;
         }
     }
     __syncthreads();
-#pragma unroll 1
-    for (int dist = 1; dist < 4; ++dist) {
-        if (warp < 4 && warp >= dist) {
-            const int I = warp, J = I - dist;
-            const int i = lane >> 1, c0 = 8 * (lane & 1);
-            float z[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) z[e] = 0.f;
-            for (int M = J; M < I; ++M)
-                for (int m = 0; m < 16; ++m) {
-                    const float a = sm.A[16 * I + i][16 * M + m];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) z[e] += a * sm.Tm[16 * M + m][16 * J + c0 + e];
-                }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) sm.Zs[warp][i][c0 + e] = z[e];
-            __syncwarp();
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                float s = 0.f;
-                for (int m = 0; m <= i; ++m) s += sm.Tm[16 * I + i][16 * I + m] * sm.Zs[warp][m][c0 + e];
-                sm.Tm[16 * I + i][16 * J + c0 + e] = -s;
-            }
-        }
-        __syncthreads();
-    }
-
-    // ---- phase 6: W = T (beta K e^G) (warps 0-3), U = T (beta V) (warps 4-7) ----
     {
-        const int I = warp & 3;
-        const bool isU = warp >= 4;
-        const __nv_bfloat16(*B)[PB] = isU ? sm.Vb : sm.KG;
-        __nv_bfloat16(*Out)[PB] = isU ? sm.Xq : sm.Xk;
-        float acc[16][4];
+        // 16-row level: T_IJ = -T_II (A_IJ T_JJ) for (I, J) = (1, 0), (3, 2)
+        const int which = tid >> 7, idx = tid & 127;
+        const int Ib = which ? 3 : 1, Jb = Ib - 1;
+        const int i = idx >> 3, cc = (idx & 7) * 2;
+        float z0 = 0.f, z1 = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-        const int bk = (lane & 7) + 8 * ((lane >> 3) & 1);
-        const int bn = 8 * (lane >> 4);
-        for (int ks = 0; ks <= I; ++ks) {
-            uint32_t a[4];
-            const int r0 = 16 * I + gid, k0 = 16 * ks + 2 * tig;
-            a[0] = pack_bf16(sm.Tm[r0][k0], sm.Tm[r0][k0 + 1]);
-            a[1] = pack_bf16(sm.Tm[r0 + 8][k0], sm.Tm[r0 + 8][k0 + 1]);
-            a[2] = pack_bf16(sm.Tm[r0][k0 + 8], sm.Tm[r0][k0 + 9]);
-            a[3] = pack_bf16(sm.Tm[r0 + 8][k0 + 8], sm.Tm[r0 + 8][k0 + 9]);
-#pragma unroll
-            for (int np = 0; np < 8; ++np) {
-                uint32_t b[4];
-                ldsm_x4_t(b, &B[16 * ks + bk][16 * np + bn]);
-                mma_bf16(acc[2 * np], a, b[0], b[1]);
-                mma_bf16(acc[2 * np + 1], a, b[2], b[3]);
-            }
+        for (int j = 0; j < 16; ++j) {
+            const float aij = Am[fsw(16 * Ib + i, 16 * Jb + j)];
+            const float2 t = *reinterpret_cast<const float2 *>(&Tm[fsw(16 * Jb + j, 16 * Jb + cc)]);
+            z0 += aij * t.x;
+            z1 += aij * t.y;
         }
-        __syncthreads();   // Xk/Xq are reused as W/U staging
+        Zs[which * 256 + i * 16 + cc] = z0;
+        Zs[which * 256 + i * 16 + cc + 1] = z1;
+        __syncthreads();
+        float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            const int i = 16 * I + gid, j = 8 * nt + 2 * tig;
-            *reinterpret_cast<uint32_t *>(&Out[i][j]) = pack_bf16(acc[nt][0], acc[nt][1]);
-            *reinterpret_cast<uint32_t *>(&Out[i + 8][j]) = pack_bf16(acc[nt][2], acc[nt][3]);
+        for (int m = 0; m < 16; ++m) {
+            const float tim = Tm[fsw(16 * Ib + i, 16 * Ib + m)];
+            y0 += tim * Zs[which * 256 + m * 16 + cc];
+            y1 += tim * Zs[which * 256 + m * 16 + cc + 1];
         }
+        Tm[fsw(16 * Ib + i, 16 * Jb + cc)] = -y0;
+        Tm[fsw(16 * Ib + i, 16 * Jb + cc + 1)] = -y1;
+    }
+    __syncthreads();
+    {
+        // 32-row level: T[32:64, 0:32] = -T[32:64, 32:64] (A[32:64, 0:32] T[0:32, 0:32])
+        const int i = tid >> 3, cc = (tid & 7) * 4;
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) {
+            const float aij = Am[fsw(32 + i, j)];
+            const float4 t = *reinterpret_cast<const float4 *>(&Tm[fsw(j, cc)]);
+            y[0] += aij * t.x; y[1] += aij * t.y; y[2] += aij * t.z; y[3] += aij * t.w;
+        }
+        *reinterpret_cast<float4 *>(&Zs[i * 32 + cc]) = make_float4(y[0], y[1], y[2], y[3]);
+        __syncthreads();
+        float z[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+        for (int m = 0; m < 32; ++m) {
+            const float tim = Tm[fsw(32 + i, 32 + m)];
+            const float4 yy = *reinterpret_cast<const float4 *>(&Zs[m * 32 + cc]);
+            z[0] += tim * yy.x; z[1] += tim * yy.y; z[2] += tim * yy.z; z[3] += tim * yy.w;
+        }
+        *reinterpret_cast<float4 *>(&Tm[fsw(32 + i, cc)]) = make_float4(-z[0], -z[1], -z[2], -z[3]);
     }
     __syncthreads();
 
-    // ---- phase 7: coalesced record stores ----
-    for (int it = tid; it < C * (D / 8); it += NT) {
-        const int r = it / (D / 8), c0 = (it % (D / 8)) * 8;
-        *reinterpret_cast<uint4 *>(rec + ws::OFF_W + ((size_t)r * D + c0) * 2) =
-            *reinterpret_cast<const uint4 *>(&sm.Xk[r][c0]);
-        *reinterpret_cast<uint4 *>(rec + ws::OFF_U + ((size_t)r * D + c0) * 2) =
-            *reinterpret_cast<const uint4 *>(&sm.Xq[r][c0]);
-    }
-    for (int it = tid; it < C * (C / 8); it += NT) {
-        const int r = it / (C / 8), c0 = (it % (C / 8)) * 8;
-        *reinterpret_cast<uint4 *>(rec + ws::OFF_P + ((size_t)r * C + c0) * 2) =
-            *reinterpret_cast<const uint4 *>(&sm.Pst[r][c0]);
+    // ---- W = T (beta K e^G) (warps 0-3), U = T (beta V) (warps 4-7) ----
+    {
+        const bool isU = warp >= 4;
+        const int qd = warp & 3;                       // 32-channel quarter
+        const unsigned char *Bs = isU ? sm.Vb : sm.KG;
+        float acc[4][4][4];
+#pragma unroll
+        for (int Ib = 0; Ib < 4; ++Ib)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[Ib][nt][e] = 0.f;
+        const int bkr = (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+        for (int Ib = 0; Ib < 4; ++Ib)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                if (ks <= Ib) {
+                    const int r0 = 16 * Ib + gid, k0 = 16 * ks + 2 * tig;
+                    uint32_t af[4];
+                    const float2 t00 = *reinterpret_cast<const float2 *>(&Tm[fsw(r0, k0)]);
+                    const float2 t10 = *reinterpret_cast<const float2 *>(&Tm[fsw(r0 + 8, k0)]);
+                    const float2 t01 = *reinterpret_cast<const float2 *>(&Tm[fsw(r0, k0 + 8)]);
+                    const float2 t11 = *reinterpret_cast<const float2 *>(&Tm[fsw(r0 + 8, k0 + 8)]);
+                    af[0] = pack_bf16(t00.x, t00.y);
+                    af[1] = pack_bf16(t10.x, t10.y);
+                    af[2] = pack_bf16(t01.x, t01.y);
+                    af[3] = pack_bf16(t11.x, t11.y);
+#pragma unroll
+                    for (int np = 0; np < 2; ++np) {
+                        uint32_t bf[4];
+                        const int kr = 16 * ks + bkr;
+                        ldsm_x4_t(bf, Bs + toff_chunk(kr, 4 * qd + 2 * np + (lane >> 4)));
+                        mma_bf16(acc[Ib][2 * np], af, bf[0], bf[1]);
+                        mma_bf16(acc[Ib][2 * np + 1], af, bf[2], bf[3]);
+                    }
+                }
+            }
+#pragma unroll
+        for (int Ib = 0; Ib < 4; ++Ib)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int r = 16 * Ib + gid + 8 * hh;
+                    const int n = 32 * qd + 8 * nt + 2 * tig;
+                    const uint32_t pk = pack_bf16(acc[Ib][nt][2 * hh], acc[Ib][nt][2 * hh + 1]);
+                    if (isU)
+                        *reinterpret_cast<uint32_t *>(rec + ws::OFF_U + (size_t)qd * ws::U_TILE + r * 64 +
+                                                      ((n & 31) << 1)) = pk;
+                    else
+                        *reinterpret_cast<uint32_t *>(rec + ws::aw_off(r, n)) = pk;
+                }
     }
 }
 

@@ -35,6 +35,13 @@ cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const
                               const float *beta, const int32_t *cu, const int32_t *coff,
                               int N, int T, int total_T, int H, int max_chunks,
                               unsigned char *wsp, cudaStream_t st);
+cudaError_t launch_chunk_chain_tc(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
+                                  const float *s0, float *sT, void *out, int N, int T,
+                                  int total_T, int H, int dvt, int max_chunks, int *err,
+                                  cudaStream_t st);
+cudaError_t launch_chunk_chain_mma(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
+                                   const float *s0, float *sT, void *out, int N, int T, int total_T,
+                                   int H, int dvt, int max_chunks, int *err, cudaStream_t st);
 cudaError_t launch_chunk_chain(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
                                const float *s0, float *sT, void *out, int N, int T, int total_T,
                                int H, int dvt, int max_chunks, int *err, cudaStream_t st);

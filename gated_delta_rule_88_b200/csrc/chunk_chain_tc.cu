@@ -48,8 +48,9 @@ struct TcLayout {
     static constexpr uint32_t B1_OFF = NS * STAGE;                 // S^bf16: K=128 x N=DVT
     static constexpr uint32_t B2_OFF = B1_OFF + 128 * DVT * 2;     // V_new: K=64 x N=DVT
     static constexpr uint32_t BAR_OFF = B2_OFF + 64 * DVT * 2;
-    static constexpr uint32_t BYTES = BAR_OFF + 8 * (2 * NS + 2) + 16;
-    static constexpr uint32_t NCOLS = 2 * DVT < 32 ? 32 : 2 * DVT;   // TMEM columns (pow2)
+    static constexpr uint32_t BYTES = BAR_OFF + 8 * (2 * NS + 3) + 16;
+    // TMEM columns: D1 double-buffered (2 x DVT) + D3 (DVT), rounded to a power of 2
+    static constexpr uint32_t NCOLS = 3 * DVT <= 32 ? 32 : 3 * DVT <= 64 ? 64 : 3 * DVT <= 128 ? 128 : 256;
     static constexpr uint32_t B1_SBO = (128 / 8) * 128;             // n-group stride
     static constexpr uint32_t B2_SBO = (64 / 8) * 128;
 };
@@ -74,8 +75,9 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::BAR_OFF);
     uint64_t *empty = full + NS;
     uint64_t *mma1 = empty + NS;
-    uint64_t *mma23 = mma1 + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma23 + 1);
+    uint64_t *mma3 = mma1 + 1;
+    uint64_t *mma2 = mma1 + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma1 + 3);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     unsigned char *B1 = sm + L::B1_OFF;
     unsigned char *B2 = sm + L::B2_OFF;
@@ -106,7 +108,8 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
         mbar_init(mma1, 1);
-        mbar_init(mma23, 1);
+        mbar_init(mma3, 1);
+        mbar_init(mma2, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -134,6 +137,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
                 bulk_g2s(st + L::U_OFF, rec + ws::OFF_U + (size_t)(n0 >> 5) * ws::U_TILE,
                          L::UT * 4096, &full[s]);
                 bulk_g2s(st + L::EGC_OFF, rec + ws::OFF_EGC, 512, &full[s]);
+                if (i + NS < nchunks) bulk_prefetch_l2(rec + (size_t)NS * rec_stride, REC_HEAD);
                 issued = i + 1;
             }
             // never leave with copies in flight into this CTA's shared memory
@@ -170,26 +174,60 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
         tc_fence_after();
 
         bool failed = false;
+        // descriptor words: A operands (K-major, 128-byte swizzle, 8-row groups
+        // 1024 B apart) relative to the ring base; B operands (MN-major
+        // interleaved, K groups 128 B apart)
+        const uint32_t sm_a = smem_u32(sm);
+        const DescParts a_sw = smem_desc_parts(sm_a, 16, 1024, 2);
+        const DescParts b1_d = smem_desc_parts(smem_u32(B1), 128, L::B1_SBO, 0);
+        const DescParts b2_d = smem_desc_parts(smem_u32(B2), 128, L::B2_SBO, 0);
+        // O of chunk ci (rows 64-127 of D1[ci & 1]) -> out; warps 2-3 only
+        auto emit_output = [&](int ci) -> bool {
+            bool okk = true;
+            if (t == 64) okk = mbar_wait(mma2, ci & 1);
+            if (named_bar_or(2, 64, !okk)) return false;
+            tc_fence_after();
+            const long long tok = bos + (long long)C * ci + (t - 64);
+            const uint32_t d1 = tmem + lane_base + (ci & 1) * DVT;
+#pragma unroll
+            for (int c16 = 0; c16 < DVT / 16; ++c16) {
+                float o[16];
+                tmem_ld16(d1 + c16 * 16, o);
+                tmem_wait_ld();
+                if (tok < eos) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)tok * H + h) * D + n0 + c16 * 16);
+                    dst[0] = make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]),
+                                        pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
+                    dst[1] = make_uint4(pack_bf16(o[8], o[9]), pack_bf16(o[10], o[11]),
+                                        pack_bf16(o[12], o[13]), pack_bf16(o[14], o[15]));
+                }
+            }
+            tc_fence_before();
+            return true;
+        };
         for (int i = 0; i < nchunks && !failed; ++i) {
             const int s = i % NS;
+            const int p = i & 1;
             unsigned char *st = sm + (size_t)s * L::STAGE;
             const uint32_t st_a = smem_u32(st);
-            const uint32_t b1_a = smem_u32(B1), b2_a = smem_u32(B2);
+            const uint32_t d1 = tmem + p * DVT;          // this chunk's [W;Qg] S accumulator
+            const uint32_t d3 = tmem + 2 * DVT;          // Kt^T V_new accumulator
             bool ok = true;
             if (t == 0) {
                 ok = mbar_wait(&full[s], (i / NS) & 1);
                 if (ok) {
                     tc_fence_after();
+                    const uint32_t a_lo = a_sw.lo + ((st_a - sm_a) >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint64_t ad = smem_desc(st_a + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, 2);
-                        const uint64_t bd = smem_desc(b1_a + kk * 256, 128, L::B1_SBO, 0);
-                        umma_bf16(tmem, ad, bd, IDESC, kk > 0);
-                    }
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_bf16_p(d1, a_lo + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), a_sw.hi,
+                                    b1_d.lo + ((kk * 256) >> 4), b1_d.hi, IDESC, kk > 0);
                     umma_commit(mma1);
-                    ok = mbar_wait(mma1, i & 1);
                 }
             }
+            // while MMA1 runs: the previous chunk's output leaves through warps 2-3
+            if (t >= 64 && i > 0 && !emit_output(i - 1)) ok = false;
+            if (t == 0 && ok) ok = mbar_wait(mma1, i & 1);
             if (named_bar_or(1, 128, !ok)) { failed = true; break; }
             tc_fence_after();
             const float eg = reinterpret_cast<const float *>(st + L::EGC_OFF)[t];
@@ -198,7 +236,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
 #pragma unroll
                 for (int c16 = 0; c16 < DVT / 16; ++c16) {
                     float x[16];
-                    tmem_ld16(tmem + lane_base + c16 * 16, x);
+                    tmem_ld16(tmem + lane_base + p * DVT + c16 * 16, x);
                     tmem_wait_ld();
                     // column (n0 % 32) + 16 c16 of the loaded U tile(s), row t
                     const int lc = (n0 & 31) + c16 * 16;
@@ -221,21 +259,20 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
             tc_fence_after();
             ok = true;
             if (t == 0) {
+                // the state update (MMA3) is on the critical path: issue it first
+                const uint32_t a_lo = a_sw.lo + ((st_a - sm_a) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bd = smem_desc(b2_a + kk * 256, 128, L::B2_SBO, 0);
-                    const uint64_t ap = smem_desc(st_a + (uint32_t)ws::OFF_P - 8192 + kk * 32, 16, 1024, 2);
-                    umma_bf16(tmem, ap, bd, IDESC, 1);
-                }
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16_p(d3, a_lo + (((uint32_t)ws::OFF_KTT + kk * 32) >> 4), a_sw.hi,
+                                b2_d.lo + ((kk * 256) >> 4), b2_d.hi, IDESC, kk > 0);
+                umma_commit(mma3);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bd = smem_desc(b2_a + kk * 256, 128, L::B2_SBO, 0);
-                    const uint64_t ak = smem_desc(st_a + (uint32_t)ws::OFF_KTT + kk * 32, 16, 1024, 2);
-                    umma_bf16(tmem + DVT, ak, bd, IDESC, kk > 0);
-                }
-                umma_commit(mma23);
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16_p(d1, a_lo + (((uint32_t)ws::OFF_P - 8192 + kk * 32) >> 4), a_sw.hi,
+                                b2_d.lo + ((kk * 256) >> 4), b2_d.hi, IDESC, 1);
+                umma_commit(mma2);
                 umma_commit(&empty[s]);
-                ok = mbar_wait(mma23, i & 1);
+                ok = mbar_wait(mma3, i & 1);
             }
             if (named_bar_or(1, 128, !ok)) { failed = true; break; }
             tc_fence_after();
@@ -243,34 +280,18 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
 #pragma unroll
             for (int c16 = 0; c16 < DVT / 16; ++c16) {
                 float z[16];
-                tmem_ld16(tmem + lane_base + DVT + c16 * 16, z);
+                tmem_ld16(tmem + lane_base + 2 * DVT + c16 * 16, z);
                 tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 16; ++e) S[c16 * 16 + e] = eg * S[c16 * 16 + e] + z[e];
             }
             write_B1();
-            if (t >= 64) {
-                // O = Qg S + P V_new for token row t - 64
-                const long long tok = bos + (long long)C * i + (t - 64);
-#pragma unroll
-                for (int c16 = 0; c16 < DVT / 16; ++c16) {
-                    float o[16];
-                    tmem_ld16(tmem + lane_base + c16 * 16, o);
-                    tmem_wait_ld();
-                    if (tok < eos) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)tok * H + h) * D + n0 + c16 * 16);
-                        dst[0] = make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]),
-                                            pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
-                        dst[1] = make_uint4(pack_bf16(o[8], o[9]), pack_bf16(o[10], o[11]),
-                                            pack_bf16(o[12], o[13]), pack_bf16(o[14], o[15]));
-                    }
-                }
-            }
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(1, 128);
             tc_fence_after();
         }
+        if (!failed && nchunks > 0 && t >= 64 && !emit_output(nchunks - 1)) failed = true;
         if (failed) {
             if (t == 0) { set_device_error(err, kErrWaitTimeout); *abort_flag = 1; }
         } else if (sT) {
@@ -304,7 +325,7 @@ cudaError_t launch_tc(const unsigned char *wsp, const int32_t *cu, const int32_t
 
 }  // namespace
 
-cudaError_t launch_chunk_chain_tc(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
+cudaError_t launch_chunk_chain(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
                                   const float *s0, float *sT, void *out, int N, int T,
                                   int total_T, int H, int dvt, int max_chunks, int *err,
                                   cudaStream_t st)

@@ -190,6 +190,7 @@ chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     }
     {
         uint32_t kt[2][8];   // Kt for (channel, token pair) -> transposed store
+        float2 kt_prev = make_float2(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int r = 16 * I + i;
@@ -206,18 +207,17 @@ chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             *reinterpret_cast<uint32_t *>(sm.Xk + o) = pack_bf16(br * kx * ai.x, br * ky * ai.y);
             *reinterpret_cast<uint32_t *>(sm.KG + o) =
                 pack_bf16(br * kx * ai.x * E.x, br * ky * ai.y * E.y);
-            *reinterpret_cast<uint32_t *>(sm.Kd + o) = pack_bf16(kx / ai.x, ky / ai.y);
+            *reinterpret_cast<uint32_t *>(sm.Kd + o) = pack_bf16(__fdividef(kx, ai.x), __fdividef(ky, ai.y));
             *reinterpret_cast<uint32_t *>(sm.Kb + o) = pack_bf16(kx * bi.x, ky * bi.y);
             *reinterpret_cast<uint32_t *>(sm.Vb + o) = pack_bf16(br * vx, br * vy);
             *reinterpret_cast<uint32_t *>(rec + ws::aw_off(64 + r, c0)) =
                 pack_bf16(qx * ai.x * E.x, qy * ai.y * E.y);
             const float ktx = kx * bi.x * F.x, kty = ky * bi.y * F.y;
             if (i & 1) {
-                kt[0][i >> 1] = pack_bf16(__low2float(*reinterpret_cast<__nv_bfloat162 *>(&kt[0][i >> 1])), ktx);
-                kt[1][i >> 1] = pack_bf16(__low2float(*reinterpret_cast<__nv_bfloat162 *>(&kt[1][i >> 1])), kty);
+                kt[0][i >> 1] = pack_bf16(kt_prev.x, ktx);
+                kt[1][i >> 1] = pack_bf16(kt_prev.y, kty);
             } else {
-                kt[0][i >> 1] = pack_bf16(ktx, 0.f);
-                kt[1][i >> 1] = pack_bf16(kty, 0.f);
+                kt_prev = make_float2(ktx, kty);
             }
         }
 #pragma unroll
@@ -256,7 +256,7 @@ chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
                     uint32_t bf[4];
                     const int br = 16 * J + bn;
                     ldsm_x4(bf, (J < Ib ? sm.Kb : sm.Kd) + toff_chunk(br, 2 * ks + bk));
-                    if (J < Ib) {
+                    if (J + 1 < Ib) {   // D_JI = 1 for adjacent blocks
                         const float *dm = sm.Dm[pair_idx(J, Ib)];
                         const float2 slo = *reinterpret_cast<const float2 *>(dm + 16 * ks + 2 * tig);
                         const float2 shi = *reinterpret_cast<const float2 *>(dm + 16 * ks + 8 + 2 * tig);

@@ -27,7 +27,8 @@ cudaError_t launch_chunk_f32(const float *q, const float *k, const float *v, con
 // buffer of per-(chunk, head) records (chunk_ws.h):
 //   chunk_plan  (varlen only) chunk offsets per sequence -> coff[N+1]
 //   chunk_prep  parallel over (chunk, head): G, A, P, T, W, U, Qg, Kt, e^{G_C}
-//   chunk_chain sequential over chunks per (sequence, head, dv tile)
+//   chunk_chain sequential over chunks per (sequence, head, dv tile),
+//               tcgen05 MMAs with TMEM accumulators (chunk_chain_tc.cu)
 size_t chunk_prep_smem_bytes();
 cudaError_t launch_chunk_plan(const int32_t *cu, int N, int total_T, int32_t *coff,
                               cudaStream_t st);
@@ -35,13 +36,6 @@ cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const
                               const float *beta, const int32_t *cu, const int32_t *coff,
                               int N, int T, int total_T, int H, int max_chunks,
                               unsigned char *wsp, cudaStream_t st);
-cudaError_t launch_chunk_chain_tc(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
-                                  const float *s0, float *sT, void *out, int N, int T,
-                                  int total_T, int H, int dvt, int max_chunks, int *err,
-                                  cudaStream_t st);
-cudaError_t launch_chunk_chain_mma(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
-                                   const float *s0, float *sT, void *out, int N, int T, int total_T,
-                                   int H, int dvt, int max_chunks, int *err, cudaStream_t st);
 cudaError_t launch_chunk_chain(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
                                const float *s0, float *sT, void *out, int N, int T, int total_T,
                                int H, int dvt, int max_chunks, int *err, cudaStream_t st);

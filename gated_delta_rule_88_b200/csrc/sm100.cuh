@@ -122,6 +122,31 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
     d |= (uint64_t)(layout & 7) << 61;
     return d;
 }
+// The same descriptor split into its two 32-bit halves: the low word holds
+// the start address (>> 4) and the leading byte offset, so stepping along K
+// is one 32-bit add on `lo` (addresses stay below 256 KiB).
+struct DescParts { uint32_t lo, hi; };
+__device__ __forceinline__ DescParts smem_desc_parts(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                                     uint32_t layout) {
+    const uint64_t d = smem_desc(saddr, lbo, sbo, layout);
+    return DescParts{(uint32_t)d, (uint32_t)(d >> 32)};
+}
+// D[tmem] (+)= A[smem] * B[smem] with descriptors given as (lo, hi) words.
+__device__ __forceinline__ void umma_bf16_p(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
+                                            uint32_t b_lo, uint32_t b_hi, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+        "mov.b64 da, {%1, %2};\n\t"
+        "mov.b64 db, {%3, %4};\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate));
+}
+// L2 prefetch of a global range (no shared-memory destination).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *gmem, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(gmem), "r"(bytes) : "memory");
+}
 // D[tmem] (+)= A[smem] * B[smem]; issued by one thread.
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                           uint32_t idesc, uint32_t accumulate) {

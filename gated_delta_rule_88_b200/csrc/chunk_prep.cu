@@ -31,8 +31,9 @@
 // m16n8k16 bf16 MMAs per row block (left operand (beta k a) or (q a), right
 // operand k b scaled by D_JI, or k / a on the diagonal block); T is formed in
 // fp32 (16x16 diagonal blocks by forward substitution, then the 2x2-block
-// recursion T21 = -T22 A21 T11 at 16 and 32 rows); W and U are m16n8k16 MMAs
-// with T rounded once to bf16.
+// recursion T21 = -T22 A21 T11 at 16 and 32 rows on tf32 tensor-core MMAs
+// with fp32 accumulation); W and U are m16n8k16 MMAs with T rounded once to
+// bf16.
 #include "chunk_ws.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -54,6 +55,27 @@ __device__ __forceinline__ int toff_chunk(int r, int j) {
 }
 // 64 x 64 fp32 matrix, column groups of 4 XOR-swizzled by row
 __device__ __forceinline__ int fsw(int i, int j) { return i * 64 + (j ^ ((i & 7) << 2)); }
+// C(16x8) += X[r0:r0+16, kx0:kx0+K] Y[ky0:ky0+K, n0:n0+8], both in the fsw layout
+template <int K>
+__device__ __forceinline__ void tile_tf32(float (&c)[4], const float *X, int r0, int kx0,
+                                          const float *Y, int ky0, int n0, int gid, int tig) {
+#pragma unroll
+    for (int ks = 0; ks < K; ks += 8) {
+        const uint32_t a[4] = {to_tf32(X[fsw(r0 + gid, kx0 + ks + tig)]),
+                               to_tf32(X[fsw(r0 + gid + 8, kx0 + ks + tig)]),
+                               to_tf32(X[fsw(r0 + gid, kx0 + ks + tig + 4)]),
+                               to_tf32(X[fsw(r0 + gid + 8, kx0 + ks + tig + 4)])};
+        mma_tf32(c, a, to_tf32(Y[fsw(ky0 + ks + tig, n0 + gid)]),
+                 to_tf32(Y[fsw(ky0 + ks + tig + 4, n0 + gid)]));
+    }
+}
+__device__ __forceinline__ void store_tile(float *Mx, const float (&c)[4], int r0, int n0,
+                                           int gid, int tig, float sgn) {
+    Mx[fsw(r0 + gid, n0 + 2 * tig)] = sgn * c[0];
+    Mx[fsw(r0 + gid, n0 + 2 * tig + 1)] = sgn * c[1];
+    Mx[fsw(r0 + gid + 8, n0 + 2 * tig)] = sgn * c[2];
+    Mx[fsw(r0 + gid + 8, n0 + 2 * tig + 1)] = sgn * c[3];
+}
 // index of the (J, I) block pair, J < I
 __device__ __forceinline__ int pair_idx(int J, int I) { return I * (I - 1) / 2 + J; }
 
@@ -97,6 +119,70 @@ __device__ __forceinline__ void locate_chunk(int chunk, const int32_t *cu, const
     }
     t0 = bos + (long long)C * cidx;
     len = (int)max(0LL, min((long long)C, eos - t0));
+}
+
+// A (isP = false: left operand beta k a) or P (isP = true: left operand q a)
+// for row block Ib: 16 rows x 16 (Ib + 1) columns, on m16n8k16 bf16 MMAs.
+// Ends with a CTA barrier (the operand tiles are then dead), after which A is
+// written as fp32 over the Xq tile and P (masked, bf16) into the record.
+template <int Ib>
+__device__ __forceinline__ void ap_block(PrepSmem &sm, unsigned char *rec, bool isP, int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+    const unsigned char *X = isP ? sm.Xq : sm.Xk;
+    float acc[Ib + 1][2][4];
+#pragma unroll
+    for (int J = 0; J <= Ib; ++J)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[J][nt][e] = 0.f;
+    const int ar = 16 * Ib + (lane & 7) + 8 * ((lane >> 3) & 1);
+    const int bn = (lane & 7) + 8 * (lane >> 4);
+    const int bk = (lane >> 3) & 1;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+        uint32_t af[4];
+        ldsm_x4(af, X + toff_chunk(ar, 2 * ks + (lane >> 4)));
+#pragma unroll
+        for (int J = 0; J <= Ib; ++J) {
+            uint32_t bf[4];
+            ldsm_x4(bf, (J < Ib ? sm.Kb : sm.Kd) + toff_chunk(16 * J + bn, 2 * ks + bk));
+            if (J + 1 < Ib) {   // D_JI = 1 for adjacent blocks
+                const float *dm = sm.Dm[pair_idx(J, Ib)];
+                const float2 slo = *reinterpret_cast<const float2 *>(dm + 16 * ks + 2 * tig);
+                const float2 shi = *reinterpret_cast<const float2 *>(dm + 16 * ks + 8 + 2 * tig);
+                bf[0] = scale_bf16x2(bf[0], slo);
+                bf[2] = scale_bf16x2(bf[2], slo);
+                bf[1] = scale_bf16x2(bf[1], shi);
+                bf[3] = scale_bf16x2(bf[3], shi);
+            }
+            mma_bf16(acc[J][0], af, bf[0], bf[1]);
+            mma_bf16(acc[J][1], af, bf[2], bf[3]);
+        }
+    }
+    __syncthreads();   // operand tiles are dead: Xq becomes A (fp32)
+    float *Am = reinterpret_cast<float *>(sm.Xq);
+#pragma unroll
+    for (int J = 0; J < 4; ++J)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int i = 16 * Ib + gid + 8 * hh;
+                const int j = 16 * J + 8 * nt + 2 * tig;
+                float v0 = 0.f, v1 = 0.f;
+                if (J <= Ib) { v0 = acc[J <= Ib ? J : 0][nt][2 * hh]; v1 = acc[J <= Ib ? J : 0][nt][2 * hh + 1]; }
+                if (!isP) {
+                    if (J <= Ib) {
+                        Am[fsw(i, j)] = (j < i) ? v0 : 0.f;
+                        Am[fsw(i, j + 1)] = (j + 1 < i) ? v1 : 0.f;
+                    }
+                } else {
+                    v0 = (j <= i) ? v0 : 0.f;
+                    v1 = (j + 1 <= i) ? v1 : 0.f;
+                    *reinterpret_cast<uint32_t *>(rec + ws::OFF_P + ws::sw128(i, j)) = pack_bf16(v0, v1);
+                }
+            }
 }
 
 __global__ void __launch_bounds__(NT, 2)
@@ -232,66 +318,11 @@ chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     __syncthreads();
 
     // ---- A (warps 0-3) and P (warps 4-7) for row block Ib = warp & 3 ----
-    {
-        const int Ib = warp & 3;
-        const bool isP = warp >= 4;
-        const unsigned char *X = isP ? sm.Xq : sm.Xk;
-        float acc[4][2][4];
-#pragma unroll
-        for (int J = 0; J < 4; ++J)
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[J][nt][e] = 0.f;
-        const int ar = 16 * Ib + (lane & 7) + 8 * ((lane >> 3) & 1);
-        const int bn = (lane & 7) + 8 * (lane >> 4);
-        const int bk = (lane >> 3) & 1;
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-            uint32_t af[4];
-            ldsm_x4(af, X + toff_chunk(ar, 2 * ks + (lane >> 4)));
-#pragma unroll
-            for (int J = 0; J < 4; ++J) {
-                if (J <= Ib) {
-                    uint32_t bf[4];
-                    const int br = 16 * J + bn;
-                    ldsm_x4(bf, (J < Ib ? sm.Kb : sm.Kd) + toff_chunk(br, 2 * ks + bk));
-                    if (J + 1 < Ib) {   // D_JI = 1 for adjacent blocks
-                        const float *dm = sm.Dm[pair_idx(J, Ib)];
-                        const float2 slo = *reinterpret_cast<const float2 *>(dm + 16 * ks + 2 * tig);
-                        const float2 shi = *reinterpret_cast<const float2 *>(dm + 16 * ks + 8 + 2 * tig);
-                        bf[0] = scale_bf16x2(bf[0], slo);
-                        bf[2] = scale_bf16x2(bf[2], slo);
-                        bf[1] = scale_bf16x2(bf[1], shi);
-                        bf[3] = scale_bf16x2(bf[3], shi);
-                    }
-                    mma_bf16(acc[J][0], af, bf[0], bf[1]);
-                    mma_bf16(acc[J][1], af, bf[2], bf[3]);
-                }
-            }
-        }
-        __syncthreads();   // operand tiles are dead: Xq becomes A (fp32)
-        float *Am = reinterpret_cast<float *>(sm.Xq);
-#pragma unroll
-        for (int J = 0; J < 4; ++J)
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int i = 16 * Ib + gid + 8 * hh;
-                    const int j = 16 * J + 8 * nt + 2 * tig;
-                    float v0 = acc[J][nt][2 * hh], v1 = acc[J][nt][2 * hh + 1];
-                    if (!isP) {
-                        if (J <= Ib) {
-                            Am[fsw(i, j)] = (j < i) ? v0 : 0.f;
-                            Am[fsw(i, j + 1)] = (j + 1 < i) ? v1 : 0.f;
-                        }
-                    } else {
-                        v0 = (J <= Ib && j <= i) ? v0 : 0.f;
-                        v1 = (J <= Ib && j + 1 <= i) ? v1 : 0.f;
-                        *reinterpret_cast<uint32_t *>(rec + ws::OFF_P + ws::sw128(i, j)) = pack_bf16(v0, v1);
-                    }
-                }
+    switch (warp & 3) {
+        case 0: ap_block<0>(sm, rec, warp >= 4, lane); break;
+        case 1: ap_block<1>(sm, rec, warp >= 4, lane); break;
+        case 2: ap_block<2>(sm, rec, warp >= 4, lane); break;
+        default: ap_block<3>(sm, rec, warp >= 4, lane); break;
     }
     __syncthreads();
 
@@ -322,53 +353,34 @@ chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
         }
     }
     __syncthreads();
-    {
-        // 16-row level: T_IJ = -T_II (A_IJ T_JJ) for (I, J) = (1, 0), (3, 2)
-        const int which = tid >> 7, idx = tid & 127;
-        const int Ib = which ? 3 : 1, Jb = Ib - 1;
-        const int i = idx >> 3, cc = (idx & 7) * 2;
-        float z0 = 0.f, z1 = 0.f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const float aij = Am[fsw(16 * Ib + i, 16 * Jb + j)];
-            const float2 t = *reinterpret_cast<const float2 *>(&Tm[fsw(16 * Jb + j, 16 * Jb + cc)]);
-            z0 += aij * t.x;
-            z1 += aij * t.y;
-        }
-        Zs[which * 256 + i * 16 + cc] = z0;
-        Zs[which * 256 + i * 16 + cc + 1] = z1;
-        __syncthreads();
-        float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const float tim = Tm[fsw(16 * Ib + i, 16 * Ib + m)];
-            y0 += tim * Zs[which * 256 + m * 16 + cc];
-            y1 += tim * Zs[which * 256 + m * 16 + cc + 1];
-        }
-        Tm[fsw(16 * Ib + i, 16 * Jb + cc)] = -y0;
-        Tm[fsw(16 * Ib + i, 16 * Jb + cc + 1)] = -y1;
+    // Off-diagonal blocks on the tensor cores (tf32, fp32 accumulate), one
+    // 16x8 output tile per warp:
+    //   16-row level: T_IJ = -T_II (A_IJ T_JJ) for (I, J) = (1, 0), (3, 2)
+    //   32-row level: T[32:64, 0:32] = -T[32:64, 32:64] (A[32:64, 0:32] T[0:32, 0:32])
+    // Zs holds the inner products at the coordinates of the block they feed.
+    if (warp < 4) {
+        const int Ib = (warp >> 1) ? 3 : 1, Jb = Ib - 1, n0 = 16 * Jb + 8 * (warp & 1);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        tile_tf32<16>(c, Am, 16 * Ib, 16 * Jb, Tm, 16 * Jb, n0, gid, tig);
+        store_tile(Zs, c, 16 * Ib, n0, gid, tig, 1.f);
+    }
+    __syncthreads();
+    if (warp < 4) {
+        const int Ib = (warp >> 1) ? 3 : 1, Jb = Ib - 1, n0 = 16 * Jb + 8 * (warp & 1);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        tile_tf32<16>(c, Tm, 16 * Ib, 16 * Ib, Zs, 16 * Ib, n0, gid, tig);
+        store_tile(Tm, c, 16 * Ib, n0, gid, tig, -1.f);
     }
     __syncthreads();
     {
-        // 32-row level: T[32:64, 0:32] = -T[32:64, 32:64] (A[32:64, 0:32] T[0:32, 0:32])
-        const int i = tid >> 3, cc = (tid & 7) * 4;
-        float y[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-        for (int j = 0; j < 32; ++j) {
-            const float aij = Am[fsw(32 + i, j)];
-            const float4 t = *reinterpret_cast<const float4 *>(&Tm[fsw(j, cc)]);
-            y[0] += aij * t.x; y[1] += aij * t.y; y[2] += aij * t.z; y[3] += aij * t.w;
-        }
-        *reinterpret_cast<float4 *>(&Zs[i * 32 + cc]) = make_float4(y[0], y[1], y[2], y[3]);
+        const int r0 = 32 + 16 * (warp >> 2), n0 = 8 * (warp & 3);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        tile_tf32<32>(c, Am, r0, 0, Tm, 0, n0, gid, tig);
+        store_tile(Zs, c, r0, n0, gid, tig, 1.f);
         __syncthreads();
         float z[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-        for (int m = 0; m < 32; ++m) {
-            const float tim = Tm[fsw(32 + i, 32 + m)];
-            const float4 yy = *reinterpret_cast<const float4 *>(&Zs[m * 32 + cc]);
-            z[0] += tim * yy.x; z[1] += tim * yy.y; z[2] += tim * yy.z; z[3] += tim * yy.w;
-        }
-        *reinterpret_cast<float4 *>(&Tm[fsw(32 + i, cc)]) = make_float4(-z[0], -z[1], -z[2], -z[3]);
+        tile_tf32<32>(z, Tm, r0, 32, Zs, 32, n0, gid, tig);
+        store_tile(Tm, z, r0, n0, gid, tig, -1.f);
     }
     __syncthreads();
 

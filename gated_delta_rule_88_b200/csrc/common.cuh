@@ -89,3 +89,23 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 }  // namespace kda
+
+namespace kda {
+// m16n8k8 tf32 MMA with fp32 accumulate.  Fragments (lane = 4*gid + tig):
+//   A 16x8: a0 (gid, tig)  a1 (gid+8, tig)  a2 (gid, tig+4)  a3 (gid+8, tig+4)
+//   B 8x8:  b0 (k = tig, n = gid)  b1 (k = tig+4, n = gid)
+//   C 16x8: as for the bf16 shape.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+}  // namespace kda

@@ -46,6 +46,30 @@ DEC_N, DEC_H = 256, 32
 DECODE_BYTES = DEC_N * DEC_H * (2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 2)
 FALLBACK_HBM_GBS = 6650.0
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# one ncu capture of each kernel on this workload (profiles/), valid only for
+# the kernel sources it was taken on: reported as null once they change.
+_SRC = os.path.join(ROOT, "gated_delta_rule_88_b200", "csrc")
+TRAFFIC = {
+    "prefill": {"files": ["chunk_prep.cu", "chunk_chain_tc.cu", "chunk_ws.h", "sm100.cuh", "common.cuh"],
+                "sha": "93f597dd29195e1a", "bytes": (342.131712 + 264.254464 + 304.178176 + 52.943872) * 1e6},
+    "decode": {"files": ["decode.cu", "common.cuh"], "sha": "5538ff5eaafbaa61",
+               "bytes": (547.416576 + 479.912448) * 1e6},
+}
+
+
+def measured_traffic(which):
+    import hashlib
+    t = TRAFFIC[which]
+    m = hashlib.sha256()
+    try:
+        for f in t["files"]:
+            with open(os.path.join(_SRC, f), "rb") as fh:
+                m.update(fh.read())
+    except OSError:
+        return None
+    return t["bytes"] if m.hexdigest()[:16] == t["sha"] else None
+
 
 def measured_peak_hbm():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -209,8 +233,11 @@ def run_ours(args):
     barrier(dist)
     e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), dist) / e2e_steps
 
-    # ---- decode leg ----
-    dec = decode_leg(kda, W, dev, dist, world, args)
+    # ---- decode leg (its timed region is sampled for clocks too) ----
+    with ClockSampler(local) as clk_dec:
+        dec = decode_leg(kda, W, dev, dist, world, args)
+    clk.samples += clk_dec.samples
+    clk.reasons |= clk_dec.reasons
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -224,7 +251,8 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "kernel": "kda_chunk_fwd (chunk_prep + chunk_chain)",
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_kind,
-                     "algorithmic_bytes_per_launch": PREFILL_BYTES, "traffic": None},
+                     "algorithmic_bytes_per_launch": PREFILL_BYTES,
+                     "traffic": measured_traffic("prefill")},
         "e2e": {"value": world * B * T / (e2e_ms * 1e-3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
@@ -268,7 +296,8 @@ def decode_leg(kda, W, dev, dist, world, args):
             "l2": "state (512 MiB) larger than L2; no flush",
             "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": ach,
                          "peak": peak, "unit": "GB/s", "frac": ach / peak, "peak_source": kind,
-                         "algorithmic_bytes_per_launch": DECODE_BYTES, "traffic": None}}
+                         "algorithmic_bytes_per_launch": DECODE_BYTES,
+                         "traffic": measured_traffic("decode")}}
 
 
 def cpu_baseline(inp_cpu, tokens=None):

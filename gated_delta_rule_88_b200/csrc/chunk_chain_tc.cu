@@ -16,13 +16,15 @@
 // 128-byte swizzle); B operands (S, V_new) are written by the threads in the
 // MN-major interleaved layout.
 //
-// Roles (160 threads): warps 0-3 own TMEM lanes 0-127 (thread t = token row
-// t for D1, channel row t for D3); thread 0 also issues the MMAs.  Warp 4
-// lane 0 streams records into an NS-stage shared-memory ring with
-// cp.async.bulk (plain, no multicast) and mbarrier transaction counts.
-// Every wait is bounded: a wait that runs out sets the device error word and
-// the whole CTA leaves its loop together (OR-reduced barrier), waits (bounded)
-// for copies in flight, frees TMEM and returns.
+// Roles (192 threads): warps 0-3 are the epilogue (thread t <-> TMEM lane t:
+// token row t of D1, channel row t of D3); warp 4 lane 0 streams records into
+// an NS-stage shared-memory ring with cp.async.bulk (plain, no multicast) and
+// mbarrier transaction counts; warp 5 lane 0 issues the MMAs.  The issuer and
+// the epilogue meet at two OR-reduced named barriers per chunk (S ready, V_new
+// ready), which also carry failures, so every party leaves the loop at the
+// same barrier.  Every wait is bounded: a wait that runs out sets the device
+// error word; the CTA then drains its copies and MMAs (bounded), frees TMEM and
+// returns.
 #include "chunk_ws.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -35,7 +37,7 @@ using namespace sm100;
 
 constexpr int C = ws::C;
 constexpr int D = ws::D;
-constexpr int NTHREADS = 160;
+constexpr int NTHREADS = 192;
 constexpr uint32_t REC_HEAD = 57344;       // [W;Qg] + Kt^T + P, contiguous in the record
 
 template <int DVT, int NS>
@@ -48,7 +50,7 @@ struct TcLayout {
     static constexpr uint32_t B1_OFF = NS * STAGE;                 // S^bf16: K=128 x N=DVT
     static constexpr uint32_t B2_OFF = B1_OFF + 128 * DVT * 2;     // V_new: K=64 x N=DVT
     static constexpr uint32_t BAR_OFF = B2_OFF + 64 * DVT * 2;
-    static constexpr uint32_t BYTES = BAR_OFF + 8 * (2 * NS + 3) + 16;
+    static constexpr uint32_t BYTES = BAR_OFF + 8 * (2 * NS + 4) + 16;
     // TMEM columns: D1 double-buffered (2 x DVT) + D3 (DVT), rounded to a power of 2
     static constexpr uint32_t NCOLS = 3 * DVT <= 32 ? 32 : 3 * DVT <= 64 ? 64 : 3 * DVT <= 128 ? 128 : 256;
     static constexpr uint32_t B1_SBO = (128 / 8) * 128;             // n-group stride
@@ -77,7 +79,8 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
     uint64_t *mma1 = empty + NS;
     uint64_t *mma3 = mma1 + 1;
     uint64_t *mma2 = mma1 + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma1 + 3);
+    uint64_t *drain = mma1 + 3;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma1 + 4);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     unsigned char *B1 = sm + L::B1_OFF;
     unsigned char *B2 = sm + L::B2_OFF;
@@ -110,6 +113,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
         mbar_init(mma1, 1);
         mbar_init(mma3, 1);
         mbar_init(mma2, 1);
+        mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -118,6 +122,8 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    constexpr int BAR_S = 1, BAR_V = 2, BAR_O = 3;     // named barriers (0 = __syncthreads)
+    constexpr int NSYNC = 160;                         // epilogue warps 0-3 + issuer warp 5
 
     if (warp == 4) {
         // ---------------- loader ----------------
@@ -144,11 +150,62 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
             for (int j = max(0, issued - NS); j < issued; ++j)
                 mbar_wait(&full[j % NS], (j / NS) & 1, 1u << 20);
         }
+    } else if (warp == 5) {
+        // ---------------- MMA issuer (lane 0; the warp joins the barriers) ----------------
+        constexpr uint32_t IDESC = idesc_bf16(128, DVT, true);
+        // A operands: K-major, 128-byte swizzle, 8-row groups 1024 B apart, relative
+        // to the ring base; B operands: MN-major interleaved, K groups 128 B apart
+        const uint32_t sm_a = smem_u32(sm);
+        const DescParts a_sw = smem_desc_parts(sm_a, 16, 1024, 2);
+        const DescParts b1_d = smem_desc_parts(smem_u32(B1), 128, L::B1_SBO, 0);
+        const DescParts b2_d = smem_desc_parts(smem_u32(B2), 128, L::B2_SBO, 0);
+        bool issued_any = false;
+        for (int i = 0; i < nchunks; ++i) {
+            const int s = i % NS;
+            const int p = i & 1;
+            const uint32_t a_lo = a_sw.lo + ((uint32_t)s * L::STAGE >> 4);
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(&full[s], (i / NS) & 1);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (named_bar_or(BAR_S, NSYNC, !ok)) break;        // S_i is in B1
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t d1 = tmem + p * DVT;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_bf16_p(d1, a_lo + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), a_sw.hi,
+                                b1_d.lo + ((kk * 256) >> 4), b1_d.hi, IDESC, kk > 0);
+                umma_commit(mma1);
+                issued_any = true;
+            }
+            __syncwarp();
+            if (named_bar_or(BAR_V, NSYNC, false)) break;      // V_new is in B2
+            tc_fence_after();
+            if (lane == 0) {
+                // the state update (MMA3) is on the critical path: issue it first
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16_p(tmem + 2 * DVT, a_lo + (((uint32_t)ws::OFF_KTT + kk * 32) >> 4),
+                                a_sw.hi, b2_d.lo + ((kk * 256) >> 4), b2_d.hi, IDESC, kk > 0);
+                umma_commit(mma3);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16_p(tmem + p * DVT, a_lo + (((uint32_t)ws::OFF_P - 8192 + kk * 32) >> 4),
+                                a_sw.hi, b2_d.lo + ((kk * 256) >> 4), b2_d.hi, IDESC, 1);
+                umma_commit(mma2);
+                umma_commit(&empty[s]);
+            }
+            __syncwarp();
+        }
+        // never free TMEM under a running MMA
+        if (lane == 0 && issued_any) {
+            umma_commit(drain);
+            mbar_wait(drain, 0, 1u << 20);
+        }
     } else {
-        // ---------------- math warps: thread t <-> TMEM lane t ----------------
+        // ---------------- epilogue warps 0-3: thread t <-> TMEM lane t ----------------
         const int t = tid;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        constexpr uint32_t IDESC = idesc_bf16(128, DVT, true);
         float S[DVT];
         {
             const size_t sb = (((size_t)seq * H + h) * D + t) * D + n0;
@@ -166,134 +223,98 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
                                       pack_bf16(S[8 * ng + 4], S[8 * ng + 5]), pack_bf16(S[8 * ng + 6], S[8 * ng + 7]));
                 *reinterpret_cast<uint4 *>(B1 + mn_off(t, ng, L::B1_SBO)) = pk;
             }
+            fence_proxy_async_smem();
         };
-        write_B1();
-        fence_proxy_async_smem();
-        tc_fence_before();
-        named_bar(1, 128);
-        tc_fence_after();
-
-        bool failed = false;
-        // descriptor words: A operands (K-major, 128-byte swizzle, 8-row groups
-        // 1024 B apart) relative to the ring base; B operands (MN-major
-        // interleaved, K groups 128 B apart)
-        const uint32_t sm_a = smem_u32(sm);
-        const DescParts a_sw = smem_desc_parts(sm_a, 16, 1024, 2);
-        const DescParts b1_d = smem_desc_parts(smem_u32(B1), 128, L::B1_SBO, 0);
-        const DescParts b2_d = smem_desc_parts(smem_u32(B2), 128, L::B2_SBO, 0);
+        // DVT columns of lane t starting at column col
+        auto tmem_row = [&](uint32_t col, float (&x)[DVT]) {
+            if constexpr (DVT == 16) {
+                tmem_ld16(tmem + lane_base + col, x);
+            } else {
+#pragma unroll
+                for (int c32 = 0; c32 < DVT / 32; ++c32)
+                    tmem_ld32(tmem + lane_base + col + 32 * c32, *reinterpret_cast<float (*)[32]>(&x[32 * c32]));
+            }
+            tmem_wait_ld();
+        };
         // O of chunk ci (rows 64-127 of D1[ci & 1]) -> out; warps 2-3 only
         auto emit_output = [&](int ci) -> bool {
             bool okk = true;
             if (t == 64) okk = mbar_wait(mma2, ci & 1);
-            if (named_bar_or(2, 64, !okk)) return false;
+            if (named_bar_or(BAR_O, 64, !okk)) return false;
             tc_fence_after();
             const long long tok = bos + (long long)C * ci + (t - 64);
-            const uint32_t d1 = tmem + lane_base + (ci & 1) * DVT;
+            float o[DVT];
+            tmem_row((ci & 1) * DVT, o);
+            if (tok < eos) {
+                uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)tok * H + h) * D + n0);
 #pragma unroll
-            for (int c16 = 0; c16 < DVT / 16; ++c16) {
-                float o[16];
-                tmem_ld16(d1 + c16 * 16, o);
-                tmem_wait_ld();
-                if (tok < eos) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)tok * H + h) * D + n0 + c16 * 16);
-                    dst[0] = make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]),
-                                        pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
-                    dst[1] = make_uint4(pack_bf16(o[8], o[9]), pack_bf16(o[10], o[11]),
-                                        pack_bf16(o[12], o[13]), pack_bf16(o[14], o[15]));
-                }
+                for (int e = 0; e < DVT / 8; ++e)
+                    dst[e] = make_uint4(pack_bf16(o[8 * e], o[8 * e + 1]), pack_bf16(o[8 * e + 2], o[8 * e + 3]),
+                                        pack_bf16(o[8 * e + 4], o[8 * e + 5]), pack_bf16(o[8 * e + 6], o[8 * e + 7]));
             }
-            tc_fence_before();
             return true;
         };
-        for (int i = 0; i < nchunks && !failed; ++i) {
+        write_B1();
+        tc_fence_before();
+        bool failed = false, ok = true;
+        for (int i = 0; i < nchunks; ++i) {
             const int s = i % NS;
             const int p = i & 1;
-            unsigned char *st = sm + (size_t)s * L::STAGE;
-            const uint32_t st_a = smem_u32(st);
-            const uint32_t d1 = tmem + p * DVT;          // this chunk's [W;Qg] S accumulator
-            const uint32_t d3 = tmem + 2 * DVT;          // Kt^T V_new accumulator
-            bool ok = true;
-            if (t == 0) {
-                ok = mbar_wait(&full[s], (i / NS) & 1);
-                if (ok) {
-                    tc_fence_after();
-                    const uint32_t a_lo = a_sw.lo + ((st_a - sm_a) >> 4);
+            const unsigned char *st = sm + (size_t)s * L::STAGE;
+            if (named_bar_or(BAR_S, NSYNC, !ok)) { failed = true; break; }
+            // this chunk's stage has landed (the issuer saw it before the barrier);
+            // U and e^{G_C} are read straight from it
+            ok = mbar_wait(&full[s], (i / NS) & 1);
+            const float eg = reinterpret_cast<const float *>(st + L::EGC_OFF)[t];
+            uint32_t u[DVT / 2];
+            if (t < 64) {
+                // column (n0 % 32) + c of the loaded U tile(s), row t
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16_p(d1, a_lo + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), a_sw.hi,
-                                    b1_d.lo + ((kk * 256) >> 4), b1_d.hi, IDESC, kk > 0);
-                    umma_commit(mma1);
+                for (int c = 0; c < DVT; c += 8) {
+                    const int lc = (n0 & 31) + c;
+                    const uint4 x = *reinterpret_cast<const uint4 *>(st + L::U_OFF + (lc >> 5) * 4096 + t * 64 + (lc & 31) * 2);
+                    u[c / 2] = x.x; u[c / 2 + 1] = x.y; u[c / 2 + 2] = x.z; u[c / 2 + 3] = x.w;
                 }
             }
-            // while MMA1 runs: the previous chunk's output leaves through warps 2-3
-            if (t >= 64 && i > 0 && !emit_output(i - 1)) ok = false;
-            if (t == 0 && ok) ok = mbar_wait(mma1, i & 1);
-            if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+            if (ok) ok = mbar_wait(mma1, i & 1);
             tc_fence_after();
-            const float eg = reinterpret_cast<const float *>(st + L::EGC_OFF)[t];
+            // the previous chunk's output leaves through warps 2-3
+            if (t >= 64 && i > 0 && !emit_output(i - 1)) ok = false;
             if (t < 64) {
                 // V_new = U - W S for token row t
+                float x[DVT];
+                tmem_row(p * DVT, x);
 #pragma unroll
-                for (int c16 = 0; c16 < DVT / 16; ++c16) {
-                    float x[16];
-                    tmem_ld16(tmem + lane_base + p * DVT + c16 * 16, x);
-                    tmem_wait_ld();
-                    // column (n0 % 32) + 16 c16 of the loaded U tile(s), row t
-                    const int lc = (n0 & 31) + c16 * 16;
-                    const unsigned char *up = st + L::U_OFF + (lc >> 5) * 4096 + t * 64 + (lc & 31) * 2;
-                    uint32_t pk[8];
+                for (int ng = 0; ng < DVT / 8; ++ng) {
+                    uint32_t pk[4];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const __nv_bfloat162 u2 = reinterpret_cast<const __nv_bfloat162 *>(up)[e];
-                        pk[e] = pack_bf16(__low2float(u2) - x[2 * e], __high2float(u2) - x[2 * e + 1]);
+                    for (int e = 0; e < 4; ++e) {
+                        const __nv_bfloat162 u2 = *reinterpret_cast<const __nv_bfloat162 *>(&u[4 * ng + e]);
+                        pk[e] = pack_bf16(__low2float(u2) - x[8 * ng + 2 * e], __high2float(u2) - x[8 * ng + 2 * e + 1]);
                     }
-                    *reinterpret_cast<uint4 *>(B2 + mn_off(t, 2 * c16, L::B2_SBO)) =
-                        make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    *reinterpret_cast<uint4 *>(B2 + mn_off(t, 2 * c16 + 1, L::B2_SBO)) =
-                        make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    *reinterpret_cast<uint4 *>(B2 + mn_off(t, ng, L::B2_SBO)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
+                fence_proxy_async_smem();
             }
-            fence_proxy_async_smem();
             tc_fence_before();
-            named_bar(1, 128);
-            tc_fence_after();
-            ok = true;
-            if (t == 0) {
-                // the state update (MMA3) is on the critical path: issue it first
-                const uint32_t a_lo = a_sw.lo + ((st_a - sm_a) >> 4);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_bf16_p(d3, a_lo + (((uint32_t)ws::OFF_KTT + kk * 32) >> 4), a_sw.hi,
-                                b2_d.lo + ((kk * 256) >> 4), b2_d.hi, IDESC, kk > 0);
-                umma_commit(mma3);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_bf16_p(d1, a_lo + (((uint32_t)ws::OFF_P - 8192 + kk * 32) >> 4), a_sw.hi,
-                                b2_d.lo + ((kk * 256) >> 4), b2_d.hi, IDESC, 1);
-                umma_commit(mma2);
-                umma_commit(&empty[s]);
-                ok = mbar_wait(mma3, i & 1);
-            }
-            if (named_bar_or(1, 128, !ok)) { failed = true; break; }
+            if (named_bar_or(BAR_V, NSYNC, !ok)) { failed = true; break; }
+            ok = mbar_wait(mma3, i & 1);
             tc_fence_after();
             // S <- Diag(e^{G_C}) S + Kt^T V_new   (channel row t)
+            {
+                float z[DVT];
+                tmem_row(2 * DVT, z);
 #pragma unroll
-            for (int c16 = 0; c16 < DVT / 16; ++c16) {
-                float z[16];
-                tmem_ld16(tmem + lane_base + 2 * DVT + c16 * 16, z);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) S[c16 * 16 + e] = eg * S[c16 * 16 + e] + z[e];
+                for (int e = 0; e < DVT; ++e) S[e] = eg * S[e] + z[e];
             }
             write_B1();
-            fence_proxy_async_smem();
             tc_fence_before();
-            named_bar(1, 128);
-            tc_fence_after();
         }
+        if (!failed && !ok) failed = true;
         if (!failed && nchunks > 0 && t >= 64 && !emit_output(nchunks - 1)) failed = true;
         if (failed) {
-            if (t == 0) { set_device_error(err, kErrWaitTimeout); *abort_flag = 1; }
+            set_device_error(err, kErrWaitTimeout);
+            *abort_flag = 1;
         } else if (sT) {
             const size_t sb = (((size_t)seq * H + h) * D + t) * D + n0;
 #pragma unroll

@@ -207,16 +207,19 @@ chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     const size_t base = ((size_t)t0 * H + h) * D;         // element offset of (t0, h, 0)
 
     // ---- stage q, k, v (zero-filled past the end) ----
-    for (int i = tid; i < 3 * C * (D / 8); i += NT) {
-        const int which = i / (C * (D / 8));
-        const int rem = i - which * (C * (D / 8));
-        const int r = rem >> 4, j = rem & 15;
-        const __nv_bfloat16 *src = which == 0 ? q : which == 1 ? k : v;
-        unsigned char *dst = which == 0 ? sm.Xq : which == 1 ? sm.Kb : sm.Vb;
-        const bool ok = r < len;
-        const __nv_bfloat16 *gp = ok ? src + base + (size_t)r * row_stride + j * 8 : src;
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(dst + toff_chunk(r, j))),
-                     "l"(gp), "r"(ok ? 16 : 0));
+    {
+        const uint32_t xq = smem_u32(sm.Xq), kb = smem_u32(sm.Kb), vb = smem_u32(sm.Vb);
+#pragma unroll
+        for (int it = 0; it < C * (D / 8) / NT; ++it) {
+            const int i = tid + it * NT;
+            const int r = i >> 4, j = i & 15;
+            const bool ok = r < len;
+            const size_t off = ok ? base + (size_t)r * row_stride + j * 8 : 0;
+            const uint32_t so = toff_chunk(r, j), n = ok ? 16 : 0;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(xq + so), "l"(q + off), "r"(n));
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(kb + so), "l"(k + off), "r"(n));
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(vb + so), "l"(v + off), "r"(n));
+        }
     }
     cp_async_commit();
 

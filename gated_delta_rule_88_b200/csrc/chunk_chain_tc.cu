@@ -37,7 +37,7 @@ using namespace sm100;
 
 constexpr int C = ws::C;
 constexpr int D = ws::D;
-constexpr int NTHREADS = 192;
+constexpr int NTHREADS = 224;
 constexpr uint32_t REC_HEAD = 57344;       // [W;Qg] + Kt^T + P, contiguous in the record
 
 template <int DVT, int NS>
@@ -48,9 +48,10 @@ struct TcLayout {
     static constexpr uint32_t STAGE = ((EGC_OFF + 512 + 1023) / 1024) * 1024;
     static constexpr uint32_t TX = REC_HEAD + UT * 4096 + 512;
     static constexpr uint32_t B1_OFF = NS * STAGE;                 // S^bf16: K=128 x N=DVT
-    static constexpr uint32_t B2_OFF = B1_OFF + 128 * DVT * 2;     // V_new: K=64 x N=DVT
-    static constexpr uint32_t BAR_OFF = B2_OFF + 64 * DVT * 2;
-    static constexpr uint32_t BYTES = BAR_OFF + 8 * (2 * NS + 4) + 16;
+    static constexpr uint32_t B2_OFF = B1_OFF + 128 * DVT * 2;     // V_new: K=64 x N=DVT, two buffers
+    static constexpr uint32_t B2_BYTES = 64 * DVT * 2;
+    static constexpr uint32_t BAR_OFF = B2_OFF + 2 * B2_BYTES;
+    static constexpr uint32_t BYTES = BAR_OFF + 8 * (2 * NS + 7) + 16;
     // TMEM columns: D1 double-buffered (2 x DVT) + D3 (DVT), rounded to a power of 2
     static constexpr uint32_t NCOLS = 3 * DVT <= 32 ? 32 : 3 * DVT <= 64 ? 64 : 3 * DVT <= 128 ? 128 : 256;
     static constexpr uint32_t B1_SBO = (128 / 8) * 128;             // n-group stride
@@ -79,8 +80,9 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
     uint64_t *mma1 = empty + NS;
     uint64_t *mma3 = mma1 + 1;
     uint64_t *mma2 = mma1 + 2;
-    uint64_t *drain = mma1 + 3;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma1 + 4);
+    uint64_t *drain = mma1 + 3;                        // [2]: one per issuer
+    uint64_t *s_go = mma1 + 5;                         // [2]: MMA3(i) issued, by i & 1
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma1 + 7);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     unsigned char *B1 = sm + L::B1_OFF;
     unsigned char *B2 = sm + L::B2_OFF;
@@ -109,11 +111,12 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
     const size_t rec_stride = (size_t)H * ws::RECORD;
 
     if (tid == 0) {
-        for (int s = 0; s < NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        // a stage is free once both issuers' MMAs on it are done
+        for (int s = 0; s < NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 2); }
         mbar_init(mma1, 1);
         mbar_init(mma3, 1);
         mbar_init(mma2, 1);
-        mbar_init(drain, 1);
+        for (int b = 0; b < 2; ++b) { mbar_init(&drain[b], 1); mbar_init(&s_go[b], 1); }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -150,17 +153,19 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
             for (int j = max(0, issued - NS); j < issued; ++j)
                 mbar_wait(&full[j % NS], (j / NS) & 1, 1u << 20);
         }
-    } else if (warp == 5) {
-        // ---------------- MMA issuer (lane 0; the warp joins the barriers) ----------------
+    } else if (warp == 5 || warp == 6) {
+        // ---------------- MMA issuers: warp 5 lane 0 the chain (MMA1, MMA3; the
+        // warp joins the barriers), warp 6 lane 0 the output product (MMA2) ----------------
         constexpr uint32_t IDESC = idesc_bf16(128, DVT, true);
         // A operands: K-major, 128-byte swizzle, 8-row groups 1024 B apart, relative
         // to the ring base; B operands: MN-major interleaved, K groups 128 B apart
         const uint32_t sm_a = smem_u32(sm);
         const DescParts a_sw = smem_desc_parts(sm_a, 16, 1024, 2);
         const DescParts b1_d = smem_desc_parts(smem_u32(B1), 128, L::B1_SBO, 0);
-        const DescParts b2_d = smem_desc_parts(smem_u32(B2), 128, L::B2_SBO, 0);
+        const DescParts b2_d0 = smem_desc_parts(smem_u32(B2), 128, L::B2_SBO, 0);
+        const DescParts b2_d1 = smem_desc_parts(smem_u32(B2 + L::B2_BYTES), 128, L::B2_SBO, 0);
         bool issued_any = false;
-        for (int i = 0; i < nchunks; ++i) {
+        if (warp == 5) for (int i = 0; i < nchunks; ++i) {
             const int s = i % NS;
             const int p = i & 1;
             const uint32_t a_lo = a_sw.lo + ((uint32_t)s * L::STAGE >> 4);
@@ -179,28 +184,50 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
                 issued_any = true;
             }
             __syncwarp();
-            if (named_bar_or(BAR_V, NSYNC, false)) break;      // V_new is in B2
+            if (named_bar_or(BAR_V, NSYNC, false)) break;      // V_new is in B2[p]
             tc_fence_after();
             if (lane == 0) {
-                // the state update (MMA3) is on the critical path: issue it first
+                // the state update (MMA3) is the sequential path; the output
+                // product (MMA2) goes to the second issuer
+                const uint32_t b2_lo = p ? b2_d1.lo : b2_d0.lo;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     umma_bf16_p(tmem + 2 * DVT, a_lo + (((uint32_t)ws::OFF_KTT + kk * 32) >> 4),
-                                a_sw.hi, b2_d.lo + ((kk * 256) >> 4), b2_d.hi, IDESC, kk > 0);
+                                a_sw.hi, b2_lo + ((kk * 256) >> 4), b2_d0.hi, IDESC, kk > 0);
                 umma_commit(mma3);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_bf16_p(tmem + p * DVT, a_lo + (((uint32_t)ws::OFF_P - 8192 + kk * 32) >> 4),
-                                a_sw.hi, b2_d.lo + ((kk * 256) >> 4), b2_d.hi, IDESC, 1);
-                umma_commit(mma2);
                 umma_commit(&empty[s]);
+                mbar_arrive(&s_go[p]);
             }
             __syncwarp();
         }
+        if (warp == 6 && lane == 0) for (int i = 0; i < nchunks; ++i) {
+            // MMA2: O rows (64-127 of D1[p]) += P V_new, once MMA3(i) is issued.
+            // s_go[p] cannot run two phases ahead: MMA3(i + 2) needs the
+            // epilogue past emit(i), which waits for this MMA2.
+            const int s = i % NS;
+            const int p = i & 1;
+            bool ok = false;
+            for (uint32_t it = 0; it < (1u << 24); ++it) {
+                if (mbar_test_wait(&s_go[p], (i >> 1) & 1)) { ok = true; break; }
+                if (*abort_flag) break;
+                if (it > 64) __nanosleep(32);
+            }
+            if (!ok) { set_device_error(err, kErrWaitTimeout); break; }
+            tc_fence_after();
+            const uint32_t a_lo = a_sw.lo + ((uint32_t)s * L::STAGE >> 4);
+            const uint32_t b2_lo = p ? b2_d1.lo : b2_d0.lo;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                umma_bf16_p(tmem + p * DVT, a_lo + (((uint32_t)ws::OFF_P - 8192 + kk * 32) >> 4),
+                            a_sw.hi, b2_lo + ((kk * 256) >> 4), b2_d0.hi, IDESC, 1);
+            umma_commit(mma2);
+            umma_commit(&empty[s]);
+            issued_any = true;
+        }
         // never free TMEM under a running MMA
         if (lane == 0 && issued_any) {
-            umma_commit(drain);
-            mbar_wait(drain, 0, 1u << 20);
+            umma_commit(&drain[warp - 5]);
+            mbar_wait(&drain[warp - 5], 0, 1u << 20);
         }
     } else {
         // ---------------- epilogue warps 0-3: thread t <-> TMEM lane t ----------------
@@ -292,7 +319,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
                         const __nv_bfloat162 u2 = *reinterpret_cast<const __nv_bfloat162 *>(&u[4 * ng + e]);
                         pk[e] = pack_bf16(__low2float(u2) - x[8 * ng + 2 * e], __high2float(u2) - x[8 * ng + 2 * e + 1]);
                     }
-                    *reinterpret_cast<uint4 *>(B2 + mn_off(t, ng, L::B2_SBO)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4 *>(B2 + p * L::B2_BYTES + mn_off(t, ng, L::B2_SBO)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
                 fence_proxy_async_smem();
             }

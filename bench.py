@@ -52,7 +52,7 @@ FALLBACK_HBM_GBS = 6650.0
 _SRC = os.path.join(ROOT, "gated_delta_rule_88_b200", "csrc")
 TRAFFIC = {
     "prefill": {"files": ["chunk_prep.cu", "chunk_chain_tc.cu", "chunk_ws.h", "sm100.cuh", "common.cuh"],
-                "sha": "93f597dd29195e1a", "bytes": (342.131712 + 264.254464 + 304.178176 + 52.943872) * 1e6},
+                "sha": "7a31f985d99e3ace", "bytes": (342.313984 + 264.840448 + 304.188416 + 55.321856) * 1e6},
     "decode": {"files": ["decode.cu", "common.cuh"], "sha": "5538ff5eaafbaa61",
                "bytes": (547.416576 + 479.912448) * 1e6},
 }

@@ -9,7 +9,9 @@ prefill tokens/s (tokens of the packed T axis, all heads) with inputs resident
 in HBM; the inputs (404 MB) are larger than the 126 MB L2, so no flush is
 needed between steps.  A second leg times the decode step on
 "decode_n256_h32_d128" (256 sequences x 32 heads, fp32 state 512 MiB in
-place) and is reported under "decode".
+place) and is reported under "decode"; a third times serving decode
+(kda_recurrent_steps: 8 tokens per sequence per call, states in a 512-entry
+pool picked by slot) under "decode_steps".
 
 Under torchrun (N > 1) every rank runs the same workload on its own GPU
 (independent replicas: the hot path has no exchange step), timing is the max
@@ -236,6 +238,7 @@ def run_ours(args):
     # ---- decode leg (its timed region is sampled for clocks too) ----
     with ClockSampler(local) as clk_dec:
         dec = decode_leg(kda, W, dev, dist, world, args)
+        dec_steps = decode_steps_leg(kda, W, dev, dist, world, args)
     clk.samples += clk_dec.samples
     clk.reasons |= clk_dec.reasons
 
@@ -259,6 +262,7 @@ def run_ours(args):
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
         "decode": dec,
+        "decode_steps": dec_steps,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(inp_cpu)
@@ -298,6 +302,47 @@ def decode_leg(kda, W, dev, dist, world, args):
                          "peak": peak, "unit": "GB/s", "frac": ach / peak, "peak_source": kind,
                          "algorithmic_bytes_per_launch": DECODE_BYTES,
                          "traffic": measured_traffic("decode")}}
+
+
+STEPS_L, STEPS_POOL = 8, 2 * DEC_N
+STEPS_BYTES = DEC_N * DEC_H * (2 * D * D * 4 + STEPS_L * (3 * D * 2 + D * 4 + 4 + D * 2)) + DEC_N * 4
+
+
+def decode_steps_leg(kda, W, dev, dist, world, args):
+    """Serving decode: 8 tokens per sequence per call (kda_recurrent_steps) for
+    the 256 x 32 decode batch, states in a pool of 512 entries picked by a
+    seeded slot permutation."""
+    pool = torch.empty(STEPS_POOL, DEC_H, D, D, dtype=torch.float32, device=dev)
+    pool.copy_(W.decode_initial_state(STEPS_POOL, DEC_H, D, D))
+    gen = torch.Generator().manual_seed(31)
+    slots = torch.randperm(STEPS_POOL, generator=gen)[:DEC_N].to(torch.int32).to(dev)
+    ring = 2
+    toks = []
+    for r in range(ring):
+        steps_r = [W.decode_tokens(r * STEPS_L + l) for l in range(STEPS_L)]
+        toks.append(tuple(torch.stack([st[i] for st in steps_r], dim=1).contiguous().to(dev)
+                          for i in range(5)))
+    out = torch.empty(DEC_N, STEPS_L, DEC_H, D, dtype=torch.bfloat16, device=dev)
+    calls = max(16, args.decode_steps // 16)
+    for i in range(max(3, args.warmup)):
+        kda.kda_recurrent_steps(*toks[i % ring], pool, slots, out=out)
+    barrier(dist)
+    s = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for i in range(calls):
+        kda.kda_recurrent_steps(*toks[i % ring], pool, slots, out=out)
+    e1.record(s)
+    barrier(dist)
+    ms = max_over_ranks(e0.elapsed_time(e1), dist) / calls
+    peak, kind = measured_peak_hbm()
+    ach = STEPS_BYTES / (ms * 1e-3) / 1e9
+    return {"workload": f"decode_steps_n{DEC_N}_l{STEPS_L}_h{DEC_H}_d{D}_pool{STEPS_POOL}",
+            "value": world * DEC_N * STEPS_L / (ms * 1e-3), "unit": UNIT, "ms_per_call": ms,
+            "calls": calls, "l2": "pool (1 GiB) larger than L2; no flush",
+            "roofline": {"bound": "hbm", "kernel": "decode_steps_kernel", "achieved": ach,
+                         "peak": peak, "unit": "GB/s", "frac": ach / peak, "peak_source": kind,
+                         "algorithmic_bytes_per_launch": STEPS_BYTES, "traffic": None}}
 
 
 def cpu_baseline(inp_cpu, tokens=None):

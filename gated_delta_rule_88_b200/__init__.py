@@ -10,6 +10,7 @@ Entry points (same names as the C ABI):
                   out=None, final_state=None, output_final_state=True)
         -> (out, final_state or None)
     kda_recurrent_step(q, k, v, g, beta, state, out=None) -> out
+    kda_recurrent_steps(q, k, v, g, beta, state_pool, slots=None, out=None) -> out
     kda_get_device_error(stream=None) -> int
 """
 from __future__ import annotations
@@ -20,7 +21,7 @@ import threading
 
 import torch
 
-__all__ = ["kda_chunk_fwd", "kda_recurrent_step", "kda_get_device_error", "KDAError",
+__all__ = ["kda_chunk_fwd", "kda_recurrent_step", "kda_recurrent_steps", "kda_get_device_error", "KDAError",
            "library_path", "load_library"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -55,6 +56,8 @@ def load_library():
         lib.kda_chunk_fwd.restype = i
         lib.kda_recurrent_step.argtypes = [vp] * 7 + [i] * 5 + [vp]
         lib.kda_recurrent_step.restype = i
+        lib.kda_recurrent_steps.argtypes = [vp] * 7 + [i] + [vp] + [i] * 6 + [vp]
+        lib.kda_recurrent_steps.restype = i
         lib.kda_get_device_error.argtypes = [vp, ctypes.POINTER(i)]
         lib.kda_get_device_error.restype = i
         lib.kda_last_error_message.restype = ctypes.c_char_p
@@ -167,6 +170,42 @@ def kda_recurrent_step(q, k, v, g, beta, state, out=None):
         rc = lib.kda_recurrent_step(_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta),
                                     _dptr(state), _dptr(out), N, H, dk, dv, _dtype_code(q),
                                     _stream_handle(dev))
+    _check(rc)
+    return out
+
+
+def kda_recurrent_steps(q, k, v, g, beta, state_pool, slots=None, out=None):
+    """L decode tokens per sequence on a slot-indexed state pool.  q,k,g
+    [N,L,H,dk]; v [N,L,H,dv]; beta [N,L,H]; state_pool [S,H,dk,dv] fp32,
+    entry slots[n] updated in place (slots: int32 [N] or None for n).
+    Returns out [N,L,H,dv]."""
+    lib = load_library()
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("kda_recurrent_steps needs CUDA tensors (no CPU path)")
+    dt = q.dtype
+    N, L, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dev, dt)
+    _need(g, "g", dev, torch.float32)
+    _need(beta, "beta", dev, torch.float32)
+    _need(state_pool, "state_pool", dev, torch.float32)
+    if state_pool.dim() != 4 or tuple(state_pool.shape[1:]) != (H, dk, dv):
+        raise ValueError(f"state_pool must be [S,{H},{dk},{dv}]")
+    if slots is not None:
+        _need(slots, "slots", dev, torch.int32)
+        if tuple(slots.shape) != (N,):
+            raise ValueError(f"slots must be [{N}]")
+    if out is None:
+        out = torch.empty(N, L, H, dv, dtype=dt, device=dev)
+    else:
+        _need(out, "out", dev, dt)
+    with torch.cuda.device(dev):
+        rc = lib.kda_recurrent_steps(_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta),
+                                     _dptr(state_pool), _dptr(slots), state_pool.shape[0],
+                                     _dptr(out), N, L, H, dk, dv, _dtype_code(q),
+                                     _stream_handle(dev))
     _check(rc)
     return out
 

@@ -148,6 +148,42 @@ kda_status kda_recurrent_step(const void *q, const void *k, const void *v, const
     return KDA_OK;
 }
 
+kda_status kda_recurrent_steps(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, float *state_pool, const int32_t *slots,
+                               int num_slots, void *out, int N, int L, int H, int dk, int dv,
+                               kda_dtype dtype, void *stream) {
+    t_msg[0] = 0;
+    if (!q || !k || !v || !g || !beta || !state_pool || !out)
+        return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_steps: null pointer argument");
+    if (N < 0 || L <= 0 || H <= 0 || dk <= 0 || dv <= 0 || num_slots <= 0)
+        return fail(KDA_ERR_INVALID_ARG,
+                    "kda_recurrent_steps: bad sizes N=%d L=%d H=%d dk=%d dv=%d num_slots=%d", N, L,
+                    H, dk, dv, num_slots);
+    if (!slots && num_slots < N)
+        return fail(KDA_ERR_INVALID_ARG,
+                    "kda_recurrent_steps: without slots the pool needs num_slots >= N (%d < %d)",
+                    num_slots, N);
+    if (dtype != KDA_F32 && dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_steps: unknown dtype %d", (int)dtype);
+    if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128)))
+        return fail(KDA_ERR_UNSUPPORTED, "kda_recurrent_steps: dk=%d dv=%d (supported: 64, 128)",
+                    dk, dv);
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) ||
+        !aligned16(state_pool) || !aligned16(out))
+        return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_steps: pointers must be 16-byte aligned");
+    if (((uintptr_t)beta & 3u) || ((uintptr_t)slots & 3u))
+        return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_steps: beta and slots must be 4-byte aligned");
+    const long long NH = (long long)N * H;
+    if (NH > 0x7fffffffLL || (long long)N * L * H > (1LL << 40))
+        return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_steps: problem too large");
+    if (NH == 0) return KDA_OK;
+    cudaError_t e = kda::launch_decode_steps(q, k, v, g, beta, state_pool, slots, num_slots, out,
+                                             N, H, L, dk, dv, dtype == KDA_BF16,
+                                             kda::error_word(), (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_steps launch");
+    return KDA_OK;
+}
+
 kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
                          const float *beta, const float *initial_state,
                          const int32_t *cu_seqlens, void *out, float *final_state, int B,

@@ -14,6 +14,7 @@ enum DeviceError : int {
     kErrNone = 0,
     kErrWaitTimeout = 1,     // an mbarrier wait exceeded its bound
     kErrBadOffsets = 2,      // cu_seqlens inconsistent (chunks beyond the records)
+    kErrBadSlot = 3,         // a state-slot index outside [0, num_slots)
 };
 
 __device__ __forceinline__ void set_device_error(int *word, int code) {

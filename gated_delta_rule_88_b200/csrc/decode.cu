@@ -105,6 +105,158 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     }
 }
 
+// L tokens per sequence against a state pool indexed by slot: the state is
+// read once, the L steps run on it in registers (the same per-token arithmetic
+// as decode_step_kernel), and it is written once.  Token l of sequence n is
+// row (n * L + l) of the token arrays; sequence n uses pool entry slots[n]
+// (n when slots is null).  A slot outside [0, num_slots) skips the sequence
+// and sets the device error word.
+template <int DK, int DV, typename Tin>
+__global__ void __launch_bounds__(256, 2)
+decode_steps_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
+                    const Tin *__restrict__ v, const float *__restrict__ g,
+                    const float *__restrict__ beta, float *__restrict__ pool,
+                    const int32_t *__restrict__ slots, int num_slots, Tin *__restrict__ out,
+                    int H, int L, int *__restrict__ err)
+{
+    constexpr int NT = 256;
+    constexpr int C4 = DV / 4;
+    constexpr int RG = NT / C4;
+    constexpr int RPT = DK / RG;
+    static_assert(NT % C4 == 0 && DK % RG == 0, "bad decode tiling");
+
+    const int n = blockIdx.x / H, h = blockIdx.x - n * H;
+    const int tid = threadIdx.x;
+    const int c4 = tid % C4;
+    const int rg = tid / C4;
+    const int slot = slots ? slots[n] : n;
+    if (slot < 0 || slot >= num_slots) {
+        if (tid == 0) set_device_error(err, kErrBadSlot);
+        return;
+    }
+
+    __shared__ float ks[DK], qs[DK], as_[DK];
+    __shared__ __align__(16) float red_k[RG][DV + 4];
+    __shared__ __align__(16) float red_q[RG][DV + 4];
+    __shared__ __align__(16) float us[DV];
+    __shared__ float qk_part[NT / 32];
+
+    float4 *Sp = reinterpret_cast<float4 *>(pool + ((size_t)slot * H + h) * (size_t)(DK * DV));
+    float4 s[RPT];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) s[r] = ld_stream(Sp + (size_t)(rg * RPT + r) * C4 + c4);
+
+    // token inputs of step l + 1 are loaded into registers while step l runs
+    float kn = 0.f, qn = 0.f, gn = 0.f, vn = 0.f, bn = 0.f;
+    auto load_token = [&](int l) {
+        const size_t row = ((size_t)n * L + l) * H + h;
+        if (tid < DK) {
+            kn = to_f(k[row * DK + tid]);
+            qn = to_f(q[row * DK + tid]);
+            gn = g[row * DK + tid];
+        }
+        if (tid < DV) {
+            vn = to_f(v[row * DV + tid]);
+            bn = beta[row];
+        }
+    };
+    load_token(0);
+    for (int l = 0; l < L; ++l) {
+        const size_t row = ((size_t)n * L + l) * H + h;
+        if (l > 0) __syncthreads();   // the previous step's readers of ks, us, qk_part
+        float qk = 0.f;
+        if (tid < DK) {
+            ks[tid] = kn;
+            qs[tid] = qn;
+            as_[tid] = expf(gn);
+            qk = kn * qn;
+        }
+        const float vcur = vn, bcur = bn;
+        if (l + 1 < L) load_token(l + 1);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, o);
+        if ((tid & 31) == 0) qk_part[tid >> 5] = qk;
+        __syncthreads();
+
+        float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            const int rr = rg * RPT + r;
+            const float a = as_[rr], kr = ks[rr], qr = qs[rr];
+            s[r].x *= a; s[r].y *= a; s[r].z *= a; s[r].w *= a;
+            pk[0] += kr * s[r].x; pk[1] += kr * s[r].y; pk[2] += kr * s[r].z; pk[3] += kr * s[r].w;
+            pq[0] += qr * s[r].x; pq[1] += qr * s[r].y; pq[2] += qr * s[r].z; pq[3] += qr * s[r].w;
+        }
+        reinterpret_cast<float4 *>(&red_k[rg][0])[c4] = make_float4(pk[0], pk[1], pk[2], pk[3]);
+        reinterpret_cast<float4 *>(&red_q[rg][0])[c4] = make_float4(pq[0], pq[1], pq[2], pq[3]);
+        __syncthreads();
+
+        if (tid < DV) {
+            float kS = 0.f, qS = 0.f;
+#pragma unroll
+            for (int i = 0; i < RG; ++i) { kS += red_k[i][tid]; qS += red_q[i][tid]; }
+            float qk_all = 0.f;
+#pragma unroll
+            for (int w = 0; w < NT / 32; ++w) qk_all += qk_part[w];
+            const float u = bcur * (vcur - kS);
+            us[tid] = u;
+            out[row * DV + tid] = from_f<Tin>(qS + qk_all * u);
+        }
+        __syncthreads();
+
+        const float4 u4 = reinterpret_cast<const float4 *>(us)[c4];
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            const float kr = ks[rg * RPT + r];
+            s[r].x += kr * u4.x; s[r].y += kr * u4.y; s[r].z += kr * u4.z; s[r].w += kr * u4.w;
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) st_stream(Sp + (size_t)(rg * RPT + r) * C4 + c4, s[r]);
+}
+
+template <int DK, int DV, typename Tin>
+static cudaError_t launch_steps_t(const void *q, const void *k, const void *v, const float *g,
+                                  const float *beta, float *pool, const int32_t *slots,
+                                  int num_slots, void *out, int N, int H, int L, int *err,
+                                  cudaStream_t st)
+{
+    decode_steps_kernel<DK, DV, Tin><<<N * H, 256, 0, st>>>(
+        (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, pool, slots, num_slots,
+        (Tin *)out, H, L, err);
+    return cudaGetLastError();
+}
+
+template <typename Tin>
+static cudaError_t launch_steps_d(const void *q, const void *k, const void *v, const float *g,
+                                  const float *beta, float *pool, const int32_t *slots,
+                                  int num_slots, void *out, int N, int H, int L, int dk, int dv,
+                                  int *err, cudaStream_t st)
+{
+#define KDA_STEPS(DK_, DV_)                                                                    \
+    if (dk == DK_ && dv == DV_)                                                                \
+        return launch_steps_t<DK_, DV_, Tin>(q, k, v, g, beta, pool, slots, num_slots, out, N, \
+                                             H, L, err, st);
+    KDA_STEPS(128, 128)
+    KDA_STEPS(64, 64)
+    KDA_STEPS(128, 64)
+    KDA_STEPS(64, 128)
+#undef KDA_STEPS
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_steps(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, float *pool, const int32_t *slots,
+                                int num_slots, void *out, int N, int H, int L, int dk, int dv,
+                                bool bf16, int *err, cudaStream_t st)
+{
+    if (bf16)
+        return launch_steps_d<__nv_bfloat16>(q, k, v, g, beta, pool, slots, num_slots, out, N, H,
+                                             L, dk, dv, err, st);
+    return launch_steps_d<float>(q, k, v, g, beta, pool, slots, num_slots, out, N, H, L, dk, dv,
+                                 err, st);
+}
+
 template <int DK, int DV, typename Tin>
 static cudaError_t launch_decode_t(const void *q, const void *k, const void *v,
                                    const float *g, const float *beta, float *state,

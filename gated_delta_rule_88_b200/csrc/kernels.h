@@ -14,6 +14,13 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const flo
                           const float *beta, float *state, void *out, int NH, int dk,
                           int dv, bool bf16, cudaStream_t st);
 
+// L decode tokens per sequence against a slot-indexed state pool
+// [num_slots, H, dk, dv]; sequence n uses pool entry slots[n] (n if null).
+cudaError_t launch_decode_steps(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, float *pool, const int32_t *slots,
+                                int num_slots, void *out, int N, int H, int L, int dk, int dv,
+                                bool bf16, int *err, cudaStream_t st);
+
 // Exact-fp32 chunked prefill (SIMT).  dk, dv in {64, 128}.
 // Token axis flattened: token t of the packed [B*T] axis, head h, channel c at
 // ((t * H) + h) * d + c.  Sequences: dense (cu == nullptr, n-th spans

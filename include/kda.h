@@ -15,12 +15,14 @@
  *                       through the chunk's transitions plus the intra-chunk
  *                       writes, via a WY-like W,U representation);
  *   kda_recurrent_step  decode: one token per sequence, the fused recurrent
- *                       form the same section names for short queries.
+ *                       form the same section names for short queries;
+ *   kda_recurrent_steps decode for serving: up to L tokens per sequence
+ *                       (short queries) on a slot-indexed state pool.
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers (cudaMalloc'd or any memory the
- *     device can address), contiguous, row-major, 16-byte aligned (beta and
- *     cu_seqlens: 4-byte aligned).  The
+ *     device can address), contiguous, row-major, 16-byte aligned (beta,
+ *     cu_seqlens and slots: 4-byte aligned).  The
  *     caller allocates and owns every buffer; the library keeps no pointer
  *     after a call returns.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
@@ -119,6 +121,38 @@ kda_status kda_recurrent_step(const void *q, const void *k, const void *v,
                               float *state_inout, void *out,
                               int N, int H, int dk, int dv,
                               kda_dtype dtype, void *stream);
+
+/*
+ * kda_recurrent_steps -- L decode tokens for each of N sequences whose states
+ * live in a slot-indexed pool (continuous batching).
+ *
+ * Source: Kimi Linear paper notes (paper-notes-site), section 2 (recurrence)
+ * and section 3 (queries of at most 64 tokens outside training take the
+ * fused recurrent mode, which keeps only the recurrent state); section 7
+ * (the serving-side wrapper owns the state's dtype and shape).  The slot
+ * array itself is a serving layout with no counterpart in the pages.
+ *
+ * Layout: q, k [N, L, H, dk] dtype; v [N, L, H, dv] dtype; g [N, L, H, dk]
+ *   float32; beta [N, L, H] float32; out [N, L, H, dv] dtype;
+ *   state_pool [num_slots, H, dk, dv] float32; slots: device int32 [N] or
+ *   NULL (sequence n uses pool entry n, which needs num_slots >= N).
+ * Computes, for each sequence n and head, the L steps of kda_recurrent_step
+ *   in order on pool entry slots[n], reading the state once and writing it
+ *   once (L tokens cost one state read and one write, not L of each).
+ * Errors: a slot outside [0, num_slots) skips that sequence (its pool entry
+ *   and outputs are not written) and sets the device error word, reported by
+ *   kda_get_device_error with code 3.  Slots must be distinct: two sequences
+ *   naming one entry race.  L >= 1 (the paper's mode switch is at 64 tokens;
+ *   longer inputs belong to kda_chunk_fwd, but any L is computed correctly).
+ * Supported: dk, dv in {64, 128}, dtype KDA_BF16 or KDA_F32.  Any finite g.
+ * Aliasing: out must not overlap any input; the pool must not overlap the
+ *   token inputs.
+ */
+kda_status kda_recurrent_steps(const void *q, const void *k, const void *v,
+                               const float *g, const float *beta,
+                               float *state_pool, const int32_t *slots, int num_slots,
+                               void *out, int N, int L, int H, int dk, int dv,
+                               kda_dtype dtype, void *stream);
 
 /*
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate

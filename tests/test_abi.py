@@ -35,7 +35,7 @@ def declared_functions():
 
 def test_header_declares_entry_points():
     names = declared_functions()
-    for n in ("kda_chunk_fwd", "kda_recurrent_step", "kda_status_string",
+    for n in ("kda_chunk_fwd", "kda_recurrent_step", "kda_recurrent_steps", "kda_status_string",
               "kda_get_device_error", "kda_last_error_message", "kda_version"):
         assert n in names
 
@@ -108,6 +108,35 @@ def test_step_unsupported_rejected(lib, kw):
 
 def test_step_empty_batch_is_a_no_op(lib):
     assert step(lib, N=0) == 0
+
+
+def steps(lib, *, q=FAKE, k=FAKE, v=FAKE, g=FAKE, b=FAKE, pool=FAKE, slots=None, S=4, out=FAKE,
+          N=1, L=2, H=1, dk=128, dv=128, dtype=1):
+    P = ctypes.c_void_p
+    return lib.kda_recurrent_steps(P(q), P(k), P(v), P(g), P(b), P(pool), P(slots), S, P(out),
+                                   N, L, H, dk, dv, dtype, None)
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "g", "b", "pool", "out"])
+def test_steps_null_pointer_rejected(lib, field):
+    assert steps(lib, **{field: 0}) == 1
+
+
+@pytest.mark.parametrize("kw", [dict(N=-1), dict(L=0), dict(H=0), dict(S=0), dict(N=5, S=4),
+                                dict(dtype=3), dict(pool=FAKE + 8), dict(b=FAKE + 1),
+                                dict(slots=FAKE + 2), dict(N=1 << 20, H=1 << 12)])
+def test_steps_bad_arguments_rejected(lib, kw):
+    assert steps(lib, **kw) == 1
+
+
+def test_steps_slots_allow_a_pool_smaller_than_the_batch(lib):
+    # with a slot array the pool size is independent of N (checked on device)
+    assert steps(lib, N=0, S=1, slots=FAKE) == 0
+
+
+@pytest.mark.parametrize("kw", [dict(dk=32), dict(dv=96)])
+def test_steps_unsupported_rejected(lib, kw):
+    assert steps(lib, **kw) == 2
 
 
 def test_python_binding_refuses_cpu_tensors():

@@ -11,6 +11,9 @@ Entry points (same names as the C ABI):
         -> (out, final_state or None)
     kda_recurrent_step(q, k, v, g, beta, state, out=None) -> out
     kda_recurrent_steps(q, k, v, g, beta, state_pool, slots=None, out=None) -> out
+    kda_chunk_fwd_host(q, k, v, g, beta, initial_state=None, out=None,
+                       final_state=None, output_final_state=True, range_tokens=0)
+        -> (out, final_state or None)   (CPU tensors; valid after the stream syncs)
     kda_get_device_error(stream=None) -> int
 """
 from __future__ import annotations
@@ -21,7 +24,8 @@ import threading
 
 import torch
 
-__all__ = ["kda_chunk_fwd", "kda_recurrent_step", "kda_recurrent_steps", "kda_get_device_error", "KDAError",
+__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_host", "kda_recurrent_step", "kda_recurrent_steps",
+           "kda_get_device_error", "KDAError",
            "library_path", "load_library"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -58,6 +62,8 @@ def load_library():
         lib.kda_recurrent_step.restype = i
         lib.kda_recurrent_steps.argtypes = [vp] * 7 + [i] + [vp] + [i] * 6 + [vp]
         lib.kda_recurrent_steps.restype = i
+        lib.kda_chunk_fwd_host.argtypes = [vp] * 8 + [i] * 7 + [vp]
+        lib.kda_chunk_fwd_host.restype = i
         lib.kda_get_device_error.argtypes = [vp, ctypes.POINTER(i)]
         lib.kda_get_device_error.restype = i
         lib.kda_last_error_message.restype = ctypes.c_char_p
@@ -141,6 +147,41 @@ def kda_chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, out=Non
                                _dptr(initial_state), _dptr(cu_seqlens), _dptr(out),
                                _dptr(final_state), B, T, H, dk, dv, N, _dtype_code(q),
                                _stream_handle(dev))
+    _check(rc)
+    return out, final_state
+
+
+def kda_chunk_fwd_host(q, k, v, g, beta, initial_state=None, out=None, final_state=None,
+                       output_final_state: bool = True, range_tokens: int = 0, device=None):
+    """kda_chunk_fwd on host (CPU) tensors, dense [B,T,H,*] layouts; the copies
+    are pipelined against the computation on ``device`` (default: the current
+    CUDA device).  Pinned tensors overlap; results are valid once the current
+    stream of that device has synchronised.  Returns (out, final_state)."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    cpu = torch.device("cpu")
+    dt = q.dtype
+    if q.dim() != 4:
+        raise ValueError("q must be [B,T,H,dk]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, cpu, dt)
+    _need(g, "g", cpu, torch.float32)
+    _need(beta, "beta", cpu, torch.float32)
+    if initial_state is not None:
+        _need(initial_state, "initial_state", cpu, torch.float32)
+    if out is None:
+        out = torch.empty(B, T, H, dv, dtype=dt, pin_memory=True)
+    else:
+        _need(out, "out", cpu, dt)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(B, H, dk, dv, dtype=torch.float32, pin_memory=True)
+    with torch.cuda.device(dev):
+        rc = lib.kda_chunk_fwd_host(_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta),
+                                    _dptr(initial_state), _dptr(out), _dptr(final_state),
+                                    B, T, H, dk, dv, _dtype_code(q), int(range_tokens),
+                                    _stream_handle(dev))
     _check(rc)
     return out, final_state
 

@@ -3,6 +3,8 @@
 // launches; nothing here touches tensor data on the host.
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include <mutex>
 
@@ -86,6 +88,12 @@ cudaError_t get_pool(cudaMemPool_t *out, int *sm_count) {
 }
 
 }  // namespace
+
+static kda_status chunk_fwd_device(const void *q, const void *k, const void *v, const float *g,
+                                   const float *beta, const float *initial_state,
+                                   const int32_t *cu_seqlens, void *out, float *final_state,
+                                   int B, int T, int H, int dk, int dv, int N, kda_dtype dtype,
+                                   cudaStream_t st);
 
 extern "C" {
 
@@ -217,8 +225,19 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const floa
     const long long total_T = (long long)B * T;
     if (total_T > 0x7fffffffLL || total_T * H > (1LL << 40))
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: problem too large (B*T=%lld)", total_T);
-    cudaStream_t st = (cudaStream_t)stream;
+    return chunk_fwd_device(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state, B, T,
+                            H, dk, dv, N, dtype, (cudaStream_t)stream);
+}
 
+}  // extern "C"
+
+// Device-side part of kda_chunk_fwd (arguments already validated).
+static kda_status chunk_fwd_device(const void *q, const void *k, const void *v, const float *g,
+                                   const float *beta, const float *initial_state,
+                                   const int32_t *cu_seqlens, void *out, float *final_state,
+                                   int B, int T, int H, int dk, int dv, int N, kda_dtype dtype,
+                                   cudaStream_t st) {
+    const long long total_T = (long long)B * T;
     if (dtype == KDA_F32) {
         if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128)))
             return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd(f32): dk=%d dv=%d (supported: 64, 128)",
@@ -271,4 +290,178 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const floa
     return KDA_OK;
 }
 
-}  // extern "C"
+// ---------------------------------------------------------------------------
+// kda_chunk_fwd_host: host buffers, pipelined over token ranges.
+namespace {
+
+struct HostPipeStreams {
+    cudaStream_t in = nullptr, out = nullptr;
+};
+std::mutex g_pipe_mu;
+HostPipeStreams g_pipe[64];
+
+cudaError_t pipe_streams(HostPipeStreams **ps) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_pipe_mu);
+    HostPipeStreams &p = g_pipe[dev];
+    if (!p.in && (e = cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if (!p.out && (e = cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    *ps = &p;
+    return cudaSuccess;
+}
+
+// rows [t0, t0 + n) of every batch: B strided blocks of n * row bytes
+cudaError_t copy_rows(void *dst, size_t dpitch, const void *src, size_t spitch, size_t width,
+                      int B, cudaStream_t st) {
+    return cudaMemcpy2DAsync(dst, dpitch, src, spitch, width, (size_t)B, cudaMemcpyDefault, st);
+}
+
+}  // namespace
+
+extern "C" kda_status kda_chunk_fwd_host(const void *q, const void *k, const void *v,
+                                         const float *g, const float *beta,
+                                         const float *initial_state, void *out,
+                                         float *final_state, int B, int T, int H, int dk, int dv,
+                                         kda_dtype dtype, int range_tokens, void *stream) {
+    t_msg[0] = 0;
+    if (!q || !k || !v || !g || !beta || !out)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: null pointer argument");
+    if (B <= 0 || B > 65535 || T < 0 || H <= 0 || H > 65535 || dk <= 0 || dv <= 0 ||
+        range_tokens < 0)
+        return fail(KDA_ERR_INVALID_ARG,
+                    "kda_chunk_fwd_host: bad sizes B=%d T=%d H=%d dk=%d dv=%d range_tokens=%d", B,
+                    T, H, dk, dv, range_tokens);
+    if (dtype != KDA_F32 && dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: unknown dtype %d", (int)dtype);
+    if (dtype == KDA_BF16 ? (dk != 128 || dv != 128)
+                          : !((dk == 64 || dk == 128) && (dv == 64 || dv == 128)))
+        return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd_host: dk=%d dv=%d not supported for %s",
+                    dk, dv, dtype == KDA_BF16 ? "bf16" : "f32");
+    const long long total_T = (long long)B * T;
+    if (total_T > 0x7fffffffLL || total_T * H > (1LL << 40))
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: problem too large (B*T=%lld)", total_T);
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t es = dtype == KDA_BF16 ? 2 : 4;
+    const size_t state_bytes = (size_t)B * H * dk * dv * sizeof(float);
+    if (T == 0) {   // nothing to process: final = initial (or zeros)
+        if (!final_state) return KDA_OK;
+        cudaError_t e = initial_state
+            ? cudaMemcpyAsync(final_state, initial_state, state_bytes, cudaMemcpyDefault, st)
+            : cudaMemsetAsync(final_state, 0, state_bytes, st);
+        if (e != cudaSuccess) {   // host memory cannot be memset by the device: zero it here
+            if (initial_state) return cuda_fail(e, "kda_chunk_fwd_host empty input");
+            cudaGetLastError();
+            if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_host");
+            memset(final_state, 0, state_bytes);
+        }
+        return KDA_OK;
+    }
+    // ranges of whole chunks, so the chunk grid is that of one call over T
+    int R = range_tokens > 0 ? range_tokens : 2048;
+    R = (R + 63) / 64 * 64;
+    if (R > T) R = (T + 63) / 64 * 64;
+    const int nr = (T + R - 1) / R;
+    // per-token row bytes of each input / output (all heads)
+    const size_t rq = (size_t)H * dk * es, rv = (size_t)H * dv * es, rg = (size_t)H * dk * 4,
+                 rb = (size_t)H * 4, ro = (size_t)H * dv * es;
+    const size_t in_bytes = (size_t)B * R * (2 * rq + rv + rg + rb);
+    const size_t out_bytes = (size_t)B * R * ro;
+    auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    // layout of one stage buffer: q k v g beta, each [B, R, H, *]
+    const size_t oq = 0, ok_ = al((size_t)B * R * rq), ov = ok_ + al((size_t)B * R * rq),
+                 og = ov + al((size_t)B * R * rv), ob = og + al((size_t)B * R * rg);
+    const size_t in_stage = ob + al((size_t)B * R * rb);
+    const size_t total = 2 * in_stage + 2 * al(out_bytes) + al(state_bytes);
+    (void)in_bytes;
+
+    HostPipeStreams *ps = nullptr;
+    cudaMemPool_t pool;
+    int sms = 148;
+    cudaError_t e = pipe_streams(&ps);
+    if (e == cudaSuccess) e = get_pool(&pool, &sms);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_host setup");
+    void *buf = nullptr;
+    if ((e = cudaMallocFromPoolAsync(&buf, total, pool, st)) != cudaSuccess)
+        return cuda_fail(e, "kda_chunk_fwd_host device buffers");
+    unsigned char *in_dev[2] = {(unsigned char *)buf, (unsigned char *)buf + in_stage};
+    unsigned char *out_dev[2] = {in_dev[1] + in_stage, in_dev[1] + in_stage + al(out_bytes)};
+    float *state_dev = (float *)(out_dev[1] + al(out_bytes));
+
+    // events: start (buffers allocated, caller's prior work done), and per range
+    // in_ready[r], done[r] (inputs of stage r % 2 free again), out_free[r]
+    const int ne = 1 + 3 * nr;
+    cudaEvent_t *ev = (cudaEvent_t *)calloc((size_t)ne, sizeof(cudaEvent_t));
+    if (!ev) { cudaFreeAsync(buf, st); return fail(KDA_ERR_CUDA, "kda_chunk_fwd_host: out of host memory"); }
+    int made = 0;
+    for (; made < ne; ++made)
+        if ((e = cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming)) != cudaSuccess) break;
+    kda_status status = KDA_OK;
+    if (e != cudaSuccess) status = cuda_fail(e, "kda_chunk_fwd_host events");
+    cudaEvent_t ev_start = ev[0];
+    auto in_ready = [&](int r) { return ev[1 + 3 * r]; };
+    auto done = [&](int r) { return ev[2 + 3 * r]; };
+    auto out_free = [&](int r) { return ev[3 + 3 * r]; };
+    auto chk = [&](cudaError_t x, const char *what) {
+        if (status == KDA_OK && x != cudaSuccess) status = cuda_fail(x, what);
+    };
+
+    if (status == KDA_OK) {
+        chk(cudaEventRecord(ev_start, st), "kda_chunk_fwd_host record");
+        chk(cudaStreamWaitEvent(ps->in, ev_start, 0), "kda_chunk_fwd_host wait");
+        chk(cudaStreamWaitEvent(ps->out, ev_start, 0), "kda_chunk_fwd_host wait");
+        if (initial_state)
+            chk(cudaMemcpyAsync(state_dev, initial_state, state_bytes, cudaMemcpyDefault, st),
+                "kda_chunk_fwd_host initial state");
+    }
+    for (int r = 0; r < nr && status == KDA_OK; ++r) {
+        const int t0 = r * R, tr = T - t0 < R ? T - t0 : R;
+        const int b = r & 1;
+        unsigned char *in = in_dev[b];
+        // copy in (the stage's previous user, range r - 2, must be done)
+        if (r >= 2) chk(cudaStreamWaitEvent(ps->in, done(r - 2), 0), "kda_chunk_fwd_host wait");
+        const struct { const void *h; size_t off, row; } srcs[5] = {
+            {q, oq, rq}, {k, ok_, rq}, {v, ov, rv}, {g, og, rg}, {beta, ob, rb}};
+        for (const auto &c : srcs)
+            chk(copy_rows(in + c.off, (size_t)tr * c.row, (const unsigned char *)c.h + (size_t)t0 * c.row,
+                          (size_t)T * c.row, (size_t)tr * c.row, B, ps->in),
+                "kda_chunk_fwd_host copy in");
+        chk(cudaEventRecord(in_ready(r), ps->in), "kda_chunk_fwd_host record");
+        // compute on the caller's stream: state in, state out, in place
+        chk(cudaStreamWaitEvent(st, in_ready(r), 0), "kda_chunk_fwd_host wait");
+        if (r >= 2) chk(cudaStreamWaitEvent(st, out_free(r - 2), 0), "kda_chunk_fwd_host wait");
+        if (status != KDA_OK) break;
+        kda_status s2 = chunk_fwd_device(in + oq, in + ok_, in + ov, (const float *)(in + og),
+                                         (const float *)(in + ob),
+                                         (r == 0 && !initial_state) ? nullptr : state_dev, nullptr,
+                                         out_dev[b], state_dev, B, tr, H, dk, dv, B, dtype, st);
+        if (s2 != KDA_OK) { status = s2; break; }
+        chk(cudaEventRecord(done(r), st), "kda_chunk_fwd_host record");
+        // copy out
+        chk(cudaStreamWaitEvent(ps->out, done(r), 0), "kda_chunk_fwd_host wait");
+        chk(copy_rows((unsigned char *)out + (size_t)t0 * ro, (size_t)T * ro, out_dev[b],
+                      (size_t)tr * ro, (size_t)tr * ro, B, ps->out),
+            "kda_chunk_fwd_host copy out");
+        chk(cudaEventRecord(out_free(r), ps->out), "kda_chunk_fwd_host record");
+    }
+    if (status == KDA_OK && final_state)
+        chk(cudaMemcpyAsync(final_state, state_dev, state_bytes, cudaMemcpyDefault, st),
+            "kda_chunk_fwd_host final state");
+    // the caller's stream ends after every copy; buffers are released on it
+    if (made == ne) {
+        for (int r = 0; r < nr; ++r) {
+            cudaStreamWaitEvent(st, in_ready(r), 0);
+            cudaStreamWaitEvent(st, out_free(r), 0);
+        }
+    } else {
+        cudaStreamSynchronize(ps->in);
+        cudaStreamSynchronize(ps->out);
+    }
+    cudaError_t ef = cudaFreeAsync(buf, st);
+    for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);
+    free(ev);
+    if (status == KDA_OK && ef != cudaSuccess) status = cuda_fail(ef, "kda_chunk_fwd_host release");
+    return status;
+}

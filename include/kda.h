@@ -17,7 +17,9 @@
  *   kda_recurrent_step  decode: one token per sequence, the fused recurrent
  *                       form the same section names for short queries;
  *   kda_recurrent_steps decode for serving: up to L tokens per sequence
- *                       (short queries) on a slot-indexed state pool.
+ *                       (short queries) on a slot-indexed state pool;
+ *   kda_chunk_fwd_host  kda_chunk_fwd on host buffers, copies pipelined
+ *                       against the computation.
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers (cudaMalloc'd or any memory the
@@ -99,6 +101,40 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v,
                          void *out, float *final_state,
                          int B, int T, int H, int dk, int dv, int num_seqs,
                          kda_dtype dtype, void *stream);
+
+/*
+ * kda_chunk_fwd_host -- kda_chunk_fwd (dense mode) on HOST buffers, with the
+ * host<->device copies pipelined against the computation.
+ *
+ * Source: as kda_chunk_fwd; the pipelining rests on the checkpoint semantics
+ * (whoami-wesleyyou blog, "context modification and checkpoint": a state
+ * summarises its prefix exactly) -- the sequence is processed in ranges of
+ * whole chunks, each range resuming from the fp32 state the previous one
+ * left on the device, so the chunk grid, and the result, are those of one
+ * kda_chunk_fwd call over the whole sequence.  The pages have no host-buffer
+ * entry point; this is a deployment variant.
+ *
+ * Pointers: q, k, v, g, beta, initial_state (nullable), out, final_state
+ *   (nullable) are HOST pointers with kda_chunk_fwd's dense layouts
+ *   ([B, T, H, *]).  Page-locked (pinned) memory lets the copies overlap the
+ *   computation; pageable memory works, with copies that do not overlap.
+ * range_tokens: tokens per pipeline stage, rounded up to a multiple of 64;
+ *   0 selects 2048 (measured best for 32 heads x d = 128 over PCIe).
+ * Streams: the computation runs on `stream`; the copies run on two streams
+ *   the library keeps per device, ordered after the work already queued on
+ *   `stream`, and `stream` is ordered after them, so the outputs are in host
+ *   memory once `stream` has completed (e.g. cudaStreamSynchronize).
+ * Memory: device buffers for two input stages, two output stages and the
+ *   state come from the library-private pool (stream-ordered, as in
+ *   kda_chunk_fwd) and are released on `stream`.
+ * Supported: as kda_chunk_fwd in dense mode (no cu_seqlens).
+ * Aliasing: out and final_state must not overlap any input.
+ */
+kda_status kda_chunk_fwd_host(const void *q, const void *k, const void *v,
+                              const float *g, const float *beta,
+                              const float *initial_state, void *out, float *final_state,
+                              int B, int T, int H, int dk, int dv,
+                              kda_dtype dtype, int range_tokens, void *stream);
 
 /*
  * kda_recurrent_step -- one decode token for each of N sequences.

@@ -35,7 +35,8 @@ def declared_functions():
 
 def test_header_declares_entry_points():
     names = declared_functions()
-    for n in ("kda_chunk_fwd", "kda_recurrent_step", "kda_recurrent_steps", "kda_status_string",
+    for n in ("kda_chunk_fwd", "kda_chunk_fwd_host", "kda_recurrent_step", "kda_recurrent_steps",
+              "kda_status_string",
               "kda_get_device_error", "kda_last_error_message", "kda_version"):
         assert n in names
 
@@ -137,6 +138,29 @@ def test_steps_slots_allow_a_pool_smaller_than_the_batch(lib):
 @pytest.mark.parametrize("kw", [dict(dk=32), dict(dv=96)])
 def test_steps_unsupported_rejected(lib, kw):
     assert steps(lib, **kw) == 2
+
+
+def host(lib, *, q=FAKE, k=FAKE, v=FAKE, g=FAKE, b=FAKE, s0=None, out=FAKE, sT=None, B=1, T=64,
+         H=1, dk=128, dv=128, dtype=1, rt=0):
+    P = ctypes.c_void_p
+    return lib.kda_chunk_fwd_host(P(q), P(k), P(v), P(g), P(b), P(s0), P(out), P(sT), B, T, H,
+                                  dk, dv, dtype, rt, None)
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "g", "b", "out"])
+def test_host_null_pointer_rejected(lib, field):
+    assert host(lib, **{field: 0}) == 1
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(T=-1), dict(H=0), dict(rt=-64), dict(dtype=9),
+                                dict(B=70000), dict(T=1 << 30, B=4)])
+def test_host_bad_arguments_rejected(lib, kw):
+    assert host(lib, **kw) == 1
+
+
+@pytest.mark.parametrize("kw", [dict(dk=64, dv=64), dict(dtype=0, dk=32, dv=64)])
+def test_host_unsupported_rejected(lib, kw):
+    assert host(lib, **kw) == 2
 
 
 def test_python_binding_refuses_cpu_tensors():

@@ -163,10 +163,16 @@ def dist_setup(n_gpus):
     return 0, 1, 0, None
 
 
+def _coll_device(dist):
+    # NCCL reduces device tensors; gloo (the CPU tests of this plumbing) host ones
+    return "cuda" if dist.get_backend() == "nccl" else "cpu"
+
+
 def max_over_ranks(x: float, dist) -> float:
+    """Max of a per-rank figure (device time) over all ranks."""
     if dist is None:
         return x
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    t = torch.tensor([x], device=_coll_device(dist), dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -174,7 +180,14 @@ def max_over_ranks(x: float, dist) -> float:
 def barrier(dist):
     if dist is not None:
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available() and torch.cuda.is_initialized():
+        torch.cuda.synchronize()
+
+
+def job_value(units_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job throughput: every rank processes the same units (replicas), in
+    ms, the max over ranks of the device time."""
+    return world * units_per_rank / (ms * 1e-3)
 
 
 def run_ours(args):
@@ -207,7 +220,7 @@ def run_ours(args):
     ms = max_over_ranks(ms_local, dist)
     ms_step = ms / args.steps
     assert kda.kda_get_device_error() == 0
-    value = world * B * T / (ms_step * 1e-3)
+    value = job_value(B * T, world, ms_step)
     peak, peak_kind = measured_peak_hbm()
     achieved = PREFILL_BYTES / (ms_step * 1e-3) / 1e9
 
@@ -256,7 +269,7 @@ def run_ours(args):
                      "frac": achieved / peak, "peak_source": peak_kind,
                      "algorithmic_bytes_per_launch": PREFILL_BYTES,
                      "traffic": measured_traffic("prefill")},
-        "e2e": {"value": world * B * T / (e2e_ms * 1e-3), "unit": UNIT,
+        "e2e": {"value": job_value(B * T, world, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "gpu_launches": 2 * args.steps,
@@ -295,7 +308,7 @@ def decode_leg(kda, W, dev, dist, world, args):
     ms = max_over_ranks(e0.elapsed_time(e1), dist) / steps
     peak, kind = measured_peak_hbm()
     ach = DECODE_BYTES / (ms * 1e-3) / 1e9
-    return {"workload": "decode_n256_h32_d128", "value": world * DEC_N / (ms * 1e-3),
+    return {"workload": "decode_n256_h32_d128", "value": job_value(DEC_N, world, ms),
             "unit": UNIT, "ms_per_step": ms, "steps": steps,
             "l2": "state (512 MiB) larger than L2; no flush",
             "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": ach,
@@ -338,7 +351,7 @@ def decode_steps_leg(kda, W, dev, dist, world, args):
     peak, kind = measured_peak_hbm()
     ach = STEPS_BYTES / (ms * 1e-3) / 1e9
     return {"workload": f"decode_steps_n{DEC_N}_l{STEPS_L}_h{DEC_H}_d{D}_pool{STEPS_POOL}",
-            "value": world * DEC_N * STEPS_L / (ms * 1e-3), "unit": UNIT, "ms_per_call": ms,
+            "value": job_value(DEC_N * STEPS_L, world, ms), "unit": UNIT, "ms_per_call": ms,
             "calls": calls, "l2": "pool (1 GiB) larger than L2; no flush",
             "roofline": {"bound": "hbm", "kernel": "decode_steps_kernel", "achieved": ach,
                          "peak": peak, "unit": "GB/s", "frac": ach / peak, "peak_source": kind,

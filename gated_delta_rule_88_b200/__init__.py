@@ -10,7 +10,11 @@ Entry points (same names as the C ABI):
                   out=None, final_state=None, output_final_state=True)
         -> (out, final_state or None)
     kda_recurrent_step(q, k, v, g, beta, state, out=None) -> out
-    kda_recurrent_steps(q, k, v, g, beta, state_pool, slots=None, out=None) -> out
+    kda_recurrent_steps(q, k, v, g, beta, state_pool, slots=None, out=None,
+                        flags=0, q_scale=1.0) -> out
+    kda_chunk_fwd_ex(..., flags=0, q_scale=1.0), kda_recurrent_step_ex(..., flags=0,
+                     q_scale=1.0): with the in-kernel input prologue
+                     (KDA_QK_L2NORM, KDA_BETA_SIGMOID)
     kda_chunk_fwd_host(q, k, v, g, beta, initial_state=None, out=None,
                        final_state=None, output_final_state=True, range_tokens=0)
         -> (out, final_state or None)   (CPU tensors; valid after the stream syncs)
@@ -24,8 +28,9 @@ import threading
 
 import torch
 
-__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_host", "kda_recurrent_step", "kda_recurrent_steps",
-           "kda_get_device_error", "KDAError",
+__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_ex", "kda_chunk_fwd_host", "kda_recurrent_step",
+           "kda_recurrent_step_ex", "kda_recurrent_steps", "kda_get_device_error", "KDAError",
+           "KDA_QK_L2NORM", "KDA_BETA_SIGMOID",
            "library_path", "load_library"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -34,6 +39,7 @@ _lib = None
 _lock = threading.Lock()
 
 KDA_F32, KDA_BF16 = 0, 1
+KDA_QK_L2NORM, KDA_BETA_SIGMOID = 1, 2     # input prologue flags (the *_ex calls)
 _STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
            3: "KDA_ERR_CUDA", 4: "KDA_ERR_DEVICE"}
 
@@ -58,9 +64,14 @@ def load_library():
         vp, i = ctypes.c_void_p, ctypes.c_int
         lib.kda_chunk_fwd.argtypes = [vp] * 9 + [i] * 7 + [vp]
         lib.kda_chunk_fwd.restype = i
+        lib.kda_chunk_fwd_ex.argtypes = [vp] * 9 + [i] * 7 + [ctypes.c_uint, ctypes.c_float, vp]
+        lib.kda_chunk_fwd_ex.restype = i
+        lib.kda_recurrent_step_ex.argtypes = [vp] * 7 + [i] * 5 + [ctypes.c_uint, ctypes.c_float, vp]
+        lib.kda_recurrent_step_ex.restype = i
         lib.kda_recurrent_step.argtypes = [vp] * 7 + [i] * 5 + [vp]
         lib.kda_recurrent_step.restype = i
-        lib.kda_recurrent_steps.argtypes = [vp] * 7 + [i] + [vp] + [i] * 6 + [vp]
+        lib.kda_recurrent_steps.argtypes = ([vp] * 7 + [i] + [vp] + [i] * 6 +
+                                            [ctypes.c_uint, ctypes.c_float, vp])
         lib.kda_recurrent_steps.restype = i
         lib.kda_chunk_fwd_host.argtypes = [vp] * 8 + [i] * 7 + [vp]
         lib.kda_chunk_fwd_host.restype = i
@@ -111,6 +122,22 @@ def kda_chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, out=Non
                   final_state=None, output_final_state: bool = True):
     """Chunkwise KDA prefill.  q,k,g [B,T,H,dk]; v [B,T,H,dv]; beta [B,T,H];
     states [N,H,dk,dv] fp32 (N = B, or len(cu_seqlens)-1 in varlen mode)."""
+    return _chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state,
+                      output_final_state, None)
+
+
+def kda_chunk_fwd_ex(q, k, v, g, beta, initial_state=None, cu_seqlens=None, out=None,
+                     final_state=None, output_final_state: bool = True, flags: int = 0,
+                     q_scale: float = 1.0):
+    """kda_chunk_fwd with the in-kernel input prologue: flags KDA_QK_L2NORM
+    (q, k L2-normalised per token and head), KDA_BETA_SIGMOID (beta given as a
+    logit); q is then scaled by q_scale."""
+    return _chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state,
+                      output_final_state, (int(flags), float(q_scale)))
+
+
+def _chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state,
+               output_final_state, pro):
     lib = load_library()
     dev = q.device
     if dev.type != "cuda":
@@ -142,11 +169,13 @@ def kda_chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, out=Non
         final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
     elif final_state is not None:
         _need(final_state, "final_state", dev, torch.float32)
+    args = (_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta), _dptr(initial_state),
+            _dptr(cu_seqlens), _dptr(out), _dptr(final_state), B, T, H, dk, dv, N, _dtype_code(q))
     with torch.cuda.device(dev):
-        rc = lib.kda_chunk_fwd(_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta),
-                               _dptr(initial_state), _dptr(cu_seqlens), _dptr(out),
-                               _dptr(final_state), B, T, H, dk, dv, N, _dtype_code(q),
-                               _stream_handle(dev))
+        if pro is None:
+            rc = lib.kda_chunk_fwd(*args, _stream_handle(dev))
+        else:
+            rc = lib.kda_chunk_fwd_ex(*args, pro[0], pro[1], _stream_handle(dev))
     _check(rc)
     return out, final_state
 
@@ -189,6 +218,15 @@ def kda_chunk_fwd_host(q, k, v, g, beta, initial_state=None, out=None, final_sta
 def kda_recurrent_step(q, k, v, g, beta, state, out=None):
     """One decode token per sequence.  q,k,g [N,H,dk]; v [N,H,dv]; beta [N,H];
     state [N,H,dk,dv] fp32 updated in place.  Returns out [N,H,dv]."""
+    return _recurrent_step(q, k, v, g, beta, state, out, None)
+
+
+def kda_recurrent_step_ex(q, k, v, g, beta, state, out=None, flags: int = 0, q_scale: float = 1.0):
+    """kda_recurrent_step with the in-kernel input prologue (see kda_chunk_fwd_ex)."""
+    return _recurrent_step(q, k, v, g, beta, state, out, (int(flags), float(q_scale)))
+
+
+def _recurrent_step(q, k, v, g, beta, state, out, pro):
     lib = load_library()
     dev = q.device
     if dev.type != "cuda":
@@ -207,15 +245,19 @@ def kda_recurrent_step(q, k, v, g, beta, state, out=None):
         out = torch.empty(N, H, dv, dtype=dt, device=dev)
     else:
         _need(out, "out", dev, dt)
+    args = (_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta), _dptr(state), _dptr(out), N, H,
+            dk, dv, _dtype_code(q))
     with torch.cuda.device(dev):
-        rc = lib.kda_recurrent_step(_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta),
-                                    _dptr(state), _dptr(out), N, H, dk, dv, _dtype_code(q),
-                                    _stream_handle(dev))
+        if pro is None:
+            rc = lib.kda_recurrent_step(*args, _stream_handle(dev))
+        else:
+            rc = lib.kda_recurrent_step_ex(*args, pro[0], pro[1], _stream_handle(dev))
     _check(rc)
     return out
 
 
-def kda_recurrent_steps(q, k, v, g, beta, state_pool, slots=None, out=None):
+def kda_recurrent_steps(q, k, v, g, beta, state_pool, slots=None, out=None, flags: int = 0,
+                        q_scale: float = 1.0):
     """L decode tokens per sequence on a slot-indexed state pool.  q,k,g
     [N,L,H,dk]; v [N,L,H,dv]; beta [N,L,H]; state_pool [S,H,dk,dv] fp32,
     entry slots[n] updated in place (slots: int32 [N] or None for n).
@@ -245,8 +287,8 @@ def kda_recurrent_steps(q, k, v, g, beta, state_pool, slots=None, out=None):
     with torch.cuda.device(dev):
         rc = lib.kda_recurrent_steps(_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta),
                                      _dptr(state_pool), _dptr(slots), state_pool.shape[0],
-                                     _dptr(out), N, L, H, dk, dv, _dtype_code(q),
-                                     _stream_handle(dev))
+                                     _dptr(out), N, L, H, dk, dv, _dtype_code(q), int(flags),
+                                     float(q_scale), _stream_handle(dev))
     _check(rc)
     return out
 

@@ -93,7 +93,20 @@ static kda_status chunk_fwd_device(const void *q, const void *k, const void *v, 
                                    const float *beta, const float *initial_state,
                                    const int32_t *cu_seqlens, void *out, float *final_state,
                                    int B, int T, int H, int dk, int dv, int N, kda_dtype dtype,
-                                   cudaStream_t st);
+                                   kda::Prologue pro, cudaStream_t st);
+
+// flags of the *_ex calls -> kernel prologue
+static kda_status make_prologue(const char *fn, unsigned flags, float q_scale,
+                                kda::Prologue *pro) {
+    if (flags & ~(unsigned)(KDA_QK_L2NORM | KDA_BETA_SIGMOID))
+        return fail(KDA_ERR_INVALID_ARG, "%s: unknown flag bits 0x%x", fn, flags);
+    if (!(q_scale == q_scale) || q_scale > 3.4e38f || q_scale < -3.4e38f)
+        return fail(KDA_ERR_INVALID_ARG, "%s: q_scale must be finite", fn);
+    pro->flags = (flags & KDA_QK_L2NORM ? kda::kProQkL2Norm : 0) |
+                 (flags & KDA_BETA_SIGMOID ? kda::kProBetaSigmoid : 0);
+    pro->q_scale = q_scale;
+    return KDA_OK;
+}
 
 extern "C" {
 
@@ -127,10 +140,10 @@ kda_status kda_get_device_error(void *stream, int *code_out) {
     return KDA_OK;
 }
 
-kda_status kda_recurrent_step(const void *q, const void *k, const void *v, const float *g,
-                              const float *beta, float *state_inout, void *out, int N,
-                              int H, int dk, int dv, kda_dtype dtype, void *stream) {
-    t_msg[0] = 0;
+static kda_status recurrent_step_impl(const void *q, const void *k, const void *v,
+                                      const float *g, const float *beta, float *state_inout,
+                                      void *out, int N, int H, int dk, int dv, kda_dtype dtype,
+                                      kda::Prologue pro, void *stream) {
     if (!q || !k || !v || !g || !beta || !state_inout || !out)
         return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_step: null pointer argument");
     if (N < 0 || H <= 0 || dk <= 0 || dv <= 0)
@@ -151,16 +164,39 @@ kda_status kda_recurrent_step(const void *q, const void *k, const void *v, const
         return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_step: N*H too large");
     if (NH == 0) return KDA_OK;
     cudaError_t e = kda::launch_decode(q, k, v, g, beta, state_inout, out, (int)NH, dk, dv,
-                                       dtype == KDA_BF16, (cudaStream_t)stream);
+                                       dtype == KDA_BF16, pro, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_step launch");
     return KDA_OK;
+}
+
+kda_status kda_recurrent_step(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, float *state_inout, void *out, int N,
+                              int H, int dk, int dv, kda_dtype dtype, void *stream) {
+    t_msg[0] = 0;
+    return recurrent_step_impl(q, k, v, g, beta, state_inout, out, N, H, dk, dv, dtype,
+                               kda::Prologue{0, 1.f}, stream);
+}
+
+kda_status kda_recurrent_step_ex(const void *q, const void *k, const void *v, const float *g,
+                                 const float *beta, float *state_inout, void *out, int N,
+                                 int H, int dk, int dv, kda_dtype dtype, unsigned flags,
+                                 float q_scale, void *stream) {
+    t_msg[0] = 0;
+    kda::Prologue pro;
+    kda_status st = make_prologue("kda_recurrent_step_ex", flags, q_scale, &pro);
+    if (st != KDA_OK) return st;
+    return recurrent_step_impl(q, k, v, g, beta, state_inout, out, N, H, dk, dv, dtype, pro,
+                               stream);
 }
 
 kda_status kda_recurrent_steps(const void *q, const void *k, const void *v, const float *g,
                                const float *beta, float *state_pool, const int32_t *slots,
                                int num_slots, void *out, int N, int L, int H, int dk, int dv,
-                               kda_dtype dtype, void *stream) {
+                               kda_dtype dtype, unsigned flags, float q_scale, void *stream) {
     t_msg[0] = 0;
+    kda::Prologue pro;
+    kda_status pst = make_prologue("kda_recurrent_steps", flags, q_scale, &pro);
+    if (pst != KDA_OK) return pst;
     if (!q || !k || !v || !g || !beta || !state_pool || !out)
         return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_steps: null pointer argument");
     if (N < 0 || L <= 0 || H <= 0 || dk <= 0 || dv <= 0 || num_slots <= 0)
@@ -187,17 +223,16 @@ kda_status kda_recurrent_steps(const void *q, const void *k, const void *v, cons
     if (NH == 0) return KDA_OK;
     cudaError_t e = kda::launch_decode_steps(q, k, v, g, beta, state_pool, slots, num_slots, out,
                                              N, H, L, dk, dv, dtype == KDA_BF16,
-                                             kda::error_word(), (cudaStream_t)stream);
+                                             kda::error_word(), pro, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_steps launch");
     return KDA_OK;
 }
 
-kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
-                         const float *beta, const float *initial_state,
-                         const int32_t *cu_seqlens, void *out, float *final_state, int B,
-                         int T, int H, int dk, int dv, int num_seqs, kda_dtype dtype,
-                         void *stream) {
-    t_msg[0] = 0;
+static kda_status chunk_fwd_impl(const void *q, const void *k, const void *v, const float *g,
+                                 const float *beta, const float *initial_state,
+                                 const int32_t *cu_seqlens, void *out, float *final_state,
+                                 int B, int T, int H, int dk, int dv, int num_seqs,
+                                 kda_dtype dtype, kda::Prologue pro, void *stream) {
     if (!q || !k || !v || !g || !beta || !out)
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: null pointer argument");
     if (B <= 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0)
@@ -226,7 +261,30 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const floa
     if (total_T > 0x7fffffffLL || total_T * H > (1LL << 40))
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: problem too large (B*T=%lld)", total_T);
     return chunk_fwd_device(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state, B, T,
-                            H, dk, dv, N, dtype, (cudaStream_t)stream);
+                            H, dk, dv, N, dtype, pro, (cudaStream_t)stream);
+}
+
+kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
+                         const float *beta, const float *initial_state,
+                         const int32_t *cu_seqlens, void *out, float *final_state, int B,
+                         int T, int H, int dk, int dv, int num_seqs, kda_dtype dtype,
+                         void *stream) {
+    t_msg[0] = 0;
+    return chunk_fwd_impl(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state, B, T,
+                          H, dk, dv, num_seqs, dtype, kda::Prologue{0, 1.f}, stream);
+}
+
+kda_status kda_chunk_fwd_ex(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, const float *initial_state,
+                            const int32_t *cu_seqlens, void *out, float *final_state, int B,
+                            int T, int H, int dk, int dv, int num_seqs, kda_dtype dtype,
+                            unsigned flags, float q_scale, void *stream) {
+    t_msg[0] = 0;
+    kda::Prologue pro;
+    kda_status st = make_prologue("kda_chunk_fwd_ex", flags, q_scale, &pro);
+    if (st != KDA_OK) return st;
+    return chunk_fwd_impl(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state, B, T,
+                          H, dk, dv, num_seqs, dtype, pro, stream);
 }
 
 }  // extern "C"
@@ -236,7 +294,7 @@ static kda_status chunk_fwd_device(const void *q, const void *k, const void *v, 
                                    const float *beta, const float *initial_state,
                                    const int32_t *cu_seqlens, void *out, float *final_state,
                                    int B, int T, int H, int dk, int dv, int N, kda_dtype dtype,
-                                   cudaStream_t st) {
+                                   kda::Prologue pro, cudaStream_t st) {
     const long long total_T = (long long)B * T;
     if (dtype == KDA_F32) {
         if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128)))
@@ -244,7 +302,7 @@ static kda_status chunk_fwd_device(const void *q, const void *k, const void *v, 
                         dk, dv);
         cudaError_t e = kda::launch_chunk_f32(
             (const float *)q, (const float *)k, (const float *)v, g, beta, initial_state,
-            cu_seqlens, (float *)out, final_state, N, T, (int)total_T, H, dk, dv, st);
+            cu_seqlens, (float *)out, final_state, N, T, (int)total_T, H, dk, dv, pro, st);
         if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd(f32) launch");
         return KDA_OK;
     }
@@ -280,7 +338,7 @@ static kda_status chunk_fwd_device(const void *q, const void *k, const void *v, 
     if (cu_seqlens) e = kda::launch_chunk_plan(cu_seqlens, N, (int)total_T, coff, st);
     if (e == cudaSuccess)
         e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, coff, N, T, (int)total_T, H,
-                                   (int)max_chunks, records, st);
+                                   (int)max_chunks, records, pro, st);
     if (e == cudaSuccess)
         e = kda::launch_chunk_chain(records, cu_seqlens, coff, initial_state, final_state, out, N,
                                     T, (int)total_T, H, dvt, (int)max_chunks, kda::error_word(), st);
@@ -436,7 +494,8 @@ extern "C" kda_status kda_chunk_fwd_host(const void *q, const void *k, const voi
         kda_status s2 = chunk_fwd_device(in + oq, in + ok_, in + ov, (const float *)(in + og),
                                          (const float *)(in + ob),
                                          (r == 0 && !initial_state) ? nullptr : state_dev, nullptr,
-                                         out_dev[b], state_dev, B, tr, H, dk, dv, B, dtype, st);
+                                         out_dev[b], state_dev, B, tr, H, dk, dv, B, dtype,
+                                         kda::Prologue{0, 1.f}, st);
         if (s2 != KDA_OK) { status = s2; break; }
         chk(cudaEventRecord(done(r), st), "kda_chunk_fwd_host record");
         // copy out

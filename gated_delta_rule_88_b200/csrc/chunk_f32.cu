@@ -56,7 +56,7 @@ chunk_f32_kernel(const float *__restrict__ q, const float *__restrict__ k,
                  const float *__restrict__ v, const float *__restrict__ g,
                  const float *__restrict__ beta, const float *__restrict__ s0,
                  const int32_t *__restrict__ cu, float *__restrict__ out,
-                 float *__restrict__ sT, int T, int total_T, int H, int dv)
+                 float *__restrict__ sT, int T, int total_T, int H, int dv, Prologue pro)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     F32Smem<DK> &sm = *reinterpret_cast<F32Smem<DK> *>(smem_raw);
@@ -102,8 +102,27 @@ chunk_f32_kernel(const float *__restrict__ q, const float *__restrict__ k,
             const int r = i / DVT, n = i % DVT;
             sm.Vs[i] = (r < len) ? v[((size_t)(t0 + r) * H + h) * dv + n0 + n] : 0.f;
         }
-        if (tid < CH) sm.bs[tid] = (tid < len) ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+        if (tid < CH) {
+            float bt = (tid < len) ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+            if ((pro.flags & kProBetaSigmoid) && tid < len) bt = sigmoid_f(bt);
+            sm.bs[tid] = bt;
+        }
         __syncthreads();
+        // ---- prologue: row factors of q (with q_scale) and k ----
+        if (pro.flags != 0 || pro.q_scale != 1.f) {
+            for (int rr = tid; rr < 2 * CH; rr += NT) {
+                float *row = rr < CH ? &sm.Qs[rr * LD] : &sm.Ks[(rr - CH) * LD];
+                float f = 1.f;
+                if (pro.flags & kProQkL2Norm) {
+                    float ss = 0.f;
+                    for (int c = 0; c < DK; ++c) ss = fmaf(row[c], row[c], ss);
+                    f = inv_norm(ss);
+                }
+                if (rr < CH) f *= pro.q_scale;
+                for (int c = 0; c < DK; ++c) row[c] *= f;
+            }
+            __syncthreads();
+        }
 
         // ---- G: chunk-local inclusive cumsum of g per channel ----
         if (tid < DK) {
@@ -215,7 +234,7 @@ template <int DK>
 cudaError_t launch_chunk_f32_t(const float *q, const float *k, const float *v, const float *g,
                                const float *beta, const float *s0, const int32_t *cu,
                                float *out, float *sT, int N, int T, int total_T, int H,
-                               int dv, cudaStream_t st)
+                               int dv, Prologue pro, cudaStream_t st)
 {
     const size_t smem = sizeof(F32Smem<DK>);
     cudaError_t e = cudaFuncSetAttribute(chunk_f32_kernel<DK>,
@@ -223,7 +242,7 @@ cudaError_t launch_chunk_f32_t(const float *q, const float *k, const float *v, c
     if (e != cudaSuccess) return e;
     dim3 grid(dv / DVT, H, N);
     chunk_f32_kernel<DK><<<grid, NT, smem, st>>>(q, k, v, g, beta, s0, cu, out, sT, T,
-                                                 total_T, H, dv);
+                                                 total_T, H, dv, pro);
     return cudaGetLastError();
 }
 
@@ -232,11 +251,11 @@ cudaError_t launch_chunk_f32_t(const float *q, const float *k, const float *v, c
 cudaError_t launch_chunk_f32(const float *q, const float *k, const float *v, const float *g,
                              const float *beta, const float *s0, const int32_t *cu,
                              float *out, float *sT, int N, int T, int total_T, int H,
-                             int dk, int dv, cudaStream_t st)
+                             int dk, int dv, Prologue pro, cudaStream_t st)
 {
     if (dv % DVT != 0) return cudaErrorInvalidValue;
-    if (dk == 64) return launch_chunk_f32_t<64>(q, k, v, g, beta, s0, cu, out, sT, N, T, total_T, H, dv, st);
-    if (dk == 128) return launch_chunk_f32_t<128>(q, k, v, g, beta, s0, cu, out, sT, N, T, total_T, H, dv, st);
+    if (dk == 64) return launch_chunk_f32_t<64>(q, k, v, g, beta, s0, cu, out, sT, N, T, total_T, H, dv, pro, st);
+    if (dk == 128) return launch_chunk_f32_t<128>(q, k, v, g, beta, s0, cu, out, sT, N, T, total_T, H, dv, pro, st);
     return cudaErrorInvalidValue;
 }
 

@@ -89,6 +89,7 @@ struct __align__(16) PrepSmem {
     float Dm[6][D];           // D_JI per channel
     float d[4][D];            // block totals
     float beta[C];
+    float rq[C], rk[C];       // prologue: per-row factors of q and k
 };
 
 __device__ __forceinline__ uint32_t scale_bf16x2(uint32_t x, float2 s) {
@@ -185,12 +186,13 @@ __device__ __forceinline__ void ap_block(PrepSmem &sm, unsigned char *rec, bool 
             }
 }
 
+template <bool PRO>
 __global__ void __launch_bounds__(NT, 2)
 chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                   const __nv_bfloat16 *__restrict__ v, const float *__restrict__ g,
                   const float *__restrict__ beta, const int32_t *__restrict__ cu,
                   const int32_t *__restrict__ coff, int N, int T, int total_T, int H, int cps,
-                  unsigned char *__restrict__ wsp)
+                  unsigned char *__restrict__ wsp, Prologue pro)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     PrepSmem &sm = *reinterpret_cast<PrepSmem *>(smem_raw);
@@ -244,9 +246,41 @@ chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     }
     sm.d[I][c0] = a[15].x;
     sm.d[I][c0 + 1] = a[15].y;
-    if (tid < C) sm.beta[tid] = (tid < len) ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+    if (tid < C) {
+        float bt = (tid < len) ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+        if (PRO && (pro.flags & kProBetaSigmoid) && tid < len) bt = sigmoid_f(bt);
+        sm.beta[tid] = bt;
+    }
     cp_async_wait<0>();
     __syncthreads();
+    if (PRO) {
+        // prologue: per-row factors (thread: tensor tid >> 7, row, half of the
+        // row); rows past the end are zero and get factor 0
+        const int tens = tid >> 7, rr = (tid >> 1) & 63, hf = tid & 1;
+        float f = 1.f;
+        if (pro.flags & kProQkL2Norm) {
+            const unsigned char *tile = tens ? sm.Kb : sm.Xq;
+            float ss = 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint4 x = *reinterpret_cast<const uint4 *>(tile + toff_chunk(rr, 8 * hf + j));
+                const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const __nv_bfloat162 p2 = *reinterpret_cast<const __nv_bfloat162 *>(&w[e]);
+                    const float a = __low2float(p2), b = __high2float(p2);
+                    ss = fmaf(a, a, fmaf(b, b, ss));
+                }
+            }
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            f = inv_norm(ss);
+        }
+        if (hf == 0) {
+            if (tens) sm.rk[rr] = f;
+            else sm.rq[rr] = f * pro.q_scale;
+        }
+        __syncthreads();
+    }
 
     float2 E = make_float2(1.f, 1.f), F = make_float2(1.f, 1.f);
     {
@@ -288,9 +322,13 @@ chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(sm.Xq + o);
             const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(sm.Kb + o);
             const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162 *>(sm.Vb + o);
-            const float qx = __low2float(q2), qy = __high2float(q2);
-            const float kx = __low2float(k2), ky = __high2float(k2);
+            float qx = __low2float(q2), qy = __high2float(q2);
+            float kx = __low2float(k2), ky = __high2float(k2);
             const float vx = __low2float(v2), vy = __high2float(v2);
+            if (PRO) {
+                const float fq = sm.rq[r], fk = sm.rk[r];
+                qx *= fq; qy *= fq; kx *= fk; ky *= fk;
+            }
             const float2 ai = a[i], bi = b[i];
             *reinterpret_cast<uint32_t *>(sm.Xq + o) = pack_bf16(qx * ai.x, qy * ai.y);
             *reinterpret_cast<uint32_t *>(sm.Xk + o) = pack_bf16(br * kx * ai.x, br * ky * ai.y);
@@ -487,17 +525,18 @@ cudaError_t launch_chunk_plan(const int32_t *cu, int N, int total_T, int32_t *co
 cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const int32_t *cu, const int32_t *coff,
                               int N, int T, int total_T, int H, int max_chunks,
-                              unsigned char *wsp, cudaStream_t st)
+                              unsigned char *wsp, Prologue pro, cudaStream_t st)
 {
     const size_t smem = sizeof(PrepSmem);
-    cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const bool use_pro = pro.flags != 0 || pro.q_scale != 1.f;
+    auto kern = use_pro ? chunk_prep_kernel<true> : chunk_prep_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int cps = (T + C - 1) / C;
     dim3 grid(max_chunks, H);
-    chunk_prep_kernel<<<grid, NT, smem, st>>>(
+    kern<<<grid, NT, smem, st>>>(
         (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, g, beta,
-        cu, coff, N, T, total_T, H, cps, wsp);
+        cu, coff, N, T, total_T, H, cps, wsp, pro);
     return cudaGetLastError();
 }
 

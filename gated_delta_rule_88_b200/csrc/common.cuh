@@ -17,6 +17,14 @@ enum DeviceError : int {
     kErrBadSlot = 3,         // a state-slot index outside [0, num_slots)
 };
 
+// Input prologue (struct Prologue, kernels.h): q <- q_scale * (QK_L2NORM ?
+// q / |q|_2 : q), k <- k / |k|_2 (QK_L2NORM; a zero row stays zero),
+// beta <- sigmoid(beta) (BETA_SIGMOID).
+constexpr int kProQkL2Norm = 1;
+constexpr int kProBetaSigmoid = 2;
+__device__ __forceinline__ float inv_norm(float sumsq) { return sumsq > 0.f ? rsqrtf(sumsq) : 0.f; }
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + expf(-x)); }
+
 __device__ __forceinline__ void set_device_error(int *word, int code) {
     if (word) atomicCAS(word, 0, code);
 }

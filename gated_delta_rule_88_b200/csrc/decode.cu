@@ -20,12 +20,12 @@
 
 namespace kda {
 
-template <int DK, int DV, typename Tin>
+template <int DK, int DV, typename Tin, bool PRO>
 __global__ void __launch_bounds__(256, 2)
 decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                    const Tin *__restrict__ v, const float *__restrict__ g,
                    const float *__restrict__ beta, float *__restrict__ state,
-                   Tin *__restrict__ out)
+                   Tin *__restrict__ out, Prologue pro)
 {
     constexpr int NT = 256;
     constexpr int C4 = DV / 4;       // float4 groups per row
@@ -42,7 +42,7 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     __shared__ __align__(16) float red_k[RG][DV + 4];
     __shared__ __align__(16) float red_q[RG][DV + 4];
     __shared__ __align__(16) float us[DV];
-    __shared__ float qk_part[NT / 32];
+    __shared__ float qk_part[NT / 32], kk_part[NT / 32], qq_part[NT / 32];
 
     // 1. Issue every state load first (64 KiB in flight per CTA at d=128).
     float4 *Sp = reinterpret_cast<float4 *>(state + nh * (size_t)(DK * DV));
@@ -51,7 +51,7 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     for (int r = 0; r < RPT; ++r) s[r] = ld_stream(Sp + (size_t)(rg * RPT + r) * C4 + c4);
 
     // 2. Token vectors; alpha = exp(g).
-    float qk = 0.f;
+    float qk = 0.f, kk = 0.f, qq = 0.f;
     if (tid < DK) {
         const float kv = to_f(k[nh * DK + tid]);
         const float qv = to_f(q[nh * DK + tid]);
@@ -59,18 +59,42 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         qs[tid] = qv;
         as_[tid] = expf(g[nh * DK + tid]);
         qk = kv * qv;
+        if (PRO) { kk = kv * kv; qq = qv * qv; }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, o);
-    if ((tid & 31) == 0) qk_part[tid >> 5] = qk;
+    for (int o = 16; o > 0; o >>= 1) {
+        qk += __shfl_xor_sync(0xffffffffu, qk, o);
+        if (PRO) {
+            kk += __shfl_xor_sync(0xffffffffu, kk, o);
+            qq += __shfl_xor_sync(0xffffffffu, qq, o);
+        }
+    }
+    if ((tid & 31) == 0) {
+        qk_part[tid >> 5] = qk;
+        if (PRO) { kk_part[tid >> 5] = kk; qq_part[tid >> 5] = qq; }
+    }
     __syncthreads();
+    // prologue factors: k <- sk k, q <- sq q
+    float sk = 1.f, sq = 1.f;
+    if (PRO) {
+        if (pro.flags & kProQkL2Norm) {
+            float ka = 0.f, qa = 0.f;
+#pragma unroll
+            for (int w = 0; w < NT / 32; ++w) { ka += kk_part[w]; qa += qq_part[w]; }
+            sk = inv_norm(ka);
+            sq = inv_norm(qa);
+        }
+        sq *= pro.q_scale;
+    }
 
     // 3. S' = Diag(a) S and the per-thread partial column sums.
     float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
         const int row = rg * RPT + r;
-        const float a = as_[row], kr = ks[row], qr = qs[row];
+        const float a = as_[row];
+        float kr = ks[row], qr = qs[row];
+        if (PRO) { kr *= sk; qr *= sq; }
         s[r].x *= a; s[r].y *= a; s[r].z *= a; s[r].w *= a;
         pk[0] += kr * s[r].x; pk[1] += kr * s[r].y; pk[2] += kr * s[r].z; pk[3] += kr * s[r].w;
         pq[0] += qr * s[r].x; pq[1] += qr * s[r].y; pq[2] += qr * s[r].z; pq[3] += qr * s[r].w;
@@ -87,7 +111,11 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         float qk_all = 0.f;
 #pragma unroll
         for (int w = 0; w < NT / 32; ++w) qk_all += qk_part[w];
-        const float b = beta[nh];
+        float b = beta[nh];
+        if (PRO) {
+            qk_all *= sk * sq;
+            if (pro.flags & kProBetaSigmoid) b = sigmoid_f(b);
+        }
         const float u = b * (to_f(v[nh * DV + tid]) - kS);
         us[tid] = u;
         out[nh * DV + tid] = from_f<Tin>(qS + qk_all * u);
@@ -98,7 +126,8 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     const float4 u4 = reinterpret_cast<const float4 *>(us)[c4];
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
-        const float kr = ks[rg * RPT + r];
+        float kr = ks[rg * RPT + r];
+        if (PRO) kr *= sk;
         float4 o4 = s[r];
         o4.x += kr * u4.x; o4.y += kr * u4.y; o4.z += kr * u4.z; o4.w += kr * u4.w;
         st_stream(Sp + (size_t)(rg * RPT + r) * C4 + c4, o4);
@@ -111,13 +140,13 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
 // row (n * L + l) of the token arrays; sequence n uses pool entry slots[n]
 // (n when slots is null).  A slot outside [0, num_slots) skips the sequence
 // and sets the device error word.
-template <int DK, int DV, typename Tin>
+template <int DK, int DV, typename Tin, bool PRO>
 __global__ void __launch_bounds__(256, 2)
 decode_steps_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                     const Tin *__restrict__ v, const float *__restrict__ g,
                     const float *__restrict__ beta, float *__restrict__ pool,
                     const int32_t *__restrict__ slots, int num_slots, Tin *__restrict__ out,
-                    int H, int L, int *__restrict__ err)
+                    int H, int L, int *__restrict__ err, Prologue pro)
 {
     constexpr int NT = 256;
     constexpr int C4 = DV / 4;
@@ -139,7 +168,7 @@ decode_steps_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     __shared__ __align__(16) float red_k[RG][DV + 4];
     __shared__ __align__(16) float red_q[RG][DV + 4];
     __shared__ __align__(16) float us[DV];
-    __shared__ float qk_part[NT / 32];
+    __shared__ float qk_part[NT / 32], kk_part[NT / 32], qq_part[NT / 32];
 
     float4 *Sp = reinterpret_cast<float4 *>(pool + ((size_t)slot * H + h) * (size_t)(DK * DV));
     float4 s[RPT];
@@ -164,25 +193,50 @@ decode_steps_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     for (int l = 0; l < L; ++l) {
         const size_t row = ((size_t)n * L + l) * H + h;
         if (l > 0) __syncthreads();   // the previous step's readers of ks, us, qk_part
-        float qk = 0.f;
+        float qk = 0.f, kk = 0.f, qq = 0.f;
         if (tid < DK) {
             ks[tid] = kn;
             qs[tid] = qn;
             as_[tid] = expf(gn);
             qk = kn * qn;
+            if (PRO) { kk = kn * kn; qq = qn * qn; }
         }
-        const float vcur = vn, bcur = bn;
+        const float vcur = vn;
+        float bcur = bn;
+        if (PRO && (pro.flags & kProBetaSigmoid)) bcur = sigmoid_f(bcur);
         if (l + 1 < L) load_token(l + 1);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, o);
-        if ((tid & 31) == 0) qk_part[tid >> 5] = qk;
+        for (int o = 16; o > 0; o >>= 1) {
+            qk += __shfl_xor_sync(0xffffffffu, qk, o);
+            if (PRO) {
+                kk += __shfl_xor_sync(0xffffffffu, kk, o);
+                qq += __shfl_xor_sync(0xffffffffu, qq, o);
+            }
+        }
+        if ((tid & 31) == 0) {
+            qk_part[tid >> 5] = qk;
+            if (PRO) { kk_part[tid >> 5] = kk; qq_part[tid >> 5] = qq; }
+        }
         __syncthreads();
+        float sk = 1.f, sq = 1.f;
+        if (PRO) {
+            if (pro.flags & kProQkL2Norm) {
+                float ka = 0.f, qa = 0.f;
+#pragma unroll
+                for (int w = 0; w < NT / 32; ++w) { ka += kk_part[w]; qa += qq_part[w]; }
+                sk = inv_norm(ka);
+                sq = inv_norm(qa);
+            }
+            sq *= pro.q_scale;
+        }
 
         float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int r = 0; r < RPT; ++r) {
             const int rr = rg * RPT + r;
-            const float a = as_[rr], kr = ks[rr], qr = qs[rr];
+            const float a = as_[rr];
+            float kr = ks[rr], qr = qs[rr];
+            if (PRO) { kr *= sk; qr *= sq; }
             s[r].x *= a; s[r].y *= a; s[r].z *= a; s[r].w *= a;
             pk[0] += kr * s[r].x; pk[1] += kr * s[r].y; pk[2] += kr * s[r].z; pk[3] += kr * s[r].w;
             pq[0] += qr * s[r].x; pq[1] += qr * s[r].y; pq[2] += qr * s[r].z; pq[3] += qr * s[r].w;
@@ -198,6 +252,7 @@ decode_steps_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
             float qk_all = 0.f;
 #pragma unroll
             for (int w = 0; w < NT / 32; ++w) qk_all += qk_part[w];
+            if (PRO) qk_all *= sk * sq;
             const float u = bcur * (vcur - kS);
             us[tid] = u;
             out[row * DV + tid] = from_f<Tin>(qS + qk_all * u);
@@ -207,7 +262,8 @@ decode_steps_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         const float4 u4 = reinterpret_cast<const float4 *>(us)[c4];
 #pragma unroll
         for (int r = 0; r < RPT; ++r) {
-            const float kr = ks[rg * RPT + r];
+            float kr = ks[rg * RPT + r];
+            if (PRO) kr *= sk;
             s[r].x += kr * u4.x; s[r].y += kr * u4.y; s[r].z += kr * u4.z; s[r].w += kr * u4.w;
         }
     }
@@ -219,11 +275,12 @@ template <int DK, int DV, typename Tin>
 static cudaError_t launch_steps_t(const void *q, const void *k, const void *v, const float *g,
                                   const float *beta, float *pool, const int32_t *slots,
                                   int num_slots, void *out, int N, int H, int L, int *err,
-                                  cudaStream_t st)
+                                  Prologue pro, cudaStream_t st)
 {
-    decode_steps_kernel<DK, DV, Tin><<<N * H, 256, 0, st>>>(
-        (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, pool, slots, num_slots,
-        (Tin *)out, H, L, err);
+    auto kern = (pro.flags != 0 || pro.q_scale != 1.f) ? decode_steps_kernel<DK, DV, Tin, true>
+                                                       : decode_steps_kernel<DK, DV, Tin, false>;
+    kern<<<N * H, 256, 0, st>>>((const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, pool,
+                                slots, num_slots, (Tin *)out, H, L, err, pro);
     return cudaGetLastError();
 }
 
@@ -231,12 +288,12 @@ template <typename Tin>
 static cudaError_t launch_steps_d(const void *q, const void *k, const void *v, const float *g,
                                   const float *beta, float *pool, const int32_t *slots,
                                   int num_slots, void *out, int N, int H, int L, int dk, int dv,
-                                  int *err, cudaStream_t st)
+                                  int *err, Prologue pro, cudaStream_t st)
 {
 #define KDA_STEPS(DK_, DV_)                                                                    \
     if (dk == DK_ && dv == DV_)                                                                \
         return launch_steps_t<DK_, DV_, Tin>(q, k, v, g, beta, pool, slots, num_slots, out, N, \
-                                             H, L, err, st);
+                                             H, L, err, pro, st);
     KDA_STEPS(128, 128)
     KDA_STEPS(64, 64)
     KDA_STEPS(128, 64)
@@ -248,43 +305,45 @@ static cudaError_t launch_steps_d(const void *q, const void *k, const void *v, c
 cudaError_t launch_decode_steps(const void *q, const void *k, const void *v, const float *g,
                                 const float *beta, float *pool, const int32_t *slots,
                                 int num_slots, void *out, int N, int H, int L, int dk, int dv,
-                                bool bf16, int *err, cudaStream_t st)
+                                bool bf16, int *err, Prologue pro, cudaStream_t st)
 {
     if (bf16)
         return launch_steps_d<__nv_bfloat16>(q, k, v, g, beta, pool, slots, num_slots, out, N, H,
-                                             L, dk, dv, err, st);
+                                             L, dk, dv, err, pro, st);
     return launch_steps_d<float>(q, k, v, g, beta, pool, slots, num_slots, out, N, H, L, dk, dv,
-                                 err, st);
+                                 err, pro, st);
 }
 
 template <int DK, int DV, typename Tin>
 static cudaError_t launch_decode_t(const void *q, const void *k, const void *v,
                                    const float *g, const float *beta, float *state,
-                                   void *out, int NH, cudaStream_t st)
+                                   void *out, int NH, Prologue pro, cudaStream_t st)
 {
-    decode_step_kernel<DK, DV, Tin><<<NH, 256, 0, st>>>(
-        (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, state, (Tin *)out);
+    auto kern = (pro.flags != 0 || pro.q_scale != 1.f) ? decode_step_kernel<DK, DV, Tin, true>
+                                                       : decode_step_kernel<DK, DV, Tin, false>;
+    kern<<<NH, 256, 0, st>>>((const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, state,
+                             (Tin *)out, pro);
     return cudaGetLastError();
 }
 
 template <typename Tin>
 static cudaError_t launch_decode_d(const void *q, const void *k, const void *v,
                                    const float *g, const float *beta, float *state,
-                                   void *out, int NH, int dk, int dv, cudaStream_t st)
+                                   void *out, int NH, int dk, int dv, Prologue pro, cudaStream_t st)
 {
-    if (dk == 128 && dv == 128) return launch_decode_t<128, 128, Tin>(q, k, v, g, beta, state, out, NH, st);
-    if (dk == 64 && dv == 64) return launch_decode_t<64, 64, Tin>(q, k, v, g, beta, state, out, NH, st);
-    if (dk == 128 && dv == 64) return launch_decode_t<128, 64, Tin>(q, k, v, g, beta, state, out, NH, st);
-    if (dk == 64 && dv == 128) return launch_decode_t<64, 128, Tin>(q, k, v, g, beta, state, out, NH, st);
+    if (dk == 128 && dv == 128) return launch_decode_t<128, 128, Tin>(q, k, v, g, beta, state, out, NH, pro, st);
+    if (dk == 64 && dv == 64) return launch_decode_t<64, 64, Tin>(q, k, v, g, beta, state, out, NH, pro, st);
+    if (dk == 128 && dv == 64) return launch_decode_t<128, 64, Tin>(q, k, v, g, beta, state, out, NH, pro, st);
+    if (dk == 64 && dv == 128) return launch_decode_t<64, 128, Tin>(q, k, v, g, beta, state, out, NH, pro, st);
     return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
                           const float *beta, float *state, void *out, int NH, int dk,
-                          int dv, bool bf16, cudaStream_t st)
+                          int dv, bool bf16, Prologue pro, cudaStream_t st)
 {
-    if (bf16) return launch_decode_d<__nv_bfloat16>(q, k, v, g, beta, state, out, NH, dk, dv, st);
-    return launch_decode_d<float>(q, k, v, g, beta, state, out, NH, dk, dv, st);
+    if (bf16) return launch_decode_d<__nv_bfloat16>(q, k, v, g, beta, state, out, NH, dk, dv, pro, st);
+    return launch_decode_d<float>(q, k, v, g, beta, state, out, NH, dk, dv, pro, st);
 }
 
 }  // namespace kda

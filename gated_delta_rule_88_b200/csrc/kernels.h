@@ -6,20 +6,28 @@
 
 namespace kda {
 
+// Input prologue applied inside the kernels (the ABI's *_ex calls): bit 0
+// L2-normalises q and k per (token, head), bit 1 takes sigmoid(beta); q is
+// then multiplied by q_scale.  {0, 1.f} is the identity.
+struct Prologue {
+    int flags;
+    float q_scale;
+};
+
 // Address of the current device's error word (see common.cuh), or nullptr.
 int *error_word();
 
 // One decode step for NH = N*H (sequence, head) pairs; state updated in place.
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
                           const float *beta, float *state, void *out, int NH, int dk,
-                          int dv, bool bf16, cudaStream_t st);
+                          int dv, bool bf16, Prologue pro, cudaStream_t st);
 
 // L decode tokens per sequence against a slot-indexed state pool
 // [num_slots, H, dk, dv]; sequence n uses pool entry slots[n] (n if null).
 cudaError_t launch_decode_steps(const void *q, const void *k, const void *v, const float *g,
                                 const float *beta, float *pool, const int32_t *slots,
                                 int num_slots, void *out, int N, int H, int L, int dk, int dv,
-                                bool bf16, int *err, cudaStream_t st);
+                                bool bf16, int *err, Prologue pro, cudaStream_t st);
 
 // Exact-fp32 chunked prefill (SIMT).  dk, dv in {64, 128}.
 // Token axis flattened: token t of the packed [B*T] axis, head h, channel c at
@@ -28,7 +36,7 @@ cudaError_t launch_decode_steps(const void *q, const void *k, const void *v, con
 cudaError_t launch_chunk_f32(const float *q, const float *k, const float *v, const float *g,
                              const float *beta, const float *s0, const int32_t *cu,
                              float *out, float *sT, int N, int T, int total_T, int H,
-                             int dk, int dv, cudaStream_t st);
+                             int dk, int dv, Prologue pro, cudaStream_t st);
 
 // bf16 tensor-core prefill (dk = dv = 128) in two launches over a scratch
 // buffer of per-(chunk, head) records (chunk_ws.h):
@@ -42,7 +50,7 @@ cudaError_t launch_chunk_plan(const int32_t *cu, int N, int total_T, int32_t *co
 cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const int32_t *cu, const int32_t *coff,
                               int N, int T, int total_T, int H, int max_chunks,
-                              unsigned char *wsp, cudaStream_t st);
+                              unsigned char *wsp, Prologue pro, cudaStream_t st);
 cudaError_t launch_chunk_chain(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
                                const float *s0, float *sT, void *out, int N, int T, int total_T,
                                int H, int dvt, int max_chunks, int *err, cudaStream_t st);

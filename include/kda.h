@@ -62,6 +62,21 @@ typedef enum {
 } kda_dtype;
 
 /*
+ * Input prologue flags of the *_ex calls (and kda_recurrent_steps), applied
+ * inside the kernels before the method runs, per (token, head):
+ *   KDA_QK_L2NORM     q <- q / |q|_2 and k <- k / |k|_2 (fp32; a zero vector
+ *                     stays zero)
+ *   KDA_BETA_SIGMOID  beta <- 1 / (1 + exp(-beta))  (beta given as a logit)
+ * and then q <- q_scale * q.  flags = 0 with q_scale = 1 is the identity.
+ * Source: Kimi Linear paper notes (paper-notes-site), section 7: the open
+ * layer hands raw projections to the KDA kernels with the q/k L2 norm done
+ * inside the kernel (use_qk_l2norm_in_kernel) and takes beta as the sigmoid
+ * of a projection; the gate activation (A_log, dt_bias) is not on the pages
+ * and is not offered.
+ */
+enum { KDA_QK_L2NORM = 1, KDA_BETA_SIGMOID = 2 };
+
+/*
  * kda_chunk_fwd -- prefill forward over whole sequences.
  *
  * Source: Kimi Linear paper notes (paper-notes-site), section 2 (recurrence)
@@ -101,6 +116,18 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v,
                          void *out, float *final_state,
                          int B, int T, int H, int dk, int dv, int num_seqs,
                          kda_dtype dtype, void *stream);
+
+/*
+ * kda_chunk_fwd_ex -- kda_chunk_fwd with the input prologue (flags, q_scale;
+ * see KDA_QK_L2NORM).  Same arguments, layouts and support otherwise;
+ * unknown flag bits or a non-finite q_scale return KDA_ERR_INVALID_ARG.
+ */
+kda_status kda_chunk_fwd_ex(const void *q, const void *k, const void *v,
+                            const float *g, const float *beta,
+                            const float *initial_state, const int32_t *cu_seqlens,
+                            void *out, float *final_state,
+                            int B, int T, int H, int dk, int dv, int num_seqs,
+                            kda_dtype dtype, unsigned flags, float q_scale, void *stream);
 
 /*
  * kda_chunk_fwd_host -- kda_chunk_fwd (dense mode) on HOST buffers, with the
@@ -159,6 +186,18 @@ kda_status kda_recurrent_step(const void *q, const void *k, const void *v,
                               kda_dtype dtype, void *stream);
 
 /*
+ * kda_recurrent_step_ex -- kda_recurrent_step with the input prologue
+ * (flags, q_scale; see KDA_QK_L2NORM).  Unknown flag bits or a non-finite
+ * q_scale return KDA_ERR_INVALID_ARG.
+ */
+kda_status kda_recurrent_step_ex(const void *q, const void *k, const void *v,
+                                 const float *g, const float *beta,
+                                 float *state_inout, void *out,
+                                 int N, int H, int dk, int dv,
+                                 kda_dtype dtype, unsigned flags, float q_scale,
+                                 void *stream);
+
+/*
  * kda_recurrent_steps -- L decode tokens for each of N sequences whose states
  * live in a slot-indexed pool (continuous batching).
  *
@@ -180,6 +219,8 @@ kda_status kda_recurrent_step(const void *q, const void *k, const void *v,
  *   kda_get_device_error with code 3.  Slots must be distinct: two sequences
  *   naming one entry race.  L >= 1 (the paper's mode switch is at 64 tokens;
  *   longer inputs belong to kda_chunk_fwd, but any L is computed correctly).
+ * Prologue: flags and q_scale as in the *_ex calls (KDA_QK_L2NORM); pass
+ *   0 and 1.0f for inputs that are already normalised.
  * Supported: dk, dv in {64, 128}, dtype KDA_BF16 or KDA_F32.  Any finite g.
  * Aliasing: out must not overlap any input; the pool must not overlap the
  *   token inputs.
@@ -188,7 +229,8 @@ kda_status kda_recurrent_steps(const void *q, const void *k, const void *v,
                                const float *g, const float *beta,
                                float *state_pool, const int32_t *slots, int num_slots,
                                void *out, int N, int L, int H, int dk, int dv,
-                               kda_dtype dtype, void *stream);
+                               kda_dtype dtype, unsigned flags, float q_scale,
+                               void *stream);
 
 /*
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate

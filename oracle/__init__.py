@@ -148,3 +148,26 @@ def decode_step(q, k, v, g, beta, state, threads: int | None = None):
                     g.unsqueeze(1), beta.unsqueeze(1), initial_state=state,
                     threads=threads)
     return o[:, 0], sT
+
+
+def prologue(q, k, beta, qk_l2norm: bool = False, beta_sigmoid: bool = False,
+             q_scale: float = 1.0):
+    """The input prologue of the library's *_ex calls, in fp64, on the values
+    as given (bf16 inputs widened exactly).  Kimi Linear paper notes, section 7:
+    the layer normalises q and k inside the kernel (use_qk_l2norm_in_kernel)
+    and takes beta as the sigmoid of a projection.  Per (token, head):
+        q <- q_scale * q / |q|_2,   k <- k / |k|_2      (qk_l2norm; 0 -> 0)
+        q <- q_scale * q                                 (otherwise)
+        beta <- 1 / (1 + exp(-beta))                     (beta_sigmoid)
+    Returns fp64 tensors (q, k, beta) of the same shapes."""
+    q64, k64, b64 = q.double(), k.double(), beta.double()
+    if qk_l2norm:
+        def unit(x):
+            n = torch.linalg.vector_norm(x, dim=-1, keepdim=True)
+            return torch.where(n > 0, x / torch.where(n > 0, n, torch.ones_like(n)),
+                               torch.zeros_like(x))
+        q64, k64 = unit(q64), unit(k64)
+    q64 = q64 * float(q_scale)
+    if beta_sigmoid:
+        b64 = 1.0 / (1.0 + torch.exp(-b64))
+    return q64, k64, b64

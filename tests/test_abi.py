@@ -35,7 +35,8 @@ def declared_functions():
 
 def test_header_declares_entry_points():
     names = declared_functions()
-    for n in ("kda_chunk_fwd", "kda_chunk_fwd_host", "kda_recurrent_step", "kda_recurrent_steps",
+    for n in ("kda_chunk_fwd", "kda_chunk_fwd_ex", "kda_chunk_fwd_host", "kda_recurrent_step",
+              "kda_recurrent_step_ex", "kda_recurrent_steps",
               "kda_status_string",
               "kda_get_device_error", "kda_last_error_message", "kda_version"):
         assert n in names
@@ -112,10 +113,10 @@ def test_step_empty_batch_is_a_no_op(lib):
 
 
 def steps(lib, *, q=FAKE, k=FAKE, v=FAKE, g=FAKE, b=FAKE, pool=FAKE, slots=None, S=4, out=FAKE,
-          N=1, L=2, H=1, dk=128, dv=128, dtype=1):
+          N=1, L=2, H=1, dk=128, dv=128, dtype=1, flags=0, q_scale=1.0):
     P = ctypes.c_void_p
     return lib.kda_recurrent_steps(P(q), P(k), P(v), P(g), P(b), P(pool), P(slots), S, P(out),
-                                   N, L, H, dk, dv, dtype, None)
+                                   N, L, H, dk, dv, dtype, flags, q_scale, None)
 
 
 @pytest.mark.parametrize("field", ["q", "k", "v", "g", "b", "pool", "out"])
@@ -125,7 +126,9 @@ def test_steps_null_pointer_rejected(lib, field):
 
 @pytest.mark.parametrize("kw", [dict(N=-1), dict(L=0), dict(H=0), dict(S=0), dict(N=5, S=4),
                                 dict(dtype=3), dict(pool=FAKE + 8), dict(b=FAKE + 1),
-                                dict(slots=FAKE + 2), dict(N=1 << 20, H=1 << 12)])
+                                dict(slots=FAKE + 2), dict(N=1 << 20, H=1 << 12),
+                                dict(flags=4), dict(q_scale=float("nan")),
+                                dict(q_scale=float("inf"))])
 def test_steps_bad_arguments_rejected(lib, kw):
     assert steps(lib, **kw) == 1
 
@@ -145,6 +148,17 @@ def host(lib, *, q=FAKE, k=FAKE, v=FAKE, g=FAKE, b=FAKE, s0=None, out=FAKE, sT=N
     P = ctypes.c_void_p
     return lib.kda_chunk_fwd_host(P(q), P(k), P(v), P(g), P(b), P(s0), P(out), P(sT), B, T, H,
                                   dk, dv, dtype, rt, None)
+
+
+@pytest.mark.parametrize("kw", [dict(flags=8), dict(flags=0xFFFFFFFF), dict(q_scale=float("nan")),
+                                dict(q_scale=float("-inf"))])
+def test_ex_prologue_arguments_rejected(lib, kw):
+    P = ctypes.c_void_p
+    flags, q_scale = kw.get("flags", 1), kw.get("q_scale", 1.0)
+    assert lib.kda_chunk_fwd_ex(P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), None, None, P(FAKE),
+                                None, 1, 64, 1, 128, 128, 1, 1, flags, q_scale, None) == 1
+    assert lib.kda_recurrent_step_ex(P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE),
+                                     1, 1, 128, 128, 1, flags, q_scale, None) == 1
 
 
 @pytest.mark.parametrize("field", ["q", "k", "v", "g", "b", "out"])

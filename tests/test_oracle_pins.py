@@ -319,3 +319,50 @@ def test_decode_step_equals_one_token_forward():
                                        g[n, h][None], beta[n, h][None], s0[n, h])
             assert np.abs(o[n, h].numpy() - o1[0]).max() == 0
             assert np.abs(s1[n, h].numpy() - S1).max() == 0
+
+
+# ---- input prologue (the *_ex calls): pinned by properties, not by retyping ----
+
+def test_prologue_l2norm_unit_rows_direction_and_zero_rows():
+    gen = torch.Generator().manual_seed(7)
+    q = torch.randn(2, 5, 3, 8, generator=gen, dtype=torch.float64) * 3.0
+    k = torch.randn(2, 5, 3, 8, generator=gen, dtype=torch.float64)
+    q[1, 2, 0] = 0.0                                    # a padding row
+    b = torch.zeros(2, 5, 3, dtype=torch.float64)
+    qn, kn, bn = oracle.prologue(q, k, b, qk_l2norm=True)
+    norms_q = torch.linalg.vector_norm(qn, dim=-1)
+    norms_k = torch.linalg.vector_norm(kn, dim=-1)
+    mask = torch.ones_like(norms_q, dtype=torch.bool)
+    mask[1, 2, 0] = False
+    assert torch.allclose(norms_q[mask], torch.ones_like(norms_q[mask]), atol=1e-14)
+    assert torch.allclose(norms_k, torch.ones_like(norms_k), atol=1e-14)
+    assert torch.all(qn[1, 2, 0] == 0)
+    # same direction: <q_hat, q> = |q|
+    dots = (qn * q).sum(-1)
+    assert torch.allclose(dots[mask], torch.linalg.vector_norm(q, dim=-1)[mask], rtol=1e-13)
+    assert torch.equal(bn, b)                          # beta untouched without the flag
+
+
+def test_prologue_q_scale_only_scales_q():
+    gen = torch.Generator().manual_seed(8)
+    q = torch.randn(1, 4, 2, 8, generator=gen, dtype=torch.float64)
+    k = torch.randn(1, 4, 2, 8, generator=gen, dtype=torch.float64)
+    b = torch.randn(1, 4, 2, generator=gen, dtype=torch.float64)
+    qs, ks, bs = oracle.prologue(q, k, b, q_scale=0.25)
+    assert torch.equal(qs, q * 0.25) and torch.equal(ks, k) and torch.equal(bs, b)
+    qn, kn, _ = oracle.prologue(q, k, b, qk_l2norm=True, q_scale=0.5)
+    assert torch.allclose(torch.linalg.vector_norm(qn, dim=-1), torch.full((1, 4, 2), 0.5,
+                          dtype=torch.float64), atol=1e-14)
+
+
+def test_prologue_sigmoid_closed_forms():
+    b = torch.tensor([0.0, math.log(3.0), -math.log(3.0), 40.0, -40.0], dtype=torch.float64)
+    _, _, s = oracle.prologue(torch.zeros(5, 1), torch.zeros(5, 1), b, beta_sigmoid=True)
+    assert s[0] == 0.5
+    assert abs(s[1] - 0.75) < 1e-15 and abs(s[2] - 0.25) < 1e-15   # sigma(ln 3) = 3/4
+    x = torch.linspace(-6, 6, 25, dtype=torch.float64)
+    _, _, sx = oracle.prologue(torch.zeros(25, 1), torch.zeros(25, 1), x, beta_sigmoid=True)
+    _, _, smx = oracle.prologue(torch.zeros(25, 1), torch.zeros(25, 1), -x, beta_sigmoid=True)
+    assert torch.allclose(sx + smx, torch.ones_like(sx), atol=1e-15)   # sigma(x) + sigma(-x) = 1
+    assert torch.all(sx[1:] > sx[:-1])                                # increasing
+    assert s[3] > 1 - 1e-15 and s[4] < 1e-15

@@ -29,7 +29,9 @@ import threading
 import torch
 
 __all__ = ["kda_chunk_fwd", "kda_chunk_fwd_ex", "kda_chunk_fwd_host", "kda_recurrent_step",
-           "kda_recurrent_step_ex", "kda_recurrent_steps", "kda_get_device_error", "KDAError",
+           "kda_recurrent_step_ex", "kda_recurrent_steps", "kda_gated_rmsnorm", "kda_state_affine",
+           "kda_get_device_error",
+           "KDAError",
            "KDA_QK_L2NORM", "KDA_BETA_SIGMOID",
            "library_path", "load_library"]
 
@@ -75,6 +77,10 @@ def load_library():
         lib.kda_recurrent_steps.restype = i
         lib.kda_chunk_fwd_host.argtypes = [vp] * 8 + [i] * 7 + [vp]
         lib.kda_chunk_fwd_host.restype = i
+        lib.kda_gated_rmsnorm.argtypes = [vp, vp, vp, ctypes.c_float, vp, ctypes.c_longlong, i, i, vp]
+        lib.kda_gated_rmsnorm.restype = i
+        lib.kda_state_affine.argtypes = [vp] * 4 + [i] * 3 + [vp]
+        lib.kda_state_affine.restype = i
         lib.kda_get_device_error.argtypes = [vp, ctypes.POINTER(i)]
         lib.kda_get_device_error.restype = i
         lib.kda_last_error_message.restype = ctypes.c_char_p
@@ -289,6 +295,59 @@ def kda_recurrent_steps(q, k, v, g, beta, state_pool, slots=None, out=None, flag
                                      _dptr(state_pool), _dptr(slots), state_pool.shape[0],
                                      _dptr(out), N, L, H, dk, dv, _dtype_code(q), int(flags),
                                      float(q_scale), _stream_handle(dev))
+    _check(rc)
+    return out
+
+
+def kda_gated_rmsnorm(x, gate, weight, eps: float = 1e-5, out=None):
+    """The layer's output epilogue: x / sqrt(mean(x^2) + eps) * weight *
+    sigmoid(gate) over the last dimension (dv = 64 or 128).  x, gate [..., dv]
+    in the output dtype; weight [dv] fp32.  out may be x (in place)."""
+    lib = load_library()
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("kda_gated_rmsnorm needs CUDA tensors (no CPU path)")
+    dv = x.shape[-1]
+    _need(x, "x", dev, x.dtype)
+    _need(gate, "gate", dev, x.dtype)
+    _need(weight, "weight", dev, torch.float32)
+    if gate.shape != x.shape or tuple(weight.shape) != (dv,):
+        raise ValueError("gate must match x and weight must be [dv]")
+    if out is None:
+        out = torch.empty_like(x)
+    else:
+        _need(out, "out", dev, x.dtype)
+    rows = x.numel() // dv
+    with torch.cuda.device(dev):
+        rc = lib.kda_gated_rmsnorm(_dptr(x), _dptr(gate), _dptr(weight), float(eps), _dptr(out),
+                                   rows, dv, _dtype_code(x), _stream_handle(dev))
+    _check(rc)
+    return out
+
+
+def kda_state_affine(M, B, S_in, out=None):
+    """S_out = M S_in + B per block: M [..., dk, dk]; B (or None), S_in
+    [..., dk, dv] fp32 CUDA tensors.  Returns S_out (a new tensor unless out
+    is given; out must not overlap S_in or M)."""
+    lib = load_library()
+    dev = S_in.device
+    if dev.type != "cuda":
+        raise ValueError("kda_state_affine needs CUDA tensors (no CPU path)")
+    dk, dv = S_in.shape[-2], S_in.shape[-1]
+    _need(M, "M", dev, torch.float32)
+    _need(S_in, "S_in", dev, torch.float32)
+    if B is not None:
+        _need(B, "B", dev, torch.float32)
+        if B.shape != S_in.shape:
+            raise ValueError("B must match S_in")
+    if M.shape[:-2] != S_in.shape[:-2] or M.shape[-2:] != (dk, dk):
+        raise ValueError("M must be [..., dk, dk] over the same blocks as S_in")
+    out = torch.empty_like(S_in) if out is None else out
+    _need(out, "out", dev, torch.float32)
+    count = S_in.numel() // (dk * dv)
+    with torch.cuda.device(dev):
+        rc = lib.kda_state_affine(_dptr(M), _dptr(B), _dptr(S_in), _dptr(out), count, dk, dv,
+                                  _stream_handle(dev))
     _check(rc)
     return out
 

@@ -348,6 +348,50 @@ static kda_status chunk_fwd_device(const void *q, const void *k, const void *v, 
     return KDA_OK;
 }
 
+extern "C" kda_status kda_gated_rmsnorm(const void *x, const void *gate, const float *weight,
+                                        float eps, void *out, long long rows, int dv,
+                                        kda_dtype dtype, void *stream) {
+    t_msg[0] = 0;
+    if (!x || !gate || !weight || !out)
+        return fail(KDA_ERR_INVALID_ARG, "kda_gated_rmsnorm: null pointer argument");
+    if (rows < 0 || rows > (1LL << 36))
+        return fail(KDA_ERR_INVALID_ARG, "kda_gated_rmsnorm: bad row count %lld", rows);
+    if (dtype != KDA_F32 && dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARG, "kda_gated_rmsnorm: unknown dtype %d", (int)dtype);
+    if (!(eps >= 0.f) || eps > 3.4e38f)
+        return fail(KDA_ERR_INVALID_ARG, "kda_gated_rmsnorm: eps must be finite and >= 0");
+    if (dv != 64 && dv != 128)
+        return fail(KDA_ERR_UNSUPPORTED, "kda_gated_rmsnorm: dv=%d (supported: 64, 128)", dv);
+    if (!aligned16(x) || !aligned16(gate) || !aligned16(out) || ((uintptr_t)weight & 3u))
+        return fail(KDA_ERR_INVALID_ARG,
+                    "kda_gated_rmsnorm: x, gate, out must be 16-byte aligned, weight 4-byte");
+    cudaError_t e = kda::launch_gated_rmsnorm(x, gate, weight, eps, out, rows, dv, dtype == KDA_BF16,
+                                              (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_gated_rmsnorm launch");
+    return KDA_OK;
+}
+
+extern "C" kda_status kda_state_affine(const float *M, const float *B, const float *S_in,
+                                       float *S_out, int count, int dk, int dv, void *stream) {
+    t_msg[0] = 0;
+    if (!M || !S_in || !S_out)
+        return fail(KDA_ERR_INVALID_ARG, "kda_state_affine: null pointer argument");
+    if (count < 0 || count > 65535 || dk <= 0 || dk > 65535 || dv <= 0 || dv > 4096)
+        return fail(KDA_ERR_INVALID_ARG, "kda_state_affine: bad sizes count=%d dk=%d dv=%d", count,
+                    dk, dv);
+    if (((uintptr_t)M | (uintptr_t)S_in | (uintptr_t)S_out | (uintptr_t)B) & 3u)
+        return fail(KDA_ERR_INVALID_ARG, "kda_state_affine: pointers must be 4-byte aligned");
+    const size_t sb = (size_t)count * dk * dv * sizeof(float), mb = (size_t)count * dk * dk * sizeof(float);
+    auto overlap = [](const void *a, size_t na, const void *b, size_t nb) {
+        return (const char *)a < (const char *)b + nb && (const char *)b < (const char *)a + na;
+    };
+    if (count > 0 && (overlap(S_out, sb, S_in, sb) || overlap(S_out, sb, M, mb)))
+        return fail(KDA_ERR_INVALID_ARG, "kda_state_affine: S_out overlaps S_in or M");
+    cudaError_t e = kda::launch_state_affine(M, B, S_in, S_out, count, dk, dv, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_state_affine launch");
+    return KDA_OK;
+}
+
 // ---------------------------------------------------------------------------
 // kda_chunk_fwd_host: host buffers, pipelined over token ranges.
 namespace {

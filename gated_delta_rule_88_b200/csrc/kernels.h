@@ -29,6 +29,15 @@ cudaError_t launch_decode_steps(const void *q, const void *k, const void *v, con
                                 int num_slots, void *out, int N, int H, int L, int dk, int dv,
                                 bool bf16, int *err, Prologue pro, cudaStream_t st);
 
+// Gated RMSNorm over rows of dv (64 or 128): y = x rsqrt(mean(x^2) + eps) w sigmoid(z).
+cudaError_t launch_gated_rmsnorm(const void *x, const void *z, const float *w, float eps, void *y,
+                                 long long rows, int dv, bool bf16, cudaStream_t st);
+
+// S_out[i] = M[i] S_in[i] + B[i] (B may be null), i < count; M [count, dk, dk],
+// B, S_in, S_out [count, dk, dv] fp32; S_out must not overlap S_in or M.
+cudaError_t launch_state_affine(const float *M, const float *B, const float *S, float *out,
+                                int count, int dk, int dv, cudaStream_t st);
+
 // Exact-fp32 chunked prefill (SIMT).  dk, dv in {64, 128}.
 // Token axis flattened: token t of the packed [B*T] axis, head h, channel c at
 // ((t * H) + h) * d + c.  Sequences: dense (cu == nullptr, n-th spans

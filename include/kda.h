@@ -19,7 +19,8 @@
  *   kda_recurrent_steps decode for serving: up to L tokens per sequence
  *                       (short queries) on a slot-indexed state pool;
  *   kda_chunk_fwd_host  kda_chunk_fwd on host buffers, copies pipelined
- *                       against the computation.
+ *                       against the computation;
+ *   kda_gated_rmsnorm   the output epilogue (RMSNorm with a sigmoid gate).
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers (cudaMalloc'd or any memory the
@@ -231,6 +232,44 @@ kda_status kda_recurrent_steps(const void *q, const void *k, const void *v,
                                void *out, int N, int L, int H, int dk, int dv,
                                kda_dtype dtype, unsigned flags, float q_scale,
                                void *stream);
+
+/*
+ * kda_gated_rmsnorm -- the layer's output epilogue: an RMSNorm with a
+ * sigmoid output gate, per row of dv values.
+ *
+ * Source: Kimi Linear paper notes (paper-notes-site), section 7: the layer
+ * passes the KDA readout through FusedRMSNormGated (sigmoid output gate)
+ * before the output projection.
+ *
+ * Computes, for each of `rows` rows (e.g. rows = B * T * H of the prefill
+ * output [B, T, H, dv], or N * H of a decode output):
+ *     out = x / sqrt(mean(x^2) + eps) * weight * 1 / (1 + exp(-gate))
+ * in fp32, rounded to nearest even for bf16.
+ * Layout: x, gate, out [rows, dv] dtype (device, 16-byte aligned); weight
+ *   [dv] float32 (device).  out may equal x (in place); it must not overlap
+ *   gate or weight otherwise.
+ * Supported: dv in {64, 128}, dtype KDA_BF16 or KDA_F32; eps finite >= 0.
+ */
+kda_status kda_gated_rmsnorm(const void *x, const void *gate, const float *weight,
+                             float eps, void *out, long long rows, int dv,
+                             kda_dtype dtype, void *stream);
+
+/*
+ * kda_state_affine -- S_out = M S_in + B for `count` independent blocks.
+ *
+ * Source: the recurrence of the paper notes (section 2) is affine in the
+ * state: a segment of tokens maps any start state S to M S + B, with B the
+ * segment's final state from S = 0 and M its final state from S = I with
+ * v = 0.  This call composes such maps, the exchange step of a sequence
+ * split across devices (gated_delta_rule_88_b200.cp); the pages describe no
+ * multi-device prefill.
+ *
+ * Layout: M [count, dk, dk]; B (nullable = 0), S_in, S_out [count, dk, dv];
+ *   float32 device memory, 4-byte aligned.  S_out must not overlap S_in or M.
+ * Supported: count <= 65535, dk <= 65535, dv <= 4096.
+ */
+kda_status kda_state_affine(const float *M, const float *B, const float *S_in,
+                            float *S_out, int count, int dk, int dv, void *stream);
 
 /*
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate

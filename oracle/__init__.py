@@ -171,3 +171,21 @@ def prologue(q, k, beta, qk_l2norm: bool = False, beta_sigmoid: bool = False,
     if beta_sigmoid:
         b64 = 1.0 / (1.0 + torch.exp(-b64))
     return q64, k64, b64
+
+
+def gated_rmsnorm(x, gate, weight, eps: float):
+    """The layer's output epilogue in fp64 (Kimi Linear paper notes, section 7:
+    FusedRMSNormGated with a sigmoid output gate), over the last dimension:
+        y = x / sqrt(mean(x^2) + eps) * weight * 1 / (1 + exp(-gate))"""
+    x64, z64, w64 = x.double(), gate.double(), weight.double()
+    r = torch.rsqrt((x64 * x64).mean(dim=-1, keepdim=True) + eps)
+    return x64 * r * w64 / (1.0 + torch.exp(-z64))
+
+
+def state_affine(M, B, S):
+    """S_out = M S + B per block in fp64: M [..., dk, dk]; B (or None), S
+    [..., dk, dv].  Kimi Linear paper notes, section 2: the recurrence is
+    affine in the state, so a segment of tokens acts on its start state as
+    such a map (used to check the context-parallel fold)."""
+    out = M.double() @ S.double()
+    return out if B is None else out + B.double()

@@ -36,7 +36,7 @@ def declared_functions():
 def test_header_declares_entry_points():
     names = declared_functions()
     for n in ("kda_chunk_fwd", "kda_chunk_fwd_ex", "kda_chunk_fwd_host", "kda_recurrent_step",
-              "kda_recurrent_step_ex", "kda_recurrent_steps",
+              "kda_recurrent_step_ex", "kda_recurrent_steps", "kda_gated_rmsnorm",
               "kda_status_string",
               "kda_get_device_error", "kda_last_error_message", "kda_version"):
         assert n in names
@@ -161,6 +161,26 @@ def test_ex_prologue_arguments_rejected(lib, kw):
                                      1, 1, 128, 128, 1, flags, q_scale, None) == 1
 
 
+def norm(lib, *, x=FAKE, z=FAKE, w=FAKE, eps=1e-5, out=FAKE, rows=4, dv=128, dtype=1):
+    P = ctypes.c_void_p
+    return lib.kda_gated_rmsnorm(P(x), P(z), P(w), eps, P(out), rows, dv, dtype, None)
+
+
+@pytest.mark.parametrize("kw", [dict(x=0), dict(z=0), dict(w=0), dict(out=0), dict(rows=-1),
+                                dict(dtype=4), dict(eps=-1.0), dict(eps=float("nan")),
+                                dict(x=FAKE + 8), dict(w=FAKE + 2)])
+def test_norm_bad_arguments_rejected(lib, kw):
+    assert norm(lib, **kw) == 1
+
+
+def test_norm_unsupported_rejected(lib):
+    assert norm(lib, dv=96) == 2
+
+
+def test_norm_empty_is_a_no_op(lib):
+    assert norm(lib, rows=0) == 0
+
+
 @pytest.mark.parametrize("field", ["q", "k", "v", "g", "b", "out"])
 def test_host_null_pointer_rejected(lib, field):
     assert host(lib, **{field: 0}) == 1
@@ -184,3 +204,19 @@ def test_python_binding_refuses_cpu_tensors():
         kda.kda_chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))
     with pytest.raises(ValueError, match="CUDA"):
         kda.kda_recurrent_step(x[0], x[0], x[0], x[0], torch.zeros(4, 1), torch.zeros(4, 1, 64, 64))
+
+
+def affine(lib, *, M=FAKE, B=0, S=FAKE + (1 << 24), out=FAKE + (1 << 25), count=2, dk=128, dv=128):
+    P = ctypes.c_void_p
+    return lib.kda_state_affine(P(M), P(B), P(S), P(out), count, dk, dv, None)
+
+
+@pytest.mark.parametrize("kw", [dict(M=0), dict(S=0), dict(out=0), dict(count=-1), dict(dk=0),
+                                dict(dv=5000), dict(M=FAKE + 2), dict(B=FAKE + 6),
+                                dict(out=FAKE + (1 << 24) + 64), dict(out=FAKE + 4)])
+def test_affine_bad_arguments_rejected(lib, kw):
+    assert affine(lib, **kw) == 1
+
+
+def test_affine_empty_is_a_no_op(lib):
+    assert affine(lib, count=0) == 0

@@ -366,3 +366,23 @@ def test_prologue_sigmoid_closed_forms():
     assert torch.allclose(sx + smx, torch.ones_like(sx), atol=1e-15)   # sigma(x) + sigma(-x) = 1
     assert torch.all(sx[1:] > sx[:-1])                                # increasing
     assert s[3] > 1 - 1e-15 and s[4] < 1e-15
+
+
+# ---- output epilogue (gated RMSNorm): pinned by properties ----
+
+def test_gated_rmsnorm_unit_rms_scale_invariance_and_gate():
+    gen = torch.Generator().manual_seed(9)
+    x = torch.randn(6, 16, generator=gen, dtype=torch.float64) * 5.0
+    ones = torch.ones(16, dtype=torch.float64)
+    big = torch.full((6, 16), 60.0, dtype=torch.float64)          # sigmoid -> 1
+    y = oracle.gated_rmsnorm(x, big, ones, 0.0)
+    assert torch.allclose(y.pow(2).mean(-1), torch.ones(6, dtype=torch.float64), atol=1e-12)
+    assert torch.allclose(oracle.gated_rmsnorm(3.7 * x, big, ones, 0.0), y, atol=1e-13)
+    half = oracle.gated_rmsnorm(x, torch.zeros(6, 16, dtype=torch.float64), ones, 0.0)
+    assert torch.allclose(half, 0.5 * y, atol=1e-13)              # sigmoid(0) = 1/2
+    w = torch.linspace(-2, 2, 16, dtype=torch.float64)
+    assert torch.allclose(oracle.gated_rmsnorm(x, big, w, 0.0), y * w, atol=1e-13)
+    # eps enters as mean(x^2) + eps: a row with mean square m maps to x / sqrt(m + eps)
+    row = torch.full((1, 16), 2.0, dtype=torch.float64)
+    assert torch.allclose(oracle.gated_rmsnorm(row, big[:1], ones, 5.0),
+                          torch.full((1, 16), 2.0 / 3.0, dtype=torch.float64), atol=1e-13)

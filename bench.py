@@ -353,7 +353,7 @@ def decode_steps_leg(kda, W, dev, dist, world, args):
     return {"workload": f"decode_steps_n{DEC_N}_l{STEPS_L}_h{DEC_H}_d{D}_pool{STEPS_POOL}",
             "value": job_value(DEC_N * STEPS_L, world, ms), "unit": UNIT, "ms_per_call": ms,
             "calls": calls, "l2": "pool (1 GiB) larger than L2; no flush",
-            "roofline": {"bound": "hbm", "kernel": "decode_steps_kernel", "achieved": ach,
+            "roofline": {"bound": "hbm", "kernel": "decode_pipe_kernel", "achieved": ach,
                          "peak": peak, "unit": "GB/s", "frac": ach / peak, "peak_source": kind,
                          "algorithmic_bytes_per_launch": STEPS_BYTES, "traffic": None}}
 

@@ -221,9 +221,9 @@ kda_status kda_recurrent_steps(const void *q, const void *k, const void *v, cons
     if (NH > 0x7fffffffLL || (long long)N * L * H > (1LL << 40))
         return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_steps: problem too large");
     if (NH == 0) return KDA_OK;
-    cudaError_t e = kda::launch_decode_steps(q, k, v, g, beta, state_pool, slots, num_slots, out,
-                                             N, H, L, dk, dv, dtype == KDA_BF16,
-                                             kda::error_word(), pro, (cudaStream_t)stream);
+    cudaError_t e = kda::launch_decode_pipe(q, k, v, g, beta, state_pool, slots, num_slots, out,
+                                            N, H, L, dk, dv, dtype == KDA_BF16,
+                                            kda::error_word(), pro, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_steps launch");
     return KDA_OK;
 }

@@ -20,12 +20,23 @@
 
 namespace kda {
 
+template <int LO, int HI, int W>
+__device__ __forceinline__ float tree_sum(const float (*red)[W], int col) {
+    if constexpr (HI - LO == 1) {
+        return red[LO][col];
+    } else {
+        constexpr int MID = (LO + HI) / 2;
+        return tree_sum<LO, MID>(red, col) + tree_sum<MID, HI>(red, col);
+    }
+}
+
 template <int DK, int DV, typename Tin, bool PRO>
 __global__ void __launch_bounds__(256, 2)
 decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                    const Tin *__restrict__ v, const float *__restrict__ g,
                    const float *__restrict__ beta, float *__restrict__ state,
-                   Tin *__restrict__ out, Prologue pro)
+                   const int32_t *__restrict__ slots, int num_slots, int H,
+                   Tin *__restrict__ out, int *__restrict__ err, Prologue pro)
 {
     constexpr int NT = 256;
     constexpr int C4 = DV / 4;       // float4 groups per row
@@ -37,6 +48,17 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     const int tid = threadIdx.x;
     const int c4 = tid % C4;
     const int rg = tid / C4;
+    // state entry: slots[n] of a [num_slots, H] pool, or nh itself
+    size_t sidx = nh;
+    if (slots) {
+        const int n = (int)(nh / H), h = (int)(nh - (size_t)n * H);
+        const int slot = slots[n];
+        if (slot < 0 || slot >= num_slots) {
+            if (tid == 0) set_device_error(err, kErrBadSlot);
+            return;
+        }
+        sidx = (size_t)slot * H + h;
+    }
 
     __shared__ float ks[DK], qs[DK], as_[DK];
     __shared__ __align__(16) float red_k[RG][DV + 4];
@@ -45,7 +67,7 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     __shared__ float qk_part[NT / 32], kk_part[NT / 32], qq_part[NT / 32];
 
     // 1. Issue every state load first (64 KiB in flight per CTA at d=128).
-    float4 *Sp = reinterpret_cast<float4 *>(state + nh * (size_t)(DK * DV));
+    float4 *Sp = reinterpret_cast<float4 *>(state + sidx * (size_t)(DK * DV));
     float4 s[RPT];
 #pragma unroll
     for (int r = 0; r < RPT; ++r) s[r] = ld_stream(Sp + (size_t)(rg * RPT + r) * C4 + c4);
@@ -96,8 +118,10 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         float kr = ks[row], qr = qs[row];
         if (PRO) { kr *= sk; qr *= sq; }
         s[r].x *= a; s[r].y *= a; s[r].z *= a; s[r].w *= a;
-        pk[0] += kr * s[r].x; pk[1] += kr * s[r].y; pk[2] += kr * s[r].z; pk[3] += kr * s[r].w;
-        pq[0] += qr * s[r].x; pq[1] += qr * s[r].y; pq[2] += qr * s[r].z; pq[3] += qr * s[r].w;
+        pk[0] = __fmaf_rn(kr, s[r].x, pk[0]); pk[1] = __fmaf_rn(kr, s[r].y, pk[1]);
+        pk[2] = __fmaf_rn(kr, s[r].z, pk[2]); pk[3] = __fmaf_rn(kr, s[r].w, pk[3]);
+        pq[0] = __fmaf_rn(qr, s[r].x, pq[0]); pq[1] = __fmaf_rn(qr, s[r].y, pq[1]);
+        pq[2] = __fmaf_rn(qr, s[r].z, pq[2]); pq[3] = __fmaf_rn(qr, s[r].w, pq[3]);
     }
     reinterpret_cast<float4 *>(&red_k[rg][0])[c4] = make_float4(pk[0], pk[1], pk[2], pk[3]);
     reinterpret_cast<float4 *>(&red_q[rg][0])[c4] = make_float4(pq[0], pq[1], pq[2], pq[3]);
@@ -105,9 +129,9 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
 
     // 4. Finish the column sums; u = beta (v - S'^T k); o = S'^T q + (q.k) u.
     if (tid < DV) {
-        float kS = 0.f, qS = 0.f;
-#pragma unroll
-        for (int i = 0; i < RG; ++i) { kS += red_k[i][tid]; qS += red_q[i][tid]; }
+        // row groups summed as a balanced tree in row-group order (the same
+        // order as the warp butterfly of the L-token kernel, decode_pipe.cu)
+        const float kS = tree_sum<0, RG>(red_k, tid), qS = tree_sum<0, RG>(red_q, tid);
         float qk_all = 0.f;
 #pragma unroll
         for (int w = 0; w < NT / 32; ++w) qk_all += qk_part[w];
@@ -118,7 +142,7 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         }
         const float u = b * (to_f(v[nh * DV + tid]) - kS);
         us[tid] = u;
-        out[nh * DV + tid] = from_f<Tin>(qS + qk_all * u);
+        out[nh * DV + tid] = from_f<Tin>(__fmaf_rn(qk_all, u, qS));
     }
     __syncthreads();
 
@@ -129,212 +153,40 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         float kr = ks[rg * RPT + r];
         if (PRO) kr *= sk;
         float4 o4 = s[r];
-        o4.x += kr * u4.x; o4.y += kr * u4.y; o4.z += kr * u4.z; o4.w += kr * u4.w;
+        o4.x = __fmaf_rn(kr, u4.x, o4.x); o4.y = __fmaf_rn(kr, u4.y, o4.y);
+        o4.z = __fmaf_rn(kr, u4.z, o4.z); o4.w = __fmaf_rn(kr, u4.w, o4.w);
         st_stream(Sp + (size_t)(rg * RPT + r) * C4 + c4, o4);
     }
-}
-
-// L tokens per sequence against a state pool indexed by slot: the state is
-// read once, the L steps run on it in registers (the same per-token arithmetic
-// as decode_step_kernel), and it is written once.  Token l of sequence n is
-// row (n * L + l) of the token arrays; sequence n uses pool entry slots[n]
-// (n when slots is null).  A slot outside [0, num_slots) skips the sequence
-// and sets the device error word.
-template <int DK, int DV, typename Tin, bool PRO>
-__global__ void __launch_bounds__(256, 2)
-decode_steps_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
-                    const Tin *__restrict__ v, const float *__restrict__ g,
-                    const float *__restrict__ beta, float *__restrict__ pool,
-                    const int32_t *__restrict__ slots, int num_slots, Tin *__restrict__ out,
-                    int H, int L, int *__restrict__ err, Prologue pro)
-{
-    constexpr int NT = 256;
-    constexpr int C4 = DV / 4;
-    constexpr int RG = NT / C4;
-    constexpr int RPT = DK / RG;
-    static_assert(NT % C4 == 0 && DK % RG == 0, "bad decode tiling");
-
-    const int n = blockIdx.x / H, h = blockIdx.x - n * H;
-    const int tid = threadIdx.x;
-    const int c4 = tid % C4;
-    const int rg = tid / C4;
-    const int slot = slots ? slots[n] : n;
-    if (slot < 0 || slot >= num_slots) {
-        if (tid == 0) set_device_error(err, kErrBadSlot);
-        return;
-    }
-
-    __shared__ float ks[DK], qs[DK], as_[DK];
-    __shared__ __align__(16) float red_k[RG][DV + 4];
-    __shared__ __align__(16) float red_q[RG][DV + 4];
-    __shared__ __align__(16) float us[DV];
-    __shared__ float qk_part[NT / 32], kk_part[NT / 32], qq_part[NT / 32];
-
-    float4 *Sp = reinterpret_cast<float4 *>(pool + ((size_t)slot * H + h) * (size_t)(DK * DV));
-    float4 s[RPT];
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) s[r] = ld_stream(Sp + (size_t)(rg * RPT + r) * C4 + c4);
-
-    // token inputs of step l + 1 are loaded into registers while step l runs
-    float kn = 0.f, qn = 0.f, gn = 0.f, vn = 0.f, bn = 0.f;
-    auto load_token = [&](int l) {
-        const size_t row = ((size_t)n * L + l) * H + h;
-        if (tid < DK) {
-            kn = to_f(k[row * DK + tid]);
-            qn = to_f(q[row * DK + tid]);
-            gn = g[row * DK + tid];
-        }
-        if (tid < DV) {
-            vn = to_f(v[row * DV + tid]);
-            bn = beta[row];
-        }
-    };
-    load_token(0);
-    for (int l = 0; l < L; ++l) {
-        const size_t row = ((size_t)n * L + l) * H + h;
-        if (l > 0) __syncthreads();   // the previous step's readers of ks, us, qk_part
-        float qk = 0.f, kk = 0.f, qq = 0.f;
-        if (tid < DK) {
-            ks[tid] = kn;
-            qs[tid] = qn;
-            as_[tid] = expf(gn);
-            qk = kn * qn;
-            if (PRO) { kk = kn * kn; qq = qn * qn; }
-        }
-        const float vcur = vn;
-        float bcur = bn;
-        if (PRO && (pro.flags & kProBetaSigmoid)) bcur = sigmoid_f(bcur);
-        if (l + 1 < L) load_token(l + 1);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            qk += __shfl_xor_sync(0xffffffffu, qk, o);
-            if (PRO) {
-                kk += __shfl_xor_sync(0xffffffffu, kk, o);
-                qq += __shfl_xor_sync(0xffffffffu, qq, o);
-            }
-        }
-        if ((tid & 31) == 0) {
-            qk_part[tid >> 5] = qk;
-            if (PRO) { kk_part[tid >> 5] = kk; qq_part[tid >> 5] = qq; }
-        }
-        __syncthreads();
-        float sk = 1.f, sq = 1.f;
-        if (PRO) {
-            if (pro.flags & kProQkL2Norm) {
-                float ka = 0.f, qa = 0.f;
-#pragma unroll
-                for (int w = 0; w < NT / 32; ++w) { ka += kk_part[w]; qa += qq_part[w]; }
-                sk = inv_norm(ka);
-                sq = inv_norm(qa);
-            }
-            sq *= pro.q_scale;
-        }
-
-        float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int r = 0; r < RPT; ++r) {
-            const int rr = rg * RPT + r;
-            const float a = as_[rr];
-            float kr = ks[rr], qr = qs[rr];
-            if (PRO) { kr *= sk; qr *= sq; }
-            s[r].x *= a; s[r].y *= a; s[r].z *= a; s[r].w *= a;
-            pk[0] += kr * s[r].x; pk[1] += kr * s[r].y; pk[2] += kr * s[r].z; pk[3] += kr * s[r].w;
-            pq[0] += qr * s[r].x; pq[1] += qr * s[r].y; pq[2] += qr * s[r].z; pq[3] += qr * s[r].w;
-        }
-        reinterpret_cast<float4 *>(&red_k[rg][0])[c4] = make_float4(pk[0], pk[1], pk[2], pk[3]);
-        reinterpret_cast<float4 *>(&red_q[rg][0])[c4] = make_float4(pq[0], pq[1], pq[2], pq[3]);
-        __syncthreads();
-
-        if (tid < DV) {
-            float kS = 0.f, qS = 0.f;
-#pragma unroll
-            for (int i = 0; i < RG; ++i) { kS += red_k[i][tid]; qS += red_q[i][tid]; }
-            float qk_all = 0.f;
-#pragma unroll
-            for (int w = 0; w < NT / 32; ++w) qk_all += qk_part[w];
-            if (PRO) qk_all *= sk * sq;
-            const float u = bcur * (vcur - kS);
-            us[tid] = u;
-            out[row * DV + tid] = from_f<Tin>(qS + qk_all * u);
-        }
-        __syncthreads();
-
-        const float4 u4 = reinterpret_cast<const float4 *>(us)[c4];
-#pragma unroll
-        for (int r = 0; r < RPT; ++r) {
-            float kr = ks[rg * RPT + r];
-            if (PRO) kr *= sk;
-            s[r].x += kr * u4.x; s[r].y += kr * u4.y; s[r].z += kr * u4.z; s[r].w += kr * u4.w;
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) st_stream(Sp + (size_t)(rg * RPT + r) * C4 + c4, s[r]);
-}
-
-template <int DK, int DV, typename Tin>
-static cudaError_t launch_steps_t(const void *q, const void *k, const void *v, const float *g,
-                                  const float *beta, float *pool, const int32_t *slots,
-                                  int num_slots, void *out, int N, int H, int L, int *err,
-                                  Prologue pro, cudaStream_t st)
-{
-    auto kern = (pro.flags != 0 || pro.q_scale != 1.f) ? decode_steps_kernel<DK, DV, Tin, true>
-                                                       : decode_steps_kernel<DK, DV, Tin, false>;
-    kern<<<N * H, 256, 0, st>>>((const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, pool,
-                                slots, num_slots, (Tin *)out, H, L, err, pro);
-    return cudaGetLastError();
-}
-
-template <typename Tin>
-static cudaError_t launch_steps_d(const void *q, const void *k, const void *v, const float *g,
-                                  const float *beta, float *pool, const int32_t *slots,
-                                  int num_slots, void *out, int N, int H, int L, int dk, int dv,
-                                  int *err, Prologue pro, cudaStream_t st)
-{
-#define KDA_STEPS(DK_, DV_)                                                                    \
-    if (dk == DK_ && dv == DV_)                                                                \
-        return launch_steps_t<DK_, DV_, Tin>(q, k, v, g, beta, pool, slots, num_slots, out, N, \
-                                             H, L, err, pro, st);
-    KDA_STEPS(128, 128)
-    KDA_STEPS(64, 64)
-    KDA_STEPS(128, 64)
-    KDA_STEPS(64, 128)
-#undef KDA_STEPS
-    return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_decode_steps(const void *q, const void *k, const void *v, const float *g,
-                                const float *beta, float *pool, const int32_t *slots,
-                                int num_slots, void *out, int N, int H, int L, int dk, int dv,
-                                bool bf16, int *err, Prologue pro, cudaStream_t st)
-{
-    if (bf16)
-        return launch_steps_d<__nv_bfloat16>(q, k, v, g, beta, pool, slots, num_slots, out, N, H,
-                                             L, dk, dv, err, pro, st);
-    return launch_steps_d<float>(q, k, v, g, beta, pool, slots, num_slots, out, N, H, L, dk, dv,
-                                 err, pro, st);
 }
 
 template <int DK, int DV, typename Tin>
 static cudaError_t launch_decode_t(const void *q, const void *k, const void *v,
                                    const float *g, const float *beta, float *state,
-                                   void *out, int NH, Prologue pro, cudaStream_t st)
+                                   const int32_t *slots, int num_slots, int H, void *out, int NH,
+                                   int *err, Prologue pro, cudaStream_t st)
 {
     auto kern = (pro.flags != 0 || pro.q_scale != 1.f) ? decode_step_kernel<DK, DV, Tin, true>
                                                        : decode_step_kernel<DK, DV, Tin, false>;
-    kern<<<NH, 256, 0, st>>>((const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, state,
-                             (Tin *)out, pro);
+    kern<<<NH, 256, 0, st>>>((const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, state, slots,
+                             num_slots, H, (Tin *)out, err, pro);
     return cudaGetLastError();
 }
 
 template <typename Tin>
 static cudaError_t launch_decode_d(const void *q, const void *k, const void *v,
                                    const float *g, const float *beta, float *state,
-                                   void *out, int NH, int dk, int dv, Prologue pro, cudaStream_t st)
+                                   const int32_t *slots, int num_slots, int H, void *out, int NH,
+                                   int dk, int dv, int *err, Prologue pro, cudaStream_t st)
 {
-    if (dk == 128 && dv == 128) return launch_decode_t<128, 128, Tin>(q, k, v, g, beta, state, out, NH, pro, st);
-    if (dk == 64 && dv == 64) return launch_decode_t<64, 64, Tin>(q, k, v, g, beta, state, out, NH, pro, st);
-    if (dk == 128 && dv == 64) return launch_decode_t<128, 64, Tin>(q, k, v, g, beta, state, out, NH, pro, st);
-    if (dk == 64 && dv == 128) return launch_decode_t<64, 128, Tin>(q, k, v, g, beta, state, out, NH, pro, st);
+#define KDA_STEP(DK_, DV_)                                                                       \
+    if (dk == DK_ && dv == DV_)                                                                  \
+        return launch_decode_t<DK_, DV_, Tin>(q, k, v, g, beta, state, slots, num_slots, H, out, \
+                                              NH, err, pro, st);
+    KDA_STEP(128, 128)
+    KDA_STEP(64, 64)
+    KDA_STEP(128, 64)
+    KDA_STEP(64, 128)
+#undef KDA_STEP
     return cudaErrorInvalidValue;
 }
 
@@ -342,8 +194,26 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const flo
                           const float *beta, float *state, void *out, int NH, int dk,
                           int dv, bool bf16, Prologue pro, cudaStream_t st)
 {
-    if (bf16) return launch_decode_d<__nv_bfloat16>(q, k, v, g, beta, state, out, NH, dk, dv, pro, st);
-    return launch_decode_d<float>(q, k, v, g, beta, state, out, NH, dk, dv, pro, st);
+    if (NH == 0) return cudaSuccess;
+    if (bf16)
+        return launch_decode_d<__nv_bfloat16>(q, k, v, g, beta, state, nullptr, 0, 1, out, NH, dk,
+                                              dv, nullptr, pro, st);
+    return launch_decode_d<float>(q, k, v, g, beta, state, nullptr, 0, 1, out, NH, dk, dv, nullptr,
+                                  pro, st);
+}
+
+cudaError_t launch_decode_slots(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, float *pool, const int32_t *slots,
+                                int num_slots, void *out, int N, int H, int dk, int dv, bool bf16,
+                                int *err, Prologue pro, cudaStream_t st)
+{
+    if (N == 0) return cudaSuccess;
+    // without slots, sequence n uses entry n: the plain layout
+    if (bf16)
+        return launch_decode_d<__nv_bfloat16>(q, k, v, g, beta, pool, slots, num_slots, H, out,
+                                              N * H, dk, dv, err, pro, st);
+    return launch_decode_d<float>(q, k, v, g, beta, pool, slots, num_slots, H, out, N * H, dk, dv,
+                                  err, pro, st);
 }
 
 }  // namespace kda

@@ -22,12 +22,24 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const flo
                           const float *beta, float *state, void *out, int NH, int dk,
                           int dv, bool bf16, Prologue pro, cudaStream_t st);
 
+// One decode token per sequence against a slot-indexed state pool
+// [num_slots, H, dk, dv] (decode_step_kernel): sequence n uses entry slots[n]
+// (n if null); a slot outside [0, num_slots) skips the sequence and sets the
+// device error word.
+cudaError_t launch_decode_slots(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, float *pool, const int32_t *slots,
+                                int num_slots, void *out, int N, int H, int dk, int dv, bool bf16,
+                                int *err, Prologue pro, cudaStream_t st);
+
 // L decode tokens per sequence against a slot-indexed state pool
 // [num_slots, H, dk, dv]; sequence n uses pool entry slots[n] (n if null).
-cudaError_t launch_decode_steps(const void *q, const void *k, const void *v, const float *g,
-                                const float *beta, float *pool, const int32_t *slots,
-                                int num_slots, void *out, int N, int H, int L, int dk, int dv,
-                                bool bf16, int *err, Prologue pro, cudaStream_t st);
+// A persistent pipelined kernel (decode_pipe.cu): the next item's state
+// arrives in shared memory while the current one is computed.  Per token the
+// arithmetic is launch_decode's, operation for operation.
+cudaError_t launch_decode_pipe(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, float *pool, const int32_t *slots, int num_slots,
+                               void *out, int N, int H, int L, int dk, int dv, bool bf16, int *err,
+                               Prologue pro, cudaStream_t st);
 
 // Gated RMSNorm over rows of dv (64 or 128): y = x rsqrt(mean(x^2) + eps) w sigmoid(z).
 cudaError_t launch_gated_rmsnorm(const void *x, const void *z, const float *w, float eps, void *y,

@@ -57,6 +57,8 @@ TRAFFIC = {
                 "sha": "7a31f985d99e3ace", "bytes": (342.313984 + 264.840448 + 304.188416 + 55.321856) * 1e6},
     "decode": {"files": ["decode.cu", "common.cuh"], "sha": "5538ff5eaafbaa61",
                "bytes": (547.416576 + 479.912448) * 1e6},
+    "decode_steps": {"files": ["decode_pipe.cu", "common.cuh", "sm100.cuh"], "sha": "",
+                     "bytes": 0.0},
 }
 
 
@@ -355,7 +357,8 @@ def decode_steps_leg(kda, W, dev, dist, world, args):
             "calls": calls, "l2": "pool (1 GiB) larger than L2; no flush",
             "roofline": {"bound": "hbm", "kernel": "decode_pipe_kernel", "achieved": ach,
                          "peak": peak, "unit": "GB/s", "frac": ach / peak, "peak_source": kind,
-                         "algorithmic_bytes_per_launch": STEPS_BYTES, "traffic": None}}
+                         "algorithmic_bytes_per_launch": STEPS_BYTES,
+                         "traffic": measured_traffic("decode_steps")}}
 
 
 def cpu_baseline(inp_cpu, tokens=None):

@@ -45,7 +45,15 @@ B, T, H, D = 1, 8192, 32, 128
 # the final fp32 state written once per (sequence, head))
 PREFILL_BYTES = B * T * H * (3 * D * 2 + D * 4 + 4 + D * 2) + B * H * D * D * 4
 DEC_N, DEC_H = 256, 32
-DECODE_BYTES = DEC_N * DEC_H * (2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 2)
+
+
+def decode_bytes(n):
+    """Algorithmic bytes of one decode step for n sequences: the fp32 state
+    read and written once, the token's q, k, v, out (bf16), g and beta (fp32)."""
+    return n * DEC_H * (2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 2)
+
+
+DECODE_BYTES = decode_bytes(DEC_N)
 FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
@@ -54,11 +62,11 @@ FALLBACK_HBM_GBS = 6650.0
 _SRC = os.path.join(ROOT, "gated_delta_rule_88_b200", "csrc")
 TRAFFIC = {
     "prefill": {"files": ["chunk_prep.cu", "chunk_chain_tc.cu", "chunk_ws.h", "sm100.cuh", "common.cuh"],
-                "sha": "7a31f985d99e3ace", "bytes": (342.313984 + 264.840448 + 304.188416 + 55.321856) * 1e6},
-    "decode": {"files": ["decode.cu", "common.cuh"], "sha": "5538ff5eaafbaa61",
-               "bytes": (547.416576 + 479.912448) * 1e6},
-    "decode_steps": {"files": ["decode_pipe.cu", "common.cuh", "sm100.cuh"], "sha": "",
-                     "bytes": 0.0},
+                "sha": "98ba6bde4155390f", "bytes": (342.247424 + 264.975872 + 304.209152 + 52.774912) * 1e6},
+    "decode": {"files": ["decode.cu", "common.cuh"], "sha": "4ceac309c0c18d2f",
+               "bytes": (547.408128 + 480.674560) * 1e6},
+    "decode_steps": {"files": ["decode_pipe.cu", "common.cuh", "sm100.cuh"], "sha": "dfd242f2df963f4b",
+                     "bytes": (621.427456 + 496.504320) * 1e6},
 }
 
 
@@ -289,11 +297,12 @@ def run_ours(args):
 
 
 def decode_leg(kda, W, dev, dist, world, args):
-    state = torch.empty(DEC_N, DEC_H, D, D, dtype=torch.float32, device=dev)
-    state.copy_(W.decode_initial_state())
+    n = args.decode_n
+    state = torch.empty(n, DEC_H, D, D, dtype=torch.float32, device=dev)
+    state.copy_(W.decode_initial_state(n))
     ring = 8
-    toks = [tuple(t.to(dev) for t in W.decode_tokens(i)) for i in range(ring)]
-    out = torch.empty(DEC_N, DEC_H, D, dtype=torch.bfloat16, device=dev)
+    toks = [tuple(t.to(dev) for t in W.decode_tokens(i, n)) for i in range(ring)]
+    out = torch.empty(n, DEC_H, D, dtype=torch.bfloat16, device=dev)
     steps = max(64, args.decode_steps)
     for i in range(max(3, args.warmup)):
         q, k, v, g, b = toks[i % ring]
@@ -309,35 +318,47 @@ def decode_leg(kda, W, dev, dist, world, args):
     barrier(dist)
     ms = max_over_ranks(e0.elapsed_time(e1), dist) / steps
     peak, kind = measured_peak_hbm()
-    ach = DECODE_BYTES / (ms * 1e-3) / 1e9
-    return {"workload": "decode_n256_h32_d128", "value": job_value(DEC_N, world, ms),
+    nbytes = decode_bytes(n)
+    ach = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": f"decode_n{n}_h{DEC_H}_d{D}", "value": job_value(n, world, ms),
             "unit": UNIT, "ms_per_step": ms, "steps": steps,
-            "l2": "state (512 MiB) larger than L2; no flush",
+            "l2": f"state ({n * DEC_H * D * D * 4 >> 20} MiB) larger than L2; no flush",
             "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": ach,
                          "peak": peak, "unit": "GB/s", "frac": ach / peak, "peak_source": kind,
-                         "algorithmic_bytes_per_launch": DECODE_BYTES,
-                         "traffic": measured_traffic("decode")}}
+                         "algorithmic_bytes_per_launch": nbytes,
+                         "traffic": measured_traffic("decode") if n == DEC_N else None}}
 
 
-STEPS_L, STEPS_POOL = 8, 2 * DEC_N
-STEPS_BYTES = DEC_N * DEC_H * (2 * D * D * 4 + STEPS_L * (3 * D * 2 + D * 4 + 4 + D * 2)) + DEC_N * 4
+STEPS_L = 8
+
+
+def steps_bytes(n):
+    """Algorithmic bytes of one serving-decode call: n pool states read and
+    written once, STEPS_L tokens' q, k, v, out (bf16), g, beta (fp32) per
+    (sequence, head), and the slot indices."""
+    return n * DEC_H * (2 * D * D * 4 + STEPS_L * (3 * D * 2 + D * 4 + 4 + D * 2)) + n * 4
+
+
+STEPS_BYTES = steps_bytes(DEC_N)
 
 
 def decode_steps_leg(kda, W, dev, dist, world, args):
     """Serving decode: 8 tokens per sequence per call (kda_recurrent_steps) for
-    the 256 x 32 decode batch, states in a pool of 512 entries picked by a
-    seeded slot permutation."""
-    pool = torch.empty(STEPS_POOL, DEC_H, D, D, dtype=torch.float32, device=dev)
-    pool.copy_(W.decode_initial_state(STEPS_POOL, DEC_H, D, D))
+    the n x 32 decode batch (n = 256 by default), states in a pool of 2n
+    entries picked by a seeded slot permutation."""
+    n = args.decode_n
+    pool_n = 2 * n
+    pool = torch.empty(pool_n, DEC_H, D, D, dtype=torch.float32, device=dev)
+    pool.copy_(W.decode_initial_state(pool_n, DEC_H, D, D))
     gen = torch.Generator().manual_seed(31)
-    slots = torch.randperm(STEPS_POOL, generator=gen)[:DEC_N].to(torch.int32).to(dev)
+    slots = torch.randperm(pool_n, generator=gen)[:n].to(torch.int32).to(dev)
     ring = 2
     toks = []
     for r in range(ring):
-        steps_r = [W.decode_tokens(r * STEPS_L + l) for l in range(STEPS_L)]
+        steps_r = [W.decode_tokens(r * STEPS_L + l, n) for l in range(STEPS_L)]
         toks.append(tuple(torch.stack([st[i] for st in steps_r], dim=1).contiguous().to(dev)
                           for i in range(5)))
-    out = torch.empty(DEC_N, STEPS_L, DEC_H, D, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(n, STEPS_L, DEC_H, D, dtype=torch.bfloat16, device=dev)
     calls = max(16, args.decode_steps // 16)
     for i in range(max(3, args.warmup)):
         kda.kda_recurrent_steps(*toks[i % ring], pool, slots, out=out)
@@ -351,14 +372,16 @@ def decode_steps_leg(kda, W, dev, dist, world, args):
     barrier(dist)
     ms = max_over_ranks(e0.elapsed_time(e1), dist) / calls
     peak, kind = measured_peak_hbm()
-    ach = STEPS_BYTES / (ms * 1e-3) / 1e9
-    return {"workload": f"decode_steps_n{DEC_N}_l{STEPS_L}_h{DEC_H}_d{D}_pool{STEPS_POOL}",
-            "value": job_value(DEC_N * STEPS_L, world, ms), "unit": UNIT, "ms_per_call": ms,
-            "calls": calls, "l2": "pool (1 GiB) larger than L2; no flush",
+    nbytes = steps_bytes(n)
+    ach = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": f"decode_steps_n{n}_l{STEPS_L}_h{DEC_H}_d{D}_pool{pool_n}",
+            "value": job_value(n * STEPS_L, world, ms), "unit": UNIT, "ms_per_call": ms,
+            "calls": calls,
+            "l2": f"pool ({pool_n * DEC_H * D * D * 4 >> 20} MiB) larger than L2; no flush",
             "roofline": {"bound": "hbm", "kernel": "decode_pipe_kernel", "achieved": ach,
                          "peak": peak, "unit": "GB/s", "frac": ach / peak, "peak_source": kind,
-                         "algorithmic_bytes_per_launch": STEPS_BYTES,
-                         "traffic": measured_traffic("decode_steps")}}
+                         "algorithmic_bytes_per_launch": nbytes,
+                         "traffic": measured_traffic("decode_steps") if n == DEC_N else None}}
 
 
 def cpu_baseline(inp_cpu, tokens=None):
@@ -418,6 +441,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-steps", type=int, default=1024)
+    ap.add_argument("--decode-n", type=int, default=DEC_N,
+                    help="sequences in the decode legs (a smaller case for profiling)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     args = ap.parse_args()
     if args.impl == "reference":

@@ -51,7 +51,7 @@ struct TcLayout {
     static constexpr uint32_t B2_OFF = B1_OFF + 128 * DVT * 2;     // V_new: K=64 x N=DVT, two buffers
     static constexpr uint32_t B2_BYTES = 64 * DVT * 2;
     static constexpr uint32_t BAR_OFF = B2_OFF + 2 * B2_BYTES;
-    static constexpr uint32_t BYTES = BAR_OFF + 8 * (2 * NS + 7) + 16;
+    static constexpr uint32_t BYTES = BAR_OFF + 8 * (2 * NS + 8) + 16;
     // TMEM columns: D1 double-buffered (2 x DVT) + D3 (DVT), rounded to a power of 2
     static constexpr uint32_t NCOLS = 3 * DVT <= 32 ? 32 : 3 * DVT <= 64 ? 64 : 3 * DVT <= 128 ? 128 : 256;
     static constexpr uint32_t B1_SBO = (128 / 8) * 128;             // n-group stride
@@ -79,10 +79,10 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
     uint64_t *empty = full + NS;
     uint64_t *mma1 = empty + NS;
     uint64_t *mma3 = mma1 + 1;
-    uint64_t *mma2 = mma1 + 2;
-    uint64_t *drain = mma1 + 3;                        // [2]: one per issuer
-    uint64_t *s_go = mma1 + 5;                         // [2]: MMA3(i) issued, by i & 1
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma1 + 7);
+    uint64_t *mma2 = mma1 + 2;                         // [2]: MMA2(i) done, by i & 1
+    uint64_t *drain = mma1 + 4;                        // [2]: one per issuer
+    uint64_t *s_go = mma1 + 6;                         // [2]: MMA3(i) issued, by i & 1
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma1 + 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     unsigned char *B1 = sm + L::B1_OFF;
     unsigned char *B2 = sm + L::B2_OFF;
@@ -115,8 +115,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
         for (int s = 0; s < NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 2); }
         mbar_init(mma1, 1);
         mbar_init(mma3, 1);
-        mbar_init(mma2, 1);
-        for (int b = 0; b < 2; ++b) { mbar_init(&drain[b], 1); mbar_init(&s_go[b], 1); }
+        for (int b = 0; b < 2; ++b) { mbar_init(&mma2[b], 1); mbar_init(&drain[b], 1); mbar_init(&s_go[b], 1); }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -203,7 +202,8 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
         if (warp == 6 && lane == 0) for (int i = 0; i < nchunks; ++i) {
             // MMA2: O rows (64-127 of D1[p]) += P V_new, once MMA3(i) is issued.
             // s_go[p] cannot run two phases ahead: MMA3(i + 2) needs the
-            // epilogue past emit(i), which waits for this MMA2.
+            // epilogue past emit(i) (after BAR_V(i + 1)), which waits for
+            // this MMA2.
             const int s = i % NS;
             const int p = i & 1;
             bool ok = false;
@@ -220,7 +220,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
             for (int kk = 0; kk < 4; ++kk)
                 umma_bf16_p(tmem + p * DVT, a_lo + (((uint32_t)ws::OFF_P - 8192 + kk * 32) >> 4),
                             a_sw.hi, b2_lo + ((kk * 256) >> 4), b2_d0.hi, IDESC, 1);
-            umma_commit(mma2);
+            umma_commit(&mma2[p]);
             umma_commit(&empty[s]);
             issued_any = true;
         }
@@ -263,10 +263,13 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
             }
             tmem_wait_ld();
         };
-        // O of chunk ci (rows 64-127 of D1[ci & 1]) -> out; warps 2-3 only
+        // O of chunk ci (rows 64-127 of D1[ci & 1]) -> out; warps 2-3 only,
+        // between BAR_S and BAR_V of chunk ci + 1.  One barrier per D1
+        // buffer: MMA2(ci + 2) needs BAR_V(ci + 2), which needs this call, so
+        // each wait is at most one phase behind.
         auto emit_output = [&](int ci) -> bool {
             bool okk = true;
-            if (t == 64) okk = mbar_wait(mma2, ci & 1);
+            if (t == 64) okk = mbar_wait(&mma2[ci & 1], (ci >> 1) & 1);
             if (named_bar_or(BAR_O, 64, !okk)) return false;
             tc_fence_after();
             const long long tok = bos + (long long)C * ci + (t - 64);
@@ -303,11 +306,13 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
                     u[c / 2] = x.x; u[c / 2 + 1] = x.y; u[c / 2 + 2] = x.z; u[c / 2 + 3] = x.w;
                 }
             }
-            if (ok) ok = mbar_wait(mma1, i & 1);
-            tc_fence_after();
-            // the previous chunk's output leaves through warps 2-3
-            if (t >= 64 && i > 0 && !emit_output(i - 1)) ok = false;
-            if (t < 64) {
+            if (t >= 64) {
+                // the previous chunk's output leaves through warps 2-3 while
+                // MMA1 runs and warps 0-1 form V_new (off the sequential path)
+                if (i > 0 && !emit_output(i - 1)) ok = false;
+            } else {
+                if (ok) ok = mbar_wait(mma1, i & 1);
+                tc_fence_after();
                 // V_new = U - W S for token row t
                 float x[DVT];
                 tmem_row(p * DVT, x);

@@ -32,7 +32,7 @@ __all__ = ["kda_chunk_fwd", "kda_chunk_fwd_ex", "kda_chunk_fwd_host", "kda_recur
            "kda_recurrent_step_ex", "kda_recurrent_steps", "kda_gated_rmsnorm", "kda_state_affine",
            "kda_get_device_error",
            "KDAError",
-           "KDA_QK_L2NORM", "KDA_BETA_SIGMOID",
+           "KDA_QK_L2NORM", "KDA_BETA_SIGMOID", "KDA_STEPS_CHUNK",
            "library_path", "load_library"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -42,6 +42,7 @@ _lock = threading.Lock()
 
 KDA_F32, KDA_BF16 = 0, 1
 KDA_QK_L2NORM, KDA_BETA_SIGMOID = 1, 2     # input prologue flags (the *_ex calls)
+KDA_STEPS_CHUNK = 4                        # kda_recurrent_steps: chunk form on tensor cores
 _STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
            3: "KDA_ERR_CUDA", 4: "KDA_ERR_DEVICE"}
 

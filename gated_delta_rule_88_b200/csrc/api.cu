@@ -195,7 +195,9 @@ kda_status kda_recurrent_steps(const void *q, const void *k, const void *v, cons
                                kda_dtype dtype, unsigned flags, float q_scale, void *stream) {
     t_msg[0] = 0;
     kda::Prologue pro;
-    kda_status pst = make_prologue("kda_recurrent_steps", flags, q_scale, &pro);
+    const bool chunk = (flags & KDA_STEPS_CHUNK) != 0;
+    kda_status pst = make_prologue("kda_recurrent_steps", flags & ~(unsigned)KDA_STEPS_CHUNK,
+                                   q_scale, &pro);
     if (pst != KDA_OK) return pst;
     if (!q || !k || !v || !g || !beta || !state_pool || !out)
         return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_steps: null pointer argument");
@@ -221,9 +223,13 @@ kda_status kda_recurrent_steps(const void *q, const void *k, const void *v, cons
     if (NH > 0x7fffffffLL || (long long)N * L * H > (1LL << 40))
         return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_steps: problem too large");
     if (NH == 0) return KDA_OK;
-    cudaError_t e = kda::launch_decode_pipe(q, k, v, g, beta, state_pool, slots, num_slots, out,
-                                            N, H, L, dk, dv, dtype == KDA_BF16,
-                                            kda::error_word(), pro, (cudaStream_t)stream);
+    const bool tc = chunk && L >= 2 && dtype == KDA_BF16 && dk == 128 && dv == 128 &&
+                    pro.flags == 0 && pro.q_scale == 1.f;
+    cudaError_t e = tc ? kda::launch_decode_chunk(q, k, v, g, beta, state_pool, slots, num_slots,
+                                                  out, N, H, L, kda::error_word(), (cudaStream_t)stream)
+                       : kda::launch_decode_pipe(q, k, v, g, beta, state_pool, slots, num_slots, out,
+                                                 N, H, L, dk, dv, dtype == KDA_BF16,
+                                                 kda::error_word(), pro, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_steps launch");
     return KDA_OK;
 }

@@ -1,0 +1,368 @@
+// decode_chunk.cu -- the L-token KDA decode on a slot-indexed state pool in
+// the chunk form, on tensor cores (bf16 operands, fp32 accumulation and
+// state), dk = dv = 128.
+//
+// Kimi Linear paper notes (paper-notes-site): section 2 gives the recurrence,
+// section 3 the chunkwise form (a WY-like representation of a chunk's
+// writes, then one product with the fixed-size state).  For a block of up
+// to 16 tokens of one (sequence, head), with G the block-local inclusive
+// cumsum of g:
+//     A_ij = beta_i sum_c k_ic k_jc e^{G_ic - G_jc}  (j < i)
+//     P_ij =        sum_c q_ic k_jc e^{G_ic - G_jc}  (j <= i)
+//     T = (I + A)^-1,  W = T (beta K e^G),  U = T (beta V)
+//     V_new = U - W S;  O = (Q e^G) S + P V_new
+//     S <- Diag(e^{G_last}) S + (K e^{G_last - G})^T V_new
+// The same algebra as the chunked prefill; here the block is at most 16
+// tokens, so A and P are formed directly from e^{G_i - G_j} <= 1 in fp32
+// (exact exponentials, no factorisation): any finite g <= 0 is accepted.
+//
+// One CTA (256 threads, 8 warps) per (sequence, head), two CTAs per SM.  The
+// fp32 state lives in registers in the m16n8k16 accumulator layout (warp w:
+// channel rows 16w .. 16w + 15, all 128 columns), so the state update is one
+// tensor-core accumulate into it; its bf16 copy in shared memory is the B
+// operand of W S and (Q e^G) S.  Rounding: the MMA operands (S, V_new, T, P
+// and the decayed forms) are bf16, as in the prefill.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace kda {
+namespace {
+
+constexpr int NT = 256;
+constexpr int D = 128;
+constexpr int BT = 16;                       // tokens per block (one MMA row tile)
+constexpr float LOG2E = 1.4426950408889634f;
+
+// 16 or 128 rows x 128 bf16, 256-byte rows, 16-byte chunk j of row r at j ^ (r & 7)
+__device__ __forceinline__ int toff(int r, int c) {
+    return r * 256 + ((((c >> 3) ^ (r & 7))) << 4) + ((c & 7) << 1);
+}
+__device__ __forceinline__ int toff_chunk(int r, int j) { return r * 256 + (((j ^ (r & 7))) << 4); }
+
+// shared-memory layout (bytes)
+constexpr int OFF_RQ = 0;                    // raw q [16][128] bf16, 256-byte rows
+constexpr int OFF_RK = OFF_RQ + 4096;
+constexpr int OFF_RV = OFF_RK + 4096;
+constexpr int OFF_G = OFF_RV + 4096;         // g, then log2e * cumsum, fp32 [16][128]
+constexpr int OFF_BETA = OFF_G + 8192;       // [16] fp32 (128 bytes reserved)
+constexpr int OFF_QG = OFF_BETA + 128;       // forms: [16][128] bf16, toff layout
+constexpr int OFF_KG = OFF_QG + 4096;        // beta k e^G
+constexpr int OFF_KT = OFF_KG + 4096;        // k e^{G_last - G}
+constexpr int OFF_BV = OFF_KT + 4096;        // beta v
+constexpr int OFF_W = OFF_BV + 4096;         // W = T (beta k e^G)
+constexpr int OFF_VN = OFF_W + 4096;         // V_new
+constexpr int OFF_SB = OFF_VN + 4096;        // state copy [128][128] bf16, toff layout
+constexpr int OFF_AM = OFF_SB + 32768;       // A, P, T: fp32 [16][16]
+constexpr int OFF_PM = OFF_AM + 1024;
+constexpr int OFF_TM = OFF_PM + 1024;
+constexpr int OFF_GAM = OFF_TM + 1024;       // e^{G_last} per channel, fp32 [128]
+constexpr int SMEM = OFF_GAM + 512;
+static_assert(OFF_QG % 16 == 0 && OFF_SB % 16 == 0 && SMEM <= 100 * 1024, "layout");
+
+__device__ __forceinline__ void cp_async16_zfill(void *smem_dst, const void *gmem_src, bool ok) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem_dst)),
+                 "l"(gmem_src), "r"(ok ? 16 : 0));
+}
+
+// A fragment (rows gid / gid + 8, k pairs) of a 16 x 16 fp32 matrix in shared memory
+__device__ __forceinline__ void frag16(uint32_t (&a)[4], const float *M, int gid, int tig) {
+    const float2 x0 = *reinterpret_cast<const float2 *>(M + gid * 16 + 2 * tig);
+    const float2 x1 = *reinterpret_cast<const float2 *>(M + (gid + 8) * 16 + 2 * tig);
+    const float2 x2 = *reinterpret_cast<const float2 *>(M + gid * 16 + 2 * tig + 8);
+    const float2 x3 = *reinterpret_cast<const float2 *>(M + (gid + 8) * 16 + 2 * tig + 8);
+    a[0] = pack_bf16(x0.x, x0.y);
+    a[1] = pack_bf16(x1.x, x1.y);
+    a[2] = pack_bf16(x2.x, x2.y);
+    a[3] = pack_bf16(x3.x, x3.y);
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(NT, 2)
+decode_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                    const __nv_bfloat16 *__restrict__ v, const float *__restrict__ g,
+                    const float *__restrict__ beta, float *__restrict__ pool,
+                    const int32_t *__restrict__ slots, int num_slots,
+                    __nv_bfloat16 *__restrict__ out, int H, int L, int *__restrict__ err)
+{
+    extern __shared__ __align__(128) unsigned char sm[];
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int n = blockIdx.x / H, h = blockIdx.x - n * H;
+    const int slot = slots ? slots[n] : n;
+    if (slot < 0 || slot >= num_slots) {
+        if (tid == 0) set_device_error(err, kErrBadSlot);
+        return;
+    }
+    float *Gs = reinterpret_cast<float *>(sm + OFF_G);
+    float *bs = reinterpret_cast<float *>(sm + OFF_BETA);
+    float *Am = reinterpret_cast<float *>(sm + OFF_AM);
+    float *Pm = reinterpret_cast<float *>(sm + OFF_PM);
+    float *Tm = reinterpret_cast<float *>(sm + OFF_TM);
+    float *gam = reinterpret_cast<float *>(sm + OFF_GAM);
+    const int nblk = (L + BT - 1) / BT;
+    auto token_row = [&](int l) -> size_t { return ((size_t)n * L + l) * H + h; };
+
+    // raw rows of block b (zero past the last token), one cp.async group
+    auto issue_raw = [&](int b) {
+        const int l0 = b * BT, nt = min(BT, L - l0);
+        for (int c = tid; c < BT * 80; c += NT) {
+            const int i = c / 80, r = c - i * 80;
+            const bool ok = i < nt;
+            const size_t row = token_row(ok ? l0 + i : l0);
+            if (r < 48) {
+                const int vec = r >> 4, j = r & 15;
+                const __nv_bfloat16 *src = (vec == 0 ? q : vec == 1 ? k : v) + row * D + j * 8;
+                cp_async16_zfill(sm + OFF_RQ + vec * 4096 + i * 256 + j * 16, src, ok);
+            } else {
+                const int j = r - 48;
+                cp_async16_zfill(sm + OFF_G + i * 512 + j * 16, g + row * D + j * 4, ok);
+            }
+        }
+        if (tid < BT) bs[tid] = tid < nt ? beta[token_row(l0 + tid)] : 0.f;
+        cp_async_commit();
+    };
+
+    // the state, fp32, in the accumulator layout: s[j] = rows (16w + gid,
+    // 16w + gid + 8) x columns (8j + 2tig, + 1)
+    float *Sg = pool + ((size_t)slot * H + h) * (size_t)(D * D);
+    const int r0 = 16 * w + gid, r1 = r0 + 8;
+    float s[16][4];
+    issue_raw(0);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const float2 x = __ldcs(reinterpret_cast<const float2 *>(Sg + (size_t)r0 * D + 8 * j + 2 * tig));
+        const float2 y = __ldcs(reinterpret_cast<const float2 *>(Sg + (size_t)r1 * D + 8 * j + 2 * tig));
+        s[j][0] = x.x; s[j][1] = x.y; s[j][2] = y.x; s[j][3] = y.y;
+    }
+    auto write_sb = [&]() {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            *reinterpret_cast<uint32_t *>(sm + OFF_SB + toff(r0, 8 * j + 2 * tig)) = pack_bf16(s[j][0], s[j][1]);
+            *reinterpret_cast<uint32_t *>(sm + OFF_SB + toff(r1, 8 * j + 2 * tig)) = pack_bf16(s[j][2], s[j][3]);
+        }
+    };
+    write_sb();
+
+    for (int b = 0; b < nblk; ++b) {
+        const int l0 = b * BT, nt = min(BT, L - l0);
+        cp_async_wait<0>();
+        __syncthreads();                       // raw rows of block b landed; S copy written
+
+        // 1. per channel: log2e-scaled inclusive cumsum of g (in place), the
+        //    block decay; meanwhile the other threads clear A and P
+        if (tid < D) {
+            float acc = 0.f;
+#pragma unroll
+            for (int i = 0; i < BT; ++i) {
+                acc = fmaf(Gs[i * D + tid], LOG2E, acc);
+                Gs[i * D + tid] = acc;
+            }
+            gam[tid] = exp2f(acc);
+        } else {
+            for (int e = tid - D; e < 512; e += NT - D) (e < 256 ? Am : Pm)[e & 255] = 0.f;
+        }
+        __syncthreads();
+
+        // 2. decayed forms (thread: token i, channel pair), A and P
+        for (int it = tid; it < BT * 64; it += NT) {
+            const int i = it >> 6, c = 2 * (it & 63);
+            const float2 gi = *reinterpret_cast<const float2 *>(Gs + i * D + c);
+            const float2 gl = *reinterpret_cast<const float2 *>(Gs + (BT - 1) * D + c);
+            const float ex = exp2f(gi.x), ey = exp2f(gi.y);
+            const float tx = exp2f(gl.x - gi.x), ty = exp2f(gl.y - gi.y);
+            const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(sm + OFF_RQ + i * 256 + 2 * c);
+            const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(sm + OFF_RK + i * 256 + 2 * c);
+            const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162 *>(sm + OFF_RV + i * 256 + 2 * c);
+            const float b_ = bs[i];
+            const float qx = __low2float(q2), qy = __high2float(q2);
+            const float kx = __low2float(k2), ky = __high2float(k2);
+            const int o = toff(i, c);
+            *reinterpret_cast<uint32_t *>(sm + OFF_QG + o) = pack_bf16(qx * ex, qy * ey);
+            *reinterpret_cast<uint32_t *>(sm + OFF_KG + o) = pack_bf16(b_ * kx * ex, b_ * ky * ey);
+            *reinterpret_cast<uint32_t *>(sm + OFF_KT + o) = pack_bf16(kx * tx, ky * ty);
+            *reinterpret_cast<uint32_t *>(sm + OFF_BV + o) =
+                pack_bf16(b_ * __low2float(v2), b_ * __high2float(v2));
+        }
+        {
+            // pairs j <= i < nt, eight slices each; slice sl of pair p takes
+            // channel pairs 2 sl + 16 m (m = 0..7), visited from a per-pair
+            // rotation so that the four pairs of a warp read different banks.
+            // The slices of a pair sit in eight consecutive lanes and meet by
+            // shuffles.
+            const int npairs = nt * (nt + 1) / 2;
+            for (int base = 0; base < npairs * 8; base += NT) {
+                const int it = base + tid;
+                const bool valid = it < npairs * 8;
+                const int p = valid ? it >> 3 : 0, sl = it & 7;
+                int i = 0;
+                while ((i + 1) * (i + 2) / 2 <= p) ++i;
+                const int j = p - i * (i + 1) / 2;
+                float a = 0.f, pp = 0.f;
+                if (valid) {
+                    const float *gi = Gs + i * D, *gj = Gs + j * D;
+                    const unsigned char *qi = sm + OFF_RQ + i * 256, *ki = sm + OFF_RK + i * 256;
+                    const unsigned char *kj = sm + OFF_RK + j * 256;
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) {
+                        const int c = 16 * ((m + p) & 7) + 2 * sl;
+                        const float2 x = *reinterpret_cast<const float2 *>(gi + c);
+                        const float2 y = *reinterpret_cast<const float2 *>(gj + c);
+                        const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(qi + 2 * c);
+                        const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(ki + 2 * c);
+                        const __nv_bfloat162 l2 = *reinterpret_cast<const __nv_bfloat162 *>(kj + 2 * c);
+                        const float e0 = exp2f(x.x - y.x), e1 = exp2f(x.y - y.y);
+                        const float kj0 = __low2float(l2), kj1 = __high2float(l2);
+                        a = fmaf(__low2float(k2) * kj0, e0, a);
+                        a = fmaf(__high2float(k2) * kj1, e1, a);
+                        pp = fmaf(__low2float(q2) * kj0, e0, pp);
+                        pp = fmaf(__high2float(q2) * kj1, e1, pp);
+                    }
+                }
+#pragma unroll
+                for (int o = 1; o < 8; o <<= 1) {
+                    a += __shfl_xor_sync(0xffffffffu, a, o);
+                    pp += __shfl_xor_sync(0xffffffffu, pp, o);
+                }
+                if (valid && sl == 0) {
+                    if (j < i) Am[i * 16 + j] = bs[i] * a;
+                    Pm[i * 16 + j] = pp;
+                }
+            }
+        }
+        __syncthreads();
+        // the raw rows are dead: the next block's arrive while this one runs
+        if (b + 1 < nblk) issue_raw(b + 1);
+
+        // 3. T = (I + A)^-1 by forward substitution, one column per thread
+        if (tid < BT) {
+            float x[BT];
+#pragma unroll
+            for (int i = 0; i < BT; ++i) {
+                float acc = 0.f;
+#pragma unroll
+                for (int j = 0; j < i; ++j) acc = fmaf(Am[i * 16 + j], x[j], acc);
+                x[i] = (i < tid) ? 0.f : (i == tid) ? 1.f : -acc;
+            }
+#pragma unroll
+            for (int i = 0; i < BT; ++i) Tm[i * 16 + tid] = x[i];
+        }
+        __syncthreads();
+
+        // 4. W = T (beta k e^G) (channel tiles 2w, 2w + 1) and U = T (beta v)
+        //    (value tiles 2w, 2w + 1; kept in registers)
+        const int kr = (lane & 7) + 8 * ((lane >> 3) & 1);
+        float u[2][4] = {}, wm[2][4] = {};
+        {
+            uint32_t ta[4], bf[4];
+            frag16(ta, Tm, gid, tig);
+            ldsm_x4_t(bf, sm + OFF_KG + toff_chunk(kr, 2 * w + (lane >> 4)));
+            mma_bf16(wm[0], ta, bf[0], bf[1]);
+            mma_bf16(wm[1], ta, bf[2], bf[3]);
+            ldsm_x4_t(bf, sm + OFF_BV + toff_chunk(kr, 2 * w + (lane >> 4)));
+            mma_bf16(u[0], ta, bf[0], bf[1]);
+            mma_bf16(u[1], ta, bf[2], bf[3]);
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int c = 16 * w + 8 * jj + 2 * tig;
+                *reinterpret_cast<uint32_t *>(sm + OFF_W + toff(gid, c)) = pack_bf16(wm[jj][0], wm[jj][1]);
+                *reinterpret_cast<uint32_t *>(sm + OFF_W + toff(gid + 8, c)) = pack_bf16(wm[jj][2], wm[jj][3]);
+            }
+        }
+        __syncthreads();
+
+        // 5. W S and (q e^G) S for value tiles 2w, 2w + 1; V_new = U - W S
+        float ws[2][4] = {}, os[2][4] = {};
+        {
+            const int ar = (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                uint32_t aw[4], aq[4], bf[4];
+                ldsm_x4_t(bf, sm + OFF_SB + toff_chunk(16 * ks + kr, 2 * w + (lane >> 4)));
+                ldsm_x4(aw, sm + OFF_W + toff_chunk(ar, 2 * ks + (lane >> 4)));
+                ldsm_x4(aq, sm + OFF_QG + toff_chunk(ar, 2 * ks + (lane >> 4)));
+                mma_bf16(ws[0], aw, bf[0], bf[1]);
+                mma_bf16(ws[1], aw, bf[2], bf[3]);
+                mma_bf16(os[0], aq, bf[0], bf[1]);
+                mma_bf16(os[1], aq, bf[2], bf[3]);
+            }
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int c = 16 * w + 8 * jj + 2 * tig;
+                *reinterpret_cast<uint32_t *>(sm + OFF_VN + toff(gid, c)) =
+                    pack_bf16(u[jj][0] - ws[jj][0], u[jj][1] - ws[jj][1]);
+                *reinterpret_cast<uint32_t *>(sm + OFF_VN + toff(gid + 8, c)) =
+                    pack_bf16(u[jj][2] - ws[jj][2], u[jj][3] - ws[jj][3]);
+            }
+        }
+        __syncthreads();
+
+        // 6. O = (q e^G) S + P V_new for value tiles 2w, 2w + 1
+        {
+            uint32_t pa[4], bf[4];
+            frag16(pa, Pm, gid, tig);
+            ldsm_x4_t(bf, sm + OFF_VN + toff_chunk(kr, 2 * w + (lane >> 4)));
+            mma_bf16(os[0], pa, bf[0], bf[1]);
+            mma_bf16(os[1], pa, bf[2], bf[3]);
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int c = 16 * w + 8 * jj + 2 * tig;
+                if (gid < nt)
+                    *reinterpret_cast<uint32_t *>(out + token_row(l0 + gid) * D + c) = pack_bf16(os[jj][0], os[jj][1]);
+                if (gid + 8 < nt)
+                    *reinterpret_cast<uint32_t *>(out + token_row(l0 + gid + 8) * D + c) = pack_bf16(os[jj][2], os[jj][3]);
+            }
+        }
+
+        // 7. S <- Diag(e^{G_last}) S + (k e^{G_last - G})^T V_new: channel rows
+        //    16w .. 16w + 15, all value tiles, accumulated into the registers
+        {
+            const float g0 = gam[r0], g1 = gam[r1];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                s[j][0] *= g0; s[j][1] *= g0; s[j][2] *= g1; s[j][3] *= g1;
+            }
+            uint32_t ka[4];
+            ldsm_x4_t(ka, sm + OFF_KT + toff_chunk((lane & 7) + 8 * (lane >> 4), 2 * w + ((lane >> 3) & 1)));
+#pragma unroll
+            for (int np = 0; np < 8; ++np) {
+                uint32_t bf[4];
+                ldsm_x4_t(bf, sm + OFF_VN + toff_chunk(kr, 2 * np + (lane >> 4)));
+                mma_bf16(s[2 * np], ka, bf[0], bf[1]);
+                mma_bf16(s[2 * np + 1], ka, bf[2], bf[3]);
+            }
+        }
+        // every warp has finished reading the old copy (step 5 precedes the
+        // barrier after V_new); write the new one for the next block
+        if (b + 1 < nblk) write_sb();
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        __stcs(reinterpret_cast<float2 *>(Sg + (size_t)r0 * D + 8 * j + 2 * tig), make_float2(s[j][0], s[j][1]));
+        __stcs(reinterpret_cast<float2 *>(Sg + (size_t)r1 * D + 8 * j + 2 * tig), make_float2(s[j][2], s[j][3]));
+    }
+}
+
+cudaError_t launch_decode_chunk(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, float *pool, const int32_t *slots,
+                                int num_slots, void *out, int N, int H, int L, int *err,
+                                cudaStream_t st)
+{
+    if (N == 0 || L == 0) return cudaSuccess;
+    static bool attr_done[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_done[dev]) {
+        e = cudaFuncSetAttribute(decode_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+        if (e != cudaSuccess) return e;
+        attr_done[dev] = true;
+    }
+    decode_chunk_kernel<<<N * H, NT, SMEM, st>>>(
+        (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, g, beta, pool,
+        slots, num_slots, (__nv_bfloat16 *)out, H, L, err);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

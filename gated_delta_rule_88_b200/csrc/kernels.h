@@ -41,6 +41,13 @@ cudaError_t launch_decode_pipe(const void *q, const void *k, const void *v, cons
                                void *out, int N, int H, int L, int dk, int dv, bool bf16, int *err,
                                Prologue pro, cudaStream_t st);
 
+// The same call in the chunk form on tensor cores (decode_chunk.cu): bf16,
+// dk = dv = 128, blocks of 16 tokens; bf16 operand rounding as in the prefill.
+cudaError_t launch_decode_chunk(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, float *pool, const int32_t *slots,
+                                int num_slots, void *out, int N, int H, int L, int *err,
+                                cudaStream_t st);
+
 // Gated RMSNorm over rows of dv (64 or 128): y = x rsqrt(mean(x^2) + eps) w sigmoid(z).
 cudaError_t launch_gated_rmsnorm(const void *x, const void *z, const float *w, float eps, void *y,
                                  long long rows, int dv, bool bf16, cudaStream_t st);

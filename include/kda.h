@@ -76,6 +76,9 @@ typedef enum {
  * and is not offered.
  */
 enum { KDA_QK_L2NORM = 1, KDA_BETA_SIGMOID = 2 };
+/* kda_recurrent_steps only: compute the L tokens in the chunk form on tensor
+ * cores (see kda_recurrent_steps). */
+enum { KDA_STEPS_CHUNK = 4 };
 
 /*
  * kda_chunk_fwd -- prefill forward over whole sequences.
@@ -225,6 +228,17 @@ kda_status kda_recurrent_step_ex(const void *q, const void *k, const void *v,
  * Supported: dk, dv in {64, 128}, dtype KDA_BF16 or KDA_F32.  Any finite g.
  * Aliasing: out must not overlap any input; the pool must not overlap the
  *   token inputs.
+ */
+/*
+ * KDA_STEPS_CHUNK in flags selects, for dtype KDA_BF16 with dk = dv = 128,
+ * L >= 2 and no prologue flags (q_scale = 1), the chunk form of the same L
+ * steps (section 3 of the notes: a WY-like representation of the block's
+ * writes, then one product with the state) in blocks of 16 tokens on tensor
+ * cores: the operands of the state products (state, V_new, T, P and the
+ * decayed k, q) are rounded to bf16 as in kda_chunk_fwd, the state stays
+ * fp32.  It needs e^{16 g} finite in fp32 for positive g (any g <= 5; gates
+ * are normally <= 0).  Other combinations run the recurrent kernel, which is
+ * bitwise equal to L calls of kda_recurrent_step.
  */
 kda_status kda_recurrent_steps(const void *q, const void *k, const void *v,
                                const float *g, const float *beta,

@@ -150,8 +150,8 @@ def host(lib, *, q=FAKE, k=FAKE, v=FAKE, g=FAKE, b=FAKE, s0=None, out=FAKE, sT=N
                                   dk, dv, dtype, rt, None)
 
 
-@pytest.mark.parametrize("kw", [dict(flags=8), dict(flags=0xFFFFFFFF), dict(q_scale=float("nan")),
-                                dict(q_scale=float("-inf"))])
+@pytest.mark.parametrize("kw", [dict(flags=8), dict(flags=4), dict(flags=0xFFFFFFFF),
+                                dict(q_scale=float("nan")), dict(q_scale=float("-inf"))])
 def test_ex_prologue_arguments_rejected(lib, kw):
     P = ctypes.c_void_p
     flags, q_scale = kw.get("flags", 1), kw.get("q_scale", 1.0)

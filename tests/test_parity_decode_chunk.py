@@ -1,0 +1,119 @@
+"""GPU parity: kda_recurrent_steps with KDA_STEPS_CHUNK (the chunk form of
+the L tokens on tensor cores, blocks of 16 tokens) vs the fp64 oracle.
+
+Kimi Linear paper notes, section 3: the chunkwise form gathers a block's
+writes in a WY-like representation and touches the state with one product;
+the result is the recurrence's.  Tolerance: the bf16 bound of the other
+parity tests (the state-product operands are bf16, as in the prefill).
+Lengths cover one partial block (2, 8), a full block (16), a block plus one
+token (17) and several blocks (40, 64); gates cover the decode workload's
+and a stronger, channel-dependent decay.
+"""
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_88_b200 import (KDA_STEPS_CHUNK, kda_get_device_error, kda_recurrent_steps)
+from gated_delta_rule_88_b200 import workloads as W
+from helpers import assert_close, rel_inf
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+BF = torch.bfloat16
+
+
+def _tokens(N, L, H, d, seed, gate="softplus8"):
+    steps = [W.decode_tokens(l, N, H, d, d, BF, seed=seed, gate=gate) for l in range(L)]
+    return [torch.stack([s[i] for s in steps], dim=1).contiguous() for i in range(5)]
+
+
+def _run(N, L, H, pool_n, seed, gate="softplus8", slots=True):
+    d = 128
+    pool0 = W.decode_initial_state(pool_n, H, d, d, seed=seed, std=0.02)
+    gen = torch.Generator().manual_seed(seed + 1)
+    sl = torch.randperm(pool_n, generator=gen)[:N].to(torch.int32) if slots else None
+    q, k, v, g, b = _tokens(N, L, H, d, seed, gate)
+    pool = pool0.to(DEV)
+    out = kda_recurrent_steps(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), b.to(DEV), pool,
+                              None if sl is None else sl.to(DEV), flags=KDA_STEPS_CHUNK)
+    torch.cuda.synchronize()
+    assert kda_get_device_error() == 0
+    idx = sl.long() if sl is not None else torch.arange(N)
+    o_ref, s_ref = oracle.forward(q, k, v, g, b, initial_state=pool0[idx].double())
+    return pool0, pool, idx, out, o_ref, s_ref, (q, k, v, g, b), sl
+
+
+@pytest.mark.parametrize("L", [2, 8, 16, 17, 40, 64])
+def test_chunk_steps_vs_oracle(L):
+    pool0, pool, idx, out, o_ref, s_ref, _, _ = _run(N=5, L=L, H=3, pool_n=9, seed=90 + L)
+    assert_close(out, o_ref, BF, "o")
+    for n in range(idx.numel()):
+        assert_close(pool[idx[n]], s_ref[n], BF, f"state {n}")
+    rest = torch.ones(pool0.shape[0], dtype=torch.bool)
+    rest[idx] = False
+    assert torch.equal(pool.cpu()[rest], pool0[rest]), "pool entries not named were written"
+
+
+@pytest.mark.parametrize("gate", ["offset16", "zero"])
+def test_chunk_steps_gates(gate):
+    _, pool, idx, out, o_ref, s_ref, _, _ = _run(N=4, L=24, H=2, pool_n=4, seed=97, gate=gate,
+                                                 slots=False)
+    assert_close(out, o_ref, BF, f"o ({gate})")
+    for n in range(idx.numel()):
+        assert_close(pool[idx[n]], s_ref[n], BF, f"state {n} ({gate})")
+
+
+def test_chunk_steps_strong_decay():
+    """g far below the prefill's range (-20 per token on every channel):
+    the block forms use e^{G_i - G_j} <= 1 directly, so nothing overflows."""
+    N, L, H, d = 3, 20, 2, 128
+    q, k, v, g, b = _tokens(N, L, H, d, seed=98)
+    g = torch.full_like(g, -20.0)
+    pool0 = W.decode_initial_state(N, H, d, d, seed=98, std=0.02)
+    pool = pool0.to(DEV)
+    out = kda_recurrent_steps(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), b.to(DEV), pool,
+                              flags=KDA_STEPS_CHUNK)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all() and torch.isfinite(pool).all()
+    o_ref, s_ref = oracle.forward(q, k, v, g, b, initial_state=pool0.double())
+    assert_close(out, o_ref, BF, "o")
+    for n in range(N):
+        assert_close(pool[n], s_ref[n], BF, f"state {n}")
+
+
+def test_chunk_steps_close_to_recurrent_on_the_decode_workload():
+    """256 x 32 heads, 8 tokens, pool of 512: the chunk form against the
+    recurrent kernel on every output (both bf16-tolerance from the oracle,
+    which a sample checks)."""
+    N, H, d, L, S = W.DECODE_N, W.DECODE_H, W.DECODE_D, 8, 2 * W.DECODE_N
+    pool0 = W.decode_initial_state(S, H, d, d)
+    gen = torch.Generator().manual_seed(31)
+    slots = torch.randperm(S, generator=gen)[:N].to(torch.int32).to(DEV)
+    q, k, v, g, b = [t.to(DEV) for t in _tokens(N, L, H, d, seed=W.DECODE_SEED)]
+    pool_c, pool_r = pool0.to(DEV), pool0.to(DEV)
+    out_c = kda_recurrent_steps(q, k, v, g, b, pool_c, slots, flags=KDA_STEPS_CHUNK)
+    out_r = kda_recurrent_steps(q, k, v, g, b, pool_r, slots)
+    torch.cuda.synchronize()
+    assert kda_get_device_error() == 0
+    assert rel_inf(out_c, out_r) <= 2e-2
+    assert rel_inf(pool_c, pool_r) <= 2e-2
+    ns = torch.randperm(N, generator=gen)[:16]
+    sl = slots.cpu()[ns].long()
+    o_ref, s_ref = oracle.forward(q.cpu()[ns], k.cpu()[ns], v.cpu()[ns], g.cpu()[ns], b.cpu()[ns],
+                                  initial_state=pool0[sl].double())
+    assert_close(out_c[ns.to(DEV)], o_ref, BF, "sampled o")
+    assert_close(pool_c[sl.to(DEV)], s_ref, BF, "sampled states")
+
+
+def test_chunk_flag_falls_back_where_unsupported():
+    """fp32 inputs or d = 64 with the flag run the recurrent kernel: bitwise
+    equal to the call without the flag."""
+    N, L, H, d = 3, 5, 2, 64
+    steps = [W.decode_tokens(l, N, H, d, d, torch.float32, seed=99) for l in range(L)]
+    q, k, v, g, b = [torch.stack([s[i] for s in steps], dim=1).contiguous().to(DEV) for i in range(5)]
+    s0 = W.decode_initial_state(N, H, d, d, seed=99).to(DEV)
+    p1, p2 = s0.clone(), s0.clone()
+    o1 = kda_recurrent_steps(q, k, v, g, b, p1, flags=KDA_STEPS_CHUNK)
+    o2 = kda_recurrent_steps(q, k, v, g, b, p2)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(p1, p2)

@@ -12,16 +12,21 @@
 //     T = (I + A)^-1,  W = T (beta K e^G),  U = T (beta V)
 //     V_new = U - W S;  O = (Q e^G) S + P V_new
 //     S <- Diag(e^{G_last}) S + (K e^{G_last - G})^T V_new
-// The same algebra as the chunked prefill; here the block is at most 16
-// tokens, so A and P are formed directly from e^{G_i - G_j} <= 1 in fp32
-// (exact exponentials, no factorisation): any finite g <= 0 is accepted.
+// The same algebra as the chunked prefill.  A and P: when every g of the
+// block is >= -5 (|G| <= 80 over 16 tokens) they are products of the forms
+// beta k e^G, q e^G and k e^{-G} on tensor cores, as in the prefill; else
+// they are formed directly from e^{G_i - G_j} <= 1 in fp32 (exact
+// exponentials, no factorisation), so any finite g <= 0 is accepted.
 //
-// One CTA (256 threads, 8 warps) per (sequence, head), two CTAs per SM.  The
-// fp32 state lives in registers in the m16n8k16 accumulator layout (warp w:
-// channel rows 16w .. 16w + 15, all 128 columns), so the state update is one
-// tensor-core accumulate into it; its bf16 copy in shared memory is the B
-// operand of W S and (Q e^G) S.  Rounding: the MMA operands (S, V_new, T, P
-// and the decayed forms) are bf16, as in the prefill.
+// Persistent CTAs (256 threads, 8 warps, one per SM) walk the (sequence,
+// head) items.  The fp32 state lives in registers in the m16n8k16
+// accumulator layout (warp w: channel rows 16w .. 16w + 15, all 128
+// columns), so the state update is one tensor-core accumulate into it; its
+// bf16 copy in shared memory is the B operand of W S and (Q e^G) S.  While an
+// item runs, each thread's share of the next item's state arrives by
+// cp.async in a thread-private shared-memory slot, and the next block's token
+// rows likewise.  Rounding: the MMA operands (S, V_new, T, P and the decayed
+// forms) are bf16, as in the prefill.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -56,9 +61,31 @@ constexpr int OFF_AM = OFF_SB + 32768;       // A, P, T: fp32 [16][16]
 constexpr int OFF_PM = OFF_AM + 1024;
 constexpr int OFF_TM = OFF_PM + 1024;
 constexpr int OFF_GAM = OFF_TM + 1024;       // e^{G_last} per channel, fp32 [128]
-constexpr int SMEM = OFF_GAM + 512;
-static_assert(OFF_QG % 16 == 0 && OFF_SB % 16 == 0 && SMEM <= 100 * 1024, "layout");
+constexpr int OFF_KD = OFF_GAM + 512;        // k e^{-G} (factorised A and P)
+constexpr int OFF_SN = OFF_KD + 4096;        // next item's state, fp32 [128][128], fsw layout
+constexpr int OFF_SO = OFF_SN + D * D * 4;   // finished item's state on its way out, fsw layout
+constexpr int SMEM = OFF_SO + D * D * 4;
+static_assert(OFF_QG % 16 == 0 && OFF_SB % 16 == 0 && OFF_KD % 16 == 0 && OFF_SN % 16 == 0 &&
+              SMEM <= 227 * 1024, "layout");
 
+// 2^x by the hardware approximation (PTX ex2.approx.ftz: relative error about
+// 2^-22, results below 2^-126 flush to zero); the operands of the products it
+// feeds are rounded to bf16 (2^-9).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ void cp_async4_zfill(void *smem_dst, const void *gmem_src, bool ok) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(smem_u32(smem_dst)),
+                 "l"(gmem_src), "r"(ok ? 4 : 0));
+}
+// fp32 [128][128] state in shared memory: 16-byte chunk j of row r at
+// j ^ 2 (r & 3), so that a half-warp reading accumulator pairs (rows
+// 16w + gid, gid = 0..3) and a warp copying one whole row are conflict-free
+__device__ __forceinline__ int fsw(int r, int c) {
+    return r * 512 + ((((c >> 2) ^ (2 * (r & 3)))) << 4) + ((c & 3) << 2);
+}
 __device__ __forceinline__ void cp_async16_zfill(void *smem_dst, const void *gmem_src, bool ok) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem_dst)),
                  "l"(gmem_src), "r"(ok ? 16 : 0));
@@ -78,22 +105,17 @@ __device__ __forceinline__ void frag16(uint32_t (&a)[4], const float *M, int gid
 
 }  // namespace
 
-__global__ void __launch_bounds__(NT, 2)
+__global__ void __launch_bounds__(NT, 1)
 decode_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                     const __nv_bfloat16 *__restrict__ v, const float *__restrict__ g,
                     const float *__restrict__ beta, float *__restrict__ pool,
                     const int32_t *__restrict__ slots, int num_slots,
-                    __nv_bfloat16 *__restrict__ out, int H, int L, int *__restrict__ err)
+                    __nv_bfloat16 *__restrict__ out, int N, int H, int L, int *__restrict__ err)
 {
     extern __shared__ __align__(128) unsigned char sm[];
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int gid = lane >> 2, tig = lane & 3;
-    const int n = blockIdx.x / H, h = blockIdx.x - n * H;
-    const int slot = slots ? slots[n] : n;
-    if (slot < 0 || slot >= num_slots) {
-        if (tid == 0) set_device_error(err, kErrBadSlot);
-        return;
-    }
+    const int items = N * H;
     float *Gs = reinterpret_cast<float *>(sm + OFF_G);
     float *bs = reinterpret_cast<float *>(sm + OFF_BETA);
     float *Am = reinterpret_cast<float *>(sm + OFF_AM);
@@ -101,15 +123,36 @@ decode_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     float *Tm = reinterpret_cast<float *>(sm + OFF_TM);
     float *gam = reinterpret_cast<float *>(sm + OFF_GAM);
     const int nblk = (L + BT - 1) / BT;
-    auto token_row = [&](int l) -> size_t { return ((size_t)n * L + l) * H + h; };
+    // the next item at or after `it` (grid stride) with a valid slot; -1 if
+    // none.  Every thread walks the same items, so the answer is uniform.
+    auto next_valid = [&](int it) -> int {
+        for (; it < items; it += gridDim.x) {
+            const int nn = it / H;
+            const int sl = slots ? slots[nn] : nn;
+            if (sl >= 0 && sl < num_slots) return it;
+            if (tid == 0) set_device_error(err, kErrBadSlot);
+        }
+        return -1;
+    };
+    auto state_of = [&](int it) -> float * {
+        const int nn = it / H, hh = it - nn * H;
+        const int sl = slots ? slots[nn] : nn;
+        return pool + ((size_t)sl * H + hh) * (size_t)(D * D);
+    };
+    // token l of item `it` is row row0(it) + l * H of the token arrays
+    auto row0 = [&](int it) -> size_t {
+        const int nn = it / H, hh = it - nn * H;
+        return (size_t)nn * L * H + hh;
+    };
 
-    // raw rows of block b (zero past the last token), one cp.async group
-    auto issue_raw = [&](int b) {
+    // raw rows of block b of item `it` (zero past the last token), one cp.async group
+    auto issue_raw = [&](int it, int b) {
         const int l0 = b * BT, nt = min(BT, L - l0);
+        const size_t base = row0(it);
         for (int c = tid; c < BT * 80; c += NT) {
             const int i = c / 80, r = c - i * 80;
             const bool ok = i < nt;
-            const size_t row = token_row(ok ? l0 + i : l0);
+            const size_t row = base + (size_t)(ok ? l0 + i : l0) * H;
             if (r < 48) {
                 const int vec = r >> 4, j = r & 15;
                 const __nv_bfloat16 *src = (vec == 0 ? q : vec == 1 ? k : v) + row * D + j * 8;
@@ -119,22 +162,25 @@ decode_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
                 cp_async16_zfill(sm + OFF_G + i * 512 + j * 16, g + row * D + j * 4, ok);
             }
         }
-        if (tid < BT) bs[tid] = tid < nt ? beta[token_row(l0 + tid)] : 0.f;
+        if (tid < BT) cp_async4_zfill(bs + tid, beta + base + (size_t)(tid < nt ? l0 + tid : l0) * H, tid < nt);
         cp_async_commit();
     };
 
     // the state, fp32, in the accumulator layout: s[j] = rows (16w + gid,
-    // 16w + gid + 8) x columns (8j + 2tig, + 1)
-    float *Sg = pool + ((size_t)slot * H + h) * (size_t)(D * D);
+    // 16w + gid + 8) x columns (8j + 2tig, + 1).  Element pair (j, half) of
+    // thread t has its own 8-byte slot in the prefetch area.
     const int r0 = 16 * w + gid, r1 = r0 + 8;
-    float s[16][4];
-    issue_raw(0);
+    // the next item's state: whole rows (one per warp and instruction) into
+    // the fsw layout; joins the next committed group
+    auto issue_state = [&](int it) {
+        const float *Sg = state_of(it);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        const float2 x = __ldcs(reinterpret_cast<const float2 *>(Sg + (size_t)r0 * D + 8 * j + 2 * tig));
-        const float2 y = __ldcs(reinterpret_cast<const float2 *>(Sg + (size_t)r1 * D + 8 * j + 2 * tig));
-        s[j][0] = x.x; s[j][1] = x.y; s[j][2] = y.x; s[j][3] = y.y;
-    }
+        for (int e = 0; e < 16; ++e) {
+            const int idx = e * NT + tid, r = idx >> 5, c = 4 * (idx & 31);
+            cp_async16(sm + OFF_SN + fsw(r, c), Sg + (size_t)r * D + c);
+        }
+    };
+    float s[16][4];
     auto write_sb = [&]() {
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -142,35 +188,54 @@ decode_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
             *reinterpret_cast<uint32_t *>(sm + OFF_SB + toff(r1, 8 * j + 2 * tig)) = pack_bf16(s[j][2], s[j][3]);
         }
     };
-    write_sb();
 
+    int cur = next_valid(blockIdx.x);
+    if (cur < 0) return;
+    issue_state(cur);
+    issue_raw(cur, 0);
+    while (cur >= 0) {
+    const int nxt = next_valid(cur + gridDim.x);
+    const size_t orow = row0(cur);
     for (int b = 0; b < nblk; ++b) {
         const int l0 = b * BT, nt = min(BT, L - l0);
         cp_async_wait<0>();
-        __syncthreads();                       // raw rows of block b landed; S copy written
+        __syncthreads();                       // raw rows of block b (and at b = 0 the state) landed
+        if (b == 0) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float2 x = *reinterpret_cast<const float2 *>(sm + OFF_SN + fsw(r0, 8 * j + 2 * tig));
+                const float2 y = *reinterpret_cast<const float2 *>(sm + OFF_SN + fsw(r1, 8 * j + 2 * tig));
+                s[j][0] = x.x; s[j][1] = x.y; s[j][2] = y.x; s[j][3] = y.y;
+            }
+            write_sb();
+        }
 
         // 1. per channel: log2e-scaled inclusive cumsum of g (in place), the
         //    block decay; meanwhile the other threads clear A and P
+        bool in_range = true;
         if (tid < D) {
             float acc = 0.f;
 #pragma unroll
             for (int i = 0; i < BT; ++i) {
-                acc = fmaf(Gs[i * D + tid], LOG2E, acc);
+                const float gv = Gs[i * D + tid];
+                in_range = in_range && gv >= -5.f;
+                acc = fmaf(gv, LOG2E, acc);
                 Gs[i * D + tid] = acc;
             }
-            gam[tid] = exp2f(acc);
+            gam[tid] = ex2(acc);
         } else {
             for (int e = tid - D; e < 512; e += NT - D) (e < 256 ? Am : Pm)[e & 255] = 0.f;
         }
-        __syncthreads();
+        // factorised A and P when every g of the block is >= -5
+        const bool fact = __syncthreads_and(in_range);
 
         // 2. decayed forms (thread: token i, channel pair), A and P
         for (int it = tid; it < BT * 64; it += NT) {
             const int i = it >> 6, c = 2 * (it & 63);
             const float2 gi = *reinterpret_cast<const float2 *>(Gs + i * D + c);
             const float2 gl = *reinterpret_cast<const float2 *>(Gs + (BT - 1) * D + c);
-            const float ex = exp2f(gi.x), ey = exp2f(gi.y);
-            const float tx = exp2f(gl.x - gi.x), ty = exp2f(gl.y - gi.y);
+            const float ex = ex2(gi.x), ey = ex2(gi.y);
+            const float tx = ex2(gl.x - gi.x), ty = ex2(gl.y - gi.y);
             const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(sm + OFF_RQ + i * 256 + 2 * c);
             const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(sm + OFF_RK + i * 256 + 2 * c);
             const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162 *>(sm + OFF_RV + i * 256 + 2 * c);
@@ -183,8 +248,9 @@ decode_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
             *reinterpret_cast<uint32_t *>(sm + OFF_KT + o) = pack_bf16(kx * tx, ky * ty);
             *reinterpret_cast<uint32_t *>(sm + OFF_BV + o) =
                 pack_bf16(b_ * __low2float(v2), b_ * __high2float(v2));
+            if (fact) *reinterpret_cast<uint32_t *>(sm + OFF_KD + o) = pack_bf16(__fdividef(kx, ex), __fdividef(ky, ey));
         }
-        {
+        if (!fact) {
             // pairs j <= i < nt, eight slices each; slice sl of pair p takes
             // channel pairs 2 sl + 16 m (m = 0..7), visited from a per-pair
             // rotation so that the four pairs of a warp read different banks.
@@ -211,7 +277,7 @@ decode_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
                         const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(qi + 2 * c);
                         const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(ki + 2 * c);
                         const __nv_bfloat162 l2 = *reinterpret_cast<const __nv_bfloat162 *>(kj + 2 * c);
-                        const float e0 = exp2f(x.x - y.x), e1 = exp2f(x.y - y.y);
+                        const float e0 = ex2(x.x - y.x), e1 = ex2(x.y - y.y);
                         const float kj0 = __low2float(l2), kj1 = __high2float(l2);
                         a = fmaf(__low2float(k2) * kj0, e0, a);
                         a = fmaf(__high2float(k2) * kj1, e1, a);
@@ -231,23 +297,74 @@ decode_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
             }
         }
         __syncthreads();
-        // the raw rows are dead: the next block's arrive while this one runs
-        if (b + 1 < nblk) issue_raw(b + 1);
+        if (fact) {
+            // A = (beta k e^G)(k e^{-G})^T, P = (q e^G)(k e^{-G})^T: warps
+            // 0-1 A, 2-3 P, one 8-column tile each
+            if (w < 4) {
+                const unsigned char *X = sm + (w < 2 ? OFF_KG : OFF_QG);
+                const int nt8 = w & 1;
+                const int ar = (lane & 7) + 8 * ((lane >> 3) & 1);
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    uint32_t af[4], bf[2];
+                    ldsm_x4(af, X + toff_chunk(ar, 2 * ks + (lane >> 4)));
+                    // B (k = channel, n = token j) from k e^{-G} stored [token][channel]
+                    bf[0] = *reinterpret_cast<const uint32_t *>(sm + OFF_KD + toff(8 * nt8 + gid, 16 * ks + 2 * tig));
+                    bf[1] = *reinterpret_cast<const uint32_t *>(sm + OFF_KD + toff(8 * nt8 + gid, 16 * ks + 8 + 2 * tig));
+                    mma_bf16(acc, af, bf[0], bf[1]);
+                }
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int i = gid + 8 * hh, j = 8 * nt8 + 2 * tig;
+                    const float v0 = acc[2 * hh], v1 = acc[2 * hh + 1];
+                    if (w < 2) {
+                        Am[i * 16 + j] = (j < i) ? v0 : 0.f;
+                        Am[i * 16 + j + 1] = (j + 1 < i) ? v1 : 0.f;
+                    } else {
+                        Pm[i * 16 + j] = (j <= i) ? v0 : 0.f;
+                        Pm[i * 16 + j + 1] = (j + 1 <= i) ? v1 : 0.f;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+        // the raw rows are dead: the next block's (or the next item's first
+        // block's) arrive while this one runs
+        if (b + 1 < nblk) issue_raw(cur, b + 1);
+        else if (nxt >= 0) issue_raw(nxt, 0);
 
         // 3. T = (I + A)^-1 by forward substitution, one column per thread
         if (tid < BT) {
+            // row i of A arrives as four vector loads before its two
+            // interleaved accumulation chains (even and odd j)
             float x[BT];
 #pragma unroll
             for (int i = 0; i < BT; ++i) {
-                float acc = 0.f;
+                float ar[BT];
 #pragma unroll
-                for (int j = 0; j < i; ++j) acc = fmaf(Am[i * 16 + j], x[j], acc);
-                x[i] = (i < tid) ? 0.f : (i == tid) ? 1.f : -acc;
+                for (int c4 = 0; c4 < BT / 4; ++c4) {
+                    const float4 t4 = *reinterpret_cast<const float4 *>(Am + i * 16 + 4 * c4);
+                    ar[4 * c4] = t4.x; ar[4 * c4 + 1] = t4.y; ar[4 * c4 + 2] = t4.z; ar[4 * c4 + 3] = t4.w;
+                }
+                float e0 = 0.f, e1 = 0.f;
+#pragma unroll
+                for (int j = 0; j < i; ++j) {
+                    if (j & 1) e1 = fmaf(ar[j], x[j], e1);
+                    else e0 = fmaf(ar[j], x[j], e0);
+                }
+                x[i] = (i < tid) ? 0.f : (i == tid) ? 1.f : -(e0 + e1);
             }
 #pragma unroll
             for (int i = 0; i < BT; ++i) Tm[i * 16 + tid] = x[i];
         }
         __syncthreads();
+        // every thread's reads of its state slots are long complete (several
+        // barriers): the next item's state may now land there
+        if (b == 0 && nxt >= 0) {
+            issue_state(nxt);
+            cp_async_commit();
+        }
 
         // 4. W = T (beta k e^G) (channel tiles 2w, 2w + 1) and U = T (beta v)
         //    (value tiles 2w, 2w + 1; kept in registers)
@@ -308,9 +425,9 @@ decode_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
             for (int jj = 0; jj < 2; ++jj) {
                 const int c = 16 * w + 8 * jj + 2 * tig;
                 if (gid < nt)
-                    *reinterpret_cast<uint32_t *>(out + token_row(l0 + gid) * D + c) = pack_bf16(os[jj][0], os[jj][1]);
+                    *reinterpret_cast<uint32_t *>(out + (orow + (size_t)(l0 + gid) * H) * D + c) = pack_bf16(os[jj][0], os[jj][1]);
                 if (gid + 8 < nt)
-                    *reinterpret_cast<uint32_t *>(out + token_row(l0 + gid + 8) * D + c) = pack_bf16(os[jj][2], os[jj][3]);
+                    *reinterpret_cast<uint32_t *>(out + (orow + (size_t)(l0 + gid + 8) * H) * D + c) = pack_bf16(os[jj][2], os[jj][3]);
             }
         }
 
@@ -336,10 +453,24 @@ decode_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         // barrier after V_new); write the new one for the next block
         if (b + 1 < nblk) write_sb();
     }
+    {
+        // out through shared memory, so that each store instruction writes
+        // whole rows
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        __stcs(reinterpret_cast<float2 *>(Sg + (size_t)r0 * D + 8 * j + 2 * tig), make_float2(s[j][0], s[j][1]));
-        __stcs(reinterpret_cast<float2 *>(Sg + (size_t)r1 * D + 8 * j + 2 * tig), make_float2(s[j][2], s[j][3]));
+        for (int j = 0; j < 16; ++j) {
+            *reinterpret_cast<float2 *>(sm + OFF_SO + fsw(r0, 8 * j + 2 * tig)) = make_float2(s[j][0], s[j][1]);
+            *reinterpret_cast<float2 *>(sm + OFF_SO + fsw(r1, 8 * j + 2 * tig)) = make_float2(s[j][2], s[j][3]);
+        }
+        __syncthreads();
+        float *Sg = state_of(cur);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int idx = e * NT + tid, r = idx >> 5, c = 4 * (idx & 31);
+            __stcs(reinterpret_cast<float4 *>(Sg + (size_t)r * D + c),
+                   *reinterpret_cast<const float4 *>(sm + OFF_SO + fsw(r, c)));
+        }
+    }
+    cur = nxt;
     }
 }
 
@@ -349,19 +480,25 @@ cudaError_t launch_decode_chunk(const void *q, const void *k, const void *v, con
                                 cudaStream_t st)
 {
     if (N == 0 || L == 0) return cudaSuccess;
-    static bool attr_done[64] = {false};
+    static int grid_for[64] = {0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_done[dev]) {
+    if (grid_for[dev] == 0) {
         e = cudaFuncSetAttribute(decode_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
         if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
+        int sms = 0, per_sm = 0;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_chunk_kernel, NT, SMEM)) != cudaSuccess)
+            return e;
+        grid_for[dev] = sms * (per_sm > 0 ? per_sm : 1);
     }
-    decode_chunk_kernel<<<N * H, NT, SMEM, st>>>(
+    const int items = N * H;
+    const int grid = items < grid_for[dev] ? items : grid_for[dev];
+    decode_chunk_kernel<<<grid, NT, SMEM, st>>>(
         (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, g, beta, pool,
-        slots, num_slots, (__nv_bfloat16 *)out, H, L, err);
+        slots, num_slots, (__nv_bfloat16 *)out, N, H, L, err);
     return cudaGetLastError();
 }
 

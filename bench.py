@@ -67,6 +67,7 @@ TRAFFIC = {
                "bytes": (547.408128 + 480.674560) * 1e6},
     "decode_steps": {"files": ["decode_pipe.cu", "common.cuh", "sm100.cuh"], "sha": "dfd242f2df963f4b",
                      "bytes": (621.427456 + 496.504320) * 1e6},
+    "decode_chunk": {"files": ["decode_chunk.cu", "common.cuh"], "sha": "", "bytes": 0.0},
 }
 
 
@@ -262,6 +263,9 @@ def run_ours(args):
     with ClockSampler(local) as clk_dec:
         dec = decode_leg(kda, W, dev, dist, world, args)
         dec_steps = decode_steps_leg(kda, W, dev, dist, world, args)
+        dec_chunk = decode_steps_leg(kda, W, dev, dist, world, args, L=CHUNK_L,
+                                     flags=kda.KDA_STEPS_CHUNK, kernel="decode_chunk_kernel",
+                                     traffic_key="decode_chunk", ring=1)
     clk.samples += clk_dec.samples
     clk.reasons |= clk_dec.reasons
 
@@ -286,6 +290,7 @@ def run_ours(args):
         "clocks": clk.summary(),
         "decode": dec,
         "decode_steps": dec_steps,
+        "decode_chunk": dec_chunk,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(inp_cpu)
@@ -329,59 +334,60 @@ def decode_leg(kda, W, dev, dist, world, args):
                          "traffic": measured_traffic("decode") if n == DEC_N else None}}
 
 
-STEPS_L = 8
+STEPS_L = 8          # tokens per call, recurrent serving leg
+CHUNK_L = 64         # tokens per call, chunk-form serving leg (the mode-switch length)
 
 
-def steps_bytes(n):
+def steps_bytes(n, L=STEPS_L):
     """Algorithmic bytes of one serving-decode call: n pool states read and
-    written once, STEPS_L tokens' q, k, v, out (bf16), g, beta (fp32) per
+    written once, L tokens' q, k, v, out (bf16), g, beta (fp32) per
     (sequence, head), and the slot indices."""
-    return n * DEC_H * (2 * D * D * 4 + STEPS_L * (3 * D * 2 + D * 4 + 4 + D * 2)) + n * 4
+    return n * DEC_H * (2 * D * D * 4 + L * (3 * D * 2 + D * 4 + 4 + D * 2)) + n * 4
 
 
 STEPS_BYTES = steps_bytes(DEC_N)
 
 
-def decode_steps_leg(kda, W, dev, dist, world, args):
-    """Serving decode: 8 tokens per sequence per call (kda_recurrent_steps) for
-    the n x 32 decode batch (n = 256 by default), states in a pool of 2n
-    entries picked by a seeded slot permutation."""
+def decode_steps_leg(kda, W, dev, dist, world, args, L=STEPS_L, flags=0,
+                     kernel="decode_pipe_kernel", traffic_key="decode_steps", ring=2):
+    """Serving decode: L tokens per sequence per call (kda_recurrent_steps,
+    with ``flags``) for the n x 32 decode batch (n = 256 by default), states
+    in a pool of 2n entries picked by a seeded slot permutation."""
     n = args.decode_n
     pool_n = 2 * n
     pool = torch.empty(pool_n, DEC_H, D, D, dtype=torch.float32, device=dev)
     pool.copy_(W.decode_initial_state(pool_n, DEC_H, D, D))
     gen = torch.Generator().manual_seed(31)
     slots = torch.randperm(pool_n, generator=gen)[:n].to(torch.int32).to(dev)
-    ring = 2
     toks = []
     for r in range(ring):
-        steps_r = [W.decode_tokens(r * STEPS_L + l, n) for l in range(STEPS_L)]
+        steps_r = [W.decode_tokens(r * L + l, n) for l in range(L)]
         toks.append(tuple(torch.stack([st[i] for st in steps_r], dim=1).contiguous().to(dev)
                           for i in range(5)))
-    out = torch.empty(n, STEPS_L, DEC_H, D, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(n, L, DEC_H, D, dtype=torch.bfloat16, device=dev)
     calls = max(16, args.decode_steps // 16)
     for i in range(max(3, args.warmup)):
-        kda.kda_recurrent_steps(*toks[i % ring], pool, slots, out=out)
+        kda.kda_recurrent_steps(*toks[i % ring], pool, slots, out=out, flags=flags)
     barrier(dist)
     s = torch.cuda.current_stream(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(s)
     for i in range(calls):
-        kda.kda_recurrent_steps(*toks[i % ring], pool, slots, out=out)
+        kda.kda_recurrent_steps(*toks[i % ring], pool, slots, out=out, flags=flags)
     e1.record(s)
     barrier(dist)
     ms = max_over_ranks(e0.elapsed_time(e1), dist) / calls
     peak, kind = measured_peak_hbm()
-    nbytes = steps_bytes(n)
+    nbytes = steps_bytes(n, L)
     ach = nbytes / (ms * 1e-3) / 1e9
-    return {"workload": f"decode_steps_n{n}_l{STEPS_L}_h{DEC_H}_d{D}_pool{pool_n}",
-            "value": job_value(n * STEPS_L, world, ms), "unit": UNIT, "ms_per_call": ms,
-            "calls": calls,
+    return {"workload": f"decode_steps_n{n}_l{L}_h{DEC_H}_d{D}_pool{pool_n}",
+            "flags": flags, "value": job_value(n * L, world, ms), "unit": UNIT,
+            "ms_per_call": ms, "calls": calls,
             "l2": f"pool ({pool_n * DEC_H * D * D * 4 >> 20} MiB) larger than L2; no flush",
-            "roofline": {"bound": "hbm", "kernel": "decode_pipe_kernel", "achieved": ach,
+            "roofline": {"bound": "hbm", "kernel": kernel, "achieved": ach,
                          "peak": peak, "unit": "GB/s", "frac": ach / peak, "peak_source": kind,
                          "algorithmic_bytes_per_launch": nbytes,
-                         "traffic": measured_traffic("decode_steps") if n == DEC_N else None}}
+                         "traffic": measured_traffic(traffic_key) if n == DEC_N else None}}
 
 
 def cpu_baseline(inp_cpu, tokens=None):

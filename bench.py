@@ -67,7 +67,8 @@ TRAFFIC = {
                "bytes": (547.408128 + 480.674560) * 1e6},
     "decode_steps": {"files": ["decode_pipe.cu", "common.cuh", "sm100.cuh"], "sha": "dfd242f2df963f4b",
                      "bytes": (621.427456 + 496.504320) * 1e6},
-    "decode_chunk": {"files": ["decode_chunk.cu", "common.cuh"], "sha": "", "bytes": 0.0},
+    "decode_chunk": {"files": ["decode_chunk.cu", "common.cuh"], "sha": "23a550bc05b00c2b",
+                     "bytes": (1210.240000 + 623.093504) * 1e6},
 }
 
 

@@ -62,7 +62,7 @@ FALLBACK_HBM_GBS = 6650.0
 _SRC = os.path.join(ROOT, "gated_delta_rule_88_b200", "csrc")
 TRAFFIC = {
     "prefill": {"files": ["chunk_prep.cu", "chunk_chain_tc.cu", "chunk_ws.h", "sm100.cuh", "common.cuh"],
-                "sha": "98ba6bde4155390f", "bytes": (342.247424 + 264.975872 + 304.209152 + 52.774912) * 1e6},
+                "sha": "a3a197b795fcf79a", "bytes": (342.108160 + 264.204800 + 304.158464 + 52.440832) * 1e6},
     "decode": {"files": ["decode.cu", "common.cuh"], "sha": "4ceac309c0c18d2f",
                "bytes": (547.408128 + 480.674560) * 1e6},
     "decode_steps": {"files": ["decode_pipe.cu", "common.cuh", "sm100.cuh"], "sha": "dfd242f2df963f4b",

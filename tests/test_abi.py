@@ -127,7 +127,7 @@ def test_steps_null_pointer_rejected(lib, field):
 @pytest.mark.parametrize("kw", [dict(N=-1), dict(L=0), dict(H=0), dict(S=0), dict(N=5, S=4),
                                 dict(dtype=3), dict(pool=FAKE + 8), dict(b=FAKE + 1),
                                 dict(slots=FAKE + 2), dict(N=1 << 20, H=1 << 12),
-                                dict(flags=4), dict(q_scale=float("nan")),
+                                dict(flags=8), dict(flags=0xFFFFFFFF), dict(q_scale=float("nan")),
                                 dict(q_scale=float("inf"))])
 def test_steps_bad_arguments_rejected(lib, kw):
     assert steps(lib, **kw) == 1

@@ -189,3 +189,52 @@ def state_affine(M, B, S):
     such a map (used to check the context-parallel fold)."""
     out = M.double() @ S.double()
     return out if B is None else out + B.double()
+
+
+def _recurrence_torch(q, k, v, g, beta, S0):
+    """The recurrence of ``recurrence`` in plain fp64 torch ops (differentiable).
+    One (sequence, head): q,k,g [T,dk]; v [T,dv]; beta [T]; S0 [dk,dv].
+    Kimi Linear paper notes, section 2: per token
+        S' = Diag(exp g) S;  S = S' + beta k (v - S'^T k)^T;  o = S^T q."""
+    S = S0
+    outs = []
+    for t in range(q.shape[0]):
+        Sp = torch.exp(g[t])[:, None] * S
+        u = beta[t] * (v[t] - Sp.T @ k[t])
+        S = Sp + torch.outer(k[t], u)
+        outs.append(S.T @ q[t])
+    return torch.stack(outs) if outs else q.new_zeros((0, v.shape[1])), S
+
+
+def backward(q, k, v, g, beta, do, initial_state=None, dsT=None):
+    """Gradients of the forward (dense layout q,k,g [B,T,H,dk]; v [B,T,H,dv];
+    beta [B,T,H]; initial_state [B,H,dk,dv] or None) for the output gradient
+    do [B,T,H,dv] and the final-state gradient dsT [B,H,dk,dv] (or None = 0):
+    returns fp64 (dq, dk, dv, dg, dbeta, ds0) of the inputs' shapes.
+
+    The chain rule through the recurrence of section 2 (``_recurrence_torch``),
+    taken by torch autograd in fp64 on the CPU; pinned against central finite
+    differences of ``recurrence`` (tests/test_oracle_pins.py)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    outs = {n: torch.zeros(x.shape, dtype=torch.float64) for n, x in
+            (("dq", q), ("dk", k), ("dv", v), ("dg", g), ("dbeta", beta))}
+    ds0 = torch.zeros(B, H, dk, dv, dtype=torch.float64)
+    for b in range(B):
+        for h in range(H):
+            xs = [x[b, :, h].detach().double().clone().requires_grad_(True) for x in (q, k, v, g)]
+            bt = beta[b, :, h].detach().double().clone().requires_grad_(True)
+            s0 = (torch.zeros(dk, dv, dtype=torch.float64) if initial_state is None
+                  else initial_state[b, h].detach().double().clone())
+            s0.requires_grad_(True)
+            o, sT = _recurrence_torch(xs[0], xs[1], xs[2], xs[3], bt, s0)
+            loss = (o * do[b, :, h].double()).sum()
+            if dsT is not None:
+                loss = loss + (sT * dsT[b, h].double()).sum()
+            grads = torch.autograd.grad(loss, xs + [bt, s0], allow_unused=True)
+            for name, gr in zip(("dq", "dk", "dv", "dg", "dbeta"), grads[:5]):
+                if gr is not None:
+                    outs[name][b, :, h] = gr
+            if grads[5] is not None:
+                ds0[b, h] = grads[5]
+    return outs["dq"], outs["dk"], outs["dv"], outs["dg"], outs["dbeta"], ds0

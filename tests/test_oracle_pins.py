@@ -386,3 +386,66 @@ def test_gated_rmsnorm_unit_rms_scale_invariance_and_gate():
     row = torch.full((1, 16), 2.0, dtype=torch.float64)
     assert torch.allclose(oracle.gated_rmsnorm(row, big[:1], ones, 5.0),
                           torch.full((1, 16), 2.0 / 3.0, dtype=torch.float64), atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# The backward oracle (autograd through the fp64 recurrence), pinned by
+# central finite differences of the C recurrence and by closed forms.
+
+def _bwd_case(seed, T=6, dk=4, dv=3, with_s0=True):
+    gen = torch.Generator().manual_seed(seed)
+    r = lambda *s: torch.randn(*s, generator=gen, dtype=torch.float64)
+    q, k, v = r(1, T, 1, dk), 0.6 * r(1, T, 1, dk), r(1, T, 1, dv)
+    g = -torch.rand(1, T, 1, dk, generator=gen, dtype=torch.float64)
+    b = torch.rand(1, T, 1, generator=gen, dtype=torch.float64)
+    s0 = r(1, 1, dk, dv) if with_s0 else None
+    do, dsT = r(1, T, 1, dv), r(1, 1, dk, dv)
+    return q, k, v, g, b, s0, do, dsT
+
+
+def _loss(q, k, v, g, b, s0, do, dsT):
+    o, sT = oracle.recurrence(q[0, :, 0], k[0, :, 0], v[0, :, 0], g[0, :, 0], b[0, :, 0],
+                              None if s0 is None else s0[0, 0])
+    return float((o * do[0, :, 0].numpy()).sum() + (sT * dsT[0, 0].numpy()).sum())
+
+
+@pytest.mark.parametrize("seed", [1, 2])
+def test_backward_matches_finite_differences(seed):
+    q, k, v, g, b, s0, do, dsT = _bwd_case(seed)
+    grads = oracle.backward(q, k, v, g, b, do, s0, dsT)
+    args = [q, k, v, g, b, s0]
+    gen = torch.Generator().manual_seed(100 + seed)
+    eps = 1e-6
+    for ai, (x, gx) in enumerate(zip(args, grads)):
+        for _ in range(4):
+            idx = tuple(int(torch.randint(0, n, (1,), generator=gen)) for n in x.shape)
+            xp, xm = x.clone(), x.clone()
+            xp[idx] += eps
+            xm[idx] -= eps
+            ap, am = list(args), list(args)
+            ap[ai], am[ai] = xp, xm
+            fd = (_loss(*ap, do, dsT) - _loss(*am, do, dsT)) / (2 * eps)
+            assert abs(fd - float(gx[idx])) <= 1e-6 * max(1.0, abs(fd)), (ai, idx, fd, float(gx[idx]))
+
+
+def test_backward_one_token_closed_form():
+    """T = 1, S0 = 0: o = beta (k.q) v, S_1 = beta k v^T, so
+    dv = beta ((k.q) do + dS^T k), dq = beta (v.do) k."""
+    q, k, v, g, b, _, do, dsT = _bwd_case(3, T=1)
+    dq, dk_, dv_, dg, db, ds0 = oracle.backward(q, k, v, g, b, do, None, dsT)
+    qq, kk, vv, bb, dd, SS = q[0, 0, 0], k[0, 0, 0], v[0, 0, 0], b[0, 0, 0], do[0, 0, 0], dsT[0, 0]
+    assert torch.allclose(dv_[0, 0, 0], bb * ((kk @ qq) * dd + SS.T @ kk), atol=1e-12)
+    assert torch.allclose(dq[0, 0, 0], bb * (vv @ dd) * kk, atol=1e-12)
+    assert torch.allclose(dg[0, 0, 0], torch.zeros_like(dg[0, 0, 0]), atol=1e-12)   # S0 = 0
+
+
+def test_backward_pure_decay_state_gradient():
+    """beta = 0: S_t = Diag(prod_{s<=t} a_s) S0 and o_t = S_t^T q_t, so
+    dS0 = sum_t Diag(prod_{s<=t} a_s) q_t do_t^T + Diag(prod_s a_s) dS_T."""
+    q, k, v, g, b, s0, do, dsT = _bwd_case(4, T=5)
+    b = torch.zeros_like(b)
+    ds0 = oracle.backward(q, k, v, g, b, do, s0, dsT)[5][0, 0]
+    a = torch.exp(torch.cumsum(g[0, :, 0], dim=0))      # [T, dk]
+    ref = sum(a[t][:, None] * torch.outer(q[0, t, 0], do[0, t, 0]) for t in range(5))
+    ref = ref + a[-1][:, None] * dsT[0, 0]
+    assert torch.allclose(ds0, ref, atol=1e-12)

@@ -30,6 +30,7 @@ import torch
 
 __all__ = ["kda_chunk_fwd", "kda_chunk_fwd_ex", "kda_chunk_fwd_host", "kda_recurrent_step",
            "kda_recurrent_step_ex", "kda_recurrent_steps", "kda_gated_rmsnorm", "kda_state_affine",
+           "kda_recurrent_bwd",
            "kda_get_device_error",
            "KDAError",
            "KDA_QK_L2NORM", "KDA_BETA_SIGMOID", "KDA_STEPS_CHUNK",
@@ -81,6 +82,8 @@ def load_library():
         lib.kda_gated_rmsnorm.argtypes = [vp, vp, vp, ctypes.c_float, vp, ctypes.c_longlong, i, i, vp]
         lib.kda_gated_rmsnorm.restype = i
         lib.kda_state_affine.argtypes = [vp] * 4 + [i] * 3 + [vp]
+        lib.kda_recurrent_bwd.argtypes = [vp] * 14 + [i] * 6 + [vp]
+        lib.kda_recurrent_bwd.restype = i
         lib.kda_state_affine.restype = i
         lib.kda_get_device_error.argtypes = [vp, ctypes.POINTER(i)]
         lib.kda_get_device_error.restype = i
@@ -324,6 +327,41 @@ def kda_gated_rmsnorm(x, gate, weight, eps: float = 1e-5, out=None):
                                    rows, dv, _dtype_code(x), _stream_handle(dev))
     _check(rc)
     return out
+
+
+def kda_recurrent_bwd(q, k, v, g, beta, do, initial_state=None, dsT=None,
+                      want_initial_state_grad: bool = True):
+    """Gradients of the recurrence (dense layout): q,k,g [B,T,H,dk]; v, do
+    [B,T,H,dv]; beta [B,T,H]; initial_state, dsT (the final-state gradient)
+    [B,H,dk,dv] fp32 or None.  Returns fp32 (dq, dk, dv, dg, dbeta, ds0)
+    (ds0 None unless wanted)."""
+    lib = load_library()
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("kda_recurrent_bwd needs CUDA tensors (no CPU path)")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    for t, name in ((k, "k"), (v, "v"), (do, "do")):
+        _need(t, name, dev, q.dtype)
+    _need(q, "q", dev)
+    _need(g, "g", dev, torch.float32)
+    _need(beta, "beta", dev, torch.float32)
+    for t, name in ((initial_state, "initial_state"), (dsT, "dsT")):
+        if t is not None:
+            _need(t, name, dev, torch.float32)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dq, dk_, dg = (torch.empty(B, T, H, dk, **f32) for _ in range(3))
+    dv_ = torch.empty(B, T, H, dv, **f32)
+    db = torch.empty(B, T, H, **f32)
+    ds0 = torch.empty(B, H, dk, dv, **f32) if want_initial_state_grad else None
+    with torch.cuda.device(dev):
+        rc = lib.kda_recurrent_bwd(_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta),
+                                   _dptr(initial_state), _dptr(do), _dptr(dsT), _dptr(dq),
+                                   _dptr(dk_), _dptr(dv_), _dptr(dg), _dptr(db), _dptr(ds0),
+                                   B, T, H, dk, dv, dt, _stream_handle(dev))
+    _check(rc)
+    return dq, dk_, dv_, dg, db, ds0
 
 
 def kda_state_affine(M, B, S_in, out=None):

@@ -377,6 +377,49 @@ extern "C" kda_status kda_gated_rmsnorm(const void *x, const void *gate, const f
     return KDA_OK;
 }
 
+extern "C" kda_status kda_recurrent_bwd(const void *q, const void *k, const void *v,
+                                        const float *g, const float *beta,
+                                        const float *initial_state, const void *dout,
+                                        const float *dfinal_state, float *dq, float *dk,
+                                        float *dv, float *dg, float *dbeta,
+                                        float *dinitial_state, int B, int T, int H, int dk_,
+                                        int dv_, kda_dtype dtype, void *stream) {
+    t_msg[0] = 0;
+    if (!q || !k || !v || !g || !beta || !dout || !dq || !dk || !dv || !dg || !dbeta)
+        return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_bwd: null pointer argument");
+    if (B <= 0 || T <= 0 || H <= 0 || dk_ <= 0 || dv_ <= 0 || B > 65535 || H > 65535)
+        return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_bwd: bad sizes B=%d T=%d H=%d dk=%d dv=%d",
+                    B, T, H, dk_, dv_);
+    if (dtype != KDA_F32 && dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_bwd: unknown dtype %d", (int)dtype);
+    if (!((dk_ == 64 || dk_ == 128) && (dv_ == 64 || dv_ == 128)))
+        return fail(KDA_ERR_UNSUPPORTED, "kda_recurrent_bwd: dk=%d dv=%d (supported: 64, 128)",
+                    dk_, dv_);
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dg) ||
+        !aligned16(initial_state) || !aligned16(dfinal_state) || !aligned16(dinitial_state))
+        return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_bwd: pointers must be 16-byte aligned");
+    if (((uintptr_t)beta & 3u) || ((uintptr_t)dbeta & 3u))
+        return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_bwd: beta and dbeta must be 4-byte aligned");
+    if ((long long)B * T * H > (1LL << 34))
+        return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_bwd: problem too large");
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaMemPool_t pool;
+    int sms = 148;
+    cudaError_t e = get_pool(&pool, &sms);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_bwd memory pool");
+    void *ws = nullptr;
+    e = cudaMallocFromPoolAsync(&ws, kda::recurrent_bwd_workspace(B, T, H, dk_, dv_), pool, st);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_bwd workspace allocation");
+    e = kda::launch_recurrent_bwd(q, k, v, g, beta, initial_state, dout, dfinal_state, dq, dk, dv,
+                                  dg, dbeta, dinitial_state, ws, B, T, H, dk_, dv_,
+                                  dtype == KDA_BF16, st);
+    cudaError_t e2 = cudaFreeAsync(ws, st);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_bwd launch");
+    if (e2 != cudaSuccess) return cuda_fail(e2, "kda_recurrent_bwd workspace release");
+    return KDA_OK;
+}
+
 extern "C" kda_status kda_state_affine(const float *M, const float *B, const float *S_in,
                                        float *S_out, int count, int dk, int dv, void *stream) {
     t_msg[0] = 0;

@@ -48,6 +48,15 @@ cudaError_t launch_decode_chunk(const void *q, const void *k, const void *v, con
                                 int num_slots, void *out, int N, int H, int L, int *err,
                                 cudaStream_t st);
 
+// Gradients of the recurrence (recurrent_bwd.cu): one warp per (sequence,
+// head, 16-column state tile), workspace of recurrent_bwd_workspace bytes.
+size_t recurrent_bwd_workspace(int B, int T, int H, int dk, int dv);
+cudaError_t launch_recurrent_bwd(const void *q, const void *k, const void *v, const float *g,
+                                 const float *beta, const float *s0, const void *dout,
+                                 const float *dsT, float *dq, float *dk, float *dv, float *dg,
+                                 float *db, float *ds0, void *ws, int B, int T, int H, int dk_,
+                                 int dv_, bool bf16, cudaStream_t st);
+
 // Gated RMSNorm over rows of dv (64 or 128): y = x rsqrt(mean(x^2) + eps) w sigmoid(z).
 cudaError_t launch_gated_rmsnorm(const void *x, const void *z, const float *w, float eps, void *y,
                                  long long rows, int dv, bool bf16, cudaStream_t st);

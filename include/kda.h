@@ -269,6 +269,38 @@ kda_status kda_gated_rmsnorm(const void *x, const void *gate, const float *weigh
                              kda_dtype dtype, void *stream);
 
 /*
+ * kda_recurrent_bwd -- gradients of kda_chunk_fwd's result (dense layout),
+ * for training.
+ *
+ * Source: Kimi Linear paper notes (paper-notes-site), section 2 (the
+ * recurrence) and section 3 (training takes the chunked kernels and their
+ * backward); the backward is the chain rule through the recurrence:
+ *   dS += q do^T;  dq = S_t do;  du = dS^T k;  dk = dS u + S' dw (dw = -beta du);
+ *   dbeta = du . (v - w);  dv = beta du;  dS' = dS + k dw^T;
+ *   dg = rowsum(dS' o S');  dS_{t-1} = Diag(exp g) dS'
+ *   with S' = Diag(exp g) S_{t-1}, w = S'^T k, u = beta (v - w), S_t = S' + k u^T,
+ * starting from dS_T = dfinal_state (or 0) and ending at dinitial_state.
+ *
+ * Layout: q, k [B, T, H, dk] dtype; v, dout [B, T, H, dv] dtype; g
+ *   [B, T, H, dk] float32; beta [B, T, H] float32; initial_state,
+ *   dfinal_state [B, H, dk, dv] float32 or NULL (zeros).  Outputs, float32,
+ *   written in full: dq, dk, dg [B, T, H, dk]; dv [B, T, H, dv]; dbeta
+ *   [B, T, H]; dinitial_state [B, H, dk, dv] or NULL (not written).
+ * Computation: one warp per (sequence, head, 16-column tile of the state) in
+ *   fp32: a forward pass storing the state every 8 tokens, then blocks in
+ *   reverse with the block's states recomputed; per-tile partial row sums
+ *   reduced by a second kernel in a fixed order (deterministic).  Workspace
+ *   from the device's stream-ordered pool on `stream`.
+ * Supported: dk, dv in {64, 128}; dtype KDA_BF16 or KDA_F32; dense only (no
+ *   cu_seqlens); no prologue flags.  Pointers 16-byte aligned (beta, dbeta 4).
+ */
+kda_status kda_recurrent_bwd(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const float *initial_state, const void *dout,
+                             const float *dfinal_state, float *dq, float *dk, float *dv,
+                             float *dg, float *dbeta, float *dinitial_state, int B, int T, int H,
+                             int dk_, int dv_, kda_dtype dtype, void *stream);
+
+/*
  * kda_state_affine -- S_out = M S_in + B for `count` independent blocks.
  *
  * Source: the recurrence of the paper notes (section 2) is affine in the

@@ -220,3 +220,26 @@ def test_affine_bad_arguments_rejected(lib, kw):
 
 def test_affine_empty_is_a_no_op(lib):
     assert affine(lib, count=0) == 0
+
+
+def bwd(lib, *, q=FAKE, k=FAKE, v=FAKE, g=FAKE, b=FAKE, s0=None, do=FAKE, dsT=None, dq=FAKE,
+        dk=FAKE, dv=FAKE, dg=FAKE, db=FAKE, ds0=None, B=1, T=8, H=1, d_k=128, d_v=128, dtype=1):
+    P = ctypes.c_void_p
+    return lib.kda_recurrent_bwd(P(q), P(k), P(v), P(g), P(b), P(s0), P(do), P(dsT), P(dq), P(dk),
+                                 P(dv), P(dg), P(db), P(ds0), B, T, H, d_k, d_v, dtype, None)
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "g", "b", "do", "dq", "dk", "dv", "dg", "db"])
+def test_bwd_null_pointer_rejected(lib, field):
+    assert bwd(lib, **{field: 0}) == 1
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(T=0), dict(H=-1), dict(dtype=5), dict(q=FAKE + 4),
+                                dict(db=FAKE + 2), dict(s0=FAKE + 8), dict(B=70000)])
+def test_bwd_bad_arguments_rejected(lib, kw):
+    assert bwd(lib, **kw) == 1
+
+
+@pytest.mark.parametrize("kw", [dict(d_k=32), dict(d_v=96), dict(d_k=256)])
+def test_bwd_unsupported_rejected(lib, kw):
+    assert bwd(lib, **kw) == 2

@@ -267,6 +267,7 @@ def run_ours(args):
         dec_chunk = decode_steps_leg(kda, W, dev, dist, world, args, L=CHUNK_L,
                                      flags=kda.KDA_STEPS_CHUNK, kernel="decode_chunk_kernel",
                                      traffic_key="decode_chunk", ring=1)
+        bwd = backward_leg(kda, inp, dev, dist, world, args)
     clk.samples += clk_dec.samples
     clk.reasons |= clk_dec.reasons
 
@@ -292,6 +293,7 @@ def run_ours(args):
         "decode": dec,
         "decode_steps": dec_steps,
         "decode_chunk": dec_chunk,
+        "backward": bwd,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(inp_cpu)
@@ -389,6 +391,40 @@ def decode_steps_leg(kda, W, dev, dist, world, args, L=STEPS_L, flags=0,
                          "peak": peak, "unit": "GB/s", "frac": ach / peak, "peak_source": kind,
                          "algorithmic_bytes_per_launch": nbytes,
                          "traffic": measured_traffic(traffic_key) if n == DEC_N else None}}
+
+
+# algorithmic bytes of one backward call on the prefill workload: q, k, v,
+# do (bf16) + g, beta (fp32) read; dq, dk, dg, dv (fp32) + dbeta written
+BWD_BYTES = B * T * H * (4 * D * 2 + D * 4 + 4 + 4 * D * 4 + 4)
+
+
+def backward_leg(kda, inp, dev, dist, world, args):
+    """Training backward (kda_recurrent_bwd) on the prefill workload with a
+    seeded output gradient; no initial or final state."""
+    gen = torch.Generator().manual_seed(41)
+    do = torch.randn(B, T, H, D, generator=gen).to(torch.bfloat16).to(dev)
+    run = lambda: kda.kda_recurrent_bwd(inp.q, inp.k, inp.v, inp.g, inp.beta, do,
+                                        want_initial_state_grad=False)
+    for _ in range(max(1, min(args.warmup, 3))):
+        run()
+    barrier(dist)
+    calls = 3
+    s = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(calls):
+        run()
+    e1.record(s)
+    barrier(dist)
+    ms = max_over_ranks(e0.elapsed_time(e1), dist) / calls
+    peak, kind = measured_peak_hbm()
+    ach = BWD_BYTES / (ms * 1e-3) / 1e9
+    return {"workload": WORKLOAD + "_backward", "value": job_value(B * T, world, ms),
+            "unit": UNIT, "ms_per_call": ms, "calls": calls,
+            "roofline": {"bound": "latency (sequential per token)", "kernel": "recurrent_bwd_kernel",
+                         "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                         "peak_source": kind, "algorithmic_bytes_per_launch": BWD_BYTES,
+                         "traffic": None}}
 
 
 def cpu_baseline(inp_cpu, tokens=None):

@@ -67,6 +67,8 @@ TRAFFIC = {
                "bytes": (547.408128 + 480.674560) * 1e6},
     "decode_steps": {"files": ["decode_pipe.cu", "common.cuh", "sm100.cuh"], "sha": "dfd242f2df963f4b",
                      "bytes": (621.427456 + 496.504320) * 1e6},
+    "backward": {"files": ["recurrent_bwd.cu", "common.cuh"], "sha": "ba9d9318f1b1cd87",
+                 "bytes": (2902.812672 + 3861.861120) * 1e6},
     "decode_chunk": {"files": ["decode_chunk.cu", "common.cuh"], "sha": "23a550bc05b00c2b",
                      "bytes": (1210.240000 + 623.093504) * 1e6},
 }
@@ -424,7 +426,7 @@ def backward_leg(kda, inp, dev, dist, world, args):
             "roofline": {"bound": "latency (sequential per token)", "kernel": "recurrent_bwd_kernel",
                          "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                          "peak_source": kind, "algorithmic_bytes_per_launch": BWD_BYTES,
-                         "traffic": None}}
+                         "traffic": measured_traffic("backward")}}
 
 
 def cpu_baseline(inp_cpu, tokens=None):

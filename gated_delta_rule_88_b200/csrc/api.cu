@@ -344,7 +344,7 @@ static kda_status chunk_fwd_device(const void *q, const void *k, const void *v, 
     if (cu_seqlens) e = kda::launch_chunk_plan(cu_seqlens, N, (int)total_T, coff, st);
     if (e == cudaSuccess)
         e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, coff, N, T, (int)total_T, H,
-                                   (int)max_chunks, records, pro, st);
+                                   (int)max_chunks, records, pro, kda::error_word(), st);
     if (e == cudaSuccess)
         e = kda::launch_chunk_chain(records, cu_seqlens, coff, initial_state, final_state, out, N,
                                     T, (int)total_T, H, dvt, (int)max_chunks, kda::error_word(), st);

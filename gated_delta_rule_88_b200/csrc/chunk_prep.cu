@@ -14,29 +14,37 @@
 //     T     = (I + A)^-1                                  (unit lower-tri.)
 //     W = T (beta K e^G),  U = T (beta V),  Qg = Q e^G,  Kt = K e^{G_C - G}
 //
-// Exponents.  The chunk is cut into four sub-chunks of 16 tokens, I = 0..3,
-// with block-end cumsums R_I (R_{-1} = 0).  Per token and channel only
-// alpha = e^g is exponentiated; everything else is a product of alphas:
-//     a_i = e^{G_i - R_{I-1}} (forward product within the block, <= 1)
-//     b_i = e^{R_I - G_i}     (backward product within the block, <= 1)
-//     d_I = e^{R_I - R_{I-1}} (block total)
-// For i in block I and j in block J:
-//     J < I:  e^{G_i - G_j} = a_i * D_JI * b_j,  D_JI = prod_{J<M<I} d_M <= 1
-//     J = I:  e^{G_i - G_j} = a_i * (1 / a_j),   1/a_j <= e^{16 * max|g|}
-// so with per-token g >= -5 no factor leaves e^{+-80}, and no 1/Gamma over the
-// whole chunk is ever formed.
+// Two ways to the same record, chosen per chunk inside one launch
+// (chunk_prep_tc_kernel):
 //
-// Work split (256 threads, two CTAs per SM): thread (I, channel pair) owns
-// one sub-chunk x two channels for the elementwise forms; A and P are
-// m16n8k16 bf16 MMAs per row block (left operand (beta k a) or (q a), right
-// operand k b scaled by D_JI, or k / a on the diagonal block); T is formed in
-// fp32 (16x16 diagonal blocks by forward substitution, then the 2x2-block
-// recursion T21 = -T22 A21 T11 at 16 and 32 rows on tf32 tensor-core MMAs
-// with fp32 accumulation); W and U are m16n8k16 MMAs with T rounded once to
-// bf16.
+// 1. Chunk-start exponents on tcgen05 (the common case).  Every decayed form
+//    is referenced at the chunk start: q e^G, beta k e^G, k e^{-G}.  Then A
+//    and P are each one product of full tiles, and A/P, W and U are three
+//    tcgen05 MMA groups with fp32 accumulators in tensor memory (see the
+//    comment above chunk_prep_tc_kernel).  Valid while every e^{+-G} and
+//    e^{G_C - G} of the chunk stays within e^{+-80}.
+//
+// 2. Sub-chunk exponents on mma.sync (prep_subchunk), for chunks outside that
+//    range.  The chunk is cut into four sub-chunks of 16 tokens, I = 0..3,
+//    with block-end cumsums R_I (R_{-1} = 0).  Per token and channel only
+//    alpha = e^g is exponentiated; everything else is a product of alphas:
+//        a_i = e^{G_i - R_{I-1}} (forward product within the block, <= 1)
+//        b_i = e^{R_I - G_i}     (backward product within the block, <= 1)
+//        d_I = e^{R_I - R_{I-1}} (block total)
+//    For i in block I and j in block J:
+//        J < I:  e^{G_i - G_j} = a_i * D_JI * b_j,  D_JI = prod_{J<M<I} d_M <= 1
+//        J = I:  e^{G_i - G_j} = a_i * (1 / a_j),   1/a_j <= e^{16 * max|g|}
+//    so with per-token g >= -5 no factor leaves e^{+-80}.
+// Neither path forms a 1/Gamma over a span that could overflow.
+//
+// Both paths form T = (I + A)^-1 in fp32 (16x16 diagonal blocks by forward
+// substitution, then the 2x2-block recursion T21 = -T22 A21 T11 at 16 and 32
+// rows on tf32 tensor-core MMAs with fp32 accumulation) and round T once to
+// bf16 for the W and U products.
 #include "chunk_ws.h"
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace kda {
 namespace {
@@ -186,20 +194,143 @@ __device__ __forceinline__ void ap_block(PrepSmem &sm, unsigned char *rec, bool 
             }
 }
 
+// T = (I + A)^-1 in fp32 for the strictly lower-triangular A (64 x 64, fsw
+// layout): 16x16 diagonal blocks by forward substitution (warps 0-1, lane ->
+// (block, column)), strictly-upper blocks zeroed (warps 2-7), then the 2x2-block
+// recursion T21 = -T22 A21 T11 at 16 and 32 rows on tf32 tensor-core MMAs with
+// fp32 accumulation.  Called by all 256 threads; ends with a CTA barrier.
+__device__ __forceinline__ void form_T(const float *Am, float *Tm, float *Zs, int tid) {
+    const int lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, tig = lane & 3;
+    if (warp < 2) {
+        // 16x16 diagonal blocks: lane -> (block, column)
+        const int Bk = 2 * warp + (lane >> 4), c = lane & 15, o = 16 * Bk;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float s = 0.f;
+#pragma unroll
+            for (int j = 0; j < i; ++j) s += Am[fsw(o + i, o + j)] * x[j];
+            x[i] = (i < c) ? 0.f : (i == c) ? 1.f : -s;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) Tm[fsw(o + i, o + c)] = x[i];
+    } else {
+        // zero the strictly-upper 16x16 blocks
+        for (int e = tid - 64; e < 6 * 256; e += NT - 64) {
+            const int blk = e >> 8, w = e & 255;
+            const int Ib = blk < 3 ? 0 : blk < 5 ? 1 : 2;
+            const int Jb = blk < 3 ? blk + 1 : blk < 5 ? blk - 1 : 3;
+            Tm[fsw(16 * Ib + (w >> 4), 16 * Jb + (w & 15))] = 0.f;
+        }
+    }
+    __syncthreads();
+    // Off-diagonal blocks on the tensor cores (tf32, fp32 accumulate), one
+    // 16x8 output tile per warp:
+    //   16-row level: T_IJ = -T_II (A_IJ T_JJ) for (I, J) = (1, 0), (3, 2)
+    //   32-row level: T[32:64, 0:32] = -T[32:64, 32:64] (A[32:64, 0:32] T[0:32, 0:32])
+    // Zs holds the inner products at the coordinates of the block they feed.
+    if (warp < 4) {
+        const int Ib = (warp >> 1) ? 3 : 1, Jb = Ib - 1, n0 = 16 * Jb + 8 * (warp & 1);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        tile_tf32<16>(c, Am, 16 * Ib, 16 * Jb, Tm, 16 * Jb, n0, gid, tig);
+        store_tile(Zs, c, 16 * Ib, n0, gid, tig, 1.f);
+    }
+    __syncthreads();
+    if (warp < 4) {
+        const int Ib = (warp >> 1) ? 3 : 1, Jb = Ib - 1, n0 = 16 * Jb + 8 * (warp & 1);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        tile_tf32<16>(c, Tm, 16 * Ib, 16 * Ib, Zs, 16 * Ib, n0, gid, tig);
+        store_tile(Tm, c, 16 * Ib, n0, gid, tig, -1.f);
+    }
+    __syncthreads();
+    {
+        const int r0 = 32 + 16 * (warp >> 2), n0 = 8 * (warp & 3);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        tile_tf32<32>(c, Am, r0, 0, Tm, 0, n0, gid, tig);
+        store_tile(Zs, c, r0, n0, gid, tig, 1.f);
+        __syncthreads();
+        float z[4] = {0.f, 0.f, 0.f, 0.f};
+        tile_tf32<32>(z, Tm, r0, 32, Zs, 32, n0, gid, tig);
+        store_tile(Tm, z, r0, n0, gid, tig, -1.f);
+    }
+    __syncthreads();
+}
+
+// form_T for the tensor-core prep: the diagonal 16x16 blocks of A come from a
+// plain padded copy Ad[4][16][17] (row stride 17 floats: immediate offsets,
+// no bank conflicts) and thread 0 first waits for its outstanding bulk
+// stores to have read their shared-memory source (the caller reuses it).
+// Zs may overlap Ad: Ad is dead after the diagonal step.
+__device__ __forceinline__ void form_T_padded_diag(const float *Am, const float *Ad, float *Tm,
+                                                   float *Zs, int tid) {
+    const int lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, tig = lane & 3;
+    if (warp < 2) {
+        const int Bk = 2 * warp + (lane >> 4), c = lane & 15, o = 16 * Bk;
+        const float *ab = Ad + Bk * (16 * 17);
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float s = 0.f;
+#pragma unroll
+            for (int j = 0; j < i; ++j) s = fmaf(ab[i * 17 + j], x[j], s);
+            x[i] = (i < c) ? 0.f : (i == c) ? 1.f : -s;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) Tm[fsw(o + i, o + c)] = x[i];
+    } else {
+        for (int e = tid - 64; e < 6 * 256; e += NT - 64) {
+            const int blk = e >> 8, w = e & 255;
+            const int Ib = blk < 3 ? 0 : blk < 5 ? 1 : 2;
+            const int Jb = blk < 3 ? blk + 1 : blk < 5 ? blk - 1 : 3;
+            Tm[fsw(16 * Ib + (w >> 4), 16 * Jb + (w & 15))] = 0.f;
+        }
+    }
+    __syncthreads();
+    if (warp < 4) {
+        const int Ib = (warp >> 1) ? 3 : 1, Jb = Ib - 1, n0 = 16 * Jb + 8 * (warp & 1);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        tile_tf32<16>(c, Am, 16 * Ib, 16 * Jb, Tm, 16 * Jb, n0, gid, tig);
+        store_tile(Zs, c, 16 * Ib, n0, gid, tig, 1.f);
+    }
+    __syncthreads();
+    if (warp < 4) {
+        const int Ib = (warp >> 1) ? 3 : 1, Jb = Ib - 1, n0 = 16 * Jb + 8 * (warp & 1);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        tile_tf32<16>(c, Tm, 16 * Ib, 16 * Ib, Zs, 16 * Ib, n0, gid, tig);
+        store_tile(Tm, c, 16 * Ib, n0, gid, tig, -1.f);
+    }
+    __syncthreads();
+    {
+        const int r0 = 32 + 16 * (warp >> 2), n0 = 8 * (warp & 3);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        tile_tf32<32>(c, Am, r0, 0, Tm, 0, n0, gid, tig);
+        store_tile(Zs, c, r0, n0, gid, tig, 1.f);
+        __syncthreads();
+        float z[4] = {0.f, 0.f, 0.f, 0.f};
+        tile_tf32<32>(z, Tm, r0, 32, Zs, 32, n0, gid, tig);
+        store_tile(Tm, z, r0, n0, gid, tig, -1.f);
+    }
+    if (tid == 0) sm100::bulk_wait_read();
+    __syncthreads();
+}
+
+// The record of one (chunk, head) with every exponent referenced inside its
+// 16-token sub-chunk (any per-token g >= -5).  The tensor-core prep below
+// calls this for the chunks whose decay over the chunk leaves its exponent
+// range.  Called by all 256 threads of the CTA; smem_raw holds a PrepSmem.
 template <bool PRO>
-__global__ void __launch_bounds__(NT, 2)
-chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                  const __nv_bfloat16 *__restrict__ v, const float *__restrict__ g,
-                  const float *__restrict__ beta, const int32_t *__restrict__ cu,
-                  const int32_t *__restrict__ coff, int N, int T, int total_T, int H, int cps,
-                  unsigned char *__restrict__ wsp, Prologue pro)
+__device__ __forceinline__ void prep_subchunk(
+    unsigned char *smem_raw, const __nv_bfloat16 *__restrict__ q,
+    const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
+    const float *__restrict__ g, const float *__restrict__ beta, const int32_t *__restrict__ cu,
+    const int32_t *__restrict__ coff, int N, int T, int total_T, int H, int cps,
+    unsigned char *__restrict__ wsp, const Prologue &pro, int chunk, int h)
 {
-    extern __shared__ __align__(1024) unsigned char smem_raw[];
     PrepSmem &sm = *reinterpret_cast<PrepSmem *>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tig = lane & 3;
-    const int chunk = blockIdx.x, h = blockIdx.y;
-    if (cu && chunk >= coff[N]) return;
 
     int len;
     long long t0;
@@ -370,60 +501,7 @@ chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     // ---- T = (I + A)^-1 in fp32 ----
     const float *Am = reinterpret_cast<const float *>(sm.Xq);
     float *Tm = reinterpret_cast<float *>(sm.Xk);
-    float *Zs = reinterpret_cast<float *>(sm.Kd);
-    if (warp < 2) {
-        // 16x16 diagonal blocks: lane -> (block, column)
-        const int Bk = 2 * warp + (lane >> 4), c = lane & 15, o = 16 * Bk;
-        float x[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float s = 0.f;
-#pragma unroll
-            for (int j = 0; j < i; ++j) s += Am[fsw(o + i, o + j)] * x[j];
-            x[i] = (i < c) ? 0.f : (i == c) ? 1.f : -s;
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) Tm[fsw(o + i, o + c)] = x[i];
-    } else {
-        // zero the strictly-upper 16x16 blocks
-        for (int e = tid - 64; e < 6 * 256; e += NT - 64) {
-            const int blk = e >> 8, w = e & 255;
-            const int Ib = blk < 3 ? 0 : blk < 5 ? 1 : 2;
-            const int Jb = blk < 3 ? blk + 1 : blk < 5 ? blk - 1 : 3;
-            Tm[fsw(16 * Ib + (w >> 4), 16 * Jb + (w & 15))] = 0.f;
-        }
-    }
-    __syncthreads();
-    // Off-diagonal blocks on the tensor cores (tf32, fp32 accumulate), one
-    // 16x8 output tile per warp:
-    //   16-row level: T_IJ = -T_II (A_IJ T_JJ) for (I, J) = (1, 0), (3, 2)
-    //   32-row level: T[32:64, 0:32] = -T[32:64, 32:64] (A[32:64, 0:32] T[0:32, 0:32])
-    // Zs holds the inner products at the coordinates of the block they feed.
-    if (warp < 4) {
-        const int Ib = (warp >> 1) ? 3 : 1, Jb = Ib - 1, n0 = 16 * Jb + 8 * (warp & 1);
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-        tile_tf32<16>(c, Am, 16 * Ib, 16 * Jb, Tm, 16 * Jb, n0, gid, tig);
-        store_tile(Zs, c, 16 * Ib, n0, gid, tig, 1.f);
-    }
-    __syncthreads();
-    if (warp < 4) {
-        const int Ib = (warp >> 1) ? 3 : 1, Jb = Ib - 1, n0 = 16 * Jb + 8 * (warp & 1);
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-        tile_tf32<16>(c, Tm, 16 * Ib, 16 * Ib, Zs, 16 * Ib, n0, gid, tig);
-        store_tile(Tm, c, 16 * Ib, n0, gid, tig, -1.f);
-    }
-    __syncthreads();
-    {
-        const int r0 = 32 + 16 * (warp >> 2), n0 = 8 * (warp & 3);
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-        tile_tf32<32>(c, Am, r0, 0, Tm, 0, n0, gid, tig);
-        store_tile(Zs, c, r0, n0, gid, tig, 1.f);
-        __syncthreads();
-        float z[4] = {0.f, 0.f, 0.f, 0.f};
-        tile_tf32<32>(z, Tm, r0, 32, Zs, 32, n0, gid, tig);
-        store_tile(Tm, z, r0, n0, gid, tig, -1.f);
-    }
-    __syncthreads();
+    form_T(Am, Tm, reinterpret_cast<float *>(sm.Kd), tid);
 
     // ---- W = T (beta K e^G) (warps 0-3), U = T (beta V) (warps 4-7) ----
     {
@@ -481,6 +559,401 @@ chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     }
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core prep: the same record, every exponent referenced at the chunk
+// start.  With G the chunk-local inclusive cumsum,
+//     A_ij = (beta_i k_i e^{G_i}) . (k_j e^{-G_j})   (j < i)
+//     P_ij = (q_i e^{G_i}) . (k_j e^{-G_j})          (j <= i)
+// exactly; the factors are formed once per token and channel, so A and P are
+// each one product of full tiles.  This is used when every e^{+-G_i} and
+// e^{G_C - G_i} of the chunk lies within e^{+-80} (normal fp32 and bf16
+// numbers; for g <= 0 that is G_C >= -80, an average per-token g >= -1.25).
+// A chunk outside that range is done by prep_subchunk in the same CTA.
+//
+// Products on tcgen05 (one issuing thread, fp32 accumulators in TMEM):
+//   MMA-AP  [beta K e^G ; Q e^G] (128 x 128) x (K e^{-G})^T  -> TMEM cols 0-63
+//           (lanes 0-63: A before masking, lanes 64-127: P before masking)
+//   MMA-W   [T ; *] (128 x 64) x beta K e^G (64 x 128)        -> cols 0-127, lanes 0-63
+//   MMA-U   [* ; T] (128 x 64) x beta V     (64 x 128)        -> cols 128-255, lanes 64-127
+// The operand tiles are 8 x 8 core matrices (8 tokens x 16 bytes) without
+// swizzle, so one tile is both a K-major A operand (token rows, channels along
+// K) and an MN-major B operand (tokens along K, channels along N).  The rows
+// marked * are whatever lies next to T in shared memory; their products land
+// in TMEM lanes that are never read.  T itself comes from form_T (fp32).
+// ---------------------------------------------------------------------------
+namespace tcp {
+constexpr int CGS = 144;               // bytes between 8-channel core-matrix columns (128 + 16 pad)
+constexpr int TGS = 16 * CGS;          // bytes between 8-token core-matrix rows
+constexpr int TILE = 8 * TGS;          // one 64 x 128 bf16 tile (18,432 B)
+constexpr int OFF_K = 0;               // k, then beta k e^G   (MMA-AP A rows 0-63; MMA-W B)
+constexpr int OFF_Q = TILE;            // q, then q e^G        (MMA-AP A rows 64-127); then T fp32
+constexpr int OFF_KI = 2 * TILE;       // k e^{-G}             (MMA-AP B); then A fp32
+constexpr int OFF_V = 3 * TILE;        // v, then beta v       (MMA-U B)
+constexpr int OFF_TB = 4 * TILE;       // T bf16, 64 x 64 K-major core matrices (8 KB)
+constexpr int OFF_Z = OFF_TB + 8192;   // form_T scratch (fp32 64 x 64)
+constexpr int OFF_GS = OFF_Z + 16384;  // per-sub-chunk sums of g [4][128]
+constexpr int OFF_BETA = OFF_GS + 4 * D * 4;
+constexpr int OFF_RQ = OFF_BETA + C * 4;
+constexpr int OFF_RK = OFF_RQ + C * 4;
+constexpr int END = OFF_RK + C * 4;
+// the mbarrier and the TMEM slot sit past both this layout and PrepSmem, so
+// the fallback never overwrites them
+constexpr int OFF_BAR = (int)((((size_t)END > sizeof(PrepSmem) ? (size_t)END : sizeof(PrepSmem)) + 15) & ~(size_t)15);
+constexpr int BYTES = OFF_BAR + 16;
+constexpr uint32_t TMEM_COLS = 256;
+constexpr float RANGE = 80.f;          // |exponent| bound of the chunk-start reference
+__device__ __forceinline__ int cm(int t, int c) {
+    return (t >> 3) * TGS + (c >> 3) * CGS + ((t & 7) << 4) + ((c & 7) << 1);
+}
+}  // namespace tcp
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t x) {
+    return make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xffff0000u));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float2 v) { return pack_bf16(v.x, v.y); }
+
+template <bool PRO>
+__global__ void __launch_bounds__(NT, 2)
+chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                     const __nv_bfloat16 *__restrict__ v, const float *__restrict__ g,
+                     const float *__restrict__ beta, const int32_t *__restrict__ cu,
+                     const int32_t *__restrict__ coff, int N, int T, int total_T, int H, int cps,
+                     unsigned char *__restrict__ wsp, Prologue pro, int *__restrict__ err)
+{
+    using namespace sm100;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int chunk = blockIdx.x, h = blockIdx.y;
+    if (cu && chunk >= coff[N]) return;
+
+    int len;
+    long long t0;
+    locate_chunk(chunk, cu, coff, N, T, total_T, cps, t0, len);
+    unsigned char *rec = wsp + ((size_t)chunk * H + h) * ws::RECORD;
+    const size_t row_stride = (size_t)H * D;
+    const size_t base = ((size_t)t0 * H + h) * D;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + tcp::OFF_BAR);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + tcp::OFF_BAR + 8);
+    float *gs = reinterpret_cast<float *>(sm + tcp::OFF_GS);
+    float *bet = reinterpret_cast<float *>(sm + tcp::OFF_BETA);
+    float *rq = reinterpret_cast<float *>(sm + tcp::OFF_RQ);
+    float *rk = reinterpret_cast<float *>(sm + tcp::OFF_RK);
+
+    // ---- stage q, k, v into core-matrix tiles (zero past the end) ----
+    {
+        const uint32_t s0 = smem_u32(sm);
+#pragma unroll
+        for (int it = 0; it < C * (D / 8) / NT; ++it) {
+            const int i = tid + it * NT;
+            const int r = i >> 4, j = i & 15;
+            const bool ok = r < len;
+            const size_t off = ok ? base + (size_t)r * row_stride + j * 8 : 0;
+            const uint32_t so = (r >> 3) * tcp::TGS + j * tcp::CGS + ((r & 7) << 4), n = ok ? 16 : 0;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s0 + tcp::OFF_Q + so), "l"(q + off), "r"(n));
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s0 + tcp::OFF_K + so), "l"(k + off), "r"(n));
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s0 + tcp::OFF_V + so), "l"(v + off), "r"(n));
+        }
+        cp_async_commit();
+    }
+
+    // ---- g: thread (sub-chunk I, channels c0, c0 + 1); local cumsum ----
+    const int I = tid >> 6, c0 = 2 * (tid & 63);
+    float2 G[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int r = 16 * I + i;
+        G[i] = make_float2(0.f, 0.f);
+        if (r < len) G[i] = *reinterpret_cast<const float2 *>(g + base + (size_t)r * row_stride + c0);
+    }
+#pragma unroll
+    for (int i = 1; i < 16; ++i) { G[i].x += G[i - 1].x; G[i].y += G[i - 1].y; }
+    *reinterpret_cast<float2 *>(gs + I * D + c0) = G[15];
+    if (tid < C) {
+        float bt = (tid < len) ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+        if (PRO && (pro.flags & kProBetaSigmoid) && tid < len) bt = sigmoid_f(bt);
+        bet[tid] = bt;
+    }
+    if (warp == 0) { tmem_alloc(tslot, tcp::TMEM_COLS); tmem_relinquish(); }
+    if (tid == 0) { mbar_init(bar, 1); fence_mbar_init(); }
+    cp_async_wait<0>();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+
+    // ---- prefix of the earlier sub-chunks; chunk total G_C; range check ----
+    float2 GC = make_float2(0.f, 0.f), PF = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int J = 0; J < 4; ++J) {
+        const float2 sj = *reinterpret_cast<const float2 *>(gs + J * D + c0);
+        if (J < I) { PF.x += sj.x; PF.y += sj.y; }
+        GC.x += sj.x; GC.y += sj.y;
+    }
+    bool bad = false;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        G[i].x += PF.x; G[i].y += PF.y;
+        bad |= !(fabsf(G[i].x) <= tcp::RANGE && fabsf(G[i].y) <= tcp::RANGE &&
+                 GC.x - G[i].x <= tcp::RANGE && GC.y - G[i].y <= tcp::RANGE);
+    }
+    if (__syncthreads_or(bad)) {
+        // out of the chunk-start range: 16-token references, mma.sync products
+        prep_subchunk<PRO>(sm, q, k, v, g, beta, cu, coff, N, T, total_T, H, cps, wsp, pro, chunk, h);
+        __syncthreads();
+        if (warp == 0) tmem_dealloc(tmem, tcp::TMEM_COLS);
+        return;
+    }
+
+    if (PRO) {
+        // per-row factors (thread: tensor tid >> 7, row, half of the row)
+        const int tens = tid >> 7, rr = (tid >> 1) & 63, hf = tid & 1;
+        float f = 1.f;
+        if (pro.flags & kProQkL2Norm) {
+            const unsigned char *tile = sm + (tens ? tcp::OFF_K : tcp::OFF_Q) + (rr >> 3) * tcp::TGS + ((rr & 7) << 4);
+            float ss = 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint4 x = *reinterpret_cast<const uint4 *>(tile + (8 * hf + j) * tcp::CGS);
+                const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 p2 = bf16x2_to_float2(w[e]);
+                    ss = fmaf(p2.x, p2.x, fmaf(p2.y, p2.y, ss));
+                }
+            }
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            f = inv_norm(ss);
+        }
+        if (hf == 0) {
+            if (tens) rk[rr] = f;
+            else rq[rr] = f * pro.q_scale;
+        }
+        __syncthreads();
+    }
+
+    // ---- decayed forms: q e^G, beta k e^G, k e^{-G}, beta v (shared memory,
+    // in place), q e^G and K e^{G_C - G} (record), e^{G_C} (record) ----
+    uint32_t qgr[16], kt[2][8];
+    {
+        constexpr float L2E = 1.4426950408889634f;
+        const float2 egc = make_float2(ex2_approx(GC.x * L2E), ex2_approx(GC.y * L2E));
+        if (I == 0) *reinterpret_cast<float2 *>(rec + ws::OFF_EGC + c0 * 4) = make_float2(expf(GC.x), expf(GC.y));
+        float2 kt_prev = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int r = 16 * I + i;
+            const int o = tcp::cm(r, c0);
+            const float2 eg = make_float2(ex2_approx(G[i].x * L2E), ex2_approx(G[i].y * L2E));
+            const float2 em = make_float2(ex2_approx(-G[i].x * L2E), ex2_approx(-G[i].y * L2E));
+            float2 qf = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(sm + tcp::OFF_Q + o));
+            float2 kf = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(sm + tcp::OFF_K + o));
+            const float2 vf = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(sm + tcp::OFF_V + o));
+            if (PRO) {
+                const float fq = rq[r], fk = rk[r];
+                qf = __fmul2_rn(qf, make_float2(fq, fq));
+                kf = __fmul2_rn(kf, make_float2(fk, fk));
+            }
+            const float br = bet[r];
+            const float2 b2 = make_float2(br, br);
+            const uint32_t qg = pack_bf16x2(__fmul2_rn(qf, eg));
+            const float2 ki = __fmul2_rn(kf, em);
+            const float2 kt2 = __fmul2_rn(ki, egc);
+            *reinterpret_cast<uint32_t *>(sm + tcp::OFF_Q + o) = qg;
+            qgr[i] = qg;
+            *reinterpret_cast<uint32_t *>(sm + tcp::OFF_K + o) = pack_bf16x2(__fmul2_rn(__fmul2_rn(kf, b2), eg));
+            *reinterpret_cast<uint32_t *>(sm + tcp::OFF_KI + o) = pack_bf16x2(ki);
+            *reinterpret_cast<uint32_t *>(sm + tcp::OFF_V + o) = pack_bf16x2(__fmul2_rn(vf, b2));
+            if (i & 1) {
+                kt[0][i >> 1] = pack_bf16(kt_prev.x, kt2.x);
+                kt[1][i >> 1] = pack_bf16(kt_prev.y, kt2.y);
+            } else {
+                kt_prev = kt2;
+            }
+        }
+        // K e^{G_C - G} transposed (channel rows, 64 tokens, 128-byte swizzle)
+        // into its record image in the scratch region
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                *reinterpret_cast<uint4 *>(sm + tcp::OFF_Z + ws::sw128(c0 + e, 16 * I + 8 * hh)) =
+                    make_uint4(kt[e][4 * hh], kt[e][4 * hh + 1], kt[e][4 * hh + 2], kt[e][4 * hh + 3]);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    const uint32_t sb = smem_u32(sm);
+    bool ok = true;
+    if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t ID_AP = idesc_bf16(128, 64, false);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+            umma_bf16(tmem, smem_desc(sb + tcp::OFF_K + kk * 2 * tcp::CGS, tcp::CGS, tcp::TGS, 0),
+                      smem_desc(sb + tcp::OFF_KI + kk * 2 * tcp::CGS, tcp::CGS, tcp::TGS, 0), ID_AP, kk > 0);
+        umma_commit(bar);
+    }
+    // record stores of q e^G (coalesced rows) overlap the MMA; K e^{G_C - G}
+    // leaves as one bulk copy of its shared-memory image
+    if (tid == 0) {
+        bulk_s2g(rec + ws::OFF_KTT, sm + tcp::OFF_Z, 16384);
+        bulk_commit();
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        *reinterpret_cast<uint32_t *>(rec + ws::aw_off(64 + 16 * I + i, c0)) = qgr[i];
+    // one thread waits for the MMA (and for the image to be read); the
+    // others sleep at the barrier
+    if (tid == 0) {
+        ok = mbar_wait(bar, 0);
+        bulk_wait_read();
+    }
+    ok = __syncthreads_and(ok);
+    tc_fence_after();
+
+    // ---- A (masked j < i) -> fp32 for form_T; P (masked j <= i) -> record ----
+    float *Am = reinterpret_cast<float *>(sm + tcp::OFF_KI);
+    float *Tm = reinterpret_cast<float *>(sm + tcp::OFF_Q);
+    float *Ad = reinterpret_cast<float *>(sm + tcp::OFF_Z);   // after the K^T image is read
+    if (ok && warp < 4) {
+        float x[64];
+        const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16);
+        tmem_ld32(ta, *reinterpret_cast<float (*)[32]>(&x[0]));
+        tmem_ld32(ta + 32, *reinterpret_cast<float (*)[32]>(&x[32]));
+        tmem_wait_ld();
+        const int i = (warp & 1) * 32 + lane;
+        if (warp < 2) {
+#pragma unroll
+            for (int j4 = 0; j4 < 16; ++j4) {
+                float4 a4;
+                a4.x = (4 * j4 < i) ? x[4 * j4] : 0.f;
+                a4.y = (4 * j4 + 1 < i) ? x[4 * j4 + 1] : 0.f;
+                a4.z = (4 * j4 + 2 < i) ? x[4 * j4 + 2] : 0.f;
+                a4.w = (4 * j4 + 3 < i) ? x[4 * j4 + 3] : 0.f;
+                *reinterpret_cast<float4 *>(Am + i * 64 + 4 * (j4 ^ (i & 7))) = a4;
+            }
+            // the row's diagonal block, padded copy for the substitution
+            float *adr = Ad + (i >> 4) * (16 * 17) + (i & 15) * 17;
+            const int B = i >> 4, ii = i & 15;
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+                const float a = B == 0 ? x[jj] : B == 1 ? x[16 + jj] : B == 2 ? x[32 + jj] : x[48 + jj];
+                adr[jj] = (jj < ii) ? a : 0.f;
+            }
+        } else {
+            unsigned char *img = sm + tcp::OFF_TB;
+#pragma unroll
+            for (int jc = 0; jc < 8; ++jc) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 8 * jc + 2 * e;
+                    pk[e] = pack_bf16(j <= i ? x[j] : 0.f, j + 1 <= i ? x[j + 1] : 0.f);
+                }
+                *reinterpret_cast<uint4 *>(img + i * 128 + ((jc ^ (i & 7)) << 4)) =
+                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+            fence_proxy_async_smem();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (ok) {
+        if (tid == 0) {
+            bulk_s2g(rec + ws::OFF_P, sm + tcp::OFF_TB, 8192);
+            bulk_commit();
+        }
+        form_T_padded_diag(Am, Ad, Tm, reinterpret_cast<float *>(sm + tcp::OFF_Z), tid);
+        // T -> bf16, K-major core matrices: (i, j) at (i/8)*1024 + (j/8)*128 + (i%8)*16 + (j%8)*2
+        {
+            const int i = tid >> 2, jq = tid & 3;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int jg = 2 * jq + hh;
+                const float4 lo = *reinterpret_cast<const float4 *>(Tm + i * 64 + 4 * ((2 * jg) ^ (i & 7)));
+                const float4 hi = *reinterpret_cast<const float4 *>(Tm + i * 64 + 4 * ((2 * jg + 1) ^ (i & 7)));
+                *reinterpret_cast<uint4 *>(sm + tcp::OFF_TB + (i >> 3) * 1024 + jg * 128 + ((i & 7) << 4)) =
+                    make_uint4(pack_bf16(lo.x, lo.y), pack_bf16(lo.z, lo.w), pack_bf16(hi.x, hi.y),
+                               pack_bf16(hi.z, hi.w));
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t ID_WU = idesc_bf16(128, 128, true);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(tmem, smem_desc(sb + tcp::OFF_TB + kk * 256, 128, 1024, 0),
+                          smem_desc(sb + tcp::OFF_K + kk * 2 * tcp::TGS, tcp::TGS, tcp::CGS, 0), ID_WU, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(tmem + 128, smem_desc(sb + tcp::OFF_TB - 8192 + kk * 256, 128, 1024, 0),
+                          smem_desc(sb + tcp::OFF_V + kk * 2 * tcp::TGS, tcp::TGS, tcp::CGS, 0), ID_WU, kk > 0);
+            umma_commit(bar);
+        }
+        if (tid == 0) ok = mbar_wait(bar, 1);
+        ok = __syncthreads_and(ok);
+        tc_fence_after();
+        if (ok) {
+            // W rows (TMEM lanes 0-63, cols 0-127) and U rows (lanes 64-127,
+            // cols 128-255); warp w: lane quarter w & 3, column half w >> 2
+            const int qd = warp & 3, hf = warp >> 2;
+            const int r = (qd & 1) * 32 + lane;
+            float x[64];
+            const uint32_t ta = tmem + ((uint32_t)(qd * 32) << 16) + (qd < 2 ? 0u : 128u) + 64u * hf;
+            tmem_ld32(ta, *reinterpret_cast<float (*)[32]>(&x[0]));
+            tmem_ld32(ta + 32, *reinterpret_cast<float (*)[32]>(&x[32]));
+            tmem_wait_ld();
+            // record images: W (rows 0-63 of both 64-channel blocks of [W; Qg])
+            // over the dead k tile, U (four 64 x 32 tiles) over the dead v tile
+            if (qd < 2) {
+                unsigned char *dst = sm + tcp::OFF_K + hf * 8192 + r * 128;
+#pragma unroll
+                for (int jc = 0; jc < 8; ++jc)
+                    *reinterpret_cast<uint4 *>(dst + ((jc ^ (r & 7)) << 4)) =
+                        make_uint4(pack_bf16(x[8 * jc], x[8 * jc + 1]), pack_bf16(x[8 * jc + 2], x[8 * jc + 3]),
+                                   pack_bf16(x[8 * jc + 4], x[8 * jc + 5]), pack_bf16(x[8 * jc + 6], x[8 * jc + 7]));
+            } else {
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt) {
+                    unsigned char *dst = sm + tcp::OFF_V + (2 * hf + tt) * ws::U_TILE + r * 64;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float *xs = x + 32 * tt + 8 * e;
+                        *reinterpret_cast<uint4 *>(dst + 16 * e) =
+                            make_uint4(pack_bf16(xs[0], xs[1]), pack_bf16(xs[2], xs[3]),
+                                       pack_bf16(xs[4], xs[5]), pack_bf16(xs[6], xs[7]));
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+        }
+        __syncthreads();
+        if (ok && tid == 0) {
+            bulk_s2g(rec + ws::OFF_AW, sm + tcp::OFF_K, 8192);
+            bulk_s2g(rec + ws::OFF_AW + 16384, sm + tcp::OFF_K + 8192, 8192);
+            bulk_s2g(rec + ws::OFF_U, sm + tcp::OFF_V, 4 * ws::U_TILE);
+            bulk_commit();
+        }
+    }
+    // the shared-memory sources of the bulk stores must be read before exit
+    if (tid == 0) bulk_wait_read();
+    if (!ok && tid == 0) set_device_error(err, kErrWaitTimeout);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, tcp::TMEM_COLS);
+}
+
 // Chunk offsets per sequence for varlen mode: coff[n] = sum_{m<n} ceil(len_m / C).
 __global__ void chunk_plan_kernel(const int32_t *__restrict__ cu, int N, int total_T,
                                   int32_t *__restrict__ coff)
@@ -513,7 +986,7 @@ __global__ void chunk_plan_kernel(const int32_t *__restrict__ cu, int N, int tot
 
 }  // namespace
 
-size_t chunk_prep_smem_bytes() { return sizeof(PrepSmem); }
+size_t chunk_prep_smem_bytes() { return tcp::BYTES + 128; }
 
 cudaError_t launch_chunk_plan(const int32_t *cu, int N, int total_T, int32_t *coff,
                               cudaStream_t st)
@@ -525,18 +998,18 @@ cudaError_t launch_chunk_plan(const int32_t *cu, int N, int total_T, int32_t *co
 cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const int32_t *cu, const int32_t *coff,
                               int N, int T, int total_T, int H, int max_chunks,
-                              unsigned char *wsp, Prologue pro, cudaStream_t st)
+                              unsigned char *wsp, Prologue pro, int *err, cudaStream_t st)
 {
-    const size_t smem = sizeof(PrepSmem);
+    const size_t smem = tcp::BYTES + 128;
     const bool use_pro = pro.flags != 0 || pro.q_scale != 1.f;
-    auto kern = use_pro ? chunk_prep_kernel<true> : chunk_prep_kernel<false>;
+    auto kern = use_pro ? chunk_prep_tc_kernel<true> : chunk_prep_tc_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int cps = (T + C - 1) / C;
     dim3 grid(max_chunks, H);
     kern<<<grid, NT, smem, st>>>(
         (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, g, beta,
-        cu, coff, N, T, total_T, H, cps, wsp, pro);
+        cu, coff, N, T, total_T, H, cps, wsp, pro, err);
     return cudaGetLastError();
 }
 

@@ -79,6 +79,7 @@ cudaError_t launch_chunk_f32(const float *q, const float *k, const float *v, con
 // buffer of per-(chunk, head) records (chunk_ws.h):
 //   chunk_plan  (varlen only) chunk offsets per sequence -> coff[N+1]
 //   chunk_prep  parallel over (chunk, head): G, A, P, T, W, U, Qg, Kt, e^{G_C}
+//               (A, P, W, U on tcgen05; err receives bounded-wait failures)
 //   chunk_chain sequential over chunks per (sequence, head, dv tile),
 //               tcgen05 MMAs with TMEM accumulators (chunk_chain_tc.cu)
 size_t chunk_prep_smem_bytes();
@@ -87,7 +88,7 @@ cudaError_t launch_chunk_plan(const int32_t *cu, int N, int total_T, int32_t *co
 cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const int32_t *cu, const int32_t *coff,
                               int N, int T, int total_T, int H, int max_chunks,
-                              unsigned char *wsp, Prologue pro, cudaStream_t st);
+                              unsigned char *wsp, Prologue pro, int *err, cudaStream_t st);
 cudaError_t launch_chunk_chain(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
                                const float *s0, float *sT, void *out, int N, int T, int total_T,
                                int H, int dvt, int max_chunks, int *err, cudaStream_t st);

@@ -57,6 +57,19 @@ def test_strongest_supported_decay():
     _check(inp)
 
 
+@pytest.mark.parametrize("g_floor", [-1.2, -1.3, -2.0])
+def test_mixed_exponent_ranges(g_floor):
+    """Chunks whose decay over the chunk stays within e^80 use one exponent
+    reference per chunk, the others 16-token references: a per-token g of
+    -1.2 on some channels keeps a 64-token chunk inside (|G_C| = 76.8),
+    -1.3 and -2 push it outside.  The strong decay sits on chunks 1 and 3 of
+    one head only, so both kinds of chunk meet in one call and in one chain."""
+    inp = W.prefill(1, 320, 3, 128, 128, BF, seed=41, initial_state_std=0.02)
+    inp.g[:, 64:128, 1, ::5] = g_floor
+    inp.g[:, 192:250, 1, 3::7] = g_floor
+    _check(inp)
+
+
 def test_varlen_with_empty_and_short_sequences():
     inp = W.prefill(1, 0, 3, 128, 128, BF, seed=21, initial_state_std=0.02,
                     seq_lens=[70, 0, 1, 128, 0, 200, 64, 65])

@@ -41,6 +41,10 @@
 // substitution, then the 2x2-block recursion T21 = -T22 A21 T11 at 16 and 32
 // rows on tf32 tensor-core MMAs with fp32 accumulation) and round T once to
 // bf16 for the W and U products.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "chunk_ws.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -570,40 +574,48 @@ __device__ __forceinline__ void prep_subchunk(
 // numbers; for g <= 0 that is G_C >= -80, an average per-token g >= -1.25).
 // A chunk outside that range is done by prep_subchunk in the same CTA.
 //
-// Products on tcgen05 (one issuing thread, fp32 accumulators in TMEM):
+// Inputs arrive by TMA (tensor maps over [tokens, heads, channels]; no
+// multicast), which keeps ~80 KB per CTA in flight where per-thread copies
+// were limited to ~20 GB/s per SM.  Products on tcgen05 (one issuing thread,
+// fp32 accumulators in TMEM):
 //   MMA-AP  [beta K e^G ; Q e^G] (128 x 128) x (K e^{-G})^T  -> TMEM cols 0-63
 //           (lanes 0-63: A before masking, lanes 64-127: P before masking)
 //   MMA-W   [T ; *] (128 x 64) x beta K e^G (64 x 128)        -> cols 0-127, lanes 0-63
 //   MMA-U   [* ; T] (128 x 64) x beta V     (64 x 128)        -> cols 128-255, lanes 64-127
-// The operand tiles are 8 x 8 core matrices (8 tokens x 16 bytes) without
-// swizzle, so one tile is both a K-major A operand (token rows, channels along
-// K) and an MN-major B operand (tokens along K, channels along N).  The rows
-// marked * are whatever lies next to T in shared memory; their products land
-// in TMEM lanes that are never read.  T itself comes from form_T (fp32).
+// The rows marked * are whatever lies next to T in shared memory; their
+// products land in TMEM lanes that are never read.  T itself comes from
+// form_T_padded_diag (fp32).  Record parts leave by bulk async stores of
+// their shared-memory images.
 // ---------------------------------------------------------------------------
 namespace tcp {
-constexpr int CGS = 144;               // bytes between 8-channel core-matrix columns (128 + 16 pad)
-constexpr int TGS = 16 * CGS;          // bytes between 8-token core-matrix rows
-constexpr int TILE = 8 * TGS;          // one 64 x 128 bf16 tile (18,432 B)
-constexpr int OFF_K = 0;               // k, then beta k e^G   (MMA-AP A rows 0-63; MMA-W B)
-constexpr int OFF_Q = TILE;            // q, then q e^G        (MMA-AP A rows 64-127); then T fp32
-constexpr int OFF_KI = 2 * TILE;       // k e^{-G}             (MMA-AP B); then A fp32
-constexpr int OFF_V = 3 * TILE;        // v, then beta v       (MMA-U B)
-constexpr int OFF_TB = 4 * TILE;       // T bf16, 64 x 64 K-major core matrices (8 KB)
-constexpr int OFF_Z = OFF_TB + 8192;   // form_T scratch (fp32 64 x 64)
-constexpr int OFF_GS = OFF_Z + 16384;  // per-sub-chunk sums of g [4][128]
+// Tiles are K-major with the 128-byte swizzle (rows of 64 bf16 = 128 bytes,
+// 16-byte chunk j of row r at j ^ (r % 8), 8-row groups 1024 bytes apart), as
+// TMA writes them with SWIZZLE_128B.  Read with rows = tokens they are the
+// K-major A operands of MMA-AP; the same bytes are the MN-major B operands of
+// MMA-W and MMA-U (tokens along K, 64-channel atoms along N).
+constexpr int OFF_KQ = 0;              // per 64-channel block b at b * 16384:
+                                       //   [k -> beta k e^G : 64 rows][q -> q e^G : 64 rows]
+constexpr int OFF_KI = 32768;          // k e^{-G} (block b at b * 8192); then A (fp32 64 x 64)
+constexpr int OFF_Z = 49152;           // K^T image; then the padded diagonal blocks; then form_T scratch
+constexpr int OFF_G = OFF_KI;          // g (fp32 [64][128], TMA) until the cumsum has read it
+constexpr int OFF_V = 65536;           // v -> beta v (block b at b * 8192)
+constexpr int OFF_TB = 81920;          // P image, then T (bf16, 64 swizzled rows)
+constexpr int OFF_TM = 90112;          // T (fp32 64 x 64); also the rows after T in MMA-W's A
+constexpr int OFF_GS = 106496;         // per-sub-chunk sums of g [4][128]
 constexpr int OFF_BETA = OFF_GS + 4 * D * 4;
 constexpr int OFF_RQ = OFF_BETA + C * 4;
 constexpr int OFF_RK = OFF_RQ + C * 4;
 constexpr int END = OFF_RK + C * 4;
-// the mbarrier and the TMEM slot sit past both this layout and PrepSmem, so
-// the fallback never overwrites them
+// mbarriers and the TMEM slot sit past both this layout and PrepSmem, so the
+// fallback never overwrites them
 constexpr int OFF_BAR = (int)((((size_t)END > sizeof(PrepSmem) ? (size_t)END : sizeof(PrepSmem)) + 15) & ~(size_t)15);
-constexpr int BYTES = OFF_BAR + 16;
+constexpr int BYTES = OFF_BAR + 32;
+constexpr uint32_t TX = 6 * 8192 + C * D * 4;   // q, k, v (two 64-channel boxes each) + g
 constexpr uint32_t TMEM_COLS = 256;
 constexpr float RANGE = 80.f;          // |exponent| bound of the chunk-start reference
-__device__ __forceinline__ int cm(int t, int c) {
-    return (t >> 3) * TGS + (c >> 3) * CGS + ((t & 7) << 4) + ((c & 7) << 1);
+// byte offset of (row r, channel c in 0..63) in a swizzled 64-channel block
+__device__ __forceinline__ int sw(int r, int c) {
+    return r * 128 + ((((c >> 3) ^ (r & 7))) << 4) + ((c & 7) << 1);
 }
 }  // namespace tcp
 
@@ -616,10 +628,21 @@ __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t x) {
     return make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xffff0000u));
 }
 __device__ __forceinline__ uint32_t pack_bf16x2(float2 v) { return pack_bf16(v.x, v.y); }
+// 3-D tiled TMA load (no multicast) completing on an mbarrier
+__device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *map, int x, int y, int z,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z),
+          "r"(smem_u32(bar))
+        : "memory");
+}
 
 template <bool PRO>
 __global__ void __launch_bounds__(NT, 2)
-chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                     const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                      const __nv_bfloat16 *__restrict__ v, const float *__restrict__ g,
                      const float *__restrict__ beta, const int32_t *__restrict__ cu,
                      const int32_t *__restrict__ coff, int N, int T, int total_T, int H, int cps,
@@ -628,7 +651,7 @@ chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *_
     using namespace sm100;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int chunk = blockIdx.x, h = blockIdx.y;
     if (cu && chunk >= coff[N]) return;
@@ -637,56 +660,60 @@ chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *_
     long long t0;
     locate_chunk(chunk, cu, coff, N, T, total_T, cps, t0, len);
     unsigned char *rec = wsp + ((size_t)chunk * H + h) * ws::RECORD;
-    const size_t row_stride = (size_t)H * D;
-    const size_t base = ((size_t)t0 * H + h) * D;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + tcp::OFF_BAR);
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + tcp::OFF_BAR + 8);
+    uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + tcp::OFF_BAR);
+    uint64_t *bar = bar_ld + 1;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + tcp::OFF_BAR + 16);
     float *gs = reinterpret_cast<float *>(sm + tcp::OFF_GS);
     float *bet = reinterpret_cast<float *>(sm + tcp::OFF_BETA);
     float *rq = reinterpret_cast<float *>(sm + tcp::OFF_RQ);
     float *rk = reinterpret_cast<float *>(sm + tcp::OFF_RK);
 
-    // ---- stage q, k, v into core-matrix tiles (zero past the end) ----
-    {
-        const uint32_t s0 = smem_u32(sm);
+    // ---- stage q, k, v (two 64-channel boxes each) and g by TMA; rows past
+    // the sequence end are masked below, rows past the tensor read as zero ----
+    if (tid == 0) {
+        mbar_init(bar_ld, 1);
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(bar_ld, tcp::TX);
+        const int tt = (int)t0;
 #pragma unroll
-        for (int it = 0; it < C * (D / 8) / NT; ++it) {
-            const int i = tid + it * NT;
-            const int r = i >> 4, j = i & 15;
-            const bool ok = r < len;
-            const size_t off = ok ? base + (size_t)r * row_stride + j * 8 : 0;
-            const uint32_t so = (r >> 3) * tcp::TGS + j * tcp::CGS + ((r & 7) << 4), n = ok ? 16 : 0;
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s0 + tcp::OFF_Q + so), "l"(q + off), "r"(n));
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s0 + tcp::OFF_K + so), "l"(k + off), "r"(n));
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s0 + tcp::OFF_V + so), "l"(v + off), "r"(n));
+        for (int b = 0; b < 2; ++b) {
+            tma_load_3d(sm + tcp::OFF_KQ + b * 16384, &tm_k, 64 * b, h, tt, bar_ld);
+            tma_load_3d(sm + tcp::OFF_KQ + b * 16384 + 8192, &tm_q, 64 * b, h, tt, bar_ld);
+            tma_load_3d(sm + tcp::OFF_V + b * 8192, &tm_v, 64 * b, h, tt, bar_ld);
         }
-        cp_async_commit();
+        tma_load_3d(sm + tcp::OFF_G, &tm_g, 0, h, tt, bar_ld);
     }
-
-    // ---- g: thread (sub-chunk I, channels c0, c0 + 1); local cumsum ----
-    const int I = tid >> 6, c0 = 2 * (tid & 63);
-    float2 G[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int r = 16 * I + i;
-        G[i] = make_float2(0.f, 0.f);
-        if (r < len) G[i] = *reinterpret_cast<const float2 *>(g + base + (size_t)r * row_stride + c0);
-    }
-#pragma unroll
-    for (int i = 1; i < 16; ++i) { G[i].x += G[i - 1].x; G[i].y += G[i - 1].y; }
-    *reinterpret_cast<float2 *>(gs + I * D + c0) = G[15];
     if (tid < C) {
         float bt = (tid < len) ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
         if (PRO && (pro.flags & kProBetaSigmoid) && tid < len) bt = sigmoid_f(bt);
         bet[tid] = bt;
     }
     if (warp == 0) { tmem_alloc(tslot, tcp::TMEM_COLS); tmem_relinquish(); }
-    if (tid == 0) { mbar_init(bar, 1); fence_mbar_init(); }
-    cp_async_wait<0>();
+    bool ok = true;
+    if (tid == 0) ok = mbar_wait(bar_ld, 0);
     tc_fence_before();
-    __syncthreads();
+    ok = __syncthreads_and(ok);
     tc_fence_after();
     const uint32_t tmem = *tslot;
+
+    // ---- g: thread (sub-chunk I, channels c0, c0 + 1); local cumsum ----
+    const int I = tid >> 6, c0 = 2 * (tid & 63);
+    const int cb = c0 >> 6, cc = c0 & 63;          // 64-channel block, channel within it
+    float2 G[16];
+    {
+        const float *gsm = reinterpret_cast<const float *>(sm + tcp::OFF_G);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int r = 16 * I + i;
+            G[i] = make_float2(0.f, 0.f);
+            if (r < len) G[i] = *reinterpret_cast<const float2 *>(gsm + r * D + c0);
+        }
+    }
+#pragma unroll
+    for (int i = 1; i < 16; ++i) { G[i].x += G[i - 1].x; G[i].y += G[i - 1].y; }
+    *reinterpret_cast<float2 *>(gs + I * D + c0) = G[15];
+    __syncthreads();
 
     // ---- prefix of the earlier sub-chunks; chunk total G_C; range check ----
     float2 GC = make_float2(0.f, 0.f), PF = make_float2(0.f, 0.f);
@@ -696,7 +723,7 @@ chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *_
         if (J < I) { PF.x += sj.x; PF.y += sj.y; }
         GC.x += sj.x; GC.y += sj.y;
     }
-    bool bad = false;
+    bool bad = !ok;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         G[i].x += PF.x; G[i].y += PF.y;
@@ -704,23 +731,25 @@ chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *_
                  GC.x - G[i].x <= tcp::RANGE && GC.y - G[i].y <= tcp::RANGE);
     }
     if (__syncthreads_or(bad)) {
-        // out of the chunk-start range: 16-token references, mma.sync products
-        prep_subchunk<PRO>(sm, q, k, v, g, beta, cu, coff, N, T, total_T, H, cps, wsp, pro, chunk, h);
+        // out of the chunk-start range (or the staging wait ran out): 16-token
+        // references, mma.sync products, its own loads
+        if (!ok && tid == 0) set_device_error(err, kErrWaitTimeout);
+        if (ok) prep_subchunk<PRO>(sm, q, k, v, g, beta, cu, coff, N, T, total_T, H, cps, wsp, pro, chunk, h);
         __syncthreads();
         if (warp == 0) tmem_dealloc(tmem, tcp::TMEM_COLS);
         return;
     }
 
     if (PRO) {
-        // per-row factors (thread: tensor tid >> 7, row, half of the row)
+        // per-row factors (thread: tensor tid >> 7, row, 64-channel block)
         const int tens = tid >> 7, rr = (tid >> 1) & 63, hf = tid & 1;
         float f = 1.f;
         if (pro.flags & kProQkL2Norm) {
-            const unsigned char *tile = sm + (tens ? tcp::OFF_K : tcp::OFF_Q) + (rr >> 3) * tcp::TGS + ((rr & 7) << 4);
+            const unsigned char *row = sm + tcp::OFF_KQ + hf * 16384 + (tens ? 0 : 8192) + rr * 128;
             float ss = 0.f;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const uint4 x = *reinterpret_cast<const uint4 *>(tile + (8 * hf + j) * tcp::CGS);
+                const uint4 x = *reinterpret_cast<const uint4 *>(row + 16 * j);
                 const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -738,23 +767,28 @@ chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *_
         __syncthreads();
     }
 
-    // ---- decayed forms: q e^G, beta k e^G, k e^{-G}, beta v (shared memory,
-    // in place), q e^G and K e^{G_C - G} (record), e^{G_C} (record) ----
-    uint32_t qgr[16], kt[2][8];
+    // ---- decayed forms: q e^G, beta k e^G, beta v (in place), k e^{-G}
+    // (over the consumed g), K e^{G_C - G} image, q e^G and e^{G_C} (record) ----
+    uint32_t qgr[16];
     {
         constexpr float L2E = 1.4426950408889634f;
         const float2 egc = make_float2(ex2_approx(GC.x * L2E), ex2_approx(GC.y * L2E));
         if (I == 0) *reinterpret_cast<float2 *>(rec + ws::OFF_EGC + c0 * 4) = make_float2(expf(GC.x), expf(GC.y));
+        uint32_t kt[2][8];
         float2 kt_prev = make_float2(0.f, 0.f);
+        unsigned char *kq = sm + tcp::OFF_KQ + cb * 16384;
+        unsigned char *ki = sm + tcp::OFF_KI + cb * 8192;
+        unsigned char *vv = sm + tcp::OFF_V + cb * 8192;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int r = 16 * I + i;
-            const int o = tcp::cm(r, c0);
+            const int o = tcp::sw(r, cc);
             const float2 eg = make_float2(ex2_approx(G[i].x * L2E), ex2_approx(G[i].y * L2E));
             const float2 em = make_float2(ex2_approx(-G[i].x * L2E), ex2_approx(-G[i].y * L2E));
-            float2 qf = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(sm + tcp::OFF_Q + o));
-            float2 kf = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(sm + tcp::OFF_K + o));
-            const float2 vf = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(sm + tcp::OFF_V + o));
+            float2 qf = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(kq + 8192 + o));
+            float2 kf = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(kq + o));
+            float2 vf = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(vv + o));
+            if (r >= len) { qf = kf = vf = make_float2(0.f, 0.f); }
             if (PRO) {
                 const float fq = rq[r], fk = rk[r];
                 qf = __fmul2_rn(qf, make_float2(fq, fq));
@@ -763,13 +797,13 @@ chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *_
             const float br = bet[r];
             const float2 b2 = make_float2(br, br);
             const uint32_t qg = pack_bf16x2(__fmul2_rn(qf, eg));
-            const float2 ki = __fmul2_rn(kf, em);
-            const float2 kt2 = __fmul2_rn(ki, egc);
-            *reinterpret_cast<uint32_t *>(sm + tcp::OFF_Q + o) = qg;
+            const float2 kinv = __fmul2_rn(kf, em);
+            const float2 kt2 = __fmul2_rn(kinv, egc);
+            *reinterpret_cast<uint32_t *>(kq + 8192 + o) = qg;
             qgr[i] = qg;
-            *reinterpret_cast<uint32_t *>(sm + tcp::OFF_K + o) = pack_bf16x2(__fmul2_rn(__fmul2_rn(kf, b2), eg));
-            *reinterpret_cast<uint32_t *>(sm + tcp::OFF_KI + o) = pack_bf16x2(ki);
-            *reinterpret_cast<uint32_t *>(sm + tcp::OFF_V + o) = pack_bf16x2(__fmul2_rn(vf, b2));
+            *reinterpret_cast<uint32_t *>(kq + o) = pack_bf16x2(__fmul2_rn(__fmul2_rn(kf, b2), eg));
+            *reinterpret_cast<uint32_t *>(ki + o) = pack_bf16x2(kinv);
+            *reinterpret_cast<uint32_t *>(vv + o) = pack_bf16x2(__fmul2_rn(vf, b2));
             if (i & 1) {
                 kt[0][i >> 1] = pack_bf16(kt_prev.x, kt2.x);
                 kt[1][i >> 1] = pack_bf16(kt_prev.y, kt2.y);
@@ -778,7 +812,7 @@ chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *_
             }
         }
         // K e^{G_C - G} transposed (channel rows, 64 tokens, 128-byte swizzle)
-        // into its record image in the scratch region
+        // into its record image
 #pragma unroll
         for (int e = 0; e < 2; ++e)
 #pragma unroll
@@ -791,26 +825,25 @@ chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *_
     __syncthreads();
 
     const uint32_t sb = smem_u32(sm);
-    bool ok = true;
     if (tid == 0) {
         tc_fence_after();
+        // A: [beta k e^G ; q e^G] K-major (M = 128), B: k e^{-G} K-major (N = 64)
         constexpr uint32_t ID_AP = idesc_bf16(128, 64, false);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-            umma_bf16(tmem, smem_desc(sb + tcp::OFF_K + kk * 2 * tcp::CGS, tcp::CGS, tcp::TGS, 0),
-                      smem_desc(sb + tcp::OFF_KI + kk * 2 * tcp::CGS, tcp::CGS, tcp::TGS, 0), ID_AP, kk > 0);
+            umma_bf16(tmem,
+                      smem_desc(sb + tcp::OFF_KQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, 2),
+                      smem_desc(sb + tcp::OFF_KI + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024, 2),
+                      ID_AP, kk > 0);
         umma_commit(bar);
-    }
-    // record stores of q e^G (coalesced rows) overlap the MMA; K e^{G_C - G}
-    // leaves as one bulk copy of its shared-memory image
-    if (tid == 0) {
         bulk_s2g(rec + ws::OFF_KTT, sm + tcp::OFF_Z, 16384);
         bulk_commit();
     }
+    // record stores of q e^G (coalesced rows) overlap the MMA
 #pragma unroll
     for (int i = 0; i < 16; ++i)
         *reinterpret_cast<uint32_t *>(rec + ws::aw_off(64 + 16 * I + i, c0)) = qgr[i];
-    // one thread waits for the MMA (and for the image to be read); the
+    // one thread waits for the MMA (and for the K^T image to be read); the
     // others sleep at the barrier
     if (tid == 0) {
         ok = mbar_wait(bar, 0);
@@ -821,8 +854,8 @@ chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *_
 
     // ---- A (masked j < i) -> fp32 for form_T; P (masked j <= i) -> record ----
     float *Am = reinterpret_cast<float *>(sm + tcp::OFF_KI);
-    float *Tm = reinterpret_cast<float *>(sm + tcp::OFF_Q);
-    float *Ad = reinterpret_cast<float *>(sm + tcp::OFF_Z);   // after the K^T image is read
+    float *Tm = reinterpret_cast<float *>(sm + tcp::OFF_TM);
+    float *Ad = reinterpret_cast<float *>(sm + tcp::OFF_Z);
     if (ok && warp < 4) {
         float x[64];
         const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16);
@@ -872,7 +905,7 @@ chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *_
             bulk_commit();
         }
         form_T_padded_diag(Am, Ad, Tm, reinterpret_cast<float *>(sm + tcp::OFF_Z), tid);
-        // T -> bf16, K-major core matrices: (i, j) at (i/8)*1024 + (j/8)*128 + (i%8)*16 + (j%8)*2
+        // T -> bf16, one swizzled 128-byte row per token row i
         {
             const int i = tid >> 2, jq = tid & 3;
 #pragma unroll
@@ -880,7 +913,7 @@ chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *_
                 const int jg = 2 * jq + hh;
                 const float4 lo = *reinterpret_cast<const float4 *>(Tm + i * 64 + 4 * ((2 * jg) ^ (i & 7)));
                 const float4 hi = *reinterpret_cast<const float4 *>(Tm + i * 64 + 4 * ((2 * jg + 1) ^ (i & 7)));
-                *reinterpret_cast<uint4 *>(sm + tcp::OFF_TB + (i >> 3) * 1024 + jg * 128 + ((i & 7) << 4)) =
+                *reinterpret_cast<uint4 *>(sm + tcp::OFF_TB + i * 128 + ((jg ^ (i & 7)) << 4)) =
                     make_uint4(pack_bf16(lo.x, lo.y), pack_bf16(lo.z, lo.w), pack_bf16(hi.x, hi.y),
                                pack_bf16(hi.z, hi.w));
             }
@@ -890,15 +923,18 @@ chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *_
         __syncthreads();
         if (tid == 0) {
             tc_fence_after();
+            // A: [T ; *] and [* ; T] K-major (K = 64 tokens in one swizzled row);
+            // B: beta k e^G and beta v as MN-major operands (tokens along K,
+            // 64-channel atoms along N: LBO = atom stride, SBO = 8-token group)
             constexpr uint32_t ID_WU = idesc_bf16(128, 128, true);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                umma_bf16(tmem, smem_desc(sb + tcp::OFF_TB + kk * 256, 128, 1024, 0),
-                          smem_desc(sb + tcp::OFF_K + kk * 2 * tcp::TGS, tcp::TGS, tcp::CGS, 0), ID_WU, kk > 0);
+                umma_bf16(tmem, smem_desc(sb + tcp::OFF_TB + kk * 32, 16, 1024, 2),
+                          smem_desc(sb + tcp::OFF_KQ + kk * 2048, 16384, 1024, 2), ID_WU, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                umma_bf16(tmem + 128, smem_desc(sb + tcp::OFF_TB - 8192 + kk * 256, 128, 1024, 0),
-                          smem_desc(sb + tcp::OFF_V + kk * 2 * tcp::TGS, tcp::TGS, tcp::CGS, 0), ID_WU, kk > 0);
+                umma_bf16(tmem + 128, smem_desc(sb + tcp::OFF_TB - 8192 + kk * 32, 16, 1024, 2),
+                          smem_desc(sb + tcp::OFF_V + kk * 2048, 8192, 1024, 2), ID_WU, kk > 0);
             umma_commit(bar);
         }
         if (tid == 0) ok = mbar_wait(bar, 1);
@@ -914,10 +950,10 @@ chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *_
             tmem_ld32(ta, *reinterpret_cast<float (*)[32]>(&x[0]));
             tmem_ld32(ta + 32, *reinterpret_cast<float (*)[32]>(&x[32]));
             tmem_wait_ld();
-            // record images: W (rows 0-63 of both 64-channel blocks of [W; Qg])
-            // over the dead k tile, U (four 64 x 32 tiles) over the dead v tile
+            // record images: W block hf (rows 0-63 of [W; Qg]) over the dead k
+            // rows of block hf, U (four 64 x 32 tiles) over the dead v tile
             if (qd < 2) {
-                unsigned char *dst = sm + tcp::OFF_K + hf * 8192 + r * 128;
+                unsigned char *dst = sm + tcp::OFF_KQ + hf * 16384 + r * 128;
 #pragma unroll
                 for (int jc = 0; jc < 8; ++jc)
                     *reinterpret_cast<uint4 *>(dst + ((jc ^ (r & 7)) << 4)) =
@@ -940,8 +976,8 @@ chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *_
         }
         __syncthreads();
         if (ok && tid == 0) {
-            bulk_s2g(rec + ws::OFF_AW, sm + tcp::OFF_K, 8192);
-            bulk_s2g(rec + ws::OFF_AW + 16384, sm + tcp::OFF_K + 8192, 8192);
+            bulk_s2g(rec + ws::OFF_AW, sm + tcp::OFF_KQ, 8192);
+            bulk_s2g(rec + ws::OFF_AW + 16384, sm + tcp::OFF_KQ + 16384, 8192);
             bulk_s2g(rec + ws::OFF_U, sm + tcp::OFF_V, 4 * ws::U_TILE);
             bulk_commit();
         }
@@ -986,7 +1022,7 @@ __global__ void chunk_plan_kernel(const int32_t *__restrict__ cu, int N, int tot
 
 }  // namespace
 
-size_t chunk_prep_smem_bytes() { return tcp::BYTES + 128; }
+size_t chunk_prep_smem_bytes() { return tcp::BYTES + 1024; }
 
 cudaError_t launch_chunk_plan(const int32_t *cu, int N, int total_T, int32_t *coff,
                               cudaStream_t st)
@@ -995,21 +1031,62 @@ cudaError_t launch_chunk_plan(const int32_t *cu, int N, int total_T, int32_t *co
     return cudaGetLastError();
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library)
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult res;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &res) == cudaSuccess &&
+            res == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Tensor map over a [total_T, H, 128] tensor of `elem`-byte elements, boxes
+// of {box_c channels, 1 head, 64 tokens}.
+static cudaError_t make_token_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem,
+                                  int H, int total_T, int box_c, CUtensorMapSwizzle swz) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)total_T};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * elem, (cuuint64_t)D * elem * H};
+    const cuuint32_t box[3] = {(cuuint32_t)box_c, 1, (cuuint32_t)C};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const int32_t *cu, const int32_t *coff,
                               int N, int T, int total_T, int H, int max_chunks,
                               unsigned char *wsp, Prologue pro, int *err, cudaStream_t st)
 {
-    const size_t smem = tcp::BYTES + 128;
+    CUtensorMap mq, mk, mv, mg;
+    cudaError_t e = make_token_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, total_T, 64,
+                                   CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e == cudaSuccess)
+        e = make_token_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, total_T, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e == cudaSuccess)
+        e = make_token_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, total_T, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e == cudaSuccess)
+        e = make_token_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, total_T, D, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (e != cudaSuccess) return e;
+    const size_t smem = tcp::BYTES + 1024;
     const bool use_pro = pro.flags != 0 || pro.q_scale != 1.f;
     auto kern = use_pro ? chunk_prep_tc_kernel<true> : chunk_prep_tc_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int cps = (T + C - 1) / C;
     dim3 grid(max_chunks, H);
     kern<<<grid, NT, smem, st>>>(
-        (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, g, beta,
-        cu, coff, N, T, total_T, H, cps, wsp, pro, err);
+        mq, mk, mv, mg, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, g,
+        beta, cu, coff, N, T, total_T, H, cps, wsp, pro, err);
     return cudaGetLastError();
 }
 

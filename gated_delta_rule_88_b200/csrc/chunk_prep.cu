@@ -612,7 +612,7 @@ constexpr int OFF_BAR = (int)((((size_t)END > sizeof(PrepSmem) ? (size_t)END : s
 constexpr int BYTES = OFF_BAR + 32;
 constexpr uint32_t TX = 6 * 8192 + C * D * 4;   // q, k, v (two 64-channel boxes each) + g
 constexpr uint32_t TMEM_COLS = 256;
-constexpr float RANGE = 80.f;          // |exponent| bound of the chunk-start reference
+constexpr float RANGE2 = 80.f * 1.4426950408889634f;   // e^{+-80} bound, in log2 units
 // byte offset of (row r, channel c in 0..63) in a swizzled 64-channel block
 __device__ __forceinline__ int sw(int r, int c) {
     return r * 128 + ((((c >> 3) ^ (r & 7))) << 4) + ((c & 7) << 1);
@@ -710,8 +710,11 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             if (r < len) G[i] = *reinterpret_cast<const float2 *>(gsm + r * D + c0);
         }
     }
+    // cumsum in log2 units (G log2(e)), so that every e^{...} below is one ex2
+    constexpr float L2E = 1.4426950408889634f;
+    G[0].x *= L2E; G[0].y *= L2E;
 #pragma unroll
-    for (int i = 1; i < 16; ++i) { G[i].x += G[i - 1].x; G[i].y += G[i - 1].y; }
+    for (int i = 1; i < 16; ++i) { G[i].x = fmaf(G[i].x, L2E, G[i - 1].x); G[i].y = fmaf(G[i].y, L2E, G[i - 1].y); }
     *reinterpret_cast<float2 *>(gs + I * D + c0) = G[15];
     __syncthreads();
 
@@ -727,8 +730,8 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         G[i].x += PF.x; G[i].y += PF.y;
-        bad |= !(fabsf(G[i].x) <= tcp::RANGE && fabsf(G[i].y) <= tcp::RANGE &&
-                 GC.x - G[i].x <= tcp::RANGE && GC.y - G[i].y <= tcp::RANGE);
+        bad |= !(fabsf(G[i].x) <= tcp::RANGE2 && fabsf(G[i].y) <= tcp::RANGE2 &&
+                 GC.x - G[i].x <= tcp::RANGE2 && GC.y - G[i].y <= tcp::RANGE2);
     }
     if (__syncthreads_or(bad)) {
         // out of the chunk-start range (or the staging wait ran out): 16-token
@@ -769,11 +772,9 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 
     // ---- decayed forms: q e^G, beta k e^G, beta v (in place), k e^{-G}
     // (over the consumed g), K e^{G_C - G} image, q e^G and e^{G_C} (record) ----
-    uint32_t qgr[16];
     {
-        constexpr float L2E = 1.4426950408889634f;
-        const float2 egc = make_float2(ex2_approx(GC.x * L2E), ex2_approx(GC.y * L2E));
-        if (I == 0) *reinterpret_cast<float2 *>(rec + ws::OFF_EGC + c0 * 4) = make_float2(expf(GC.x), expf(GC.y));
+        const float2 egc = make_float2(ex2_approx(GC.x), ex2_approx(GC.y));
+        if (I == 0) *reinterpret_cast<float2 *>(rec + ws::OFF_EGC + c0 * 4) = make_float2(exp2f(GC.x), exp2f(GC.y));
         uint32_t kt[2][8];
         float2 kt_prev = make_float2(0.f, 0.f);
         unsigned char *kq = sm + tcp::OFF_KQ + cb * 16384;
@@ -783,8 +784,8 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         for (int i = 0; i < 16; ++i) {
             const int r = 16 * I + i;
             const int o = tcp::sw(r, cc);
-            const float2 eg = make_float2(ex2_approx(G[i].x * L2E), ex2_approx(G[i].y * L2E));
-            const float2 em = make_float2(ex2_approx(-G[i].x * L2E), ex2_approx(-G[i].y * L2E));
+            const float2 eg = make_float2(ex2_approx(G[i].x), ex2_approx(G[i].y));
+            const float2 em = make_float2(ex2_approx(-G[i].x), ex2_approx(-G[i].y));
             float2 qf = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(kq + 8192 + o));
             float2 kf = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(kq + o));
             float2 vf = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(vv + o));
@@ -800,7 +801,6 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const float2 kinv = __fmul2_rn(kf, em);
             const float2 kt2 = __fmul2_rn(kinv, egc);
             *reinterpret_cast<uint32_t *>(kq + 8192 + o) = qg;
-            qgr[i] = qg;
             *reinterpret_cast<uint32_t *>(kq + o) = pack_bf16x2(__fmul2_rn(__fmul2_rn(kf, b2), eg));
             *reinterpret_cast<uint32_t *>(ki + o) = pack_bf16x2(kinv);
             *reinterpret_cast<uint32_t *>(vv + o) = pack_bf16x2(__fmul2_rn(vf, b2));
@@ -836,13 +836,13 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                       smem_desc(sb + tcp::OFF_KI + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024, 2),
                       ID_AP, kk > 0);
         umma_commit(bar);
+        // record parts that are final now: K^T (its image) and q e^G (the
+        // swizzled q e^G tile is already the record's layout for rows 64-127)
         bulk_s2g(rec + ws::OFF_KTT, sm + tcp::OFF_Z, 16384);
+        bulk_s2g(rec + ws::OFF_AW + 8192, sm + tcp::OFF_KQ + 8192, 8192);
+        bulk_s2g(rec + ws::OFF_AW + 16384 + 8192, sm + tcp::OFF_KQ + 16384 + 8192, 8192);
         bulk_commit();
     }
-    // record stores of q e^G (coalesced rows) overlap the MMA
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-        *reinterpret_cast<uint32_t *>(rec + ws::aw_off(64 + 16 * I + i, c0)) = qgr[i];
     // one thread waits for the MMA (and for the K^T image to be read); the
     // others sleep at the barrier
     if (tid == 0) {

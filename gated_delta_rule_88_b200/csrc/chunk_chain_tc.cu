@@ -37,12 +37,16 @@ using namespace sm100;
 
 constexpr int C = ws::C;
 constexpr int D = ws::D;
-constexpr int NTHREADS = 224;
 constexpr uint32_t REC_HEAD = 57344;       // [W;Qg] + Kt^T + P, contiguous in the record
 
 template <int DVT, int NS>
 struct TcLayout {
-    static constexpr int UT = DVT > 32 ? 2 : 1;
+    // epilogue: one warp per (TMEM lane quarter, group of CPT columns)
+    static constexpr int CPT = DVT < 32 ? DVT : 32;          // columns per epilogue thread
+    static constexpr int CGRP = DVT / CPT;                   // column groups
+    static constexpr int EPI = 4 * CGRP;                     // epilogue warps
+    static constexpr int NTHREADS = 32 * (EPI + 3);          // + loader + two MMA issuers
+    static constexpr int UT = DVT > 32 ? DVT / 32 : 1;
     static constexpr uint32_t U_OFF = REC_HEAD;
     static constexpr uint32_t EGC_OFF = REC_HEAD + UT * 4096;
     static constexpr uint32_t STAGE = ((EGC_OFF + 512 + 1023) / 1024) * 1024;
@@ -53,7 +57,8 @@ struct TcLayout {
     static constexpr uint32_t BAR_OFF = B2_OFF + 2 * B2_BYTES;
     static constexpr uint32_t BYTES = BAR_OFF + 8 * (2 * NS + 8) + 16;
     // TMEM columns: D1 double-buffered (2 x DVT) + D3 (DVT), rounded to a power of 2
-    static constexpr uint32_t NCOLS = 3 * DVT <= 32 ? 32 : 3 * DVT <= 64 ? 64 : 3 * DVT <= 128 ? 128 : 256;
+    static constexpr uint32_t NCOLS = 3 * DVT <= 32 ? 32 : 3 * DVT <= 64 ? 64 : 3 * DVT <= 128 ? 128
+                                    : 3 * DVT <= 256 ? 256 : 512;
     static constexpr uint32_t B1_SBO = (128 / 8) * 128;             // n-group stride
     static constexpr uint32_t B2_SBO = (64 / 8) * 128;
 };
@@ -65,7 +70,7 @@ __device__ __forceinline__ uint32_t mn_off(int k, int ng, uint32_t sbo) {
 }
 
 template <int DVT, int NS>
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __launch_bounds__(TcLayout<DVT, NS>::NTHREADS, 1)
 chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__restrict__ cu,
                       const int32_t *__restrict__ coff, const float *__restrict__ s0,
                       float *__restrict__ sT, __nv_bfloat16 *__restrict__ out, int T, int total_T,
@@ -125,9 +130,11 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     constexpr int BAR_S = 1, BAR_V = 2, BAR_O = 3;     // named barriers (0 = __syncthreads)
-    constexpr int NSYNC = 160;                         // epilogue warps 0-3 + issuer warp 5
+    constexpr int EPI = L::EPI, CPT = L::CPT;
+    constexpr int NSYNC = 32 * EPI + 32;               // epilogue warps + the chain issuer warp
+    constexpr int NOUT = 32 * EPI / 2;                 // epilogue threads on TMEM lanes 64-127
 
-    if (warp == 4) {
+    if (warp == EPI) {
         // ---------------- loader ----------------
         if (lane == 0) {
             int issued = 0;
@@ -145,16 +152,16 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
                 bulk_g2s(st + L::U_OFF, rec + ws::OFF_U + (size_t)(n0 >> 5) * ws::U_TILE,
                          L::UT * 4096, &full[s]);
                 bulk_g2s(st + L::EGC_OFF, rec + ws::OFF_EGC, 512, &full[s]);
-                if (i + NS < nchunks) bulk_prefetch_l2(rec + (size_t)NS * rec_stride, REC_HEAD);
+                if (i + NS < nchunks) bulk_prefetch_l2(rec + (size_t)NS * rec_stride, ws::RECORD);
                 issued = i + 1;
             }
             // never leave with copies in flight into this CTA's shared memory
             for (int j = max(0, issued - NS); j < issued; ++j)
                 mbar_wait(&full[j % NS], (j / NS) & 1, 1u << 20);
         }
-    } else if (warp == 5 || warp == 6) {
-        // ---------------- MMA issuers: warp 5 lane 0 the chain (MMA1, MMA3; the
-        // warp joins the barriers), warp 6 lane 0 the output product (MMA2) ----------------
+    } else if (warp == EPI + 1 || warp == EPI + 2) {
+        // ---------------- MMA issuers: warp EPI + 1 lane 0 the chain (MMA1, MMA3;
+        // the warp joins the barriers), warp EPI + 2 lane 0 the output product (MMA2) ----------------
         constexpr uint32_t IDESC = idesc_bf16(128, DVT, true);
         // A operands: K-major, 128-byte swizzle, 8-row groups 1024 B apart, relative
         // to the ring base; B operands: MN-major interleaved, K groups 128 B apart
@@ -164,7 +171,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
         const DescParts b2_d0 = smem_desc_parts(smem_u32(B2), 128, L::B2_SBO, 0);
         const DescParts b2_d1 = smem_desc_parts(smem_u32(B2 + L::B2_BYTES), 128, L::B2_SBO, 0);
         bool issued_any = false;
-        if (warp == 5) for (int i = 0; i < nchunks; ++i) {
+        if (warp == EPI + 1) for (int i = 0; i < nchunks; ++i) {
             const int s = i % NS;
             const int p = i & 1;
             const uint32_t a_lo = a_sw.lo + ((uint32_t)s * L::STAGE >> 4);
@@ -199,7 +206,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
             }
             __syncwarp();
         }
-        if (warp == 6 && lane == 0) for (int i = 0; i < nchunks; ++i) {
+        if (warp == EPI + 2 && lane == 0) for (int i = 0; i < nchunks; ++i) {
             // MMA2: O rows (64-127 of D1[p]) += P V_new, once MMA3(i) is issued.
             // s_go[p] cannot run two phases ahead: MMA3(i + 2) needs the
             // epilogue past emit(i) (after BAR_V(i + 1)), which waits for
@@ -226,18 +233,21 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
         }
         // never free TMEM under a running MMA
         if (lane == 0 && issued_any) {
-            umma_commit(&drain[warp - 5]);
-            mbar_wait(&drain[warp - 5], 0, 1u << 20);
+            umma_commit(&drain[warp - EPI - 1]);
+            mbar_wait(&drain[warp - EPI - 1], 0, 1u << 20);
         }
     } else {
-        // ---------------- epilogue warps 0-3: thread t <-> TMEM lane t ----------------
-        const int t = tid;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        float S[DVT];
+        // ---------------- epilogue warps 0 .. EPI-1: thread <-> TMEM lane t =
+        // 32 (warp % 4) + lane (token row t of D1, channel row t of D3), columns
+        // cb .. cb + CPT - 1 of the tile with cb = CPT (warp / 4) ----------------
+        const int t = 32 * (warp & 3) + lane;
+        const int cb = CPT * (warp >> 2);
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        float S[CPT];
         {
-            const size_t sb = (((size_t)seq * H + h) * D + t) * D + n0;
+            const size_t sb = (((size_t)seq * H + h) * D + t) * D + n0 + cb;
 #pragma unroll
-            for (int j = 0; j < DVT; j += 4) {
+            for (int j = 0; j < CPT; j += 4) {
                 float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (s0) x = *reinterpret_cast<const float4 *>(s0 + sb + j);
                 S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
@@ -245,40 +255,38 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
         }
         auto write_B1 = [&]() {
 #pragma unroll
-            for (int ng = 0; ng < DVT / 8; ++ng) {
+            for (int ng = 0; ng < CPT / 8; ++ng) {
                 uint4 pk = make_uint4(pack_bf16(S[8 * ng], S[8 * ng + 1]), pack_bf16(S[8 * ng + 2], S[8 * ng + 3]),
                                       pack_bf16(S[8 * ng + 4], S[8 * ng + 5]), pack_bf16(S[8 * ng + 6], S[8 * ng + 7]));
-                *reinterpret_cast<uint4 *>(B1 + mn_off(t, ng, L::B1_SBO)) = pk;
+                *reinterpret_cast<uint4 *>(B1 + mn_off(t, cb / 8 + ng, L::B1_SBO)) = pk;
             }
             fence_proxy_async_smem();
         };
-        // DVT columns of lane t starting at column col
-        auto tmem_row = [&](uint32_t col, float (&x)[DVT]) {
-            if constexpr (DVT == 16) {
-                tmem_ld16(tmem + lane_base + col, x);
+        // CPT columns of lane t starting at tile column col + cb
+        auto tmem_row = [&](uint32_t col, float (&x)[CPT]) {
+            if constexpr (CPT == 16) {
+                tmem_ld16(tmem + lane_base + col + cb, x);
             } else {
-#pragma unroll
-                for (int c32 = 0; c32 < DVT / 32; ++c32)
-                    tmem_ld32(tmem + lane_base + col + 32 * c32, *reinterpret_cast<float (*)[32]>(&x[32 * c32]));
+                tmem_ld32(tmem + lane_base + col + cb, x);
             }
             tmem_wait_ld();
         };
-        // O of chunk ci (rows 64-127 of D1[ci & 1]) -> out; warps 2-3 only,
-        // between BAR_S and BAR_V of chunk ci + 1.  One barrier per D1
-        // buffer: MMA2(ci + 2) needs BAR_V(ci + 2), which needs this call, so
-        // each wait is at most one phase behind.
+        // O of chunk ci (rows 64-127 of D1[ci & 1]) -> out; the warps on TMEM
+        // lanes 64-127 only, between BAR_S and BAR_V of chunk ci + 1.  One
+        // barrier per D1 buffer: MMA2(ci + 2) needs BAR_V(ci + 2), which needs
+        // this call, so each wait is at most one phase behind.
         auto emit_output = [&](int ci) -> bool {
             bool okk = true;
-            if (t == 64) okk = mbar_wait(&mma2[ci & 1], (ci >> 1) & 1);
-            if (named_bar_or(BAR_O, 64, !okk)) return false;
+            if (t == 64 && cb == 0) okk = mbar_wait(&mma2[ci & 1], (ci >> 1) & 1);
+            if (named_bar_or(BAR_O, NOUT, !okk)) return false;
             tc_fence_after();
             const long long tok = bos + (long long)C * ci + (t - 64);
-            float o[DVT];
+            float o[CPT];
             tmem_row((ci & 1) * DVT, o);
             if (tok < eos) {
-                uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)tok * H + h) * D + n0);
+                uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)tok * H + h) * D + n0 + cb);
 #pragma unroll
-                for (int e = 0; e < DVT / 8; ++e)
+                for (int e = 0; e < CPT / 8; ++e)
                     dst[e] = make_uint4(pack_bf16(o[8 * e], o[8 * e + 1]), pack_bf16(o[8 * e + 2], o[8 * e + 3]),
                                         pack_bf16(o[8 * e + 4], o[8 * e + 5]), pack_bf16(o[8 * e + 6], o[8 * e + 7]));
             }
@@ -296,35 +304,36 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
             // U and e^{G_C} are read straight from it
             ok = mbar_wait(&full[s], (i / NS) & 1);
             const float eg = reinterpret_cast<const float *>(st + L::EGC_OFF)[t];
-            uint32_t u[DVT / 2];
+            uint32_t u[CPT / 2];
             if (t < 64) {
-                // column (n0 % 32) + c of the loaded U tile(s), row t
+                // column (n0 % 32) + cb + c of the loaded U tile(s), row t
 #pragma unroll
-                for (int c = 0; c < DVT; c += 8) {
-                    const int lc = (n0 & 31) + c;
+                for (int c = 0; c < CPT; c += 8) {
+                    const int lc = (n0 & 31) + cb + c;
                     const uint4 x = *reinterpret_cast<const uint4 *>(st + L::U_OFF + (lc >> 5) * 4096 + t * 64 + (lc & 31) * 2);
                     u[c / 2] = x.x; u[c / 2 + 1] = x.y; u[c / 2 + 2] = x.z; u[c / 2 + 3] = x.w;
                 }
             }
             if (t >= 64) {
-                // the previous chunk's output leaves through warps 2-3 while
-                // MMA1 runs and warps 0-1 form V_new (off the sequential path)
+                // the previous chunk's output leaves through the lane 64-127
+                // warps while MMA1 runs and the others form V_new (off the
+                // sequential path)
                 if (i > 0 && !emit_output(i - 1)) ok = false;
             } else {
                 if (ok) ok = mbar_wait(mma1, i & 1);
                 tc_fence_after();
                 // V_new = U - W S for token row t
-                float x[DVT];
+                float x[CPT];
                 tmem_row(p * DVT, x);
 #pragma unroll
-                for (int ng = 0; ng < DVT / 8; ++ng) {
+                for (int ng = 0; ng < CPT / 8; ++ng) {
                     uint32_t pk[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const __nv_bfloat162 u2 = *reinterpret_cast<const __nv_bfloat162 *>(&u[4 * ng + e]);
                         pk[e] = pack_bf16(__low2float(u2) - x[8 * ng + 2 * e], __high2float(u2) - x[8 * ng + 2 * e + 1]);
                     }
-                    *reinterpret_cast<uint4 *>(B2 + p * L::B2_BYTES + mn_off(t, ng, L::B2_SBO)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4 *>(B2 + p * L::B2_BYTES + mn_off(t, cb / 8 + ng, L::B2_SBO)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
                 fence_proxy_async_smem();
             }
@@ -334,10 +343,10 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
             tc_fence_after();
             // S <- Diag(e^{G_C}) S + Kt^T V_new   (channel row t)
             {
-                float z[DVT];
+                float z[CPT];
                 tmem_row(2 * DVT, z);
 #pragma unroll
-                for (int e = 0; e < DVT; ++e) S[e] = eg * S[e] + z[e];
+                for (int e = 0; e < CPT; ++e) S[e] = eg * S[e] + z[e];
             }
             write_B1();
             tc_fence_before();
@@ -348,9 +357,9 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
             set_device_error(err, kErrWaitTimeout);
             *abort_flag = 1;
         } else if (sT) {
-            const size_t sb = (((size_t)seq * H + h) * D + t) * D + n0;
+            const size_t sb = (((size_t)seq * H + h) * D + t) * D + n0 + cb;
 #pragma unroll
-            for (int j = 0; j < DVT; j += 4)
+            for (int j = 0; j < CPT; j += 4)
                 *reinterpret_cast<float4 *>(sT + sb + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
         }
     }
@@ -371,7 +380,7 @@ cudaError_t launch_tc(const unsigned char *wsp, const int32_t *cu, const int32_t
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(D / DVT, H, N);
-    chunk_chain_tc_kernel<DVT, NS><<<grid, NTHREADS, smem, st>>>(
+    chunk_chain_tc_kernel<DVT, NS><<<grid, L::NTHREADS, smem, st>>>(
         wsp, cu, coff, s0, sT, (__nv_bfloat16 *)out, T, total_T, H, (T + C - 1) / C, max_chunks, err);
     return cudaGetLastError();
 }

@@ -13,8 +13,8 @@
 //           S <- Diag(e^{G_C}) S + D3 (threads 0-127, one channel row each)
 // The state stays in fp32 registers for the whole sequence; its bf16 copy is
 // the B operand of MMA1.  A operands come straight from the record (K-major,
-// 128-byte swizzle); B operands (S, V_new) are written by the threads in the
-// MN-major interleaved layout.
+// 128-byte swizzle); B operands (S, V_new) are written by the threads as
+// MN-major operands swizzled to the tile width (rows of 32 to 128 bytes).
 //
 // Roles (192 threads): warps 0-3 are the epilogue (thread t <-> TMEM lane t:
 // token row t of D1, channel row t of D3); warp 4 lane 0 streams records into
@@ -59,15 +59,17 @@ struct TcLayout {
     // TMEM columns: D1 double-buffered (2 x DVT) + D3 (DVT), rounded to a power of 2
     static constexpr uint32_t NCOLS = 3 * DVT <= 32 ? 32 : 3 * DVT <= 64 ? 64 : 3 * DVT <= 128 ? 128
                                     : 3 * DVT <= 256 ? 256 : 512;
-    static constexpr uint32_t B1_SBO = (128 / 8) * 128;             // n-group stride
-    static constexpr uint32_t B2_SBO = (64 / 8) * 128;
+    // B operands S and V_new: MN-major, one swizzle atom wide (rows of DVT
+    // bf16 = 32, 64 or 128 bytes), 8-row groups contiguous
+    static constexpr uint32_t BW = DVT * 2;
+    static constexpr uint32_t B_SBO = 8 * BW;
+    static constexpr uint32_t B_LAYOUT = DVT == 64 ? 2 : DVT == 32 ? 4 : 6;   // 128 / 64 / 32-byte swizzle
+    static constexpr int B_SWZ = DVT == 64 ? 7 : DVT == 32 ? 3 : 1;
+    // byte offset of the 16-byte chunk `chunk` (8 columns) of K row k
+    static __device__ __forceinline__ uint32_t b_off(int k, int chunk) {
+        return (k >> 3) * B_SBO + (k & 7) * BW + ((chunk ^ ((((k & 7) * BW) >> 7) & B_SWZ)) << 4);
+    }
 };
-
-// MN-major interleaved core-matrix layout: element (n, k) of a K x N operand
-// at (n / 8) * SBO + (k / 8) * 128 + (k % 8) * 16 + (n % 8) * 2.
-__device__ __forceinline__ uint32_t mn_off(int k, int ng, uint32_t sbo) {
-    return ng * sbo + (k >> 3) * 128 + (k & 7) * 16;
-}
 
 template <int DVT, int NS>
 __global__ void __launch_bounds__(TcLayout<DVT, NS>::NTHREADS, 1)
@@ -164,12 +166,13 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
         // the warp joins the barriers), warp EPI + 2 lane 0 the output product (MMA2) ----------------
         constexpr uint32_t IDESC = idesc_bf16(128, DVT, true);
         // A operands: K-major, 128-byte swizzle, 8-row groups 1024 B apart, relative
-        // to the ring base; B operands: MN-major interleaved, K groups 128 B apart
+        // to the ring base; B operands: MN-major, swizzled to the tile width
         const uint32_t sm_a = smem_u32(sm);
         const DescParts a_sw = smem_desc_parts(sm_a, 16, 1024, 2);
-        const DescParts b1_d = smem_desc_parts(smem_u32(B1), 128, L::B1_SBO, 0);
-        const DescParts b2_d0 = smem_desc_parts(smem_u32(B2), 128, L::B2_SBO, 0);
-        const DescParts b2_d1 = smem_desc_parts(smem_u32(B2 + L::B2_BYTES), 128, L::B2_SBO, 0);
+        const DescParts b1_d = smem_desc_parts(smem_u32(B1), L::B_SBO, L::B_SBO, L::B_LAYOUT);
+        const DescParts b2_d0 = smem_desc_parts(smem_u32(B2), L::B_SBO, L::B_SBO, L::B_LAYOUT);
+        const DescParts b2_d1 = smem_desc_parts(smem_u32(B2 + L::B2_BYTES), L::B_SBO, L::B_SBO, L::B_LAYOUT);
+        constexpr uint32_t BK = (2 * L::B_SBO) >> 4;       // descriptor step per 16 K rows
         bool issued_any = false;
         if (warp == EPI + 1) for (int i = 0; i < nchunks; ++i) {
             const int s = i % NS;
@@ -185,7 +188,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     umma_bf16_p(d1, a_lo + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), a_sw.hi,
-                                b1_d.lo + ((kk * 256) >> 4), b1_d.hi, IDESC, kk > 0);
+                                b1_d.lo + (kk * BK), b1_d.hi, IDESC, kk > 0);
                 umma_commit(mma1);
                 issued_any = true;
             }
@@ -199,7 +202,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     umma_bf16_p(tmem + 2 * DVT, a_lo + (((uint32_t)ws::OFF_KTT + kk * 32) >> 4),
-                                a_sw.hi, b2_lo + ((kk * 256) >> 4), b2_d0.hi, IDESC, kk > 0);
+                                a_sw.hi, b2_lo + (kk * BK), b2_d0.hi, IDESC, kk > 0);
                 umma_commit(mma3);
                 umma_commit(&empty[s]);
                 mbar_arrive(&s_go[p]);
@@ -226,7 +229,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 umma_bf16_p(tmem + p * DVT, a_lo + (((uint32_t)ws::OFF_P - 8192 + kk * 32) >> 4),
-                            a_sw.hi, b2_lo + ((kk * 256) >> 4), b2_d0.hi, IDESC, 1);
+                            a_sw.hi, b2_lo + (kk * BK), b2_d0.hi, IDESC, 1);
             umma_commit(&mma2[p]);
             umma_commit(&empty[s]);
             issued_any = true;
@@ -258,7 +261,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
             for (int ng = 0; ng < CPT / 8; ++ng) {
                 uint4 pk = make_uint4(pack_bf16(S[8 * ng], S[8 * ng + 1]), pack_bf16(S[8 * ng + 2], S[8 * ng + 3]),
                                       pack_bf16(S[8 * ng + 4], S[8 * ng + 5]), pack_bf16(S[8 * ng + 6], S[8 * ng + 7]));
-                *reinterpret_cast<uint4 *>(B1 + mn_off(t, cb / 8 + ng, L::B1_SBO)) = pk;
+                *reinterpret_cast<uint4 *>(B1 + L::b_off(t, cb / 8 + ng)) = pk;
             }
             fence_proxy_async_smem();
         };
@@ -333,7 +336,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
                         const __nv_bfloat162 u2 = *reinterpret_cast<const __nv_bfloat162 *>(&u[4 * ng + e]);
                         pk[e] = pack_bf16(__low2float(u2) - x[8 * ng + 2 * e], __high2float(u2) - x[8 * ng + 2 * e + 1]);
                     }
-                    *reinterpret_cast<uint4 *>(B2 + p * L::B2_BYTES + mn_off(t, cb / 8 + ng, L::B2_SBO)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4 *>(B2 + p * L::B2_BYTES + L::b_off(t, cb / 8 + ng)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
                 fence_proxy_async_smem();
             }

@@ -62,11 +62,11 @@ FALLBACK_HBM_GBS = 6650.0
 _SRC = os.path.join(ROOT, "gated_delta_rule_88_b200", "csrc")
 TRAFFIC = {
     "prefill": {"files": ["chunk_prep.cu", "chunk_chain_tc.cu", "chunk_ws.h", "sm100.cuh", "common.cuh"],
-                "sha": "a3a197b795fcf79a", "bytes": (342.108160 + 264.204800 + 304.158464 + 52.440832) * 1e6},
+                "sha": "358fe9eded9e9d6b", "bytes": (338.166528 + 254.972928 + 304.168960 + 49.464832) * 1e6},
     "decode": {"files": ["decode.cu", "common.cuh"], "sha": "4ceac309c0c18d2f",
                "bytes": (547.408128 + 480.674560) * 1e6},
-    "decode_steps": {"files": ["decode_pipe.cu", "common.cuh", "sm100.cuh"], "sha": "dfd242f2df963f4b",
-                     "bytes": (621.427456 + 496.504320) * 1e6},
+    "decode_steps": {"files": ["decode_pipe.cu", "common.cuh", "sm100.cuh"], "sha": "d9cf376f965488af",
+                     "bytes": (621.110016 + 492.918016) * 1e6},
     "backward": {"files": ["recurrent_bwd.cu", "common.cuh"], "sha": "ba9d9318f1b1cd87",
                  "bytes": (2902.812672 + 3861.861120) * 1e6},
     "decode_chunk": {"files": ["decode_chunk.cu", "common.cuh"], "sha": "23a550bc05b00c2b",

@@ -585,7 +585,8 @@ __device__ __forceinline__ void prep_subchunk(
 // The rows marked * are whatever lies next to T in shared memory; their
 // products land in TMEM lanes that are never read.  T itself comes from
 // form_T_padded_diag (fp32).  Record parts leave by bulk async stores of
-// their shared-memory images.
+// their shared-memory images (W and U, the last, by a coalesced copy of all
+// threads so that the CTA need not wait for a bulk copy to read them).
 // ---------------------------------------------------------------------------
 namespace tcp {
 // Tiles are K-major with the 128-byte swizzle (rows of 64 bf16 = 128 bytes,
@@ -873,13 +874,18 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 a4.w = (4 * j4 + 3 < i) ? x[4 * j4 + 3] : 0.f;
                 *reinterpret_cast<float4 *>(Am + i * 64 + 4 * (j4 ^ (i & 7))) = a4;
             }
-            // the row's diagonal block, padded copy for the substitution
+            // the row's diagonal block, padded copy for the substitution: warp
+            // w holds rows 32w..32w+31, i.e. diagonal blocks 2w (lanes 0-15)
+            // and 2w + 1 (lanes 16-31)
             float *adr = Ad + (i >> 4) * (16 * 17) + (i & 15) * 17;
-            const int B = i >> 4, ii = i & 15;
+            const int ii = i & 15;
+            const bool upper = lane >= 16;
+            if (warp == 0) {
 #pragma unroll
-            for (int jj = 0; jj < 16; ++jj) {
-                const float a = B == 0 ? x[jj] : B == 1 ? x[16 + jj] : B == 2 ? x[32 + jj] : x[48 + jj];
-                adr[jj] = (jj < ii) ? a : 0.f;
+                for (int jj = 0; jj < 16; ++jj) adr[jj] = (jj < ii) ? (upper ? x[16 + jj] : x[jj]) : 0.f;
+            } else {
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) adr[jj] = (jj < ii) ? (upper ? x[48 + jj] : x[32 + jj]) : 0.f;
             }
         } else {
             unsigned char *img = sm + tcp::OFF_TB;
@@ -951,7 +957,8 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             tmem_ld32(ta + 32, *reinterpret_cast<float (*)[32]>(&x[32]));
             tmem_wait_ld();
             // record images: W block hf (rows 0-63 of [W; Qg]) over the dead k
-            // rows of block hf, U (four 64 x 32 tiles) over the dead v tile
+            // rows of block hf, U (four 64 x 32 tiles) over the dead v tile;
+            // copied out below by all threads
             if (qd < 2) {
                 unsigned char *dst = sm + tcp::OFF_KQ + hf * 16384 + r * 128;
 #pragma unroll
@@ -972,14 +979,21 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     }
                 }
             }
-            fence_proxy_async_smem();
         }
         __syncthreads();
-        if (ok && tid == 0) {
-            bulk_s2g(rec + ws::OFF_AW, sm + tcp::OFF_KQ, 8192);
-            bulk_s2g(rec + ws::OFF_AW + 16384, sm + tcp::OFF_KQ + 16384, 8192);
-            bulk_s2g(rec + ws::OFF_U, sm + tcp::OFF_V, 4 * ws::U_TILE);
-            bulk_commit();
+        if (ok) {
+            // all threads copy the 32 KB of images out with coalesced 16-byte
+            // accesses (W block 0, W block 1, the four U tiles); nothing is
+            // left in flight that reads shared memory
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int c = tid + NT * j;                   // 16-byte chunk, 0..2047
+                const int src = c < 512 ? tcp::OFF_KQ + 16 * c
+                              : c < 1024 ? tcp::OFF_KQ + 16384 + 16 * (c - 512) : tcp::OFF_V + 16 * (c - 1024);
+                const size_t dst = c < 512 ? ws::OFF_AW + 16 * c
+                                 : c < 1024 ? ws::OFF_AW + 16384 + 16 * (c - 512) : ws::OFF_U + 16 * (c - 1024);
+                *reinterpret_cast<uint4 *>(rec + dst) = *reinterpret_cast<const uint4 *>(sm + src);
+            }
         }
     }
     // the shared-memory sources of the bulk stores must be read before exit

@@ -61,6 +61,24 @@ def test_chunk_prologue(dtype, d, flags):
     assert_close(s, s_ref, dtype if dtype == torch.bfloat16 else torch.float32, "final state")
 
 
+def test_chunk_prologue_with_strong_decay_chunks():
+    """bf16 prefill with the prologue where chunk 1 of head 0 decays by more
+    than e^80 (g = -2 on some channels): that chunk takes the 16-token
+    exponent path, the others the chunk-start path, both normalising q, k
+    and taking the sigmoid of beta inside the kernel."""
+    B, T, H, d = 1, 256, 2, 128
+    q, k, v, g, b = _raw((B, T, H), d, d, torch.bfloat16, seed=57)
+    g[:, 64:128, 0, ::4] = -2.0
+    qs = 1.0 / math.sqrt(d)
+    o, s = kda_chunk_fwd_ex(*[t.to(DEV) for t in (q, k, v, g, b)], flags=ALL, q_scale=qs)
+    torch.cuda.synchronize()
+    qp, kp, bp = oracle.prologue(q, k, b, qk_l2norm=True, beta_sigmoid=True, q_scale=qs)
+    o_ref, s_ref = oracle.forward(qp, kp, v, g, bp)
+    assert not torch.isnan(o).any()
+    assert_close(o, o_ref, torch.bfloat16, "o")
+    assert_close(s, s_ref, torch.bfloat16, "final state")
+
+
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_chunk_prologue_identity_is_bitwise_the_plain_call(dtype):
     from gated_delta_rule_88_b200 import workloads as W

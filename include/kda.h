@@ -107,7 +107,10 @@ enum { KDA_STEPS_CHUNK = 4 };
  *   KDA_F32 with dk, dv in {64, 128} (exact fp32 path).  Others return
  *   KDA_ERR_UNSUPPORTED.
  * Numerical range (bf16 path): per-token g >= -5 keeps every exponent the
- *   chunk form takes within fp32 range (sub-chunks of 16 tokens).
+ *   chunk form takes within fp32 range.  A chunk whose decay over its 64
+ *   tokens stays within e^{+-80} references its exponents at the chunk start
+ *   (the fast path); any other chunk references them per 16-token sub-chunk,
+ *   inside the same call, with the same result up to rounding.
  * Aliasing: out must not overlap any input.
  * Memory: the bf16 path takes a stream-ordered scratch buffer from a
  *   library-private pool on the current device (cudaMallocFromPoolAsync on

@@ -654,7 +654,11 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int chunk = blockIdx.x, h = blockIdx.y;
+    // heads fastest and chunks last-to-first: the records written last, still
+    // in L2 when the chain starts, are the first chunks of every head, the
+    // ones the chain reads first
+    const int lin = blockIdx.y * gridDim.x + blockIdx.x;
+    const int h = lin % H, chunk = gridDim.x - 1 - lin / H;
     if (cu && chunk >= coff[N]) return;
 
     int len;

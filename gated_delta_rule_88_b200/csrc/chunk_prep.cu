@@ -325,7 +325,7 @@ __device__ __forceinline__ void form_T_padded_diag(const float *Am, const float 
 // calls this for the chunks whose decay over the chunk leaves its exponent
 // range.  Called by all 256 threads of the CTA; smem_raw holds a PrepSmem.
 template <bool PRO>
-__device__ __forceinline__ void prep_subchunk(
+__device__ __noinline__ void prep_subchunk(
     unsigned char *smem_raw, const __nv_bfloat16 *__restrict__ q,
     const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
     const float *__restrict__ g, const float *__restrict__ beta, const int32_t *__restrict__ cu,

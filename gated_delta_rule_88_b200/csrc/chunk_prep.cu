@@ -611,7 +611,8 @@ constexpr int END = OFF_RK + C * 4;
 // fallback never overwrites them
 constexpr int OFF_BAR = (int)((((size_t)END > sizeof(PrepSmem) ? (size_t)END : sizeof(PrepSmem)) + 15) & ~(size_t)15);
 constexpr int BYTES = OFF_BAR + 32;
-constexpr uint32_t TX = 6 * 8192 + C * D * 4;   // q, k, v (two 64-channel boxes each) + g
+constexpr uint32_t TX_QKV = 6 * 8192;          // q, k, v: two 64-channel boxes each
+constexpr uint32_t TX_G = C * D * 4;            // g
 constexpr uint32_t TMEM_COLS = 256;
 constexpr float RANGE2 = 80.f * 1.4426950408889634f;   // e^{+-80} bound, in log2 units
 // byte offset of (row r, channel c in 0..63) in a swizzled 64-channel block
@@ -667,6 +668,7 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     unsigned char *rec = wsp + ((size_t)chunk * H + h) * ws::RECORD;
     uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + tcp::OFF_BAR);
     uint64_t *bar = bar_ld + 1;
+    uint64_t *bar_g = bar_ld + 3;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + tcp::OFF_BAR + 16);
     float *gs = reinterpret_cast<float *>(sm + tcp::OFF_GS);
     float *bet = reinterpret_cast<float *>(sm + tcp::OFF_BETA);
@@ -678,16 +680,20 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (tid == 0) {
         mbar_init(bar_ld, 1);
         mbar_init(bar, 1);
+        mbar_init(bar_g, 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(bar_ld, tcp::TX);
+        // g first, on its own barrier: the cumsum and the range check run
+        // while q, k and v are still arriving
+        mbar_arrive_expect_tx(bar_g, tcp::TX_G);
         const int tt = (int)t0;
+        tma_load_3d(sm + tcp::OFF_G, &tm_g, 0, h, tt, bar_g);
+        mbar_arrive_expect_tx(bar_ld, tcp::TX_QKV);
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
             tma_load_3d(sm + tcp::OFF_KQ + b * 16384, &tm_k, 64 * b, h, tt, bar_ld);
             tma_load_3d(sm + tcp::OFF_KQ + b * 16384 + 8192, &tm_q, 64 * b, h, tt, bar_ld);
             tma_load_3d(sm + tcp::OFF_V + b * 8192, &tm_v, 64 * b, h, tt, bar_ld);
         }
-        tma_load_3d(sm + tcp::OFF_G, &tm_g, 0, h, tt, bar_ld);
     }
     if (tid < C) {
         float bt = (tid < len) ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
@@ -696,7 +702,7 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
     if (warp == 0) { tmem_alloc(tslot, tcp::TMEM_COLS); tmem_relinquish(); }
     bool ok = true;
-    if (tid == 0) ok = mbar_wait(bar_ld, 0);
+    if (tid == 0) ok = mbar_wait(bar_g, 0);
     tc_fence_before();
     ok = __syncthreads_and(ok);
     tc_fence_after();
@@ -738,8 +744,12 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         bad |= !(fabsf(G[i].x) <= tcp::RANGE2 && fabsf(G[i].y) <= tcp::RANGE2 &&
                  GC.x - G[i].x <= tcp::RANGE2 && GC.y - G[i].y <= tcp::RANGE2);
     }
-    if (__syncthreads_or(bad)) {
-        // out of the chunk-start range (or the staging wait ran out): 16-token
+    // q, k, v have landed before anything (this path or the fallback, which
+    // reuses the shared memory) touches their tiles
+    if (tid == 0 && ok) ok = mbar_wait(bar_ld, 0);
+    ok = __syncthreads_and(ok);
+    if (__syncthreads_or(bad || !ok)) {
+        // out of the chunk-start range (or a staging wait ran out): 16-token
         // references, mma.sync products, its own loads
         if (!ok && tid == 0) set_device_error(err, kErrWaitTimeout);
         if (ok) prep_subchunk<PRO>(sm, q, k, v, g, beta, cu, coff, N, T, total_T, H, cps, wsp, pro, chunk, h);

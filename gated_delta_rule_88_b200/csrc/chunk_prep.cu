@@ -844,12 +844,12 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         tc_fence_after();
         // A: [beta k e^G ; q e^G] K-major (M = 128), B: k e^{-G} K-major (N = 64)
         constexpr uint32_t ID_AP = idesc_bf16(128, 64, false);
+        const DescParts da = smem_desc_parts(sb + tcp::OFF_KQ, 16, 1024, 2);
+        const DescParts db = smem_desc_parts(sb + tcp::OFF_KI, 16, 1024, 2);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-            umma_bf16(tmem,
-                      smem_desc(sb + tcp::OFF_KQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, 2),
-                      smem_desc(sb + tcp::OFF_KI + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024, 2),
-                      ID_AP, kk > 0);
+            umma_bf16_p(tmem, da.lo + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), da.hi,
+                        db.lo + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), db.hi, ID_AP, kk > 0);
         umma_commit(bar);
         // record parts that are final now: K^T (its image) and q e^G (the
         // swizzled q e^G tile is already the record's layout for rows 64-127)
@@ -947,14 +947,17 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             // B: beta k e^G and beta v as MN-major operands (tokens along K,
             // 64-channel atoms along N: LBO = atom stride, SBO = 8-token group)
             constexpr uint32_t ID_WU = idesc_bf16(128, 128, true);
+            const DescParts ta = smem_desc_parts(sb + tcp::OFF_TB, 16, 1024, 2);
+            const DescParts tu = smem_desc_parts(sb + tcp::OFF_TB - 8192, 16, 1024, 2);
+            const DescParts bw = smem_desc_parts(sb + tcp::OFF_KQ, 16384, 1024, 2);
+            const DescParts bu = smem_desc_parts(sb + tcp::OFF_V, 8192, 1024, 2);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                umma_bf16(tmem, smem_desc(sb + tcp::OFF_TB + kk * 32, 16, 1024, 2),
-                          smem_desc(sb + tcp::OFF_KQ + kk * 2048, 16384, 1024, 2), ID_WU, kk > 0);
+                umma_bf16_p(tmem, ta.lo + ((kk * 32) >> 4), ta.hi, bw.lo + ((kk * 2048) >> 4), bw.hi, ID_WU, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                umma_bf16(tmem + 128, smem_desc(sb + tcp::OFF_TB - 8192 + kk * 32, 16, 1024, 2),
-                          smem_desc(sb + tcp::OFF_V + kk * 2048, 8192, 1024, 2), ID_WU, kk > 0);
+                umma_bf16_p(tmem + 128, tu.lo + ((kk * 32) >> 4), tu.hi, bu.lo + ((kk * 2048) >> 4), bu.hi, ID_WU,
+                            kk > 0);
             umma_commit(bar);
         }
         if (tid == 0) ok = mbar_wait(bar, 1);

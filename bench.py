@@ -62,7 +62,7 @@ FALLBACK_HBM_GBS = 6650.0
 _SRC = os.path.join(ROOT, "gated_delta_rule_88_b200", "csrc")
 TRAFFIC = {
     "prefill": {"files": ["chunk_prep.cu", "chunk_chain_tc.cu", "chunk_ws.h", "sm100.cuh", "common.cuh"],
-                "sha": "71761dcb2469b150", "bytes": (338.203392 + 255.355392 + 304.178688 + 49.751808) * 1e6},
+                "sha": "8b788aa77014ac59", "bytes": (336.785152 + 254.092800 + 304.155648 + 49.041920) * 1e6},
     "decode": {"files": ["decode.cu", "common.cuh"], "sha": "4ceac309c0c18d2f",
                "bytes": (547.408128 + 480.674560) * 1e6},
     "decode_steps": {"files": ["decode_pipe.cu", "common.cuh", "sm100.cuh"], "sha": "d9cf376f965488af",

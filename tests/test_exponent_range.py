@@ -50,7 +50,7 @@ def test_chunk_start_factors_keep_bf16_accuracy_up_to_80():
         assert float(G.abs().max()) <= 80.0
         exact, approx = _pairwise(G, x, y)
         err = _lower_rel_err(exact, approx)
-        assert err < 2e-2, (total, err)          # bf16 operands, fp32 accumulation
+        assert err < 1e-2, (total, err)          # bf16 operands, fp32 accumulation
 
 
 def test_chunk_start_factor_overflows_past_the_bound():

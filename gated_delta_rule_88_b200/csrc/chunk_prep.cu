@@ -1053,6 +1053,7 @@ __global__ void chunk_plan_kernel(const int32_t *__restrict__ cu, int N, int tot
 
 }  // namespace
 
+size_t chunk_prep_smem_bytes() { return tcp::BYTES + 1024; }
 
 cudaError_t launch_chunk_plan(const int32_t *cu, int N, int total_T, int32_t *coff,
                               cudaStream_t st)

@@ -82,6 +82,7 @@ cudaError_t launch_chunk_f32(const float *q, const float *k, const float *v, con
 //               (A, P, W, U on tcgen05; err receives bounded-wait failures)
 //   chunk_chain sequential over chunks per (sequence, head, dv tile),
 //               tcgen05 MMAs with TMEM accumulators (chunk_chain_tc.cu)
+size_t chunk_prep_smem_bytes();
 cudaError_t launch_chunk_plan(const int32_t *cu, int N, int total_T, int32_t *coff,
                               cudaStream_t st);
 cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const float *g,

@@ -6,6 +6,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include <cuda_runtime.h>
@@ -21,15 +22,18 @@ namespace kda {
 __device__ int g_device_error = 0;
 
 int *error_word() {
-    static int *addr[64] = {nullptr};
+    // per-device cache; threads that race on first use store the same address
+    static std::atomic<int *> addr[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-        addr[dev] = (int *)p;
+    int *p = addr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        void *s = nullptr;
+        if (cudaGetSymbolAddress(&s, g_device_error) != cudaSuccess) return nullptr;
+        p = (int *)s;
+        addr[dev].store(p, std::memory_order_release);
     }
-    return addr[dev];
+    return p;
 }
 }  // namespace kda
 

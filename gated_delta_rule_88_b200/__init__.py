@@ -18,6 +18,13 @@ Entry points (same names as the C ABI):
     kda_chunk_fwd_host(q, k, v, g, beta, initial_state=None, out=None,
                        final_state=None, output_final_state=True, range_tokens=0)
         -> (out, final_state or None)   (CPU tensors; valid after the stream syncs)
+    kda_chunk_fwd_noalloc(...): kda_chunk_fwd over the library's fixed
+                     scratch array (bf16, dk = dv = 128; pass out and
+                     final_state to keep the call free of allocations)
+    kda_gated_rmsnorm(x, gate, weight, eps=1e-5, out=None) -> out
+    kda_recurrent_bwd(q, k, v, g, beta, do, initial_state=None, dsT=None)
+        -> (dq, dk, dv, dg, dbeta, ds0)
+    kda_state_affine(M, B, S_in, out=None) -> S_out
     kda_get_device_error(stream=None) -> int
 """
 from __future__ import annotations
@@ -28,7 +35,8 @@ import threading
 
 import torch
 
-__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_ex", "kda_chunk_fwd_host", "kda_recurrent_step",
+__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_ex", "kda_chunk_fwd_host", "kda_chunk_fwd_noalloc",
+           "kda_recurrent_step",
            "kda_recurrent_step_ex", "kda_recurrent_steps", "kda_gated_rmsnorm", "kda_state_affine",
            "kda_recurrent_bwd",
            "kda_get_device_error",
@@ -70,6 +78,8 @@ def load_library():
         lib.kda_chunk_fwd.restype = i
         lib.kda_chunk_fwd_ex.argtypes = [vp] * 9 + [i] * 7 + [ctypes.c_uint, ctypes.c_float, vp]
         lib.kda_chunk_fwd_ex.restype = i
+        lib.kda_chunk_fwd_noalloc.argtypes = [vp] * 9 + [i] * 7 + [vp]
+        lib.kda_chunk_fwd_noalloc.restype = i
         lib.kda_recurrent_step_ex.argtypes = [vp] * 7 + [i] * 5 + [ctypes.c_uint, ctypes.c_float, vp]
         lib.kda_recurrent_step_ex.restype = i
         lib.kda_recurrent_step.argtypes = [vp] * 7 + [i] * 5 + [vp]
@@ -146,8 +156,18 @@ def kda_chunk_fwd_ex(q, k, v, g, beta, initial_state=None, cu_seqlens=None, out=
                       output_final_state, (int(flags), float(q_scale)))
 
 
+def kda_chunk_fwd_noalloc(q, k, v, g, beta, initial_state=None, cu_seqlens=None, out=None,
+                          final_state=None, output_final_state: bool = True):
+    """kda_chunk_fwd through the allocation-free entry point: the library
+    allocates nothing (its scratch is a fixed 32 MiB array); bf16 with
+    dk = dv = 128.  Pass out (and final_state) to make the whole call
+    allocation-free; otherwise they are allocated here, as torch tensors."""
+    return _chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state,
+                      output_final_state, None, noalloc=True)
+
+
 def _chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state,
-               output_final_state, pro):
+               output_final_state, pro, noalloc: bool = False):
     lib = load_library()
     dev = q.device
     if dev.type != "cuda":
@@ -182,7 +202,9 @@ def _chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state,
     args = (_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta), _dptr(initial_state),
             _dptr(cu_seqlens), _dptr(out), _dptr(final_state), B, T, H, dk, dv, N, _dtype_code(q))
     with torch.cuda.device(dev):
-        if pro is None:
+        if noalloc:
+            rc = lib.kda_chunk_fwd_noalloc(*args, _stream_handle(dev))
+        elif pro is None:
             rc = lib.kda_chunk_fwd(*args, _stream_handle(dev))
         else:
             rc = lib.kda_chunk_fwd_ex(*args, pro[0], pro[1], _stream_handle(dev))

@@ -42,6 +42,21 @@ def test_header_declares_entry_points():
         assert n in names
 
 
+def test_every_computing_entry_point_has_a_binding_of_the_same_name():
+    """The Python package binds every entry point of the C ABI that computes
+    (the status helpers are used internally), under the same name, and each
+    refuses CPU tensors instead of computing on the host."""
+    import torch
+    helpers = {"kda_status_string", "kda_last_error_message", "kda_version"}
+    for n in declared_functions():
+        if n in helpers:
+            continue
+        assert hasattr(kda, n) and n in kda.__all__, f"{n} has no Python binding"
+    x = torch.zeros(1, 4, 1, 128)
+    with pytest.raises(ValueError, match="CUDA"):
+        kda.kda_chunk_fwd_noalloc(x, x, x, x, torch.zeros(1, 4, 1))
+
+
 def test_library_exports_every_declared_symbol(lib):
     for n in declared_functions():
         assert hasattr(lib, n), f"{n} declared in include/ but not exported"

@@ -15,7 +15,7 @@ Entry points (same names as the C ABI):
     kda_chunk_fwd_ex(..., flags=0, q_scale=1.0), kda_recurrent_step_ex(..., flags=0,
                      q_scale=1.0): with the in-kernel input prologue
                      (KDA_QK_L2NORM, KDA_BETA_SIGMOID)
-    kda_chunk_fwd_host(q, k, v, g, beta, initial_state=None, out=None,
+    kda_chunk_fwd_host(q, k, v, g, beta, initial_state=None, cu_seqlens=None, out=None,
                        final_state=None, output_final_state=True, range_tokens=0)
         -> (out, final_state or None)   (CPU tensors; valid after the stream syncs)
     kda_chunk_fwd_noalloc(...): kda_chunk_fwd over the library's fixed
@@ -87,7 +87,7 @@ def load_library():
         lib.kda_recurrent_steps.argtypes = ([vp] * 7 + [i] + [vp] + [i] * 6 +
                                             [ctypes.c_uint, ctypes.c_float, vp])
         lib.kda_recurrent_steps.restype = i
-        lib.kda_chunk_fwd_host.argtypes = [vp] * 8 + [i] * 7 + [vp]
+        lib.kda_chunk_fwd_host.argtypes = [vp] * 9 + [i] * 8 + [vp]
         lib.kda_chunk_fwd_host.restype = i
         lib.kda_gated_rmsnorm.argtypes = [vp, vp, vp, ctypes.c_float, vp, ctypes.c_longlong, i, i, vp]
         lib.kda_gated_rmsnorm.restype = i
@@ -212,12 +212,14 @@ def _chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state,
     return out, final_state
 
 
-def kda_chunk_fwd_host(q, k, v, g, beta, initial_state=None, out=None, final_state=None,
-                       output_final_state: bool = True, range_tokens: int = 0, device=None):
-    """kda_chunk_fwd on host (CPU) tensors, dense [B,T,H,*] layouts; the copies
-    are pipelined against the computation on ``device`` (default: the current
-    CUDA device).  Pinned tensors overlap; results are valid once the current
-    stream of that device has synchronised.  Returns (out, final_state)."""
+def kda_chunk_fwd_host(q, k, v, g, beta, initial_state=None, cu_seqlens=None, out=None,
+                       final_state=None, output_final_state: bool = True, range_tokens: int = 0,
+                       device=None):
+    """kda_chunk_fwd on host (CPU) tensors, dense [B,T,H,*] layouts or (with a
+    CPU int32 ``cu_seqlens``) varlen [1,T,H,*]; the copies are pipelined
+    against the computation on ``device`` (default: the current CUDA device).
+    Pinned tensors overlap; results are valid once the current stream of that
+    device has synchronised.  Returns (out, final_state)."""
     lib = load_library()
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     cpu = torch.device("cpu")
@@ -230,6 +232,10 @@ def kda_chunk_fwd_host(q, k, v, g, beta, initial_state=None, out=None, final_sta
         _need(t, n, cpu, dt)
     _need(g, "g", cpu, torch.float32)
     _need(beta, "beta", cpu, torch.float32)
+    N = B
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", cpu, torch.int32)
+        N = cu_seqlens.numel() - 1
     if initial_state is not None:
         _need(initial_state, "initial_state", cpu, torch.float32)
     if out is None:
@@ -237,12 +243,12 @@ def kda_chunk_fwd_host(q, k, v, g, beta, initial_state=None, out=None, final_sta
     else:
         _need(out, "out", cpu, dt)
     if final_state is None and output_final_state:
-        final_state = torch.empty(B, H, dk, dv, dtype=torch.float32, pin_memory=True)
+        final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, pin_memory=True)
     with torch.cuda.device(dev):
         rc = lib.kda_chunk_fwd_host(_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta),
-                                    _dptr(initial_state), _dptr(out), _dptr(final_state),
-                                    B, T, H, dk, dv, _dtype_code(q), int(range_tokens),
-                                    _stream_handle(dev))
+                                    _dptr(initial_state), _dptr(cu_seqlens), _dptr(out),
+                                    _dptr(final_state), B, T, H, dk, dv, N, _dtype_code(q),
+                                    int(range_tokens), _stream_handle(dev))
     _check(rc)
     return out, final_state
 

@@ -6,8 +6,10 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include <cuda_runtime.h>
 
@@ -468,19 +470,14 @@ cudaError_t pipe_streams(HostPipeStreams **ps) {
     return cudaSuccess;
 }
 
-// rows [t0, t0 + n) of every batch: B strided blocks of n * row bytes
-cudaError_t copy_rows(void *dst, size_t dpitch, const void *src, size_t spitch, size_t width,
-                      int B, cudaStream_t st) {
-    return cudaMemcpy2DAsync(dst, dpitch, src, spitch, width, (size_t)B, cudaMemcpyDefault, st);
-}
-
 }  // namespace
 
 extern "C" kda_status kda_chunk_fwd_host(const void *q, const void *k, const void *v,
                                          const float *g, const float *beta,
-                                         const float *initial_state, void *out,
-                                         float *final_state, int B, int T, int H, int dk, int dv,
-                                         kda_dtype dtype, int range_tokens, void *stream) {
+                                         const float *initial_state, const int32_t *cu_seqlens,
+                                         void *out, float *final_state, int B, int T, int H,
+                                         int dk, int dv, int num_seqs, kda_dtype dtype,
+                                         int range_tokens, void *stream) {
     t_msg[0] = 0;
     if (!q || !k || !v || !g || !beta || !out)
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: null pointer argument");
@@ -498,10 +495,27 @@ extern "C" kda_status kda_chunk_fwd_host(const void *q, const void *k, const voi
     const long long total_T = (long long)B * T;
     if (total_T > 0x7fffffffLL || total_T * H > (1LL << 40))
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: problem too large (B*T=%lld)", total_T);
+    // sequences on the packed token axis: dense [B, T] is B sequences of T
+    int N = B;
+    if (cu_seqlens) {
+        if (B != 1)
+            return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: varlen mode requires B == 1 (got %d)", B);
+        if (num_seqs <= 0 || num_seqs > 65535)
+            return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: num_seqs=%d out of [1, 65535]", num_seqs);
+        N = num_seqs;
+        // a host array: checked in full here
+        if (cu_seqlens[0] != 0 || cu_seqlens[N] != T)
+            return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: cu_seqlens must run from 0 to T=%d", T);
+        for (int n = 0; n < N; ++n)
+            if (cu_seqlens[n + 1] < cu_seqlens[n])
+                return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: cu_seqlens decreases at %d", n);
+    }
+    auto seq_start = [&](int n) -> long long { return cu_seqlens ? cu_seqlens[n] : (long long)n * T; };
     cudaStream_t st = (cudaStream_t)stream;
     const size_t es = dtype == KDA_BF16 ? 2 : 4;
-    const size_t state_bytes = (size_t)B * H * dk * dv * sizeof(float);
-    if (T == 0) {   // nothing to process: final = initial (or zeros)
+    const size_t one_state = (size_t)H * dk * dv * sizeof(float);
+    const size_t state_bytes = (size_t)N * one_state;
+    if (total_T == 0) {   // nothing to process: final = initial (or zeros)
         if (!final_state) return KDA_OK;
         cudaError_t e = initial_state
             ? cudaMemcpyAsync(final_state, initial_state, state_bytes, cudaMemcpyDefault, st)
@@ -514,23 +528,62 @@ extern "C" kda_status kda_chunk_fwd_host(const void *q, const void *k, const voi
         }
         return KDA_OK;
     }
-    // ranges of whole chunks, so the chunk grid is that of one call over T
+    // Ranges of the packed token axis that end at a sequence end or at a whole
+    // number of chunks into a sequence, so every sequence keeps the chunk grid
+    // of one call over it.  Range r covers tokens [cut[r], cut[r + 1]) and
+    // the sequences first[r] .. last[r].
     int R = range_tokens > 0 ? range_tokens : 2048;
     R = (R + 63) / 64 * 64;
-    if (R > T) R = (T + 63) / 64 * 64;
-    const int nr = (T + R - 1) / R;
+    auto seq_of = [&](long long p) -> int {   // the sequence holding token p
+        if (!cu_seqlens) return (int)(p / T);
+        int lo = 0, hi = N - 1;               // the last n with cu[n] <= p
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) / 2;
+            if (cu_seqlens[mid] <= p) lo = mid; else hi = mid - 1;
+        }
+        return lo;
+    };
+    std::vector<long long> cut{0};
+    std::vector<int> first, last;
+    for (long long t0 = 0; t0 < total_T;) {
+        long long c = t0 + R;
+        if (c >= total_T) {
+            c = total_T;
+        } else {   // back to the last chunk boundary of the sequence holding c
+            const long long s = seq_start(seq_of(c));
+            c = s + (c - s) / 64 * 64;    // > t0: t0 is itself such a boundary
+        }
+        first.push_back(seq_of(t0));
+        last.push_back(seq_of(c - 1));
+        cut.push_back(c);
+        t0 = c;
+    }
+    const int nr = (int)first.size();
+    long long max_tokens = 64;
+    for (int r = 0; r < nr; ++r) max_tokens = std::max(max_tokens, cut[r + 1] - cut[r]);
     // per-token row bytes of each input / output (all heads)
     const size_t rq = (size_t)H * dk * es, rv = (size_t)H * dv * es, rg = (size_t)H * dk * 4,
                  rb = (size_t)H * 4, ro = (size_t)H * dv * es;
-    const size_t in_bytes = (size_t)B * R * (2 * rq + rv + rg + rb);
-    const size_t out_bytes = (size_t)B * R * ro;
     auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    // layout of one stage buffer: q k v g beta, each [B, R, H, *]
-    const size_t oq = 0, ok_ = al((size_t)B * R * rq), ov = ok_ + al((size_t)B * R * rq),
-                 og = ov + al((size_t)B * R * rv), ob = og + al((size_t)B * R * rg);
-    const size_t in_stage = ob + al((size_t)B * R * rb);
-    const size_t total = 2 * in_stage + 2 * al(out_bytes) + al(state_bytes);
-    (void)in_bytes;
+    const size_t Rt = (size_t)max_tokens;
+    // one stage buffer: q k v g beta, each [range tokens, H, *]
+    const size_t oq = 0, ok_ = al(Rt * rq), ov = ok_ + al(Rt * rq), og = ov + al(Rt * rv),
+                 ob = og + al(Rt * rg);
+    const size_t in_stage = ob + al(Rt * rb);
+    const size_t out_stage = al(Rt * ro);
+    // range-local offsets: nr arrays of (sequences + 1) int32
+    std::vector<int32_t> local_cu;
+    std::vector<size_t> cu_off(nr);
+    for (int r = 0; r < nr; ++r) {
+        cu_off[r] = local_cu.size();
+        local_cu.push_back(0);
+        for (int n = first[r]; n <= last[r]; ++n) {
+            long long e_ = std::min(seq_start(n + 1), cut[r + 1]) - cut[r];
+            local_cu.push_back((int32_t)e_);
+        }
+    }
+    const size_t cu_bytes = al(local_cu.size() * sizeof(int32_t));
+    const size_t total = 2 * in_stage + 2 * out_stage + al(state_bytes) + cu_bytes;
 
     HostPipeStreams *ps = nullptr;
     cudaMemPool_t pool;
@@ -542,14 +595,14 @@ extern "C" kda_status kda_chunk_fwd_host(const void *q, const void *k, const voi
     if ((e = cudaMallocFromPoolAsync(&buf, total, pool, st)) != cudaSuccess)
         return cuda_fail(e, "kda_chunk_fwd_host device buffers");
     unsigned char *in_dev[2] = {(unsigned char *)buf, (unsigned char *)buf + in_stage};
-    unsigned char *out_dev[2] = {in_dev[1] + in_stage, in_dev[1] + in_stage + al(out_bytes)};
-    float *state_dev = (float *)(out_dev[1] + al(out_bytes));
+    unsigned char *out_dev[2] = {in_dev[1] + in_stage, in_dev[1] + in_stage + out_stage};
+    float *state_dev = (float *)(out_dev[1] + out_stage);
+    int32_t *cu_dev = (int32_t *)((unsigned char *)state_dev + al(state_bytes));
 
     // events: start (buffers allocated, caller's prior work done), and per range
     // in_ready[r], done[r] (inputs of stage r % 2 free again), out_free[r]
     const int ne = 1 + 3 * nr;
-    cudaEvent_t *ev = (cudaEvent_t *)calloc((size_t)ne, sizeof(cudaEvent_t));
-    if (!ev) { cudaFreeAsync(buf, st); return fail(KDA_ERR_CUDA, "kda_chunk_fwd_host: out of host memory"); }
+    std::vector<cudaEvent_t> ev((size_t)ne);
     int made = 0;
     for (; made < ne; ++made)
         if ((e = cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming)) != cudaSuccess) break;
@@ -567,12 +620,18 @@ extern "C" kda_status kda_chunk_fwd_host(const void *q, const void *k, const voi
         chk(cudaEventRecord(ev_start, st), "kda_chunk_fwd_host record");
         chk(cudaStreamWaitEvent(ps->in, ev_start, 0), "kda_chunk_fwd_host wait");
         chk(cudaStreamWaitEvent(ps->out, ev_start, 0), "kda_chunk_fwd_host wait");
-        if (initial_state)
-            chk(cudaMemcpyAsync(state_dev, initial_state, state_bytes, cudaMemcpyDefault, st),
-                "kda_chunk_fwd_host initial state");
+        // every sequence's state lives in state_dev for the whole call
+        chk(initial_state
+                ? cudaMemcpyAsync(state_dev, initial_state, state_bytes, cudaMemcpyDefault, st)
+                : cudaMemsetAsync(state_dev, 0, state_bytes, st),
+            "kda_chunk_fwd_host initial state");
+        chk(cudaMemcpyAsync(cu_dev, local_cu.data(), local_cu.size() * sizeof(int32_t),
+                            cudaMemcpyHostToDevice, st),
+            "kda_chunk_fwd_host range offsets");
     }
     for (int r = 0; r < nr && status == KDA_OK; ++r) {
-        const int t0 = r * R, tr = T - t0 < R ? T - t0 : R;
+        const long long t0 = cut[r];
+        const int tr = (int)(cut[r + 1] - t0);
         const int b = r & 1;
         unsigned char *in = in_dev[b];
         // copy in (the stage's previous user, range r - 2, must be done)
@@ -580,25 +639,27 @@ extern "C" kda_status kda_chunk_fwd_host(const void *q, const void *k, const voi
         const struct { const void *h; size_t off, row; } srcs[5] = {
             {q, oq, rq}, {k, ok_, rq}, {v, ov, rv}, {g, og, rg}, {beta, ob, rb}};
         for (const auto &c : srcs)
-            chk(copy_rows(in + c.off, (size_t)tr * c.row, (const unsigned char *)c.h + (size_t)t0 * c.row,
-                          (size_t)T * c.row, (size_t)tr * c.row, B, ps->in),
+            chk(cudaMemcpyAsync(in + c.off, (const unsigned char *)c.h + (size_t)t0 * c.row,
+                                (size_t)tr * c.row, cudaMemcpyDefault, ps->in),
                 "kda_chunk_fwd_host copy in");
         chk(cudaEventRecord(in_ready(r), ps->in), "kda_chunk_fwd_host record");
-        // compute on the caller's stream: state in, state out, in place
+        // compute on the caller's stream; the states of the range's sequences
+        // are resumed and written back in place
         chk(cudaStreamWaitEvent(st, in_ready(r), 0), "kda_chunk_fwd_host wait");
         if (r >= 2) chk(cudaStreamWaitEvent(st, out_free(r - 2), 0), "kda_chunk_fwd_host wait");
         if (status != KDA_OK) break;
+        float *sr = state_dev + (size_t)first[r] * (one_state / sizeof(float));
+        const int nseq = last[r] - first[r] + 1;
         kda_status s2 = chunk_fwd_device(in + oq, in + ok_, in + ov, (const float *)(in + og),
-                                         (const float *)(in + ob),
-                                         (r == 0 && !initial_state) ? nullptr : state_dev, nullptr,
-                                         out_dev[b], state_dev, B, tr, H, dk, dv, B, dtype,
+                                         (const float *)(in + ob), sr, cu_dev + cu_off[r],
+                                         out_dev[b], sr, 1, tr, H, dk, dv, nseq, dtype,
                                          kda::Prologue{0, 1.f}, st);
         if (s2 != KDA_OK) { status = s2; break; }
         chk(cudaEventRecord(done(r), st), "kda_chunk_fwd_host record");
         // copy out
         chk(cudaStreamWaitEvent(ps->out, done(r), 0), "kda_chunk_fwd_host wait");
-        chk(copy_rows((unsigned char *)out + (size_t)t0 * ro, (size_t)T * ro, out_dev[b],
-                      (size_t)tr * ro, (size_t)tr * ro, B, ps->out),
+        chk(cudaMemcpyAsync((unsigned char *)out + (size_t)t0 * ro, out_dev[b], (size_t)tr * ro,
+                            cudaMemcpyDefault, ps->out),
             "kda_chunk_fwd_host copy out");
         chk(cudaEventRecord(out_free(r), ps->out), "kda_chunk_fwd_host record");
     }
@@ -617,7 +678,6 @@ extern "C" kda_status kda_chunk_fwd_host(const void *q, const void *k, const voi
     }
     cudaError_t ef = cudaFreeAsync(buf, st);
     for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);
-    free(ev);
     if (status == KDA_OK && ef != cudaSuccess) status = cuda_fail(ef, "kda_chunk_fwd_host release");
     return status;
 }

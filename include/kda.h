@@ -137,37 +137,43 @@ kda_status kda_chunk_fwd_ex(const void *q, const void *k, const void *v,
                             kda_dtype dtype, unsigned flags, float q_scale, void *stream);
 
 /*
- * kda_chunk_fwd_host -- kda_chunk_fwd (dense mode) on HOST buffers, with the
- * host<->device copies pipelined against the computation.
+ * kda_chunk_fwd_host -- kda_chunk_fwd on HOST buffers, with the host<->device
+ * copies pipelined against the computation.
  *
  * Source: as kda_chunk_fwd; the pipelining rests on the checkpoint semantics
  * (whoami-wesleyyou blog, "context modification and checkpoint": a state
- * summarises its prefix exactly) -- the sequence is processed in ranges of
- * whole chunks, each range resuming from the fp32 state the previous one
- * left on the device, so the chunk grid, and the result, are those of one
- * kda_chunk_fwd call over the whole sequence.  The pages have no host-buffer
- * entry point; this is a deployment variant.
+ * summarises its prefix exactly) -- the packed token axis is processed in
+ * ranges, each range resuming its sequences from the fp32 states the
+ * previous range left on the device.  A range ends at a sequence end or a
+ * whole number of chunks into a sequence, so every sequence keeps the chunk
+ * grid, and the result, of one kda_chunk_fwd call.  The pages have no
+ * host-buffer entry point; this is a deployment variant.
  *
  * Pointers: q, k, v, g, beta, initial_state (nullable), out, final_state
- *   (nullable) are HOST pointers with kda_chunk_fwd's dense layouts
- *   ([B, T, H, *]).  Page-locked (pinned) memory lets the copies overlap the
- *   computation; pageable memory works, with copies that do not overlap.
+ *   (nullable) are HOST pointers with kda_chunk_fwd's layouts (dense [B, T,
+ *   H, *], or varlen [1, T, H, *] with states [num_seqs, H, dk, dv]).
+ *   cu_seqlens (nullable = dense mode) is a HOST int32 array [num_seqs + 1],
+ *   checked in full (cu[0] = 0, non-decreasing, cu[num_seqs] = T; else
+ *   KDA_ERR_INVALID_ARG).  Page-locked (pinned) memory lets the copies
+ *   overlap the computation; pageable memory works, with copies that do not
+ *   overlap.
  * range_tokens: tokens per pipeline stage, rounded up to a multiple of 64;
  *   0 selects 2048 (measured best for 32 heads x d = 128 over PCIe).
  * Streams: the computation runs on `stream`; the copies run on two streams
  *   the library keeps per device, ordered after the work already queued on
  *   `stream`, and `stream` is ordered after them, so the outputs are in host
  *   memory once `stream` has completed (e.g. cudaStreamSynchronize).
- * Memory: device buffers for two input stages, two output stages and the
- *   state come from the library-private pool (stream-ordered, as in
- *   kda_chunk_fwd) and are released on `stream`.
- * Supported: as kda_chunk_fwd in dense mode (no cu_seqlens).
+ * Memory: device buffers for two input stages, two output stages, every
+ *   sequence's state and the ranges' offsets come from the library-private
+ *   pool (stream-ordered, as in kda_chunk_fwd) and are released on `stream`.
+ * Supported: as kda_chunk_fwd.
  * Aliasing: out and final_state must not overlap any input.
  */
 kda_status kda_chunk_fwd_host(const void *q, const void *k, const void *v,
                               const float *g, const float *beta,
-                              const float *initial_state, void *out, float *final_state,
-                              int B, int T, int H, int dk, int dv,
+                              const float *initial_state, const int32_t *cu_seqlens,
+                              void *out, float *final_state,
+                              int B, int T, int H, int dk, int dv, int num_seqs,
                               kda_dtype dtype, int range_tokens, void *stream);
 
 /*

@@ -158,11 +158,12 @@ def test_steps_unsupported_rejected(lib, kw):
     assert steps(lib, **kw) == 2
 
 
-def host(lib, *, q=FAKE, k=FAKE, v=FAKE, g=FAKE, b=FAKE, s0=None, out=FAKE, sT=None, B=1, T=64,
-         H=1, dk=128, dv=128, dtype=1, rt=0):
+def host(lib, *, q=FAKE, k=FAKE, v=FAKE, g=FAKE, b=FAKE, s0=None, cu=None, out=FAKE, sT=None,
+         B=1, T=64, H=1, dk=128, dv=128, N=1, dtype=1, rt=0):
     P = ctypes.c_void_p
-    return lib.kda_chunk_fwd_host(P(q), P(k), P(v), P(g), P(b), P(s0), P(out), P(sT), B, T, H,
-                                  dk, dv, dtype, rt, None)
+    cu_arr = None if cu is None else (ctypes.c_int32 * len(cu))(*cu)
+    return lib.kda_chunk_fwd_host(P(q), P(k), P(v), P(g), P(b), P(s0), cu_arr, P(out), P(sT), B,
+                                  T, H, dk, dv, N, dtype, rt, None)
 
 
 @pytest.mark.parametrize("kw", [dict(flags=8), dict(flags=4), dict(flags=0xFFFFFFFF),
@@ -204,6 +205,13 @@ def test_host_null_pointer_rejected(lib, field):
 @pytest.mark.parametrize("kw", [dict(B=0), dict(T=-1), dict(H=0), dict(rt=-64), dict(dtype=9),
                                 dict(B=70000), dict(T=1 << 30, B=4)])
 def test_host_bad_arguments_rejected(lib, kw):
+    assert host(lib, **kw) == 1
+
+
+@pytest.mark.parametrize("kw", [dict(cu=[1, 64], N=1), dict(cu=[0, 32], N=1), dict(cu=[0, 40, 30, 64], N=3),
+                                dict(cu=[0, 64], N=0), dict(cu=[0, 64], N=1, B=2)])
+def test_host_bad_varlen_offsets_rejected(lib, kw):
+    # cu_seqlens is a host array here: it is checked in full before any CUDA call
     assert host(lib, **kw) == 1
 
 

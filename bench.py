@@ -270,6 +270,7 @@ def run_ours(args):
                                      flags=kda.KDA_STEPS_CHUNK, kernel="decode_chunk_kernel",
                                      traffic_key="decode_chunk", ring=1)
         bwd = backward_leg(kda, inp, dev, dist, world, args)
+        bwd_chunk = backward_leg(kda, inp, dev, dist, world, args, chunked=True)
     clk.samples += clk_dec.samples
     clk.reasons |= clk_dec.reasons
 
@@ -296,6 +297,7 @@ def run_ours(args):
         "decode_steps": dec_steps,
         "decode_chunk": dec_chunk,
         "backward": bwd,
+        "backward_chunk": bwd_chunk,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(inp_cpu)
@@ -400,13 +402,14 @@ def decode_steps_leg(kda, W, dev, dist, world, args, L=STEPS_L, flags=0,
 BWD_BYTES = B * T * H * (4 * D * 2 + D * 4 + 4 + 4 * D * 4 + 4)
 
 
-def backward_leg(kda, inp, dev, dist, world, args):
-    """Training backward (kda_recurrent_bwd) on the prefill workload with a
-    seeded output gradient; no initial or final state."""
+def backward_leg(kda, inp, dev, dist, world, args, chunked=False):
+    """Training backward on the prefill workload with a seeded output
+    gradient; no initial or final state.  chunked: kda_chunk_bwd (tensor
+    cores), else kda_recurrent_bwd."""
     gen = torch.Generator().manual_seed(41)
     do = torch.randn(B, T, H, D, generator=gen).to(torch.bfloat16).to(dev)
-    run = lambda: kda.kda_recurrent_bwd(inp.q, inp.k, inp.v, inp.g, inp.beta, do,
-                                        want_initial_state_grad=False)
+    fn = kda.kda_chunk_bwd if chunked else kda.kda_recurrent_bwd
+    run = lambda: fn(inp.q, inp.k, inp.v, inp.g, inp.beta, do, want_initial_state_grad=False)
     for _ in range(max(1, min(args.warmup, 3))):
         run()
     barrier(dist)
@@ -421,12 +424,17 @@ def backward_leg(kda, inp, dev, dist, world, args):
     ms = max_over_ranks(e0.elapsed_time(e1), dist) / calls
     peak, kind = measured_peak_hbm()
     ach = BWD_BYTES / (ms * 1e-3) / 1e9
+    if chunked:
+        bound, kernel, traffic = "hbm", "kda_chunk_bwd (prep, chain, reverse chain, per-chunk pass)", None
+    else:
+        bound, kernel = "latency (sequential per token)", "recurrent_bwd_kernel"
+        traffic = measured_traffic("backward")
     return {"workload": WORKLOAD + "_backward", "value": job_value(B * T, world, ms),
             "unit": UNIT, "ms_per_call": ms, "calls": calls,
-            "roofline": {"bound": "latency (sequential per token)", "kernel": "recurrent_bwd_kernel",
+            "roofline": {"bound": bound, "kernel": kernel,
                          "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                          "peak_source": kind, "algorithmic_bytes_per_launch": BWD_BYTES,
-                         "traffic": measured_traffic("backward")}}
+                         "traffic": traffic}}
 
 
 def cpu_baseline(inp_cpu, tokens=None):

@@ -24,6 +24,8 @@ Entry points (same names as the C ABI):
     kda_gated_rmsnorm(x, gate, weight, eps=1e-5, out=None) -> out
     kda_recurrent_bwd(q, k, v, g, beta, do, initial_state=None, dsT=None)
         -> (dq, dk, dv, dg, dbeta, ds0)
+    kda_chunk_bwd(..., cu_seqlens=None): the same gradients by the chunked form
+                     (bf16, dk = dv = 128; tensor cores)
     kda_state_affine(M, B, S_in, out=None) -> S_out
     kda_get_device_error(stream=None) -> int
 """
@@ -38,7 +40,7 @@ import torch
 __all__ = ["kda_chunk_fwd", "kda_chunk_fwd_ex", "kda_chunk_fwd_host", "kda_chunk_fwd_noalloc",
            "kda_recurrent_step",
            "kda_recurrent_step_ex", "kda_recurrent_steps", "kda_gated_rmsnorm", "kda_state_affine",
-           "kda_recurrent_bwd",
+           "kda_recurrent_bwd", "kda_chunk_bwd",
            "kda_get_device_error",
            "KDAError",
            "KDA_QK_L2NORM", "KDA_BETA_SIGMOID", "KDA_STEPS_CHUNK",
@@ -94,6 +96,8 @@ def load_library():
         lib.kda_state_affine.argtypes = [vp] * 4 + [i] * 3 + [vp]
         lib.kda_recurrent_bwd.argtypes = [vp] * 14 + [i] * 6 + [vp]
         lib.kda_recurrent_bwd.restype = i
+        lib.kda_chunk_bwd.argtypes = [vp] * 15 + [i] * 7 + [vp]
+        lib.kda_chunk_bwd.restype = i
         lib.kda_state_affine.restype = i
         lib.kda_get_device_error.argtypes = [vp, ctypes.POINTER(i)]
         lib.kda_get_device_error.restype = i
@@ -388,6 +392,44 @@ def kda_recurrent_bwd(q, k, v, g, beta, do, initial_state=None, dsT=None,
                                    _dptr(initial_state), _dptr(do), _dptr(dsT), _dptr(dq),
                                    _dptr(dk_), _dptr(dv_), _dptr(dg), _dptr(db), _dptr(ds0),
                                    B, T, H, dk, dv, dt, _stream_handle(dev))
+    _check(rc)
+    return dq, dk_, dv_, dg, db, ds0
+
+
+def kda_chunk_bwd(q, k, v, g, beta, do, initial_state=None, dsT=None, cu_seqlens=None,
+                  want_initial_state_grad: bool = True):
+    """Gradients by the chunked form on the tensor cores (bf16, dk = dv = 128):
+    arguments and results as kda_recurrent_bwd, plus cu_seqlens (varlen, B == 1;
+    states then [N,H,dk,dv])."""
+    lib = load_library()
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("kda_chunk_bwd needs CUDA tensors (no CPU path)")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    for t, name in ((k, "k"), (v, "v"), (do, "do")):
+        _need(t, name, dev, q.dtype)
+    _need(q, "q", dev)
+    _need(g, "g", dev, torch.float32)
+    _need(beta, "beta", dev, torch.float32)
+    N = B
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", dev, torch.int32)
+        N = cu_seqlens.numel() - 1
+    for t, name in ((initial_state, "initial_state"), (dsT, "dsT")):
+        if t is not None:
+            _need(t, name, dev, torch.float32)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dq, dk_, dg = (torch.empty(B, T, H, dk, **f32) for _ in range(3))
+    dv_ = torch.empty(B, T, H, dv, **f32)
+    db = torch.empty(B, T, H, **f32)
+    ds0 = torch.empty(N, H, dk, dv, **f32) if want_initial_state_grad else None
+    with torch.cuda.device(dev):
+        rc = lib.kda_chunk_bwd(_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta),
+                               _dptr(initial_state), _dptr(cu_seqlens), _dptr(do), _dptr(dsT),
+                               _dptr(dq), _dptr(dk_), _dptr(dv_), _dptr(dg), _dptr(db), _dptr(ds0),
+                               B, T, H, dk, dv, N, dt, _stream_handle(dev))
     _check(rc)
     return dq, dk_, dv_, dg, db, ds0
 

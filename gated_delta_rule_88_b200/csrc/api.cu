@@ -383,6 +383,98 @@ extern "C" kda_status kda_gated_rmsnorm(const void *x, const void *gate, const f
     return KDA_OK;
 }
 
+extern "C" kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const float *g,
+                                    const float *beta, const float *initial_state,
+                                    const int32_t *cu_seqlens, const void *dout,
+                                    const float *dfinal_state, float *dq, float *dk, float *dv,
+                                    float *dg, float *dbeta, float *dinitial_state, int B, int T,
+                                    int H, int dk_, int dv_, int num_seqs, kda_dtype dtype,
+                                    void *stream) {
+    t_msg[0] = 0;
+    if (!q || !k || !v || !g || !beta || !dout || !dq || !dk || !dv || !dg || !dbeta)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: null pointer argument");
+    if (B <= 0 || T < 0 || H <= 0 || dk_ <= 0 || dv_ <= 0 || B > 65535 || H > 65535)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: bad sizes B=%d T=%d H=%d dk=%d dv=%d", B,
+                    T, H, dk_, dv_);
+    if (dtype != KDA_F32 && dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: unknown dtype %d", (int)dtype);
+    if (dtype != KDA_BF16 || dk_ != 128 || dv_ != 128)
+        return fail(KDA_ERR_UNSUPPORTED,
+                    "kda_chunk_bwd: dtype=%d dk=%d dv=%d (supported: bf16 with dk = dv = 128)",
+                    (int)dtype, dk_, dv_);
+    int N = B;
+    if (cu_seqlens) {
+        if (B != 1)
+            return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: varlen mode requires B == 1 (got %d)", B);
+        if (num_seqs <= 0 || num_seqs > 65535)
+            return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: num_seqs=%d out of [1, 65535]", num_seqs);
+        N = num_seqs;
+    }
+    const void *ptrs[] = {q, k, v, g, dout, dq, dk, dv, dg, initial_state, dfinal_state, dinitial_state};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p))
+            return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: pointers must be 16-byte aligned");
+    if (((uintptr_t)beta & 3u) || ((uintptr_t)dbeta & 3u) || ((uintptr_t)cu_seqlens & 3u))
+        return fail(KDA_ERR_INVALID_ARG,
+                    "kda_chunk_bwd: beta, dbeta and cu_seqlens must be 4-byte aligned");
+    const long long total_T = (long long)B * T;
+    if (total_T > 0x7fffffffLL || total_T * H > (1LL << 34))
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: problem too large (B*T=%lld)", total_T);
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t sbytes = (size_t)N * H * 128 * 128 * sizeof(float);
+    if (total_T == 0) {
+        // no tokens: the initial state's gradient is the final state's
+        cudaError_t e = cudaSuccess;
+        if (dinitial_state)
+            e = dfinal_state ? cudaMemcpyAsync(dinitial_state, dfinal_state, sbytes,
+                                               cudaMemcpyDeviceToDevice, st)
+                             : cudaMemsetAsync(dinitial_state, 0, sbytes, st);
+        return e == cudaSuccess ? KDA_OK : cuda_fail(e, "kda_chunk_bwd empty input");
+    }
+    const long long max_chunks = cu_seqlens ? (total_T + 63) / 64 + N : (long long)B * ((T + 63) / 64);
+    const size_t slots = (size_t)max_chunks * H;
+    const size_t coff_bytes = (((size_t)N + 1) * sizeof(int32_t) + 255) & ~(size_t)255;
+    const size_t bytes = coff_bytes + slots * (kda::ws::RECORD + 2 * 32768 + 2 * 16384);
+    cudaMemPool_t pool;
+    int sms = 148;
+    cudaError_t e = get_pool(&pool, &sms);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_bwd memory pool");
+    void *scratch = nullptr;
+    e = cudaMallocFromPoolAsync(&scratch, bytes, pool, st);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_bwd scratch allocation");
+    int32_t *coff = (int32_t *)scratch;
+    unsigned char *records = (unsigned char *)scratch + coff_bytes;
+    unsigned char *s_img = records + slots * kda::ws::RECORD;
+    unsigned char *dsp_img = s_img + slots * 32768;
+    unsigned char *v_img = dsp_img + slots * 32768;
+    unsigned char *dvn_img = v_img + slots * 16384;
+    kda::Prologue pro{0, 1.f};
+    int *err = kda::error_word();
+    if (cu_seqlens) e = kda::launch_chunk_plan(cu_seqlens, N, (int)total_T, coff, st);
+    // forward recompute: records, then the chain storing S and V_new per chunk
+    if (e == cudaSuccess)
+        e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, cu_seqlens ? coff : nullptr, N, T,
+                                   (int)total_T, H, (int)max_chunks, records, pro, err, st);
+    if (e == cudaSuccess)
+        e = kda::launch_chunk_chain(records, cu_seqlens, cu_seqlens ? coff : nullptr, initial_state,
+                                    nullptr, nullptr, N, T, (int)total_T, H, 32, (int)max_chunks, err,
+                                    st, s_img, v_img);
+    // reverse chain, then the per-(chunk, head) gradients
+    if (e == cudaSuccess)
+        e = kda::launch_chunk_chain_bwd(dout, records, cu_seqlens, cu_seqlens ? coff : nullptr,
+                                        dfinal_state, dinitial_state, dsp_img, dvn_img, N, T,
+                                        (int)total_T, H, (int)max_chunks, err, st);
+    if (e == cudaSuccess)
+        e = kda::launch_chunk_bwd_local(q, k, v, g, beta, dout, cu_seqlens,
+                                        cu_seqlens ? coff : nullptr, N, T, (int)total_T, H,
+                                        (int)max_chunks, s_img, v_img, dsp_img, dvn_img, dq, dk, dv,
+                                        dg, dbeta, err, st);
+    cudaError_t e2 = cudaFreeAsync(scratch, st);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_bwd launch");
+    if (e2 != cudaSuccess) return cuda_fail(e2, "kda_chunk_bwd scratch release");
+    return KDA_OK;
+}
+
 extern "C" kda_status kda_recurrent_bwd(const void *q, const void *k, const void *v,
                                         const float *g, const float *beta,
                                         const float *initial_state, const void *dout,

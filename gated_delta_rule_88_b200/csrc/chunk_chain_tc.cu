@@ -76,7 +76,8 @@ __global__ void __launch_bounds__(TcLayout<DVT, NS>::NTHREADS, 1)
 chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__restrict__ cu,
                       const int32_t *__restrict__ coff, const float *__restrict__ s0,
                       float *__restrict__ sT, __nv_bfloat16 *__restrict__ out, int T, int total_T,
-                      int H, int cps, int max_chunks, int *__restrict__ err)
+                      int H, int cps, int max_chunks, int *__restrict__ err,
+                      unsigned char *__restrict__ s_img, unsigned char *__restrict__ v_img)
 {
     using L = TcLayout<DVT, NS>;
     extern __shared__ unsigned char smem_raw[];
@@ -256,12 +257,20 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
                 S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
             }
         }
-        auto write_B1 = [&]() {
+        // S entering chunk ci -> B1; with s_img (the backward's forward pass)
+        // also its bf16 image [dk][dv], K-major SW128 in 64-column blocks
+        auto write_B1 = [&](int ci) {
+            unsigned char *img = (s_img && ci < nchunks)
+                                     ? s_img + ((size_t)(max(c_begin, 0) + ci) * H + h) * 32768 : nullptr;
 #pragma unroll
             for (int ng = 0; ng < CPT / 8; ++ng) {
                 uint4 pk = make_uint4(pack_bf16(S[8 * ng], S[8 * ng + 1]), pack_bf16(S[8 * ng + 2], S[8 * ng + 3]),
                                       pack_bf16(S[8 * ng + 4], S[8 * ng + 5]), pack_bf16(S[8 * ng + 6], S[8 * ng + 7]));
                 *reinterpret_cast<uint4 *>(B1 + L::b_off(t, cb / 8 + ng)) = pk;
+                if (img) {
+                    const int n = n0 + cb + 8 * ng;
+                    *reinterpret_cast<uint4 *>(img + (size_t)(n >> 6) * 16384 + ws::sw128(t, n & 63)) = pk;
+                }
             }
             fence_proxy_async_smem();
         };
@@ -286,7 +295,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
             const long long tok = bos + (long long)C * ci + (t - 64);
             float o[CPT];
             tmem_row((ci & 1) * DVT, o);
-            if (tok < eos) {
+            if (out && tok < eos) {        // out == nullptr: the backward's recompute pass
                 uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)tok * H + h) * D + n0 + cb);
 #pragma unroll
                 for (int e = 0; e < CPT / 8; ++e)
@@ -295,7 +304,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
             }
             return true;
         };
-        write_B1();
+        write_B1(0);
         tc_fence_before();
         bool failed = false, ok = true;
         for (int i = 0; i < nchunks; ++i) {
@@ -337,6 +346,13 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
                         pk[e] = pack_bf16(__low2float(u2) - x[8 * ng + 2 * e], __high2float(u2) - x[8 * ng + 2 * e + 1]);
                     }
                     *reinterpret_cast<uint4 *>(B2 + p * L::B2_BYTES + L::b_off(t, cb / 8 + ng)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    if (v_img) {
+                        // the backward's V_new image [C][dv], K-major SW128
+                        const int n = n0 + cb + 8 * ng;
+                        *reinterpret_cast<uint4 *>(v_img + ((size_t)(max(c_begin, 0) + i) * H + h) * 16384 +
+                                                   (size_t)(n >> 6) * 8192 + ws::sw128(t, n & 63)) =
+                            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
                 }
                 fence_proxy_async_smem();
             }
@@ -351,7 +367,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
 #pragma unroll
                 for (int e = 0; e < CPT; ++e) S[e] = eg * S[e] + z[e];
             }
-            write_B1();
+            write_B1(i + 1);
             tc_fence_before();
         }
         if (!failed && !ok) failed = true;
@@ -375,7 +391,8 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
 template <int DVT, int NS>
 cudaError_t launch_tc(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
                       const float *s0, float *sT, void *out, int N, int T, int total_T, int H,
-                      int max_chunks, int *err, cudaStream_t st)
+                      int max_chunks, int *err, cudaStream_t st, unsigned char *s_img,
+                      unsigned char *v_img)
 {
     using L = TcLayout<DVT, NS>;
     const size_t smem = L::BYTES + 1024;
@@ -384,7 +401,8 @@ cudaError_t launch_tc(const unsigned char *wsp, const int32_t *cu, const int32_t
     if (e != cudaSuccess) return e;
     dim3 grid(D / DVT, H, N);
     chunk_chain_tc_kernel<DVT, NS><<<grid, L::NTHREADS, smem, st>>>(
-        wsp, cu, coff, s0, sT, (__nv_bfloat16 *)out, T, total_T, H, (T + C - 1) / C, max_chunks, err);
+        wsp, cu, coff, s0, sT, (__nv_bfloat16 *)out, T, total_T, H, (T + C - 1) / C, max_chunks, err,
+        s_img, v_img);
     return cudaGetLastError();
 }
 
@@ -393,12 +411,12 @@ cudaError_t launch_tc(const unsigned char *wsp, const int32_t *cu, const int32_t
 cudaError_t launch_chunk_chain(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
                                   const float *s0, float *sT, void *out, int N, int T,
                                   int total_T, int H, int dvt, int max_chunks, int *err,
-                                  cudaStream_t st)
+                                  cudaStream_t st, unsigned char *s_img, unsigned char *v_img)
 {
     switch (dvt) {
-        case 16: return launch_tc<16, 3>(wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st);
-        case 32: return launch_tc<32, 3>(wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st);
-        case 64: return launch_tc<64, 2>(wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st);
+        case 16: return launch_tc<16, 3>(wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st, s_img, v_img);
+        case 32: return launch_tc<32, 3>(wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st, s_img, v_img);
+        case 64: return launch_tc<64, 2>(wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st, s_img, v_img);
     }
     return cudaErrorInvalidValue;
 }

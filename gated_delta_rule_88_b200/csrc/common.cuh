@@ -15,6 +15,7 @@ enum DeviceError : int {
     kErrWaitTimeout = 1,     // an mbarrier wait exceeded its bound
     kErrBadOffsets = 2,      // cu_seqlens inconsistent (chunks beyond the records)
     kErrBadSlot = 3,         // a state-slot index outside [0, num_slots)
+    kErrBwdRange = 4,        // chunked backward: a chunk's decay leaves e^{+-80} (chunk skipped)
 };
 
 // Input prologue (struct Prologue, kernels.h): q <- q_scale * (QK_L2NORM ?

@@ -89,8 +89,26 @@ cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const
                               const float *beta, const int32_t *cu, const int32_t *coff,
                               int N, int T, int total_T, int H, int max_chunks,
                               unsigned char *wsp, Prologue pro, int *err, cudaStream_t st);
+// s_img / v_img (nullable): per-(chunk, head) bf16 images of the state
+// entering each chunk (32 KiB) and of V_new (16 KiB), for the backward
 cudaError_t launch_chunk_chain(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
                                const float *s0, float *sT, void *out, int N, int T, int total_T,
-                               int H, int dvt, int max_chunks, int *err, cudaStream_t st);
+                               int H, int dvt, int max_chunks, int *err, cudaStream_t st,
+                               unsigned char *s_img = nullptr, unsigned char *v_img = nullptr);
+
+// Chunked backward (bf16, dk = dv = 128): the reverse chain over the forward
+// records (gradient images dS' 32 KiB and dV_new 16 KiB per (chunk, head)),
+// then the per-(chunk, head) gradient pass.
+cudaError_t launch_chunk_chain_bwd(const void *dout, const unsigned char *wsp, const int32_t *cu,
+                                   const int32_t *coff, const float *dsT, float *ds0,
+                                   unsigned char *dsp_img, unsigned char *dvn_img, int N, int T,
+                                   int total_T, int H, int max_chunks, int *err, cudaStream_t st);
+cudaError_t launch_chunk_bwd_local(const void *q, const void *k, const void *v, const float *g,
+                                   const float *beta, const void *dout, const int32_t *cu,
+                                   const int32_t *coff, int N, int T, int total_T, int H,
+                                   int max_chunks, const unsigned char *s_img,
+                                   const unsigned char *v_img, const unsigned char *dsp_img,
+                                   const unsigned char *dvn_img, float *dq, float *dk, float *dv,
+                                   float *dg, float *dbeta, int *err, cudaStream_t st);
 
 }  // namespace kda

@@ -310,6 +310,45 @@ kda_status kda_recurrent_bwd(const void *q, const void *k, const void *v, const 
                              int dk_, int dv_, kda_dtype dtype, void *stream);
 
 /*
+ * kda_chunk_bwd -- gradients of kda_chunk_fwd's result by the chunked form on
+ * the tensor cores, for training (bf16, dk = dv = 128).
+ *
+ * Source: Kimi Linear paper notes (paper-notes-site), section 3 (training
+ * takes the chunked kernels and their backward); the equations are reverse
+ * mode through the chunk form of section 3 (derived from the section 2
+ * recurrence).  Per chunk, S the state entering it and dS' the gradient of
+ * the state leaving it (dS' = dfinal_state, or 0, for the last chunk):
+ *   dV_new = P^T dO + Kt dS',  dS = Qg^T dO + Diag(e^{G_C}) dS' - W^T dV_new
+ * (last chunk first), then per chunk dP = tril0(dO V_new^T), dKt = V_new dS'^T,
+ *   dW = -dV_new S^T, dT = dV_new (beta V)^T + dW (beta K e^G)^T,
+ *   dA = tril_-1(-T^T dT T^T), and the gradients of the decayed forms down to
+ *   dq, dk, dv, dbeta and dg (the in-chunk reverse cumsum of dG).
+ * Computation: the forward prep and chain recomputed (the chain also storing
+ *   S and V_new per chunk as bf16), a reverse chain over chunks per (sequence,
+ *   head, 32-column tile), and one CTA per (chunk, head) for the rest; bf16
+ *   tensor-core operands, fp32 accumulation and state gradient.  Workspace
+ *   from the device's stream-ordered pool on `stream`: 168.5 KiB per (chunk,
+ *   head).
+ * Layout: as kda_chunk_fwd for q, k, v, g, beta, initial_state, cu_seqlens
+ *   (varlen: B == 1, num_seqs sequences); dout [B, T, H, dv] bf16;
+ *   dfinal_state, dinitial_state [N, H, dk, dv] float32 or NULL (zeros / not
+ *   written).  Outputs, float32, written for every token: dq, dk, dg
+ *   [B, T, H, dk]; dv [B, T, H, dv]; dbeta [B, T, H].
+ * Range: a chunk in which some |G| or G_C - G exceeds 80 (an average per-token
+ *   log-decay below -1.25 on a channel over 64 tokens) sets the device error
+ *   word (kda_get_device_error returns KDA_ERR_DEVICE) and its gradients are
+ *   not written; kda_recurrent_bwd covers such inputs.
+ * Supported: KDA_BF16 with dk = dv = 128 (else KDA_ERR_UNSUPPORTED).
+ *   Pointers 16-byte aligned (beta, dbeta, cu_seqlens 4).
+ */
+kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const float *g,
+                         const float *beta, const float *initial_state,
+                         const int32_t *cu_seqlens, const void *dout, const float *dfinal_state,
+                         float *dq, float *dk, float *dv, float *dg, float *dbeta,
+                         float *dinitial_state, int B, int T, int H, int dk_, int dv_,
+                         int num_seqs, kda_dtype dtype, void *stream);
+
+/*
  * kda_state_affine -- S_out = M S_in + B for `count` independent blocks.
  *
  * Source: the recurrence of the paper notes (section 2) is affine in the

@@ -266,3 +266,28 @@ def test_bwd_bad_arguments_rejected(lib, kw):
 @pytest.mark.parametrize("kw", [dict(d_k=32), dict(d_v=96), dict(d_k=256)])
 def test_bwd_unsupported_rejected(lib, kw):
     assert bwd(lib, **kw) == 2
+
+
+def cbwd(lib, *, q=FAKE, k=FAKE, v=FAKE, g=FAKE, b=FAKE, s0=None, cu=None, do=FAKE, dsT=None,
+         dq=FAKE, dk=FAKE, dv=FAKE, dg=FAKE, db=FAKE, ds0=None, B=1, T=8, H=1, d_k=128, d_v=128,
+         N=1, dtype=1):
+    P = ctypes.c_void_p
+    return lib.kda_chunk_bwd(P(q), P(k), P(v), P(g), P(b), P(s0), P(cu), P(do), P(dsT), P(dq),
+                             P(dk), P(dv), P(dg), P(db), P(ds0), B, T, H, d_k, d_v, N, dtype, None)
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "g", "b", "do", "dq", "dk", "dv", "dg", "db"])
+def test_chunk_bwd_null_pointer_rejected(lib, field):
+    assert cbwd(lib, **{field: 0}) == 1
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(T=-1), dict(H=-1), dict(dtype=5), dict(q=FAKE + 4),
+                                dict(db=FAKE + 2), dict(s0=FAKE + 8), dict(B=70000),
+                                dict(cu=FAKE, B=2), dict(cu=FAKE, N=0), dict(cu=FAKE + 2)])
+def test_chunk_bwd_bad_arguments_rejected(lib, kw):
+    assert cbwd(lib, **kw) == 1
+
+
+@pytest.mark.parametrize("kw", [dict(d_k=64), dict(d_v=64), dict(dtype=0)])
+def test_chunk_bwd_unsupported_rejected(lib, kw):
+    assert cbwd(lib, **kw) == 2

@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "chunk_ws.h"
+#include "api_internal.h"
 
 namespace kda {
 // The per-device error word (see common.cuh).  Host code reaches it through
@@ -44,9 +45,7 @@ namespace kda {
 thread_local char t_msg[512] = "";
 }  // namespace kda
 
-namespace {
-using kda::t_msg;
-
+namespace kda {
 kda_status fail(kda_status s, const char *fmt, ...) {
     va_list ap;
     va_start(ap, fmt);
@@ -54,6 +53,11 @@ kda_status fail(kda_status s, const char *fmt, ...) {
     va_end(ap);
     return s;
 }
+}  // namespace kda
+
+namespace {
+using kda::t_msg;
+using kda::fail;
 
 kda_status cuda_fail(cudaError_t e, const char *what) {
     return fail(KDA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
@@ -245,33 +249,11 @@ static kda_status chunk_fwd_impl(const void *q, const void *k, const void *v, co
                                  const int32_t *cu_seqlens, void *out, float *final_state,
                                  int B, int T, int H, int dk, int dv, int num_seqs,
                                  kda_dtype dtype, kda::Prologue pro, void *stream) {
-    if (!q || !k || !v || !g || !beta || !out)
-        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: null pointer argument");
-    if (B <= 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0)
-        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: bad sizes B=%d T=%d H=%d dk=%d dv=%d",
-                    B, T, H, dk, dv);
-    if (dtype != KDA_F32 && dtype != KDA_BF16)
-        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: unknown dtype %d", (int)dtype);
-    int N = B;
-    if (cu_seqlens) {
-        if (B != 1)
-            return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: varlen mode requires B == 1 (got %d)", B);
-        if (num_seqs <= 0 || num_seqs > 65535)
-            return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: num_seqs=%d out of [1, 65535]", num_seqs);
-        N = num_seqs;
-    } else if (B > 65535) {
-        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: B=%d exceeds 65535", B);
-    }
-    if (H > 65535) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: H=%d exceeds 65535", H);
-    const void *ptrs[] = {q, k, v, g, out, initial_state, final_state};
-    for (const void *p : ptrs)
-        if (p && !aligned16(p))
-            return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: pointers must be 16-byte aligned");
-    if (((uintptr_t)beta & 3u) || (cu_seqlens && ((uintptr_t)cu_seqlens & 3u)))
-        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: beta and cu_seqlens must be 4-byte aligned");
-    const long long total_T = (long long)B * T;
-    if (total_T > 0x7fffffffLL || total_T * H > (1LL << 40))
-        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: problem too large (B*T=%lld)", total_T);
+    int N = 0;
+    kda_status s = kda::check_chunk_fwd_args("kda_chunk_fwd", q, k, v, g, beta, initial_state,
+                                             cu_seqlens, out, final_state, B, T, H, dk, dv,
+                                             num_seqs, dtype, &N);
+    if (s != KDA_OK) return s;
     return chunk_fwd_device(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state, B, T,
                             H, dk, dv, N, dtype, pro, (cudaStream_t)stream);
 }
@@ -301,6 +283,88 @@ kda_status kda_chunk_fwd_ex(const void *q, const void *k, const void *v, const f
 
 }  // extern "C"
 
+namespace kda {
+
+kda_status check_chunk_fwd_args(const char *fn, const void *q, const void *k, const void *v,
+                                const float *g, const float *beta, const float *initial_state,
+                                const int32_t *cu_seqlens, const void *out,
+                                const float *final_state, int B, int T, int H, int dk, int dv,
+                                int num_seqs, kda_dtype dtype, int *N_out) {
+    if (!q || !k || !v || !g || !beta || !out)
+        return fail(KDA_ERR_INVALID_ARG, "%s: null pointer argument", fn);
+    if (B <= 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0)
+        return fail(KDA_ERR_INVALID_ARG, "%s: bad sizes B=%d T=%d H=%d dk=%d dv=%d", fn, B, T, H,
+                    dk, dv);
+    if (dtype != KDA_F32 && dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, (int)dtype);
+    int N = B;
+    if (cu_seqlens) {
+        if (B != 1)
+            return fail(KDA_ERR_INVALID_ARG, "%s: varlen mode requires B == 1 (got %d)", fn, B);
+        if (num_seqs <= 0 || num_seqs > 65535)
+            return fail(KDA_ERR_INVALID_ARG, "%s: num_seqs=%d out of [1, 65535]", fn, num_seqs);
+        N = num_seqs;
+    } else if (B > 65535) {
+        return fail(KDA_ERR_INVALID_ARG, "%s: B=%d exceeds 65535", fn, B);
+    }
+    if (H > 65535) return fail(KDA_ERR_INVALID_ARG, "%s: H=%d exceeds 65535", fn, H);
+    const void *ptrs[] = {q, k, v, g, out, initial_state, final_state};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p))
+            return fail(KDA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", fn);
+    if (((uintptr_t)beta & 3u) || (cu_seqlens && ((uintptr_t)cu_seqlens & 3u)))
+        return fail(KDA_ERR_INVALID_ARG, "%s: beta and cu_seqlens must be 4-byte aligned", fn);
+    const long long total_T = (long long)B * T;
+    if (total_T > 0x7fffffffLL || total_T * H > (1LL << 40))
+        return fail(KDA_ERR_INVALID_ARG, "%s: problem too large (B*T=%lld)", fn, total_T);
+    *N_out = N;
+    return KDA_OK;
+}
+
+size_t bf16_prefill_scratch_bytes(int N, int B, int T, int H, bool varlen, long long *max_chunks) {
+    const long long total_T = (long long)B * T;
+    const long long mc = varlen ? (total_T + 63) / 64 + N : (long long)B * ((T + 63) / 64);
+    if (max_chunks) *max_chunks = mc;
+    const size_t coff_bytes = (((size_t)N + 1) * sizeof(int32_t) + 255) & ~(size_t)255;
+    return coff_bytes + (size_t)mc * H * ws::RECORD;
+}
+
+cudaError_t bf16_prefill_no_tokens(const float *initial_state, float *final_state, int N, int H,
+                                   cudaStream_t st) {
+    // nothing to process: final = initial (or zeros)
+    if (!final_state) return cudaSuccess;
+    const size_t bytes = (size_t)N * H * 128 * 128 * sizeof(float);
+    if (!initial_state) return cudaMemsetAsync(final_state, 0, bytes, st);
+    if (initial_state == final_state) return cudaSuccess;
+    return cudaMemcpyAsync(final_state, initial_state, bytes, cudaMemcpyDeviceToDevice, st);
+}
+
+cudaError_t launch_bf16_prefill(unsigned char *scratch, const void *q, const void *k,
+                                const void *v, const float *g, const float *beta,
+                                const float *initial_state, const int32_t *cu_seqlens, void *out,
+                                float *final_state, int B, int T, int H, int N, Prologue pro,
+                                int sms, cudaStream_t st) {
+    const long long total_T = (long long)B * T;
+    long long max_chunks = 0;
+    bf16_prefill_scratch_bytes(N, B, T, H, cu_seqlens != nullptr, &max_chunks);
+    const size_t coff_bytes = (((size_t)N + 1) * sizeof(int32_t) + 255) & ~(size_t)255;
+    int32_t *coff = (int32_t *)scratch;
+    unsigned char *records = scratch + coff_bytes;
+    const long long units = (long long)N * H;
+    const int dvt = units * 8 <= sms ? 16 : units * 4 <= sms ? 32 : 64;
+    cudaError_t e = cudaSuccess;
+    if (cu_seqlens) e = launch_chunk_plan(cu_seqlens, N, (int)total_T, coff, st);
+    if (e == cudaSuccess)
+        e = launch_chunk_prep(q, k, v, g, beta, cu_seqlens, coff, N, T, (int)total_T, H,
+                              (int)max_chunks, records, pro, error_word(), st);
+    if (e == cudaSuccess)
+        e = launch_chunk_chain(records, cu_seqlens, coff, initial_state, final_state, out, N, T,
+                               (int)total_T, H, dvt, (int)max_chunks, error_word(), st);
+    return e;
+}
+
+}  // namespace kda
+
 // Device-side part of kda_chunk_fwd (arguments already validated).
 static kda_status chunk_fwd_device(const void *q, const void *k, const void *v, const float *g,
                                    const float *beta, const float *initial_state,
@@ -322,20 +386,11 @@ static kda_status chunk_fwd_device(const void *q, const void *k, const void *v, 
         return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd(bf16): dk=%d dv=%d (supported: 128, 128)",
                     dk, dv);
     if (N == 0 || total_T == 0) {
-        // nothing to process: final = initial (or zeros)
-        if (final_state) {
-            const size_t bytes = (size_t)N * H * dk * dv * sizeof(float);
-            cudaError_t e = initial_state
-                ? (initial_state == final_state ? cudaSuccess
-                   : cudaMemcpyAsync(final_state, initial_state, bytes, cudaMemcpyDeviceToDevice, st))
-                : cudaMemsetAsync(final_state, 0, bytes, st);
-            if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd(bf16) empty input");
-        }
+        cudaError_t e = kda::bf16_prefill_no_tokens(initial_state, final_state, N, H, st);
+        if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd(bf16) empty input");
         return KDA_OK;
     }
-    const long long max_chunks = cu_seqlens ? (total_T + 63) / 64 + N : (long long)B * ((T + 63) / 64);
-    const size_t coff_bytes = (((size_t)N + 1) * sizeof(int32_t) + 255) & ~(size_t)255;
-    const size_t bytes = coff_bytes + (size_t)max_chunks * H * kda::ws::RECORD;
+    const size_t bytes = kda::bf16_prefill_scratch_bytes(N, B, T, H, cu_seqlens != nullptr, nullptr);
     cudaMemPool_t pool;
     int sms = 148;
     cudaError_t e = get_pool(&pool, &sms);
@@ -343,17 +398,8 @@ static kda_status chunk_fwd_device(const void *q, const void *k, const void *v, 
     void *scratch = nullptr;
     e = cudaMallocFromPoolAsync(&scratch, bytes, pool, st);
     if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd(bf16) scratch allocation");
-    int32_t *coff = (int32_t *)scratch;
-    unsigned char *records = (unsigned char *)scratch + coff_bytes;
-    const long long units = (long long)N * H;
-    const int dvt = units * 8 <= sms ? 16 : units * 4 <= sms ? 32 : 64;
-    if (cu_seqlens) e = kda::launch_chunk_plan(cu_seqlens, N, (int)total_T, coff, st);
-    if (e == cudaSuccess)
-        e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, coff, N, T, (int)total_T, H,
-                                   (int)max_chunks, records, pro, kda::error_word(), st);
-    if (e == cudaSuccess)
-        e = kda::launch_chunk_chain(records, cu_seqlens, coff, initial_state, final_state, out, N,
-                                    T, (int)total_T, H, dvt, (int)max_chunks, kda::error_word(), st);
+    e = kda::launch_bf16_prefill((unsigned char *)scratch, q, k, v, g, beta, initial_state,
+                                 cu_seqlens, out, final_state, B, T, H, N, pro, sms, st);
     cudaError_t e2 = cudaFreeAsync(scratch, st);
     if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd(bf16) launch");
     if (e2 != cudaSuccess) return cuda_fail(e2, "kda_chunk_fwd(bf16) scratch release");

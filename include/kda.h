@@ -376,8 +376,12 @@ kda_status kda_state_affine(const float *M, const float *B, const float *S_in,
  * breaks its accounting), and code on paths where an allocation call is not
  * permitted.  This entry point calls no cudaMalloc, cudaFree or other
  * allocating routine; its scratch is a fixed 32 MiB device array inside the
- * library (allocated once on every device that loads the library, kept until
- * the process exits).
+ * library, kept until the process exits.  The CUDA runtime reserves the array
+ * on a device when it loads the library's module there: at load time, or,
+ * under lazy module loading (CUDA_MODULE_LOADING=LAZY, the default since CUDA
+ * 12.2), at this entry point's first call on the device.  A caller that
+ * reserves its whole device budget up front should make one call (e.g. a
+ * small warm-up) before it does.
  *
  * Arguments, layouts and results are those of kda_chunk_fwd.  Supported:
  * KDA_BF16 with dk = dv = 128 only (other dtypes/dims: KDA_ERR_UNSUPPORTED).

@@ -2,24 +2,32 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {ours,reference}]
 
-One step = one kda_chunk_fwd over the prefill workload
-"prefill_t8192_h32_d128" (B=1, T=8192, H=32, dk=dv=128, bf16 q/k/v, fp32 g,
-beta, zero initial state, final state written).  `value` is whole-job
-prefill tokens/s (tokens of the packed T axis, all heads) with inputs resident
-in HBM; the inputs (404 MB) are larger than the 126 MB L2, so no flush is
-needed between steps.  A second leg times the decode step on
+One step = one kda_chunk_fwd over the headline prefill workload
+"varlen8_h32_d128_resume": 8 packed sequences (lengths drawn uniformly in
+[1024, 32768], 146,875 tokens), H=32, dk=dv=128, bf16 q/k/v, fp32 g and beta,
+a per-sequence fp32 initial state resumed and the 8 final states written.
+`value` is whole-job prefill tokens/s (tokens of the packed T axis, all heads)
+with inputs resident in HBM; the inputs (7.2 GB) are far larger than the
+126 MB L2, so no flush is needed between steps.  `e2e` is the same workload
+through the host-buffer entry point (kda_chunk_fwd_host) from pinned host
+memory, copies inside the timed region.
+
+Further legs: the dense prefill workloads "prefill_t8192_h32_d128" and
+"prefill_t65536_h32_d128" (each with its own roofline); the decode step on
 "decode_n256_h32_d128" (256 sequences x 32 heads, fp32 state 512 MiB in
-place) and is reported under "decode"; a third times serving decode
-(kda_recurrent_steps: 8 tokens per sequence per call, states in a 512-entry
-pool picked by slot) under "decode_steps".
+place); serving decode (kda_recurrent_steps: 8 tokens per call recurrent, 64
+tokens per call in the chunk form, states in a 512-entry pool picked by slot);
+the training backward (recurrent and chunked) on prefill_t8192_h32_d128.
 
 Under torchrun (N > 1) every rank runs the same workload on its own GPU
 (independent replicas: the hot path has no exchange step), timing is the max
 over ranks, and `value` sums all ranks' tokens ("scaling": "weak").
 
 --impl reference times the fp64 CPU oracle (tests' reference implementation)
-on the host cores, each step a bounded sample of the same workload (the first
-1024 tokens of all 32 heads), reported in the same metric and unit.
+on the host cores, each step a bounded sample of the headline workload (the
+first 256 tokens of each of its 8 sequences, all 32 heads), reported in the
+same metric and unit.  Under torchrun only rank 0 runs it, on the host's
+cores, so its value is one host's throughput whatever N is.
 """
 from __future__ import annotations
 
@@ -39,11 +47,31 @@ sys.path.insert(0, ROOT)
 
 METRIC = "KDA tokens/s (prefill chunk fwd, decode step) at 1 B200; % of roofline"
 UNIT = "tokens/s"
-WORKLOAD = "prefill_t8192_h32_d128"
-B, T, H, D = 1, 8192, 32, 128
-# algorithmic bytes (bf16 q,k,v,out + fp32 g + fp32 beta per token-head, plus
-# the final fp32 state written once per (sequence, head))
-PREFILL_BYTES = B * T * H * (3 * D * 2 + D * 4 + 4 + D * 2) + B * H * D * D * 4
+WORKLOAD = "varlen8_h32_d128_resume"      # the headline (largest single-GPU config)
+DENSE_LEGS = ("prefill_t8192_h32_d128", "prefill_t65536_h32_d128")
+H, D, C = 32, 128, 64
+# per token-head: bf16 q, k, v, out + fp32 g + fp32 beta
+TOKEN_BYTES = 3 * D * 2 + D * 4 + 4 + D * 2
+STATE_BYTES = D * D * 4
+# FLOPs per chunk-head of the chunk form, triangle-aware (2 per multiply-add):
+# A (strict lower) and P (lower) C x C x dk; T = (I + A)^-1 ~C^3/6; W, U with
+# the unit-lower T; W S, (q e^G) S and the state update C x dk x dv each;
+# P V_new lower C x C x dv
+CHUNK_FLOPS = 2 * (C * (C - 1) // 2 * D + C * (C + 1) // 2 * D + C ** 3 // 6
+                   + 2 * C * (C + 1) // 2 * D + 3 * C * D * D + C * (C + 1) // 2 * D)
+
+
+def prefill_bytes(tokens, nseq, initial_state):
+    """Algorithmic bytes of one prefill call: every token-head's inputs and
+    output once, the final states written, the initial states read if given."""
+    return tokens * H * TOKEN_BYTES + nseq * H * STATE_BYTES * (2 if initial_state else 1)
+
+
+def prefill_flops(lens):
+    """Chunk-form FLOPs of one call (partial chunks counted as whole ones)."""
+    return sum((n + C - 1) // C for n in lens) * H * CHUNK_FLOPS
+
+
 DEC_N, DEC_H = 256, 32
 
 
@@ -55,14 +83,18 @@ def decode_bytes(n):
 
 DECODE_BYTES = decode_bytes(DEC_N)
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
 # one ncu capture of each kernel on this workload (profiles/), valid only for
 # the kernel sources it was taken on: reported as null once they change.
 _SRC = os.path.join(ROOT, "gated_delta_rule_88_b200", "csrc")
+PREFILL_SRC = ["chunk_prep.cu", "prep_common.cuh", "chunk_chain_tc.cu", "chunk_ws.h", "sm100.cuh",
+               "common.cuh"]
 TRAFFIC = {
-    "prefill": {"files": ["chunk_prep.cu", "chunk_chain_tc.cu", "chunk_ws.h", "sm100.cuh", "common.cuh"],
-                "sha": "8b788aa77014ac59", "bytes": (336.785152 + 254.092800 + 304.155648 + 49.041920) * 1e6},
+    "prefill_t8192_h32_d128": {"files": PREFILL_SRC, "sha": "", "bytes": 0.0},
+    "prefill_t65536_h32_d128": {"files": PREFILL_SRC, "sha": "", "bytes": 0.0},
+    "varlen8_h32_d128_resume": {"files": PREFILL_SRC, "sha": "", "bytes": 0.0},
     "decode": {"files": ["decode.cu", "common.cuh"], "sha": "4ceac309c0c18d2f",
                "bytes": (547.408128 + 480.674560) * 1e6},
     "decode_steps": {"files": ["decode_pipe.cu", "common.cuh", "sm100.cuh"], "sha": "d9cf376f965488af",
@@ -76,7 +108,9 @@ TRAFFIC = {
 
 def measured_traffic(which):
     import hashlib
-    t = TRAFFIC[which]
+    t = TRAFFIC.get(which)
+    if not t or not t["sha"]:
+        return None
     m = hashlib.sha256()
     try:
         for f in t["files"]:
@@ -94,6 +128,17 @@ def measured_peak_hbm():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_peak_bf16():
+    """Dense bf16 tensor peak (TFLOP/s): the burst figure, for a kernel timed
+    on its own."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 class ClockSampler:
@@ -204,21 +249,97 @@ def job_value(units_per_rank: float, world: int, ms: float) -> float:
     return world * units_per_rank / (ms * 1e-3)
 
 
+def time_calls(fn, steps, warmup, stream, dist):
+    """Device time per call (ms, max over ranks) of `steps` calls after
+    `warmup` untimed ones, bracketed by barrier + synchronize."""
+    for _ in range(max(warmup, 0)):
+        fn()
+    barrier(dist)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    barrier(dist)
+    return max_over_ranks(e0.elapsed_time(e1), dist) / steps
+
+
+def prefill_roofline(name, inp, ms):
+    """Both sides of the prefill roofline for one call: the algorithmic bytes
+    at the measured HBM bandwidth and the chunk-form FLOPs at the measured
+    dense bf16 peak; the bound is the slower of the two."""
+    lens = seq_lens(inp)
+    nbytes = prefill_bytes(sum(lens), len(lens), inp.initial_state is not None)
+    flops = prefill_flops(lens)
+    hbm, hbm_kind = measured_peak_hbm()
+    tc, tc_kind = measured_peak_bf16()
+    t_hbm, t_tc = nbytes / (hbm * 1e9), flops / (tc * 1e12)
+    ach = nbytes / (ms * 1e-3) / 1e9
+    line = {"bound": "hbm" if t_hbm >= t_tc else "tensor",
+            "kernel": "kda_chunk_fwd (chunk_prep_tc_kernel + chunk_chain_tc_kernel"
+                      + (" + chunk_plan_kernel)" if inp.cu_seqlens is not None else ")"),
+            "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+            "peak_source": hbm_kind, "algorithmic_bytes_per_launch": nbytes,
+            "traffic": measured_traffic(name),
+            "tensor_side": {"flops_per_launch": flops, "achieved_tflops": flops / (ms * 1e-3) / 1e12,
+                            "peak_tflops": tc, "peak_source": tc_kind,
+                            "frac": flops / (ms * 1e-3) / 1e12 / tc,
+                            "t_hbm_us": t_hbm * 1e6, "t_tensor_us": t_tc * 1e6}}
+    return line
+
+
+def seq_lens(inp):
+    if inp.cu_seqlens is None:
+        return [inp.q.shape[1]] * inp.q.shape[0]
+    cu = inp.cu_seqlens.cpu().tolist()
+    return [cu[i + 1] - cu[i] for i in range(len(cu) - 1)]
+
+
+def prefill_call(kda, inp, out, sT):
+    return lambda: kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.initial_state,
+                                     inp.cu_seqlens, out, sT)
+
+
+def prefill_leg(kda, W, name, dev, dist, world, args):
+    """A dense prefill workload as a leg: device time per call and roofline."""
+    inp = W.named_prefill(name).to(dev)
+    Bq, Tq = inp.q.shape[:2]
+    out = torch.empty(Bq, Tq, H, D, dtype=torch.bfloat16, device=dev)
+    sT = torch.empty(inp.num_seqs, H, D, D, dtype=torch.float32, device=dev)
+    steps = max(3, min(args.steps, 20))
+    ms = time_calls(prefill_call(kda, inp, out, sT), steps, max(3, args.warmup),
+                    torch.cuda.current_stream(dev), dist)
+    assert kda.kda_get_device_error() == 0
+    tokens = Bq * Tq
+    gb = tokens * H * TOKEN_BYTES / 1e9
+    res = {"workload": name, "value": job_value(tokens, world, ms), "unit": UNIT, "ms_per_call": ms,
+           "calls": steps, "B": Bq, "T": Tq, "H": H, "dk": D, "dv": D,
+           "initial_state": "zeros (NULL)", "final_state": "written",
+           "l2": f"inputs ({gb:.2f} GB) larger than L2 (126 MB); no flush",
+           "roofline": prefill_roofline(name, inp, ms)}
+    del inp, out, sT
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     import gated_delta_rule_88_b200 as kda
     from gated_delta_rule_88_b200 import workloads as W
 
     rank, world, local, dist = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
-    inp_cpu = W.named_prefill(WORKLOAD)
-    inp = inp_cpu.to(dev)
-    out = torch.empty(B, T, H, D, dtype=torch.bfloat16, device=dev)
-    sT = torch.empty(B, H, D, D, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.g, inp.beta, None, None, out, sT)
+    # ---- the dense legs first, so their buffers are gone before the headline's ----
+    dense = {name: prefill_leg(kda, W, name, dev, dist, world, args) for name in DENSE_LEGS}
 
+    inp_cpu = W.named_prefill(WORKLOAD)
+    inp = inp_cpu.to(dev)
+    lens = seq_lens(inp_cpu)
+    tokens, nseq = sum(lens), len(lens)
+    out = torch.empty(1, tokens, H, D, dtype=torch.bfloat16, device=dev)
+    sT = torch.empty(nseq, H, D, D, dtype=torch.float32, device=dev)
+    step = prefill_call(kda, inp, out, sT)
     for _ in range(max(args.warmup, 0)):
         step()
     barrier(dist)
@@ -230,47 +351,41 @@ def run_ours(args):
             step()
         ev1.record(stream)
         barrier(dist)
-    ms_local = ev0.elapsed_time(ev1)
-    ms = max_over_ranks(ms_local, dist)
-    ms_step = ms / args.steps
+    ms_step = max_over_ranks(ev0.elapsed_time(ev1), dist) / args.steps
     assert kda.kda_get_device_error() == 0
-    value = job_value(B * T, world, ms_step)
-    peak, peak_kind = measured_peak_hbm()
-    achieved = PREFILL_BYTES / (ms_step * 1e-3) / 1e9
+    value = job_value(tokens, world, ms_step)
+    roof = prefill_roofline(WORKLOAD, inp, ms_step)
 
     # ---- end to end through the public API with host buffers ----
-    pin = {n: getattr(inp_cpu, n).pin_memory() for n in ("q", "k", "v", "g", "beta")}
-    out_h = torch.empty(B, T, H, D, dtype=torch.bfloat16).pin_memory()
-    sT_h = torch.empty(B, H, D, D, dtype=torch.float32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    pin = {n: getattr(inp_cpu, n).pin_memory() for n in ("q", "k", "v", "g", "beta", "initial_state")}
+    cu_h = inp_cpu.cu_seqlens.contiguous()
+    out_h = torch.empty(1, tokens, H, D, dtype=torch.bfloat16).pin_memory()
+    sT_h = torch.empty(nseq, H, D, D, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pin.values()) + cu_h.numel() * 4
     d2h = out_h.numel() * out_h.element_size() + sT_h.numel() * sT_h.element_size()
 
     def e2e_step():
         # the public host-buffer entry point: the copies of each token range
         # overlap the computation of the previous one
         kda.kda_chunk_fwd_host(pin["q"], pin["k"], pin["v"], pin["g"], pin["beta"],
+                               initial_state=pin["initial_state"], cu_seqlens=cu_h,
                                out=out_h, final_state=sT_h, device=dev)
 
-    for _ in range(2):
-        e2e_step()
-    barrier(dist)
-    e2e_steps = max(3, min(args.steps, 20))
-    ev0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    ev1.record(stream)
-    barrier(dist)
-    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), dist) / e2e_steps
+    e2e_ms = time_calls(e2e_step, max(3, min(args.steps, 10)), 2, stream, dist)
+    del inp, out, sT
+    torch.cuda.empty_cache()
 
-    # ---- decode leg (its timed region is sampled for clocks too) ----
+    # ---- decode and backward legs (their timed regions are sampled for clocks too) ----
     with ClockSampler(local) as clk_dec:
         dec = decode_leg(kda, W, dev, dist, world, args)
         dec_steps = decode_steps_leg(kda, W, dev, dist, world, args)
         dec_chunk = decode_steps_leg(kda, W, dev, dist, world, args, L=CHUNK_L,
                                      flags=kda.KDA_STEPS_CHUNK, kernel="decode_chunk_kernel",
                                      traffic_key="decode_chunk", ring=1)
-        bwd = backward_leg(kda, inp, dev, dist, world, args)
-        bwd_chunk = backward_leg(kda, inp, dev, dist, world, args, chunked=True)
+        bwd_inp = W.named_prefill(BWD_WORKLOAD).to(dev)
+        bwd = backward_leg(kda, bwd_inp, dev, dist, world, args)
+        bwd_chunk = backward_leg(kda, bwd_inp, dev, dist, world, args, chunked=True)
+        del bwd_inp
     clk.samples += clk_dec.samples
     clk.reasons |= clk_dec.reasons
 
@@ -279,20 +394,20 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "B": B, "T": T, "H": H, "dk": D, "dv": D, "chunk": 64,
-                   "initial_state": "zeros (NULL)", "final_state": "written",
-                   "l2": "inputs (404 MB) larger than L2 (126 MB); no flush",
+        "config": {"workload": WORKLOAD, "num_seqs": nseq, "seq_lens": lens, "T": tokens, "H": H,
+                   "dk": D, "dv": D, "chunk": C,
+                   "initial_state": "per sequence, 0.02 N(0,1), resumed",
+                   "final_state": "written (8 states)",
+                   "l2": f"inputs ({tokens * H * TOKEN_BYTES / 1e9:.2f} GB) larger than L2 (126 MB); no flush",
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
-        "roofline": {"bound": "hbm", "kernel": "kda_chunk_fwd (chunk_prep + chunk_chain)",
-                     "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "peak_source": peak_kind,
-                     "algorithmic_bytes_per_launch": PREFILL_BYTES,
-                     "traffic": measured_traffic("prefill")},
-        "e2e": {"value": job_value(B * T, world, e2e_ms), "unit": UNIT,
+        "roofline": roof,
+        "e2e": {"value": job_value(tokens, world, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms},
-        "gpu_launches": 2 * args.steps,
+                "ms_per_step": e2e_ms, "entry_point": "kda_chunk_fwd_host (pinned host buffers)"},
+        "gpu_launches": 3 * args.steps,
         "clocks": clk.summary(),
+        "prefill_t8192": dense["prefill_t8192_h32_d128"],
+        "prefill_t65536": dense["prefill_t65536_h32_d128"],
         "decode": dec,
         "decode_steps": dec_steps,
         "decode_chunk": dec_chunk,
@@ -397,39 +512,34 @@ def decode_steps_leg(kda, W, dev, dist, world, args, L=STEPS_L, flags=0,
                          "traffic": measured_traffic(traffic_key) if n == DEC_N else None}}
 
 
-# algorithmic bytes of one backward call on the prefill workload: q, k, v,
-# do (bf16) + g, beta (fp32) read; dq, dk, dg, dv (fp32) + dbeta written
-BWD_BYTES = B * T * H * (4 * D * 2 + D * 4 + 4 + 4 * D * 4 + 4)
+# the backward legs run on the 8192-token dense workload
+BWD_WORKLOAD = "prefill_t8192_h32_d128"
+BWD_T = 8192
+# algorithmic bytes of one backward call: q, k, v, do (bf16) + g, beta (fp32)
+# read; dq, dk, dg, dv (fp32) + dbeta written
+BWD_BYTES = BWD_T * H * (4 * D * 2 + D * 4 + 4 + 4 * D * 4 + 4)
 
 
 def backward_leg(kda, inp, dev, dist, world, args, chunked=False):
-    """Training backward on the prefill workload with a seeded output
+    """Training backward on the 8192-token workload with a seeded output
     gradient; no initial or final state.  chunked: kda_chunk_bwd (tensor
     cores), else kda_recurrent_bwd."""
     gen = torch.Generator().manual_seed(41)
-    do = torch.randn(B, T, H, D, generator=gen).to(torch.bfloat16).to(dev)
+    do = torch.randn(1, BWD_T, H, D, generator=gen).to(torch.bfloat16).to(dev)
     fn = kda.kda_chunk_bwd if chunked else kda.kda_recurrent_bwd
     run = lambda: fn(inp.q, inp.k, inp.v, inp.g, inp.beta, do, want_initial_state_grad=False)
-    for _ in range(max(1, min(args.warmup, 3))):
-        run()
-    barrier(dist)
-    calls = 3
-    s = torch.cuda.current_stream(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s)
-    for _ in range(calls):
-        run()
-    e1.record(s)
-    barrier(dist)
-    ms = max_over_ranks(e0.elapsed_time(e1), dist) / calls
+    calls = 3 if not chunked else 10
+    ms = time_calls(run, calls, max(1, min(args.warmup, 3)), torch.cuda.current_stream(dev), dist)
+    assert kda.kda_get_device_error() == 0
     peak, kind = measured_peak_hbm()
     ach = BWD_BYTES / (ms * 1e-3) / 1e9
     if chunked:
-        bound, kernel, traffic = "hbm", "kda_chunk_bwd (prep, chain, reverse chain, per-chunk pass)", None
+        bound, kernel = "hbm", "kda_chunk_bwd (prep, chain, reverse chain, per-chunk pass)"
+        traffic = measured_traffic("backward_chunk")
     else:
         bound, kernel = "latency (sequential per token)", "recurrent_bwd_kernel"
         traffic = measured_traffic("backward")
-    return {"workload": WORKLOAD + "_backward", "value": job_value(B * T, world, ms),
+    return {"workload": BWD_WORKLOAD + "_backward", "value": job_value(BWD_T, world, ms),
             "unit": UNIT, "ms_per_call": ms, "calls": calls,
             "roofline": {"bound": bound, "kernel": kernel,
                          "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
@@ -437,20 +547,42 @@ def backward_leg(kda, inp, dev, dist, world, args, chunked=False):
                          "traffic": traffic}}
 
 
-def cpu_baseline(inp_cpu, tokens=None):
-    """The fp64 oracle, as it stands, on the host cores."""
+def _oracle_sample(inp, per_seq):
+    """The first `per_seq` tokens of every sequence of a varlen workload, as a
+    packed varlen batch (host tensors)."""
+    cu = inp.cu_seqlens.tolist()
+    idx = torch.cat([torch.arange(cu[i], cu[i] + min(per_seq, cu[i + 1] - cu[i]))
+                     for i in range(len(cu) - 1)])
+    lens = [min(per_seq, cu[i + 1] - cu[i]) for i in range(len(cu) - 1)]
+    cu_s = torch.zeros(len(lens) + 1, dtype=torch.int32)
+    cu_s[1:] = torch.cumsum(torch.tensor(lens), 0).to(torch.int32)
+    pick = lambda x: x[:, idx].contiguous()
+    return (pick(inp.q), pick(inp.k), pick(inp.v), pick(inp.g), pick(inp.beta),
+            inp.initial_state.double(), cu_s, sum(lens))
+
+
+def cpu_baseline(inp_cpu, per_seq=2048, per_seq_1thread=128):
+    """The fp64 oracle, as it stands, on the host cores (all threads, and one
+    thread on a smaller sample)."""
     import oracle
     threads = os.cpu_count() or 1
-    n = T if tokens is None else tokens
-    sl = lambda x: x[:, :n].contiguous()
     oracle.build()
+    q, k, v, g, b, s0, cu, n = _oracle_sample(inp_cpu, per_seq)
     t0 = time.perf_counter()
-    oracle.forward(sl(inp_cpu.q), sl(inp_cpu.k), sl(inp_cpu.v), sl(inp_cpu.g), sl(inp_cpu.beta),
-                   None, None, threads=threads)
+    oracle.forward(q, k, v, g, b, s0, cu, threads=threads)
     dt = time.perf_counter() - t0
-    return {"value": B * n / dt, "unit": UNIT, "cores": min(threads, B * H), "kind": "oracle",
-            "sample": f"first {n} tokens of all {H} heads of {WORKLOAD} (fp64, token by token), "
-                      f"{dt:.2f} s wall"}
+    q, k, v, g, b, s0, cu, n1 = _oracle_sample(inp_cpu, per_seq_1thread)
+    t0 = time.perf_counter()
+    oracle.forward(q, k, v, g, b, s0, cu, threads=1)
+    dt1 = time.perf_counter() - t0
+    nseq = inp_cpu.num_seqs
+    return {"value": n / dt, "unit": UNIT, "cores": min(threads, nseq * H), "kind": "oracle",
+            "sample": f"first {per_seq} tokens of each of the {nseq} sequences of {WORKLOAD}, "
+                      f"all {H} heads, initial states resumed ({n} tokens, fp64, token by token), "
+                      f"{dt:.2f} s wall",
+            "one_thread": {"value": n1 / dt1, "unit": UNIT, "cores": 1,
+                           "sample": f"first {per_seq_1thread} tokens of each sequence, all {H} "
+                                     f"heads ({n1} tokens), {dt1:.2f} s wall"}}
 
 
 def run_reference(args):
@@ -462,26 +594,30 @@ def run_reference(args):
     import oracle
     oracle.build()
     inp = W.named_prefill(WORKLOAD)
-    n = 1024
-    sl = lambda x: x[:, :n].contiguous()
-    q, k, v, g, b = (sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.g), sl(inp.beta))
+    per_seq = 256
+    q, k, v, g, b, s0, cu, n = _oracle_sample(inp, per_seq)
     threads = os.cpu_count() or 1
     for _ in range(max(args.warmup, 0)):
-        oracle.forward(q, k, v, g, b, threads=threads)
+        oracle.forward(q, k, v, g, b, s0, cu, threads=threads)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.forward(q, k, v, g, b, threads=threads)
+        oracle.forward(q, k, v, g, b, s0, cu, threads=threads)
     dt = (time.perf_counter() - t0) / max(args.steps, 1)
-    value = B * n / dt
+    value = n / dt
+    nseq = inp.num_seqs
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "B": B, "T": T, "H": H, "dk": D, "dv": D,
+        "config": {"workload": WORKLOAD, "num_seqs": nseq, "H": H, "dk": D, "dv": D,
                    "sample_tokens_per_step": n},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(threads, H), "kind": "oracle",
-                         "sample": f"first {n} tokens of all {H} heads per step"},
+        # rank 0 alone works, on the host's cores: one host's figure at any N
+        "host": {"ranks_working": 1, "ranks_launched": world},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(threads, nseq * H),
+                         "kind": "oracle",
+                         "sample": f"first {per_seq} tokens of each of the {nseq} sequences, "
+                                   f"all {H} heads, per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

@@ -28,6 +28,8 @@ Entry points (same names as the C ABI):
                      (bf16, dk = dv = 128; tensor cores)
     kda_state_affine(M, B, S_in, out=None) -> S_out
     kda_get_device_error(stream=None) -> int
+    kda_selftest_bounded_wait(limit=1000): one CTA's bounded wait that always
+                     runs out (sets device error code 1; no fault)
 """
 from __future__ import annotations
 
@@ -41,7 +43,7 @@ __all__ = ["kda_chunk_fwd", "kda_chunk_fwd_ex", "kda_chunk_fwd_host", "kda_chunk
            "kda_recurrent_step",
            "kda_recurrent_step_ex", "kda_recurrent_steps", "kda_gated_rmsnorm", "kda_state_affine",
            "kda_recurrent_bwd", "kda_chunk_bwd",
-           "kda_get_device_error",
+           "kda_get_device_error", "kda_selftest_bounded_wait",
            "KDAError",
            "KDA_QK_L2NORM", "KDA_BETA_SIGMOID", "KDA_STEPS_CHUNK",
            "library_path", "load_library"]
@@ -100,6 +102,8 @@ def load_library():
         lib.kda_chunk_bwd.restype = i
         lib.kda_state_affine.restype = i
         lib.kda_get_device_error.argtypes = [vp, ctypes.POINTER(i)]
+        lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp]
+        lib.kda_selftest_bounded_wait.restype = i
         lib.kda_get_device_error.restype = i
         lib.kda_last_error_message.restype = ctypes.c_char_p
         lib.kda_status_string.restype = ctypes.c_char_p
@@ -471,3 +475,12 @@ def kda_get_device_error(stream=None) -> int:
     if rc not in (0, 4):
         _check(rc)
     return code.value
+
+
+def kda_selftest_bounded_wait(limit: int = 1000, device=None) -> None:
+    """Launch one CTA whose bounded mbarrier wait always runs out: it sets the
+    device error word to 1 (read it with kda_get_device_error) and returns."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _check(lib.kda_selftest_bounded_wait(int(limit), _stream_handle(dev)))

@@ -14,6 +14,9 @@
 
 namespace kda {
 
+// Detail of the calling thread's last failing call (kda_last_error_message).
+extern thread_local char t_msg[512];
+
 // Records the message for kda_last_error_message() and returns s.
 kda_status fail(kda_status s, const char *fmt, ...);
 

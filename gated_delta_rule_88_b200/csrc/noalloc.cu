@@ -28,10 +28,6 @@
 #include "api_internal.h"
 #include "common.cuh"
 
-namespace kda {
-extern thread_local char t_msg[512];
-}
-
 namespace {
 
 constexpr size_t kStaticScratchBytes = 32u << 20;   // 32 MiB

@@ -405,6 +405,20 @@ kda_status kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
                                  int B, int T, int H, int dk, int dv, int num_seqs,
                                  kda_dtype dtype, void *stream);
 
+/*
+ * kda_selftest_bounded_wait -- a diagnostic for the library's failure path.
+ * The paper has no counterpart.
+ *
+ * Every kernel here that waits on an mbarrier polls it at most a bounded
+ * number of times; when the bound runs out it sets the device error word to 1
+ * (a wait timed out) and returns instead of hanging or trapping.  This call
+ * launches one CTA that waits, polling at most `limit` times, on an mbarrier
+ * nothing arrives on (no copy or MMA in flight), so it always times out: the
+ * next kda_get_device_error() on the device reports code 1 and clears it, and
+ * the context stays usable.  limit: 1 .. 65536 (else KDA_ERR_INVALID_ARG).
+ */
+kda_status kda_selftest_bounded_wait(unsigned limit, void *stream);
+
 /* Static string for a status code. */
 const char *kda_status_string(kda_status s);
 

@@ -74,7 +74,9 @@ def test_reference_arm_prints_on_rank0_only():
                 "vs_baseline", "dtype", "data", "config"):
         assert key in line, key
     assert line["steps"] == 1 and line["warmup"] == 0 and line["higher_is_better"] is True
-    assert "workload" in line["config"]
+    assert line["config"]["workload"] == "varlen8_h32_d128_resume"
+    # rank 0 alone works: the value is one host's throughput, not scaled by N
+    assert line["host"] == {"ranks_working": 1, "ranks_launched": 2}
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == line["value"]
     e2e = line["e2e"]

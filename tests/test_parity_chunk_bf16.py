@@ -132,19 +132,29 @@ def test_prefill_t8192_h32_full():
           f"S rel {rel_inf(sT, s_ref):.2e}")
 
 
-def test_prefill_t65536_h32_sampled_heads():
-    """The T = 65536, H = 32 long-memory workload; four heads, full length."""
+def _margins(name, o, sT, o_ref, s_ref):
+    msg = (f"{name}: o rel-inf {rel_inf(o, o_ref):.2e} rms {rms_rel(o, o_ref):.2e}; "
+           f"S rel-inf {rel_inf(sT, s_ref):.2e} rms {rms_rel(sT, s_ref):.2e}")
+    print(msg)
+    return msg
+
+
+def test_prefill_t65536_h32_all_heads():
+    """The T = 65536, H = 32 long-memory workload, every head against the
+    oracle over the full length."""
     inp = W.named_prefill("prefill_t65536_h32_d128")
-    _check(inp, heads=[0, 9, 22, 31])
+    o, sT, o_ref, s_ref = _check(inp)
+    _margins("prefill_t65536_h32_d128", o, sT, o_ref, s_ref)
 
 
-def test_varlen8_resume_sampled_heads():
-    """8 packed sequences, lengths U[1024, 32768], per-sequence initial states.
-    Each sequence is also split at a non-multiple of 64 and resumed; the
-    resumed run must match the unsplit one and the oracle."""
+def test_varlen8_resume_all_heads():
+    """8 packed sequences, lengths U[1024, 32768], per-sequence initial states,
+    every head of every sequence against the oracle.  Each sequence is also
+    split at a non-multiple of 64 and resumed; the resumed run must match the
+    oracle too."""
     inp = W.named_prefill("varlen8_h32_d128_resume")
-    heads = [0, 13, 31]
-    o, sT, o_ref, s_ref = _check(inp, heads=heads)
+    o, sT, o_ref, s_ref = _check(inp)
+    _margins("varlen8_h32_d128_resume", o, sT, o_ref, s_ref)
     d = inp.to(DEV)
     cu = inp.cu_seqlens.tolist()
     for n in range(8):
@@ -155,6 +165,5 @@ def test_varlen8_resume_sampled_heads():
                               sl(d.beta, s, cut), d.initial_state[n:n + 1].contiguous())
         ob, sb = kda_chunk_fwd(sl(d.q, cut, e), sl(d.k, cut, e), sl(d.v, cut, e), sl(d.g, cut, e),
                                sl(d.beta, cut, e), sa)
-        # o_ref / s_ref are already restricted to `heads`
-        assert_close(sb[0][heads], s_ref[n], BF, f"resumed state {n}")
-        assert_close(ob[:, :, heads], o_ref[:, cut:e], BF, f"resumed o {n}")
+        assert_close(sb[0], s_ref[n], BF, f"resumed state {n}")
+        assert_close(ob, o_ref[:, cut:e], BF, f"resumed o {n}")

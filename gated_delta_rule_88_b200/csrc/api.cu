@@ -372,19 +372,17 @@ static kda_status chunk_fwd_device(const void *q, const void *k, const void *v, 
                                    int B, int T, int H, int dk, int dv, int N, kda_dtype dtype,
                                    kda::Prologue pro, cudaStream_t st) {
     const long long total_T = (long long)B * T;
-    if (dtype == KDA_F32) {
-        if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128)))
-            return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd(f32): dk=%d dv=%d (supported: 64, 128)",
-                        dk, dv);
-        cudaError_t e = kda::launch_chunk_f32(
-            (const float *)q, (const float *)k, (const float *)v, g, beta, initial_state,
-            cu_seqlens, (float *)out, final_state, N, T, (int)total_T, H, dk, dv, pro, st);
-        if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd(f32) launch");
+    if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128)))
+        return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd: dk=%d dv=%d (supported: 64, 128)", dk, dv);
+    if (dtype == KDA_F32 || dk != 128 || dv != 128) {
+        // fp32 arithmetic on the CUDA cores: fp32 inputs, and bf16 inputs at
+        // head dimensions the tensor-core kernels do not take
+        cudaError_t e = kda::launch_chunk_f32(q, k, v, g, beta, initial_state, cu_seqlens, out,
+                                              final_state, N, T, (int)total_T, H, dk, dv,
+                                              dtype == KDA_BF16, pro, st);
+        if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd(simt) launch");
         return KDA_OK;
     }
-    if (dk != 128 || dv != 128)
-        return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd(bf16): dk=%d dv=%d (supported: 128, 128)",
-                    dk, dv);
     if (N == 0 || total_T == 0) {
         cudaError_t e = kda::bf16_prefill_no_tokens(initial_state, final_state, N, H, st);
         if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd(bf16) empty input");
@@ -626,10 +624,9 @@ extern "C" kda_status kda_chunk_fwd_host(const void *q, const void *k, const voi
                     T, H, dk, dv, range_tokens);
     if (dtype != KDA_F32 && dtype != KDA_BF16)
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: unknown dtype %d", (int)dtype);
-    if (dtype == KDA_BF16 ? (dk != 128 || dv != 128)
-                          : !((dk == 64 || dk == 128) && (dv == 64 || dv == 128)))
-        return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd_host: dk=%d dv=%d not supported for %s",
-                    dk, dv, dtype == KDA_BF16 ? "bf16" : "f32");
+    if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128)))
+        return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd_host: dk=%d dv=%d (supported: 64, 128)",
+                    dk, dv);
     const long long total_T = (long long)B * T;
     if (total_T > 0x7fffffffLL || total_T * H > (1LL << 40))
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: problem too large (B*T=%lld)", total_T);

@@ -1,7 +1,10 @@
 // chunk_f32.cu -- exact-fp32 chunkwise KDA prefill (SIMT, no tensor cores).
 //
 // Serves fp32 inputs, where the tolerance is an absolute 1e-3 and bf16
-// tensor-core operands would not do.  It is the chunkwise form of the Kimi
+// tensor-core operands would not do, and bf16 inputs at head dimensions the
+// tensor-core kernels do not take (dk or dv = 64): the bf16 values are
+// widened on load, every step is fp32, and the output is rounded to nearest
+// even on store.  It is the chunkwise form of the Kimi
 // Linear paper notes, section 3: within a chunk of C = 64 tokens the old
 // state's contribution goes through the chunk's transitions and the
 // intra-chunk writes are gathered by a WY-like transform.  With G the
@@ -50,12 +53,13 @@ struct F32Smem {
     float GC[DK];           // G_C, the cumsum at the chunk's last row
 };
 
-template <int DK>
+// TI: the type of q, k, v and out (float or __nv_bfloat16)
+template <int DK, typename TI>
 __global__ void __launch_bounds__(NT)
-chunk_f32_kernel(const float *__restrict__ q, const float *__restrict__ k,
-                 const float *__restrict__ v, const float *__restrict__ g,
+chunk_f32_kernel(const TI *__restrict__ q, const TI *__restrict__ k,
+                 const TI *__restrict__ v, const float *__restrict__ g,
                  const float *__restrict__ beta, const float *__restrict__ s0,
-                 const int32_t *__restrict__ cu, float *__restrict__ out,
+                 const int32_t *__restrict__ cu, TI *__restrict__ out,
                  float *__restrict__ sT, int T, int total_T, int H, int dv, Prologue pro)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -94,13 +98,13 @@ chunk_f32_kernel(const float *__restrict__ q, const float *__restrict__ k,
             float qv = 0.f, kv = 0.f, gv = 0.f;
             if (r < len) {
                 const size_t off = ((size_t)(t0 + r) * H + h) * DK + c;
-                qv = q[off]; kv = k[off]; gv = g[off];
+                qv = to_f(q[off]); kv = to_f(k[off]); gv = g[off];
             }
             sm.Qs[r * LD + c] = qv; sm.Ks[r * LD + c] = kv; sm.Gs[r * LD + c] = gv;
         }
         for (int i = tid; i < CH * DVT; i += NT) {
             const int r = i / DVT, n = i % DVT;
-            sm.Vs[i] = (r < len) ? v[((size_t)(t0 + r) * H + h) * dv + n0 + n] : 0.f;
+            sm.Vs[i] = (r < len) ? to_f(v[((size_t)(t0 + r) * H + h) * dv + n0 + n]) : 0.f;
         }
         if (tid < CH) {
             float bt = (tid < len) ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
@@ -212,7 +216,7 @@ chunk_f32_kernel(const float *__restrict__ q, const float *__restrict__ k,
             for (int i = tid / DVT; i < len; i += NT / DVT) {
                 float acc = sm.Am[i * LDA + n];
                 for (int j = 0; j <= i; ++j) acc += sm.Pm[i * LDA + j] * sm.Vs[j * DVT + n];
-                out[((size_t)(t0 + i) * H + h) * dv + n0 + n] = acc;
+                out[((size_t)(t0 + i) * H + h) * dv + n0 + n] = from_f<TI>(acc);
             }
             for (int c = tid / DVT; c < DK; c += NT / DVT) {
                 float acc = sm.eGC[c] * sm.Ss[c * DVT + n];
@@ -230,33 +234,46 @@ chunk_f32_kernel(const float *__restrict__ q, const float *__restrict__ k,
     }
 }
 
-template <int DK>
-cudaError_t launch_chunk_f32_t(const float *q, const float *k, const float *v, const float *g,
+template <int DK, typename TI>
+cudaError_t launch_chunk_f32_t(const TI *q, const TI *k, const TI *v, const float *g,
                                const float *beta, const float *s0, const int32_t *cu,
-                               float *out, float *sT, int N, int T, int total_T, int H,
+                               TI *out, float *sT, int N, int T, int total_T, int H,
                                int dv, Prologue pro, cudaStream_t st)
 {
     const size_t smem = sizeof(F32Smem<DK>);
-    cudaError_t e = cudaFuncSetAttribute(chunk_f32_kernel<DK>,
+    cudaError_t e = cudaFuncSetAttribute(chunk_f32_kernel<DK, TI>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(dv / DVT, H, N);
-    chunk_f32_kernel<DK><<<grid, NT, smem, st>>>(q, k, v, g, beta, s0, cu, out, sT, T,
-                                                 total_T, H, dv, pro);
+    chunk_f32_kernel<DK, TI><<<grid, NT, smem, st>>>(q, k, v, g, beta, s0, cu, out, sT, T,
+                                                     total_T, H, dv, pro);
     return cudaGetLastError();
+}
+
+template <typename TI>
+cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, const float *s0, const int32_t *cu, void *out,
+                              float *sT, int N, int T, int total_T, int H, int dk, int dv,
+                              Prologue pro, cudaStream_t st)
+{
+    if (dv % DVT != 0) return cudaErrorInvalidValue;
+    const TI *q_ = (const TI *)q, *k_ = (const TI *)k, *v_ = (const TI *)v;
+    if (dk == 64)
+        return launch_chunk_f32_t<64, TI>(q_, k_, v_, g, beta, s0, cu, (TI *)out, sT, N, T, total_T, H, dv, pro, st);
+    if (dk == 128)
+        return launch_chunk_f32_t<128, TI>(q_, k_, v_, g, beta, s0, cu, (TI *)out, sT, N, T, total_T, H, dv, pro, st);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_chunk_f32(const float *q, const float *k, const float *v, const float *g,
+cudaError_t launch_chunk_f32(const void *q, const void *k, const void *v, const float *g,
                              const float *beta, const float *s0, const int32_t *cu,
-                             float *out, float *sT, int N, int T, int total_T, int H,
-                             int dk, int dv, Prologue pro, cudaStream_t st)
+                             void *out, float *sT, int N, int T, int total_T, int H,
+                             int dk, int dv, bool bf16, Prologue pro, cudaStream_t st)
 {
-    if (dv % DVT != 0) return cudaErrorInvalidValue;
-    if (dk == 64) return launch_chunk_f32_t<64>(q, k, v, g, beta, s0, cu, out, sT, N, T, total_T, H, dv, pro, st);
-    if (dk == 128) return launch_chunk_f32_t<128>(q, k, v, g, beta, s0, cu, out, sT, N, T, total_T, H, dv, pro, st);
-    return cudaErrorInvalidValue;
+    return bf16 ? launch_chunk_simt<__nv_bfloat16>(q, k, v, g, beta, s0, cu, out, sT, N, T, total_T, H, dk, dv, pro, st)
+                : launch_chunk_simt<float>(q, k, v, g, beta, s0, cu, out, sT, N, T, total_T, H, dk, dv, pro, st);
 }
 
 }  // namespace kda

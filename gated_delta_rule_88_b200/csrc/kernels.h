@@ -70,10 +70,10 @@ cudaError_t launch_state_affine(const float *M, const float *B, const float *S, 
 // Token axis flattened: token t of the packed [B*T] axis, head h, channel c at
 // ((t * H) + h) * d + c.  Sequences: dense (cu == nullptr, n-th spans
 // [n*T, n*T+T)) or varlen (cu[n], cu[n+1]).
-cudaError_t launch_chunk_f32(const float *q, const float *k, const float *v, const float *g,
+cudaError_t launch_chunk_f32(const void *q, const void *k, const void *v, const float *g,
                              const float *beta, const float *s0, const int32_t *cu,
-                             float *out, float *sT, int N, int T, int total_T, int H,
-                             int dk, int dv, Prologue pro, cudaStream_t st);
+                             void *out, float *sT, int N, int T, int total_T, int H,
+                             int dk, int dv, bool bf16, Prologue pro, cudaStream_t st);
 
 // bf16 tensor-core prefill (dk = dv = 128) in two launches over a scratch
 // buffer of per-(chunk, head) records (chunk_ws.h):

@@ -101,7 +101,7 @@ def test_chunk_bad_arguments_rejected(lib, kw):
     assert chunk(lib, **kw) == 1
 
 
-@pytest.mark.parametrize("kw", [dict(dk=96, dv=96), dict(dk=128, dv=64), dict(dk=64, dv=64),
+@pytest.mark.parametrize("kw", [dict(dk=96, dv=96), dict(dk=32, dv=64), dict(dk=128, dv=256),
                                 dict(dtype=0, dk=32, dv=64), dict(dtype=0, dk=128, dv=256)])
 def test_chunk_unsupported_rejected(lib, kw):
     assert chunk(lib, **kw) == 2
@@ -215,7 +215,7 @@ def test_host_bad_varlen_offsets_rejected(lib, kw):
     assert host(lib, **kw) == 1
 
 
-@pytest.mark.parametrize("kw", [dict(dk=64, dv=64), dict(dtype=0, dk=32, dv=64)])
+@pytest.mark.parametrize("kw", [dict(dk=96, dv=96), dict(dtype=0, dk=32, dv=64)])
 def test_host_unsupported_rejected(lib, kw):
     assert host(lib, **kw) == 2
 

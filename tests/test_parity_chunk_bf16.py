@@ -167,3 +167,31 @@ def test_varlen8_resume_all_heads():
                                sl(d.beta, cut, e), sa)
         assert_close(sb[0], s_ref[n], BF, f"resumed state {n}")
         assert_close(ob, o_ref[:, cut:e], BF, f"resumed o {n}")
+
+
+# ---- bf16 inputs at head dimension 64 (fp32 arithmetic on the CUDA cores) ----
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64)])
+def test_head_dim_64_ragged(T, dk, dv):
+    _check(W.prefill(2, T, 3, dk, dv, BF, seed=700 + T + dk + dv, initial_state_std=0.02))
+
+
+def test_head_dim_64_varlen_and_resume():
+    """Varlen with an empty and a one-token sequence, then each sequence split
+    at a non-multiple of 64 and resumed from its checkpoint."""
+    inp = W.prefill(1, 0, 4, 64, 64, BF, seed=710, initial_state_std=0.05,
+                    seq_lens=[300, 0, 1, 129])
+    o, sT, o_ref, s_ref = _check(inp)
+    d = inp.to(DEV)
+    cu = inp.cu_seqlens.tolist()
+    for n in (0, 3):
+        s, e = cu[n], cu[n + 1]
+        cut = s + 77
+        sl = lambda x, a, b: x[:, a:b].contiguous()
+        _, sa = kda_chunk_fwd(sl(d.q, s, cut), sl(d.k, s, cut), sl(d.v, s, cut), sl(d.g, s, cut),
+                              sl(d.beta, s, cut), d.initial_state[n:n + 1].contiguous())
+        ob, sb = kda_chunk_fwd(sl(d.q, cut, e), sl(d.k, cut, e), sl(d.v, cut, e), sl(d.g, cut, e),
+                               sl(d.beta, cut, e), sa)
+        assert_close(sb[0], s_ref[n], BF, f"resumed state {n}")
+        assert_close(ob, o_ref[:, cut:e], BF, f"resumed o {n}")

@@ -321,12 +321,14 @@ kda_status check_chunk_fwd_args(const char *fn, const void *q, const void *k, co
     return KDA_OK;
 }
 
+// chunk offsets coff[N + 1], then (varlen) the sequence order[N], 256-byte rounded
+static size_t plan_bytes(int N) { return (((size_t)2 * N + 1) * sizeof(int32_t) + 255) & ~(size_t)255; }
+
 size_t bf16_prefill_scratch_bytes(int N, int B, int T, int H, bool varlen, long long *max_chunks) {
     const long long total_T = (long long)B * T;
     const long long mc = varlen ? (total_T + 63) / 64 + N : (long long)B * ((T + 63) / 64);
     if (max_chunks) *max_chunks = mc;
-    const size_t coff_bytes = (((size_t)N + 1) * sizeof(int32_t) + 255) & ~(size_t)255;
-    return coff_bytes + (size_t)mc * H * ws::RECORD;
+    return plan_bytes(N) + (size_t)mc * H * ws::RECORD;
 }
 
 cudaError_t bf16_prefill_no_tokens(const float *initial_state, float *final_state, int N, int H,
@@ -339,6 +341,12 @@ cudaError_t bf16_prefill_no_tokens(const float *initial_state, float *final_stat
     return cudaMemcpyAsync(final_state, initial_state, bytes, cudaMemcpyDeviceToDevice, st);
 }
 
+int bf16_prefill_dvt(long long units, int sms) {
+    // the widest state tile that still gives every SM a chain: one CTA per
+    // (sequence, head) once there are more of those than half the SMs
+    return units * 8 <= sms ? 16 : units * 4 <= sms ? 32 : units * 2 <= sms ? 64 : 128;
+}
+
 cudaError_t launch_bf16_prefill(unsigned char *scratch, const void *q, const void *k,
                                 const void *v, const float *g, const float *beta,
                                 const float *initial_state, const int32_t *cu_seqlens, void *out,
@@ -347,19 +355,19 @@ cudaError_t launch_bf16_prefill(unsigned char *scratch, const void *q, const voi
     const long long total_T = (long long)B * T;
     long long max_chunks = 0;
     bf16_prefill_scratch_bytes(N, B, T, H, cu_seqlens != nullptr, &max_chunks);
-    const size_t coff_bytes = (((size_t)N + 1) * sizeof(int32_t) + 255) & ~(size_t)255;
     int32_t *coff = (int32_t *)scratch;
-    unsigned char *records = scratch + coff_bytes;
-    const long long units = (long long)N * H;
-    const int dvt = units * 8 <= sms ? 16 : units * 4 <= sms ? 32 : 64;
+    int32_t *order = cu_seqlens ? coff + N + 1 : nullptr;
+    unsigned char *records = scratch + plan_bytes(N);
+    const int dvt = bf16_prefill_dvt((long long)N * H, sms);
     cudaError_t e = cudaSuccess;
-    if (cu_seqlens) e = launch_chunk_plan(cu_seqlens, N, (int)total_T, coff, st);
+    if (cu_seqlens) e = launch_chunk_plan(cu_seqlens, N, (int)total_T, coff, st, order);
     if (e == cudaSuccess)
         e = launch_chunk_prep(q, k, v, g, beta, cu_seqlens, coff, N, T, (int)total_T, H,
                               (int)max_chunks, records, pro, error_word(), st);
     if (e == cudaSuccess)
         e = launch_chunk_chain(records, cu_seqlens, coff, initial_state, final_state, out, N, T,
-                               (int)total_T, H, dvt, (int)max_chunks, error_word(), st);
+                               (int)total_T, H, dvt, (int)max_chunks, error_word(), st, nullptr,
+                               nullptr, order);
     return e;
 }
 

@@ -29,10 +29,15 @@ kda_status check_chunk_fwd_args(const char *fn, const void *q, const void *k, co
                                 const float *final_state, int B, int T, int H, int dk, int dv,
                                 int num_seqs, kda_dtype dtype, int *N_out);
 
-// Scratch bytes of the bf16 (dk = dv = 128) prefill: 256-byte-rounded chunk
-// offsets, then one record per (chunk slot, head).  *max_chunks (nullable)
+// Scratch bytes of the bf16 (dk = dv = 128) prefill: the chunk offsets and
+// the sequence order (256-byte rounded), then one record per (chunk slot,
+// head).  *max_chunks (nullable)
 // receives the chunk slots.
 size_t bf16_prefill_scratch_bytes(int N, int B, int T, int H, bool varlen, long long *max_chunks);
+
+// State-tile width (dv columns per chain CTA) for `units` (sequence, head)
+// pairs on `sms` SMs.
+int bf16_prefill_dvt(long long units, int sms);
 
 // The bf16 prefill with no tokens: final = initial, or zeros.
 cudaError_t bf16_prefill_no_tokens(const float *initial_state, float *final_state, int N, int H,

@@ -59,15 +59,26 @@ struct TcLayout {
     // TMEM columns: D1 double-buffered (2 x DVT) + D3 (DVT), rounded to a power of 2
     static constexpr uint32_t NCOLS = 3 * DVT <= 32 ? 32 : 3 * DVT <= 64 ? 64 : 3 * DVT <= 128 ? 128
                                     : 3 * DVT <= 256 ? 256 : 512;
-    // B operands S and V_new: MN-major, one swizzle atom wide (rows of DVT
-    // bf16 = 32, 64 or 128 bytes), 8-row groups contiguous
-    static constexpr uint32_t BW = DVT * 2;
+    // B operands S and V_new: MN-major, swizzled to the tile width (rows of
+    // DVT bf16 = 32, 64 or 128 bytes; at DVT = 128 two 64-column atoms of
+    // 128-byte rows, the second B1_ATOM / B2_ATOM bytes after the first),
+    // 8-row groups contiguous
+    static constexpr int NATOM = DVT > 64 ? DVT / 64 : 1;
+    static constexpr uint32_t BW = DVT > 64 ? 128 : DVT * 2;
     static constexpr uint32_t B_SBO = 8 * BW;
-    static constexpr uint32_t B_LAYOUT = DVT == 64 ? 2 : DVT == 32 ? 4 : 6;   // 128 / 64 / 32-byte swizzle
-    static constexpr int B_SWZ = DVT == 64 ? 7 : DVT == 32 ? 3 : 1;
-    // byte offset of the 16-byte chunk `chunk` (8 columns) of K row k
+    static constexpr uint32_t B1_ATOM = 128 * BW;                  // K = 128 channel rows
+    static constexpr uint32_t B2_ATOM = 64 * BW;                   // K = 64 token rows
+    static constexpr uint32_t B1_LBO = NATOM > 1 ? B1_ATOM : B_SBO;
+    static constexpr uint32_t B2_LBO = NATOM > 1 ? B2_ATOM : B_SBO;
+    static constexpr uint32_t B_LAYOUT = DVT >= 64 ? 2 : DVT == 32 ? 4 : 6;   // 128 / 64 / 32-byte swizzle
+    static constexpr int B_SWZ = DVT >= 64 ? 7 : DVT == 32 ? 3 : 1;
+    // byte offset of the 16-byte chunk `chunk` (8 columns) of K row k, in an
+    // operand whose 64-column atoms are ATOM bytes apart
+    template <uint32_t ATOM>
     static __device__ __forceinline__ uint32_t b_off(int k, int chunk) {
-        return (k >> 3) * B_SBO + (k & 7) * BW + ((chunk ^ ((((k & 7) * BW) >> 7) & B_SWZ)) << 4);
+        const uint32_t a = NATOM > 1 ? (uint32_t)(chunk >> 3) * ATOM : 0u;
+        const int j = NATOM > 1 ? (chunk & 7) : chunk;
+        return a + (k >> 3) * B_SBO + (k & 7) * BW + ((j ^ ((((k & 7) * BW) >> 7) & B_SWZ)) << 4);
     }
 };
 
@@ -77,7 +88,8 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
                       const int32_t *__restrict__ coff, const float *__restrict__ s0,
                       float *__restrict__ sT, __nv_bfloat16 *__restrict__ out, int T, int total_T,
                       int H, int cps, int max_chunks, int *__restrict__ err,
-                      unsigned char *__restrict__ s_img, unsigned char *__restrict__ v_img)
+                      unsigned char *__restrict__ s_img, unsigned char *__restrict__ v_img,
+                      const int32_t *__restrict__ order)
 {
     using L = TcLayout<DVT, NS>;
     extern __shared__ unsigned char smem_raw[];
@@ -96,7 +108,10 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
     unsigned char *B2 = sm + L::B2_OFF;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n0 = blockIdx.x * DVT, h = blockIdx.y, seq = blockIdx.z;
+    // varlen: sequences longest first (order from chunk_plan_kernel), so the
+    // longest chains start in the first wave
+    const int n0 = blockIdx.x * DVT, h = blockIdx.y;
+    const int seq = order ? order[blockIdx.z] : blockIdx.z;
 
     long long bos, eos;
     int c_begin;
@@ -170,9 +185,9 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
         // to the ring base; B operands: MN-major, swizzled to the tile width
         const uint32_t sm_a = smem_u32(sm);
         const DescParts a_sw = smem_desc_parts(sm_a, 16, 1024, 2);
-        const DescParts b1_d = smem_desc_parts(smem_u32(B1), L::B_SBO, L::B_SBO, L::B_LAYOUT);
-        const DescParts b2_d0 = smem_desc_parts(smem_u32(B2), L::B_SBO, L::B_SBO, L::B_LAYOUT);
-        const DescParts b2_d1 = smem_desc_parts(smem_u32(B2 + L::B2_BYTES), L::B_SBO, L::B_SBO, L::B_LAYOUT);
+        const DescParts b1_d = smem_desc_parts(smem_u32(B1), L::B1_LBO, L::B_SBO, L::B_LAYOUT);
+        const DescParts b2_d0 = smem_desc_parts(smem_u32(B2), L::B2_LBO, L::B_SBO, L::B_LAYOUT);
+        const DescParts b2_d1 = smem_desc_parts(smem_u32(B2 + L::B2_BYTES), L::B2_LBO, L::B_SBO, L::B_LAYOUT);
         constexpr uint32_t BK = (2 * L::B_SBO) >> 4;       // descriptor step per 16 K rows
         bool issued_any = false;
         if (warp == EPI + 1) for (int i = 0; i < nchunks; ++i) {
@@ -266,7 +281,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
             for (int ng = 0; ng < CPT / 8; ++ng) {
                 uint4 pk = make_uint4(pack_bf16(S[8 * ng], S[8 * ng + 1]), pack_bf16(S[8 * ng + 2], S[8 * ng + 3]),
                                       pack_bf16(S[8 * ng + 4], S[8 * ng + 5]), pack_bf16(S[8 * ng + 6], S[8 * ng + 7]));
-                *reinterpret_cast<uint4 *>(B1 + L::b_off(t, cb / 8 + ng)) = pk;
+                *reinterpret_cast<uint4 *>(B1 + L::template b_off<L::B1_ATOM>(t, cb / 8 + ng)) = pk;
                 if (img) {
                     const int n = n0 + cb + 8 * ng;
                     *reinterpret_cast<uint4 *>(img + (size_t)(n >> 6) * 16384 + ws::sw128(t, n & 63)) = pk;
@@ -345,7 +360,8 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
                         const __nv_bfloat162 u2 = *reinterpret_cast<const __nv_bfloat162 *>(&u[4 * ng + e]);
                         pk[e] = pack_bf16(__low2float(u2) - x[8 * ng + 2 * e], __high2float(u2) - x[8 * ng + 2 * e + 1]);
                     }
-                    *reinterpret_cast<uint4 *>(B2 + p * L::B2_BYTES + L::b_off(t, cb / 8 + ng)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4 *>(B2 + p * L::B2_BYTES + L::template b_off<L::B2_ATOM>(t, cb / 8 + ng)) =
+                        make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     if (v_img) {
                         // the backward's V_new image [C][dv], K-major SW128
                         const int n = n0 + cb + 8 * ng;
@@ -392,7 +408,7 @@ template <int DVT, int NS>
 cudaError_t launch_tc(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
                       const float *s0, float *sT, void *out, int N, int T, int total_T, int H,
                       int max_chunks, int *err, cudaStream_t st, unsigned char *s_img,
-                      unsigned char *v_img)
+                      unsigned char *v_img, const int32_t *order)
 {
     using L = TcLayout<DVT, NS>;
     const size_t smem = L::BYTES + 1024;
@@ -402,7 +418,7 @@ cudaError_t launch_tc(const unsigned char *wsp, const int32_t *cu, const int32_t
     dim3 grid(D / DVT, H, N);
     chunk_chain_tc_kernel<DVT, NS><<<grid, L::NTHREADS, smem, st>>>(
         wsp, cu, coff, s0, sT, (__nv_bfloat16 *)out, T, total_T, H, (T + C - 1) / C, max_chunks, err,
-        s_img, v_img);
+        s_img, v_img, order);
     return cudaGetLastError();
 }
 
@@ -411,12 +427,14 @@ cudaError_t launch_tc(const unsigned char *wsp, const int32_t *cu, const int32_t
 cudaError_t launch_chunk_chain(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
                                   const float *s0, float *sT, void *out, int N, int T,
                                   int total_T, int H, int dvt, int max_chunks, int *err,
-                                  cudaStream_t st, unsigned char *s_img, unsigned char *v_img)
+                                  cudaStream_t st, unsigned char *s_img, unsigned char *v_img,
+                                  const int32_t *order)
 {
     switch (dvt) {
-        case 16: return launch_tc<16, 3>(wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st, s_img, v_img);
-        case 32: return launch_tc<32, 3>(wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st, s_img, v_img);
-        case 64: return launch_tc<64, 2>(wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st, s_img, v_img);
+        case 16: return launch_tc<16, 3>(wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st, s_img, v_img, order);
+        case 32: return launch_tc<32, 3>(wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st, s_img, v_img, order);
+        case 64: return launch_tc<64, 2>(wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st, s_img, v_img, order);
+        case 128: return launch_tc<128, 2>(wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st, s_img, v_img, order);
     }
     return cudaErrorInvalidValue;
 }

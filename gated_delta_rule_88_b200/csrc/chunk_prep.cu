@@ -896,7 +896,7 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 
 // Chunk offsets per sequence for varlen mode: coff[n] = sum_{m<n} ceil(len_m / C).
 __global__ void chunk_plan_kernel(const int32_t *__restrict__ cu, int N, int total_T,
-                                  int32_t *__restrict__ coff)
+                                  int32_t *__restrict__ coff, int32_t *__restrict__ order)
 {
     __shared__ int part[1024];
     const int tid = threadIdx.x;
@@ -922,6 +922,26 @@ __global__ void chunk_plan_kernel(const int32_t *__restrict__ cu, int N, int tot
         run += e > b ? (e - b + C - 1) / C : 0;
     }
     if (tid == 1023) coff[N] = part[1023];
+    if (order) {
+        // rank of each sequence by decreasing length, ties by index (a
+        // permutation); quadratic, so only for up to 4096 sequences
+        for (int n = tid; n < N; n += 1024) {
+            int rank = n;
+            if (N <= 4096) {
+                auto len = [&](int m) {
+                    const int b = min(max(cu[m], 0), total_T), e = min(max(cu[m + 1], 0), total_T);
+                    return e > b ? e - b : 0;
+                };
+                const int ln = len(n);
+                rank = 0;
+                for (int m = 0; m < N; ++m) {
+                    const int lm = len(m);
+                    rank += (lm > ln || (lm == ln && m < n)) ? 1 : 0;
+                }
+            }
+            order[rank] = n;
+        }
+    }
 }
 
 }  // namespace
@@ -929,9 +949,9 @@ __global__ void chunk_plan_kernel(const int32_t *__restrict__ cu, int N, int tot
 size_t chunk_prep_smem_bytes() { return tcp::BYTES + 1024; }
 
 cudaError_t launch_chunk_plan(const int32_t *cu, int N, int total_T, int32_t *coff,
-                              cudaStream_t st)
+                              cudaStream_t st, int32_t *order)
 {
-    chunk_plan_kernel<<<1, 1024, 0, st>>>(cu, N, total_T, coff);
+    chunk_plan_kernel<<<1, 1024, 0, st>>>(cu, N, total_T, coff, order);
     return cudaGetLastError();
 }
 

@@ -83,8 +83,10 @@ cudaError_t launch_chunk_f32(const void *q, const void *k, const void *v, const 
 //   chunk_chain sequential over chunks per (sequence, head, dv tile),
 //               tcgen05 MMAs with TMEM accumulators (chunk_chain_tc.cu)
 size_t chunk_prep_smem_bytes();
+// order (nullable): also the sequences sorted by decreasing length (ties by
+// index; the identity order when N > 4096)
 cudaError_t launch_chunk_plan(const int32_t *cu, int N, int total_T, int32_t *coff,
-                              cudaStream_t st);
+                              cudaStream_t st, int32_t *order = nullptr);
 cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const int32_t *cu, const int32_t *coff,
                               int N, int T, int total_T, int H, int max_chunks,
@@ -94,7 +96,8 @@ cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const
 cudaError_t launch_chunk_chain(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
                                const float *s0, float *sT, void *out, int N, int T, int total_T,
                                int H, int dvt, int max_chunks, int *err, cudaStream_t st,
-                               unsigned char *s_img = nullptr, unsigned char *v_img = nullptr);
+                               unsigned char *s_img = nullptr, unsigned char *v_img = nullptr,
+                               const int32_t *order = nullptr);
 
 // Chunked backward (bf16, dk = dv = 128): the reverse chain over the forward
 // records (gradient images dS' 32 KiB and dV_new 16 KiB per (chunk, head)),

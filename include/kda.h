@@ -387,7 +387,7 @@ kda_status kda_state_affine(const float *M, const float *B, const float *S_in,
  * KDA_BF16 with dk = dv = 128 only (other dtypes/dims: KDA_ERR_UNSUPPORTED).
  * Size limit: it returns KDA_ERR_INVALID_ARG, with the needed and the
  * available byte counts in kda_last_error_message(), when
- *     roundup256(4 * (N + 1)) + slots * H * 74240 > 32 MiB,
+ *     roundup256(4 * (2 N + 1)) + slots * H * 74240 > 32 MiB,
  * where slots = B * ceil(T / 64) in dense mode and ceil(T / 64) + num_seqs in
  * varlen mode (e.g. 451 (chunk, head) slots: T = 1024 with H <= 28).
  * First call on a device: it looks up the array's device address there

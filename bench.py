@@ -330,6 +330,23 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
 
+    if args.only_prefill:
+        # profiling: just the prefill calls of one workload (no legs, no e2e)
+        inp = W.named_prefill(args.only_prefill).to(dev)
+        lens = seq_lens(inp)
+        out = torch.empty(*inp.q.shape[:3], D, dtype=torch.bfloat16, device=dev)
+        sT = torch.empty(len(lens), H, D, D, dtype=torch.float32, device=dev)
+        ms = time_calls(prefill_call(kda, inp, out, sT), args.steps, args.warmup, stream, dist)
+        assert kda.kda_get_device_error() == 0
+        if rank == 0:
+            print(json.dumps({"workload": args.only_prefill, "ms_per_call": ms,
+                              "value": job_value(sum(lens), world, ms), "unit": UNIT,
+                              "roofline": prefill_roofline(args.only_prefill, inp, ms)}), flush=True)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
     # ---- the dense legs first, so their buffers are gone before the headline's ----
     dense = {name: prefill_leg(kda, W, name, dev, dist, world, args) for name in DENSE_LEGS}
 
@@ -633,6 +650,9 @@ def main():
     ap.add_argument("--decode-n", type=int, default=DEC_N,
                     help="sequences in the decode legs (a smaller case for profiling)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--only-prefill", metavar="WORKLOAD", default=None,
+                    help="profiling: time only kda_chunk_fwd on this named workload "
+                         "(e.g. varlen8_h32_d128_resume) and print its line")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

@@ -476,9 +476,10 @@ __device__ __noinline__ void prep_subchunk(
 //   MMA-U   [* ; T] (128 x 64) x beta V     (64 x 128)        -> cols 128-255, lanes 64-127
 // The rows marked * are whatever lies next to T in shared memory; their
 // products land in TMEM lanes that are never read.  T itself comes from
-// form_T_padded_diag (fp32).  Record parts leave by bulk async stores of
-// their shared-memory images (W and U, the last, by a coalesced copy of all
-// threads so that the CTA need not wait for a bulk copy to read them).
+// form_T_padded_diag (fp32).  K^T leaves from the registers of the forms
+// pass; q e^G and P by bulk async stores of their shared-memory images; W
+// and U, the last, by a coalesced copy of all threads so that the CTA need
+// not wait for a bulk copy to read them.
 // ---------------------------------------------------------------------------
 namespace tcp {
 // Tiles are K-major with the 128-byte swizzle (rows of 64 bf16 = 128 bytes,
@@ -489,7 +490,7 @@ namespace tcp {
 constexpr int OFF_KQ = 0;              // per 64-channel block b at b * 16384:
                                        //   [k -> beta k e^G : 64 rows][q -> q e^G : 64 rows]
 constexpr int OFF_KI = 32768;          // k e^{-G} (block b at b * 8192); then A (fp32 64 x 64)
-constexpr int OFF_Z = 49152;           // K^T image; then the padded diagonal blocks; then form_T scratch
+constexpr int OFF_Z = 49152;           // the padded diagonal blocks of A; then form_T scratch
 constexpr int OFF_G = OFF_KI;          // g (fp32 [64][128], TMA) until the cumsum has read it
 constexpr int OFF_V = 65536;           // v -> beta v (block b at b * 8192)
 constexpr int OFF_TB = 81920;          // P image, then T (bf16, 64 swizzled rows)
@@ -700,12 +701,13 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             }
         }
         // K e^{G_C - G} transposed (channel rows, 64 tokens, 128-byte swizzle)
-        // into its record image
+        // straight into the record: each 16-byte piece is half a sector, the
+        // other half follows from the same thread
 #pragma unroll
         for (int e = 0; e < 2; ++e)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh)
-                *reinterpret_cast<uint4 *>(sm + tcp::OFF_Z + ws::sw128(c0 + e, 16 * I + 8 * hh)) =
+                *reinterpret_cast<uint4 *>(rec + ws::OFF_KTT + ws::sw128(c0 + e, 16 * I + 8 * hh)) =
                     make_uint4(kt[e][4 * hh], kt[e][4 * hh + 1], kt[e][4 * hh + 2], kt[e][4 * hh + 3]);
     }
     fence_proxy_async_smem();
@@ -724,19 +726,15 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             umma_bf16_p(tmem, da.lo + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), da.hi,
                         db.lo + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), db.hi, ID_AP, kk > 0);
         umma_commit(bar);
-        // record parts that are final now: K^T (its image) and q e^G (the
-        // swizzled q e^G tile is already the record's layout for rows 64-127)
-        bulk_s2g(rec + ws::OFF_KTT, sm + tcp::OFF_Z, 16384);
+        // the record part that is final now: q e^G (the swizzled q e^G tile
+        // is already the record's layout for rows 64-127; nothing overwrites
+        // it before form_T waits for the reads)
         bulk_s2g(rec + ws::OFF_AW + 8192, sm + tcp::OFF_KQ + 8192, 8192);
         bulk_s2g(rec + ws::OFF_AW + 16384 + 8192, sm + tcp::OFF_KQ + 16384 + 8192, 8192);
         bulk_commit();
     }
-    // one thread waits for the MMA (and for the K^T image to be read); the
-    // others sleep at the barrier
-    if (tid == 0) {
-        ok = mbar_wait(bar, 0);
-        bulk_wait_read();
-    }
+    // one thread waits for the MMA; the others sleep at the barrier
+    if (tid == 0) ok = mbar_wait(bar, 0);
     ok = __syncthreads_and(ok);
     tc_fence_after();
 

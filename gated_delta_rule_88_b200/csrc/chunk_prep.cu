@@ -212,10 +212,70 @@ __device__ __forceinline__ void form_T(const float *Am, float *Tm, float *Zs, in
     __syncthreads();
 }
 
+// Diagonal 16x16 blocks of A (fp32, fsw layout over Am) and of P (bf16, into
+// the record) for a chunk whose decay inside a sub-chunk is so strong that
+// the factorised form e^{G_i - G_j} = a_i (1 / a_j) leaves the fp32 range:
+// every factor is formed directly as e^{G_i - G_j} = exp(sum of g over tokens
+// j+1 .. i) <= 1 (for g <= 0), from q, k and g read again from global memory.
+// Warp w takes the (block, column) tasks w, w + 8, ...; lane l the channels
+// 4l .. 4l + 3.  Called by all 256 threads.
+template <bool PRO>
+__device__ __forceinline__ void ap_diag_direct(
+    float *Am, unsigned char *rec, const float *sbeta, const float *srq, const float *srk,
+    const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+    const float *__restrict__ g, size_t base, size_t row_stride, int len)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int c = 4 * lane;
+    auto ld4 = [&](const __nv_bfloat16 *p, int r) {
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < len) {
+            const uint2 w = *reinterpret_cast<const uint2 *>(p + base + (size_t)r * row_stride + c);
+            const float2 lo = bf16x2_to_float2(w.x), hi = bf16x2_to_float2(w.y);
+            x = make_float4(lo.x, lo.y, hi.x, hi.y);
+        }
+        return x;
+    };
+    for (int task = warp; task < 64; task += NT / 32) {
+        const int I = task >> 4, jj = task & 15, j = 16 * I + jj;
+        float4 kj = ld4(k, j);
+        if (PRO) { const float f = srk[j]; kj.x *= f; kj.y *= f; kj.z *= f; kj.w *= f; }
+        float4 sg = make_float4(0.f, 0.f, 0.f, 0.f);      // sum of g over tokens j+1 .. i
+        for (int ii = jj; ii < 16; ++ii) {
+            const int i = 16 * I + ii;
+            if (ii > jj && i < len) {
+                const float4 gi = *reinterpret_cast<const float4 *>(g + base + (size_t)i * row_stride + c);
+                sg.x += gi.x; sg.y += gi.y; sg.z += gi.z; sg.w += gi.w;
+            }
+            float4 qi = ld4(q, i), ki = ld4(k, i);
+            if (PRO) {
+                const float fq = srq[i], fk = srk[i];
+                qi.x *= fq; qi.y *= fq; qi.z *= fq; qi.w *= fq;
+                ki.x *= fk; ki.y *= fk; ki.z *= fk; ki.w *= fk;
+            }
+            const float4 e = make_float4(expf(sg.x), expf(sg.y), expf(sg.z), expf(sg.w));
+            const float4 ke = make_float4(kj.x * e.x, kj.y * e.y, kj.z * e.z, kj.w * e.w);
+            float a = ki.x * ke.x + ki.y * ke.y + ki.z * ke.z + ki.w * ke.w;
+            float pp = qi.x * ke.x + qi.y * ke.y + qi.z * ke.z + qi.w * ke.w;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                a += __shfl_xor_sync(0xffffffffu, a, o);
+                pp += __shfl_xor_sync(0xffffffffu, pp, o);
+            }
+            if (lane == 0) {
+                Am[fsw(i, j)] = ii > jj ? sbeta[i] * a : 0.f;
+                *reinterpret_cast<__nv_bfloat16 *>(rec + ws::OFF_P + ws::sw128(i, j)) = __float2bfloat16_rn(pp);
+            }
+        }
+    }
+}
+
 // The record of one (chunk, head) with every exponent referenced inside its
-// 16-token sub-chunk (any per-token g >= -5).  The tensor-core prep below
-// calls this for the chunks whose decay over the chunk leaves its exponent
-// range.  Called by all 256 threads of the CTA; smem_raw holds a PrepSmem.
+// 16-token sub-chunk.  The tensor-core prep below calls this for the chunks
+// whose decay over the chunk leaves its exponent range.  Any g <= 0 is taken:
+// when a sub-chunk's own decay underflows the factor a_j (1 / a_j would
+// overflow), its diagonal blocks of A and P are formed directly
+// (ap_diag_direct).  Called by all 256 threads of the CTA; smem_raw holds a PrepSmem.
 template <bool PRO>
 __device__ __noinline__ void prep_subchunk(
     unsigned char *smem_raw, const __nv_bfloat16 *__restrict__ q,
@@ -255,6 +315,7 @@ __device__ __noinline__ void prep_subchunk(
     // ---- elementwise ownership: sub-chunk I, channels c0, c0 + 1 ----
     const int I = tid >> 6, c0 = 2 * (tid & 63);
     float2 a[16], b[16];
+    bool tiny_a;
     {
         float2 al[16];
 #pragma unroll
@@ -267,6 +328,7 @@ __device__ __noinline__ void prep_subchunk(
         float2 run = make_float2(1.f, 1.f);
 #pragma unroll
         for (int i = 0; i < 16; ++i) { run.x *= al[i].x; run.y *= al[i].y; a[i] = run; }
+        tiny_a = !(run.x >= 0x1p-60f && run.y >= 0x1p-60f);   // a is smallest at the block end
         run = make_float2(1.f, 1.f);
 #pragma unroll
         for (int i = 15; i >= 0; --i) { b[i] = run; run.x *= al[i].x; run.y *= al[i].y; }
@@ -392,7 +454,12 @@ __device__ __noinline__ void prep_subchunk(
         case 2: ap_block<2>(sm, rec, warp >= 4, lane); break;
         default: ap_block<3>(sm, rec, warp >= 4, lane); break;
     }
-    __syncthreads();
+    // a sub-chunk decay below 2^-60 makes 1 / a_j unusable: diagonal blocks directly
+    if (__syncthreads_or(tiny_a)) {
+        ap_diag_direct<PRO>(reinterpret_cast<float *>(sm.Xq), rec, sm.beta, sm.rq, sm.rk, q, k, g,
+                            base, row_stride, len);
+        __syncthreads();
+    }
 
     // ---- T = (I + A)^-1 in fp32 ----
     const float *Am = reinterpret_cast<const float *>(sm.Xq);

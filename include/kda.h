@@ -106,11 +106,13 @@ enum { KDA_STEPS_CHUNK = 4 };
  * Supported: dtype KDA_BF16 with dk = dv = 128 (tensor-core path), and
  *   KDA_F32 with dk, dv in {64, 128} (exact fp32 path).  Others return
  *   KDA_ERR_UNSUPPORTED.
- * Numerical range (bf16 path): per-token g >= -5 keeps every exponent the
- *   chunk form takes within fp32 range.  A chunk whose decay over its 64
- *   tokens stays within e^{+-80} references its exponents at the chunk start
- *   (the fast path); any other chunk references them per 16-token sub-chunk,
- *   inside the same call, with the same result up to rounding.
+ * Numerical range (bf16 path): any finite per-token g <= 0, and g <= 5 for
+ *   positive gates.  A chunk whose decay over its 64 tokens stays within
+ *   e^{+-80} references its exponents at the chunk start (the fast path);
+ *   any other chunk references them per 16-token sub-chunk, inside the same
+ *   call, and a sub-chunk whose own decay falls below 2^-60 has its diagonal
+ *   blocks formed from e^{G_i - G_j} directly; the result is the same up to
+ *   rounding.
  * Aliasing: out must not overlap any input.
  * Memory: the bf16 path takes a stream-ordered scratch buffer from a
  *   library-private pool on the current device (cudaMallocFromPoolAsync on
@@ -242,12 +244,16 @@ kda_status kda_recurrent_step_ex(const void *q, const void *k, const void *v,
  * KDA_STEPS_CHUNK in flags selects, for dtype KDA_BF16 with dk = dv = 128,
  * L >= 2 and no prologue flags (q_scale = 1), the chunk form of the same L
  * steps (section 3 of the notes: a WY-like representation of the block's
- * writes, then one product with the state) in blocks of 16 tokens on tensor
- * cores: the operands of the state products (state, V_new, T, P and the
- * decayed k, q) are rounded to bf16 as in kda_chunk_fwd, the state stays
- * fp32.  It needs e^{16 g} finite in fp32 for positive g (any g <= 5; gates
- * are normally <= 0).  Other combinations run the recurrent kernel, which is
- * bitwise equal to L calls of kda_recurrent_step.
+ * writes, then one product with the state) on tensor cores: the operands of
+ * the state products (state, V_new, T, P and the decayed k, q) are rounded
+ * to bf16 as in kda_chunk_fwd, the state stays fp32.  For L <= 32 it runs in
+ * blocks of 16 tokens in one kernel that allocates nothing; from L = 33 on
+ * it runs kda_chunk_fwd's kernels over the N sequences of L tokens with each
+ * state resumed from and written back to its pool entry, and takes their
+ * scratch (N * ceil(L / 64) * H * 74,240 bytes) from the library-private
+ * stream-ordered pool, as kda_chunk_fwd does.  Any finite g <= 0, and
+ * g <= 5 for positive gates.  Other combinations run the recurrent kernel,
+ * which is bitwise equal to L calls of kda_recurrent_step.
  */
 kda_status kda_recurrent_steps(const void *q, const void *k, const void *v,
                                const float *g, const float *beta,

@@ -57,6 +57,37 @@ def test_strongest_supported_decay():
     _check(inp)
 
 
+@pytest.mark.parametrize("g_strong", [-6.0, -20.0, -90.0])
+def test_any_decay_below_the_factorised_range(g_strong):
+    """per-token g far below -5 on some channels and heads (down to a decay of
+    e^-90 per token): the sub-chunk factor 1 / a_j would overflow, so those
+    sub-chunks' diagonal blocks of A and P are formed from e^{G_i - G_j}
+    directly; mixed with ordinary chunks in one call"""
+    inp = W.prefill(1, 333, 3, 128, 128, BF, seed=44, initial_state_std=0.02)
+    inp.g[:, :, 0, ::4] = g_strong          # every chunk of head 0
+    inp.g[:, 100:180, 2, 1::3] = g_strong   # a span of head 2 (chunks 1 and 2)
+    o, sT, _, _ = _check(inp)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(sT).all()
+
+
+def test_any_decay_prologue_path():
+    """the same with the in-kernel prologue (the fallback re-reads q and k
+    and applies the L2-norm factors itself)"""
+    from gated_delta_rule_88_b200 import kda_chunk_fwd_ex, KDA_QK_L2NORM
+    inp = W.prefill(1, 150, 2, 128, 128, BF, seed=45, initial_state_std=0.02)
+    inp.g[:, :, 1, ::2] = -30.0
+    raw_q = (inp.q.float() * 3.0).to(BF)     # not normalised: the prologue does it
+    d = inp.to(DEV)
+    o, sT = kda_chunk_fwd_ex(raw_q.to(DEV), d.k, d.v, d.g, d.beta, d.initial_state,
+                             flags=KDA_QK_L2NORM, q_scale=1.0 / 128 ** 0.5)
+    torch.cuda.synchronize()
+    assert kda_get_device_error() == 0
+    qn, kn, _ = oracle.prologue(raw_q, inp.k, inp.beta, qk_l2norm=True, q_scale=1.0 / 128 ** 0.5)
+    o_ref, s_ref = oracle.forward(qn, kn, inp.v, inp.g, inp.beta, inp.initial_state)
+    assert_close(o, o_ref, BF, "o (prologue, strong decay)")
+    assert_close(sT[0], s_ref[0], BF, "state (prologue, strong decay)")
+
+
 @pytest.mark.parametrize("g_floor", [-1.2, -1.3, -2.0])
 def test_mixed_exponent_ranges(g_floor):
     """Chunks whose decay over the chunk stays within e^80 use one exponent

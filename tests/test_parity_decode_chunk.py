@@ -6,8 +6,9 @@ writes in a WY-like representation and touches the state with one product;
 the result is the recurrence's.  Tolerance: the bf16 bound of the other
 parity tests (the state-product operands are bf16, as in the prefill).
 Lengths cover one partial block (2, 8), a full block (16), a block plus one
-token (17) and several blocks (40, 64); gates cover the decode workload's
-and a stronger, channel-dependent decay.
+token (17) and several blocks (40, 64, 100: from 33 tokens on the call runs
+the prefill's kernels on the pool); gates cover the decode workload's and a
+stronger, channel-dependent decay.
 """
 import pytest
 import torch
@@ -43,7 +44,7 @@ def _run(N, L, H, pool_n, seed, gate="softplus8", slots=True):
     return pool0, pool, idx, out, o_ref, s_ref, (q, k, v, g, b), sl
 
 
-@pytest.mark.parametrize("L", [2, 8, 16, 17, 40, 64])
+@pytest.mark.parametrize("L", [2, 8, 16, 17, 32, 33, 40, 64, 100])
 def test_chunk_steps_vs_oracle(L):
     pool0, pool, idx, out, o_ref, s_ref, _, _ = _run(N=5, L=L, H=3, pool_n=9, seed=90 + L)
     assert_close(out, o_ref, BF, "o")
@@ -63,10 +64,12 @@ def test_chunk_steps_gates(gate):
         assert_close(pool[idx[n]], s_ref[n], BF, f"state {n} ({gate})")
 
 
-def test_chunk_steps_strong_decay():
-    """g far below the prefill's range (-20 per token on every channel):
-    the block forms use e^{G_i - G_j} <= 1 directly, so nothing overflows."""
-    N, L, H, d = 3, 20, 2, 128
+@pytest.mark.parametrize("L", [20, 70])
+def test_chunk_steps_strong_decay(L):
+    """g = -20 per token on every channel: the block forms use e^{G_i - G_j}
+    <= 1 directly (16-token blocks at L = 20; the prefill kernels' direct
+    diagonal blocks at L = 70), so nothing overflows."""
+    N, H, d = 3, 2, 128
     q, k, v, g, b = _tokens(N, L, H, d, seed=98)
     g = torch.full_like(g, -20.0)
     pool0 = W.decode_initial_state(N, H, d, d, seed=98, std=0.02)
@@ -117,3 +120,25 @@ def test_chunk_flag_falls_back_where_unsupported():
     o2 = kda_recurrent_steps(q, k, v, g, b, p2)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(p1, p2)
+
+
+def test_chunk_steps_bad_slot_reported_and_skipped_long():
+    """From 33 tokens on (the prefill kernels on the pool): a slot outside the
+    pool skips its sequence (no output, no pool entry written) and reports
+    device error code 3; the other sequences are computed."""
+    N, L, H, d, S = 4, 40, 2, 128, 6
+    q, k, v, g, b = [t.to(DEV) for t in _tokens(N, L, H, d, seed=26)]
+    pool0 = W.decode_initial_state(S, H, d, d, seed=26)
+    pool = pool0.to(DEV)
+    slots = torch.tensor([2, -1, 5, 6], dtype=torch.int32, device=DEV)   # -1 and 6 are invalid
+    out = torch.full((N, L, H, d), 7.0, dtype=BF, device=DEV)
+    kda_recurrent_steps(q, k, v, g, b, pool, slots, out=out, flags=KDA_STEPS_CHUNK)
+    assert kda_get_device_error() == 3
+    assert torch.all(out[1] == 7.0) and torch.all(out[3] == 7.0)
+    ok = torch.tensor([0, 2])
+    o_ref, s_ref = oracle.forward(q.cpu()[ok], k.cpu()[ok], v.cpu()[ok], g.cpu()[ok], b.cpu()[ok],
+                                  initial_state=pool0[[2, 5]].double())
+    assert_close(out[ok.to(DEV)], o_ref, BF, "o of the valid sequences")
+    assert_close(pool[[2, 5]], s_ref, BF, "their pool entries")
+    keep = [0, 1, 3, 4]
+    assert torch.equal(pool.cpu()[keep], pool0[keep])

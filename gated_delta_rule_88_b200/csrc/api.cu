@@ -65,11 +65,6 @@ kda_status cuda_fail(cudaError_t e, const char *what) {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-// kda_recurrent_steps in the chunk form: from this many tokens per call on,
-// the prefill's two kernels (64-token chunks, records in scratch) beat the
-// 16-token-block decode kernel
-constexpr int kStepsViaPrefillMinL = 33;
-
 // Library-private stream-ordered memory pool per device.  Its release
 // threshold is unbounded, so scratch freed at the end of a call stays
 // reserved for the next one instead of returning to the driver.
@@ -240,26 +235,6 @@ kda_status kda_recurrent_steps(const void *q, const void *k, const void *v, cons
     if (NH == 0) return KDA_OK;
     const bool tc = chunk && L >= 2 && dtype == KDA_BF16 && dk == 128 && dv == 128 &&
                     pro.flags == 0 && pro.q_scale == 1.f;
-    if (tc && L >= kStepsViaPrefillMinL) {
-        // longer blocks: the prefill's kernels on [N, L] as N sequences of L
-        // tokens, each state resumed from and written back to its pool entry
-        cudaStream_t st = (cudaStream_t)stream;
-        cudaMemPool_t pool;
-        int sms = 148;
-        cudaError_t e = get_pool(&pool, &sms);
-        if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_steps memory pool");
-        const size_t bytes = kda::bf16_prefill_scratch_bytes(N, N, L, H, false, nullptr);
-        void *scratch = nullptr;
-        e = cudaMallocFromPoolAsync(&scratch, bytes, pool, st);
-        if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_steps scratch allocation");
-        e = kda::launch_bf16_prefill((unsigned char *)scratch, q, k, v, g, beta, state_pool, nullptr,
-                                     out, state_pool, N, L, H, N, pro, sms, st,
-                                     slots ? slots : nullptr, slots ? num_slots : N);
-        cudaError_t e2 = cudaFreeAsync(scratch, st);
-        if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_steps launch");
-        if (e2 != cudaSuccess) return cuda_fail(e2, "kda_recurrent_steps scratch release");
-        return KDA_OK;
-    }
     cudaError_t e = tc ? kda::launch_decode_chunk(q, k, v, g, beta, state_pool, slots, num_slots,
                                                   out, N, H, L, kda::error_word(), (cudaStream_t)stream)
                        : kda::launch_decode_pipe(q, k, v, g, beta, state_pool, slots, num_slots, out,
@@ -376,7 +351,7 @@ cudaError_t launch_bf16_prefill(unsigned char *scratch, const void *q, const voi
                                 const void *v, const float *g, const float *beta,
                                 const float *initial_state, const int32_t *cu_seqlens, void *out,
                                 float *final_state, int B, int T, int H, int N, Prologue pro,
-                                int sms, cudaStream_t st, const int32_t *slots, int num_slots) {
+                                int sms, cudaStream_t st) {
     const long long total_T = (long long)B * T;
     long long max_chunks = 0;
     bf16_prefill_scratch_bytes(N, B, T, H, cu_seqlens != nullptr, &max_chunks);
@@ -392,7 +367,7 @@ cudaError_t launch_bf16_prefill(unsigned char *scratch, const void *q, const voi
     if (e == cudaSuccess)
         e = launch_chunk_chain(records, cu_seqlens, coff, initial_state, final_state, out, N, T,
                                (int)total_T, H, dvt, (int)max_chunks, error_word(), st, nullptr,
-                               nullptr, order, slots, num_slots);
+                               nullptr, order);
     return e;
 }
 

@@ -44,13 +44,11 @@ cudaError_t bf16_prefill_no_tokens(const float *initial_state, float *final_stat
                                    cudaStream_t st);
 
 // The bf16 prefill's launches (plan if varlen, prep, chain) on `scratch` of
-// bf16_prefill_scratch_bytes() bytes.  slots (nullable): sequence n's
-// initial and final state are entry slots[n] of a pool of num_slots entries.
+// bf16_prefill_scratch_bytes() bytes.
 cudaError_t launch_bf16_prefill(unsigned char *scratch, const void *q, const void *k,
                                 const void *v, const float *g, const float *beta,
                                 const float *initial_state, const int32_t *cu_seqlens, void *out,
                                 float *final_state, int B, int T, int H, int N, Prologue pro,
-                                int sms, cudaStream_t st, const int32_t *slots = nullptr,
-                                int num_slots = 0);
+                                int sms, cudaStream_t st);
 
 }  // namespace kda

@@ -89,8 +89,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
                       float *__restrict__ sT, __nv_bfloat16 *__restrict__ out, int T, int total_T,
                       int H, int cps, int max_chunks, int *__restrict__ err,
                       unsigned char *__restrict__ s_img, unsigned char *__restrict__ v_img,
-                      const int32_t *__restrict__ order, const int32_t *__restrict__ slots,
-                      int num_slots)
+                      const int32_t *__restrict__ order)
 {
     using L = TcLayout<DVT, NS>;
     extern __shared__ unsigned char smem_raw[];
@@ -113,17 +112,6 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
     // longest chains start in the first wave
     const int n0 = blockIdx.x * DVT, h = blockIdx.y;
     const int seq = order ? order[blockIdx.z] : blockIdx.z;
-    // the state's entry: sequence seq's own, or (serving decode) the pool
-    // entry slots[seq]; an entry outside the pool skips the sequence (no
-    // state or output written) and reports it
-    int st_idx = seq;
-    if (slots) {
-        st_idx = slots[seq];
-        if (st_idx < 0 || st_idx >= num_slots) {
-            if (threadIdx.x == 0) set_device_error(err, kErrBadSlot);
-            return;
-        }
-    }
 
     long long bos, eos;
     int c_begin;
@@ -276,7 +264,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         float S[CPT];
         {
-            const size_t sb = (((size_t)st_idx * H + h) * D + t) * D + n0 + cb;
+            const size_t sb = (((size_t)seq * H + h) * D + t) * D + n0 + cb;
 #pragma unroll
             for (int j = 0; j < CPT; j += 4) {
                 float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -404,7 +392,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
             set_device_error(err, kErrWaitTimeout);
             *abort_flag = 1;
         } else if (sT) {
-            const size_t sb = (((size_t)st_idx * H + h) * D + t) * D + n0 + cb;
+            const size_t sb = (((size_t)seq * H + h) * D + t) * D + n0 + cb;
 #pragma unroll
             for (int j = 0; j < CPT; j += 4)
                 *reinterpret_cast<float4 *>(sT + sb + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
@@ -420,8 +408,7 @@ template <int DVT, int NS>
 cudaError_t launch_tc(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
                       const float *s0, float *sT, void *out, int N, int T, int total_T, int H,
                       int max_chunks, int *err, cudaStream_t st, unsigned char *s_img,
-                      unsigned char *v_img, const int32_t *order, const int32_t *slots,
-                      int num_slots)
+                      unsigned char *v_img, const int32_t *order)
 {
     using L = TcLayout<DVT, NS>;
     const size_t smem = L::BYTES + 1024;
@@ -431,7 +418,7 @@ cudaError_t launch_tc(const unsigned char *wsp, const int32_t *cu, const int32_t
     dim3 grid(D / DVT, H, N);
     chunk_chain_tc_kernel<DVT, NS><<<grid, L::NTHREADS, smem, st>>>(
         wsp, cu, coff, s0, sT, (__nv_bfloat16 *)out, T, total_T, H, (T + C - 1) / C, max_chunks, err,
-        s_img, v_img, order, slots, num_slots);
+        s_img, v_img, order);
     return cudaGetLastError();
 }
 
@@ -441,9 +428,9 @@ cudaError_t launch_chunk_chain(const unsigned char *wsp, const int32_t *cu, cons
                                   const float *s0, float *sT, void *out, int N, int T,
                                   int total_T, int H, int dvt, int max_chunks, int *err,
                                   cudaStream_t st, unsigned char *s_img, unsigned char *v_img,
-                                  const int32_t *order, const int32_t *slots, int num_slots)
+                                  const int32_t *order)
 {
-#define KDA_CHAIN_ARGS wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st, s_img, v_img, order, slots, num_slots
+#define KDA_CHAIN_ARGS wsp, cu, coff, s0, sT, out, N, T, total_T, H, max_chunks, err, st, s_img, v_img, order
     switch (dvt) {
         case 16: return launch_tc<16, 3>(KDA_CHAIN_ARGS);
         case 32: return launch_tc<32, 3>(KDA_CHAIN_ARGS);

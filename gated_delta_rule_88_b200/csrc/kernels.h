@@ -94,15 +94,11 @@ cudaError_t launch_chunk_prep(const void *q, const void *k, const void *v, const
 // s_img / v_img (nullable): per-(chunk, head) bf16 images of the state
 // entering each chunk (32 KiB) and of V_new (16 KiB), for the backward.
 // order (nullable): the sequences in launch order (longest first).
-// slots (nullable): sequence n's state is entry slots[n] of s0 / sT (a pool
-// of num_slots entries); an entry outside the pool skips the sequence and
-// sets kErrBadSlot.
 cudaError_t launch_chunk_chain(const unsigned char *wsp, const int32_t *cu, const int32_t *coff,
                                const float *s0, float *sT, void *out, int N, int T, int total_T,
                                int H, int dvt, int max_chunks, int *err, cudaStream_t st,
                                unsigned char *s_img = nullptr, unsigned char *v_img = nullptr,
-                               const int32_t *order = nullptr, const int32_t *slots = nullptr,
-                               int num_slots = 0);
+                               const int32_t *order = nullptr);
 
 // Chunked backward (bf16, dk = dv = 128): the reverse chain over the forward
 // records (gradient images dS' 32 KiB and dV_new 16 KiB per (chunk, head)),

@@ -244,16 +244,12 @@ kda_status kda_recurrent_step_ex(const void *q, const void *k, const void *v,
  * KDA_STEPS_CHUNK in flags selects, for dtype KDA_BF16 with dk = dv = 128,
  * L >= 2 and no prologue flags (q_scale = 1), the chunk form of the same L
  * steps (section 3 of the notes: a WY-like representation of the block's
- * writes, then one product with the state) on tensor cores: the operands of
- * the state products (state, V_new, T, P and the decayed k, q) are rounded
- * to bf16 as in kda_chunk_fwd, the state stays fp32.  For L <= 32 it runs in
- * blocks of 16 tokens in one kernel that allocates nothing; from L = 33 on
- * it runs kda_chunk_fwd's kernels over the N sequences of L tokens with each
- * state resumed from and written back to its pool entry, and takes their
- * scratch (N * ceil(L / 64) * H * 74,240 bytes) from the library-private
- * stream-ordered pool, as kda_chunk_fwd does.  Any finite g <= 0, and
- * g <= 5 for positive gates.  Other combinations run the recurrent kernel,
- * which is bitwise equal to L calls of kda_recurrent_step.
+ * writes, then one product with the state) in blocks of 16 tokens on tensor
+ * cores: the operands of the state products (state, V_new, T, P and the
+ * decayed k, q) are rounded to bf16 as in kda_chunk_fwd, the state stays
+ * fp32.  Any finite g <= 0, and g <= 5 for positive gates.  Other
+ * combinations run the recurrent kernel, which is bitwise equal to L calls
+ * of kda_recurrent_step.
  */
 kda_status kda_recurrent_steps(const void *q, const void *k, const void *v,
                                const float *g, const float *beta,

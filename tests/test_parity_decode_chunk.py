@@ -6,9 +6,8 @@ writes in a WY-like representation and touches the state with one product;
 the result is the recurrence's.  Tolerance: the bf16 bound of the other
 parity tests (the state-product operands are bf16, as in the prefill).
 Lengths cover one partial block (2, 8), a full block (16), a block plus one
-token (17) and several blocks (40, 64, 100: from 33 tokens on the call runs
-the prefill's kernels on the pool); gates cover the decode workload's and a
-stronger, channel-dependent decay.
+token (17) and several blocks (32, 33, 40, 64, 100); gates cover the decode
+workload's and a stronger, channel-dependent decay.
 """
 import pytest
 import torch
@@ -67,8 +66,7 @@ def test_chunk_steps_gates(gate):
 @pytest.mark.parametrize("L", [20, 70])
 def test_chunk_steps_strong_decay(L):
     """g = -20 per token on every channel: the block forms use e^{G_i - G_j}
-    <= 1 directly (16-token blocks at L = 20; the prefill kernels' direct
-    diagonal blocks at L = 70), so nothing overflows."""
+    <= 1 directly, so nothing overflows."""
     N, H, d = 3, 2, 128
     q, k, v, g, b = _tokens(N, L, H, d, seed=98)
     g = torch.full_like(g, -20.0)
@@ -123,9 +121,9 @@ def test_chunk_flag_falls_back_where_unsupported():
 
 
 def test_chunk_steps_bad_slot_reported_and_skipped_long():
-    """From 33 tokens on (the prefill kernels on the pool): a slot outside the
-    pool skips its sequence (no output, no pool entry written) and reports
-    device error code 3; the other sequences are computed."""
+    """A slot outside the pool skips its sequence (no output, no pool entry
+    written) and reports device error code 3; the other sequences are
+    computed (several 16-token blocks per call)."""
     N, L, H, d, S = 4, 40, 2, 128, 6
     q, k, v, g, b = [t.to(DEV) for t in _tokens(N, L, H, d, seed=26)]
     pool0 = W.decode_initial_state(S, H, d, d, seed=26)

@@ -330,6 +330,17 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
 
+    if args.only_backward:
+        # profiling: just the chunked backward on its workload
+        bwd_inp = W.named_prefill(BWD_WORKLOAD).to(dev)
+        res = backward_leg(kda, bwd_inp, dev, dist, world, args, chunked=True)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
     if args.only_prefill:
         # profiling: just the prefill calls of one workload (no legs, no e2e)
         inp = W.named_prefill(args.only_prefill).to(dev)
@@ -650,6 +661,8 @@ def main():
     ap.add_argument("--decode-n", type=int, default=DEC_N,
                     help="sequences in the decode legs (a smaller case for profiling)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--only-backward", action="store_true",
+                    help="profiling: time only kda_chunk_bwd on the 8192-token workload")
     ap.add_argument("--only-prefill", metavar="WORKLOAD", default=None,
                     help="profiling: time only kda_chunk_fwd on this named workload "
                          "(e.g. varlen8_h32_d128_resume) and print its line")

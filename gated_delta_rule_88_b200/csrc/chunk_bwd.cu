@@ -75,6 +75,9 @@ __device__ __forceinline__ uint32_t mnmaj(int kk) { return (kk * 2048) >> 4; }
 __device__ __forceinline__ uint32_t img_off(int r, int c, uint32_t bs) {
     return (c >> 6) * bs + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1);
 }
+// fp32 [64][128] tile with the column XOR-swizzled by the row: 16 lanes on
+// 16 consecutive rows and one column hit 16 different banks
+__device__ __forceinline__ int gsw(int r, int c) { return r * 128 + (c ^ ((r & 15) << 1)); }
 // 8 floats -> one 16-byte chunk of bf16
 __device__ __forceinline__ uint4 pack8(const float *x, float s) {
     return make_uint4(pack_bf16(s * x[0], s * x[1]), pack_bf16(s * x[2], s * x[3]), pack_bf16(s * x[4], s * x[5]),
@@ -182,7 +185,7 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             Gv[i].x += PF.x; Gv[i].y += PF.y;
             bad |= !(fabsf(Gv[i].x) <= RANGE2 && fabsf(Gv[i].y) <= RANGE2 &&
                      GC.x - Gv[i].x <= RANGE2 && GC.y - Gv[i].y <= RANGE2);
-            *reinterpret_cast<float2 *>(G2 + (16 * I + i) * D + c0) = Gv[i];
+            *reinterpret_cast<float2 *>(G2 + gsw(16 * I + i, c0)) = Gv[i];
         }
     }
     if (tid == 0 && ok) ok = mbar_wait(bar_ld, 0);
@@ -204,7 +207,7 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         for (int i = 0; i < 16; ++i) {
             const int r = 16 * I + i;
             const int o = sw(r, cc);
-            const float2 Gi = *reinterpret_cast<const float2 *>(G2 + r * D + c0);
+            const float2 Gi = *reinterpret_cast<const float2 *>(G2 + gsw(r, c0));
             const float2 eg = make_float2(ex2_approx(Gi.x), ex2_approx(Gi.y));
             const float2 em = make_float2(ex2_approx(-Gi.x), ex2_approx(-Gi.y));
             float2 qf = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(kq + 8192 + o));
@@ -531,6 +534,9 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 kb[j] = __shfl_xor_sync(0xffffffffu, b[j], 16);
                 vc[j] = __shfl_xor_sync(0xffffffffu, c[j], 16);
             }
+            float ktv[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) ktv[j] = 0.f;
             if (hi == pass) {
             // owner: lanes < 16 hold (Q, Kt, bV) in a, b, c and (Kinv, bKg) in kb, vc;
             // lanes >= 16 the other way round
@@ -560,15 +566,15 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                             const float dKinv = hi ? b[j] : kb[j];
                             const float dbV = hi ? vc[j] : c[j];
                             const float dbKg = hi ? c[j] : vc[j];
-                            const float g2 = G2[i * D + ch], gc2 = G2[63 * D + ch];
+                            const float g2 = G2[gsw(i, ch)], gc2 = G2[gsw(63, ch)];
                             const float eg = ex2_approx(g2), em = ex2_approx(-g2), egc = ex2_approx(gc2);
                             const float kt = ks[w2] * em * egc;
                             oq[2 * u + w2] = dQg * eg;
                             ok_[2 * u + w2] = dbKg * br * eg + (dKinv + dKt * egc) * em;
                             ov[2 * u + w2] = dbV * br;
                             dbp = fmaf(dbKg * ks[w2], eg, fmaf(dbV, vs[w2], dbp));
-                            dG[i * D + ch] = dQg * qs[w2] * eg + dbKg * br * ks[w2] * eg - dKinv * ks[w2] * em - dKt * kt;
-                            atomicAdd(kts + ch, dKt * kt);
+                            dG[gsw(i, ch)] = dQg * qs[w2] * eg + dbKg * br * ks[w2] * eg - dKinv * ks[w2] * em - dKt * kt;
+                            ktv[j] = dKt * kt;
                         }
                     }
                     float4 *pq = reinterpret_cast<float4 *>(dq + grow + 8 * e);
@@ -581,19 +587,31 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 atomicAdd(dbs + i, dbp);
             } else {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) dG[i * D + ch0 + j] = 0.f;
+                for (int j = 0; j < 16; ++j) dG[gsw(i, ch0 + j)] = 0.f;
             }
+            }
+            // sum over the 16 token rows of the owner half (lanes outside it
+            // hold zeros; the xor steps stay inside each half), one shared
+            // atomic per channel and warp
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                float t = ktv[j];
+                t += __shfl_xor_sync(0xffffffffu, t, 1);
+                t += __shfl_xor_sync(0xffffffffu, t, 2);
+                t += __shfl_xor_sync(0xffffffffu, t, 4);
+                t += __shfl_xor_sync(0xffffffffu, t, 8);
+                if (l16 == 0 && hi == pass) atomicAdd(kts + ch0 + j, t);
             }
         }
     }
     __syncthreads();
     if (ok && tid < 128) {
         const int c = tid;
-        const float gc2 = G2[63 * D + c];
+        const float gc2 = G2[gsw(63, c)];
         float acc = kts[c] + degc[c] * ex2_approx(gc2);
         // the G_C terms sit on the last row; reverse cumsum inside the chunk
         for (int t = 63; t >= 0; --t) {
-            acc += dG[t * D + c];
+            acc += dG[gsw(t, c)];
             if (t < len) dg[((size_t)(t0 + t) * H + h) * D + c] = acc;
         }
     } else if (ok && tid >= 128 && tid - 128 < len) {

@@ -111,6 +111,7 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 
     uint64_t *bar_g = reinterpret_cast<uint64_t *>(sm + bl::BAR);
     uint64_t *bar_ld = bar_g + 1, *bar_in2 = bar_g + 2, *bar_in3 = bar_g + 3, *bar_mma = bar_g + 4;
+    uint64_t *bar_fin = bar_g + 5;      // q, k, v again, for the finale
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + bl::TSLOT);
     float *bet = reinterpret_cast<float *>(sm + bl::BETA);
     float *degc = reinterpret_cast<float *>(sm + bl::DEGC);
@@ -119,7 +120,7 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     float *G2 = reinterpret_cast<float *>(sm + bl::G);
 
     if (tid == 0) {
-        for (int b = 0; b < 5; ++b) mbar_init(bar_g + b, 1);
+        for (int b = 0; b < 6; ++b) mbar_init(bar_g + b, 1);
         fence_mbar_init();
         const int tt = (int)t0;
         mbar_arrive_expect_tx(bar_g, bl::TX_G);
@@ -347,6 +348,19 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         if (b == 0) degc[c] = s;
     }
     ok = mma_done(ok);
+    // dO, V_new and beta v are dead: q, k and v come again (raw, by TMA) into
+    // their places for the finale, while the products below run
+    bool fin_issued = false;
+    if (tid == 0 && ok) {
+        fin_issued = true;
+        mbar_arrive_expect_tx(bar_fin, bl::TX_QKV);
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+            tma_load_3d(sm + bl::DO + b * 8192, &tm_q, 64 * b, h, (int)t0, bar_fin);
+            tma_load_3d(sm + bl::VN + b * 8192, &tm_k, 64 * b, h, (int)t0, bar_fin);
+            tma_load_3d(sm + bl::V + b * 8192, &tm_v, 64 * b, h, (int)t0, bar_fin);
+        }
+    }
 
     // ---- readback: dW = -D_W (lanes +16, cols 0-127) -> DW image; dP = tril0(D_P) -> DP image ----
     const int sub = warp & 3, l16 = lane & 15, hi = lane >> 4;
@@ -514,6 +528,8 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     ok = mma_done(ok);
 
     // ---- finale: per token row and 32-channel group ----
+    if (tid == 0 && ok) ok = mbar_wait(bar_fin, 0);
+    ok = __syncthreads_and(ok);
     float *dG = reinterpret_cast<float *>(sm + bl::KQ);        // [64][128] fp32 (bKg, Qg are dead)
     if (ok) {
         const int csel = warp >> 2;
@@ -547,9 +563,11 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 float dbp = 0.f;
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const uint4 qx = *reinterpret_cast<const uint4 *>(q + grow + 8 * e);
-                    const uint4 kx = *reinterpret_cast<const uint4 *>(k + grow + 8 * e);
-                    const uint4 vx = *reinterpret_cast<const uint4 *>(v + grow + 8 * e);
+                    const int cq = ch0 + 8 * e;
+                    const uint32_t so = (cq >> 6) * 8192 + sw(i, cq & 63);
+                    const uint4 qx = *reinterpret_cast<const uint4 *>(sm + bl::DO + so);
+                    const uint4 kx = *reinterpret_cast<const uint4 *>(sm + bl::VN + so);
+                    const uint4 vx = *reinterpret_cast<const uint4 *>(sm + bl::V + so);
                     const uint32_t qw[4] = {qx.x, qx.y, qx.z, qx.w}, kw[4] = {kx.x, kx.y, kx.z, kx.w},
                                    vw[4] = {vx.x, vx.y, vx.z, vx.w};
                     float oq[8], ok_[8], ov[8];
@@ -605,17 +623,28 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         }
     }
     __syncthreads();
-    if (ok && tid < 128) {
-        const int c = tid;
-        const float gc2 = G2[gsw(63, c)];
-        float acc = kts[c] + degc[c] * ex2_approx(gc2);
-        // the G_C terms sit on the last row; reverse cumsum inside the chunk
-        for (int t = 63; t >= 0; --t) {
+    // dg = reverse cumsum of dG inside the chunk, the G_C terms on the last
+    // row: two threads per channel, rows 32-63 (hf = 1) and 0-31 (hf = 0),
+    // meeting once through shared memory (the upper half's total)
+    if (ok) {
+        const int c = tid & 127, hf = tid >> 7;
+        const float base_c = kts[c] + degc[c] * ex2_approx(G2[gsw(63, c)]);
+        float up = base_c;
+        if (hf) {
+#pragma unroll 8
+            for (int t = 32; t < 64; ++t) up += dG[gsw(t, c)];
+        }
+        __syncthreads();                         // kts read by every thread
+        if (hf) kts[c] = up;
+        __syncthreads();
+        float acc = hf ? base_c : kts[c];
+        const int t_hi = hf ? 63 : 31;
+#pragma unroll 8
+        for (int t = t_hi; t > t_hi - 32; --t) {
             acc += dG[gsw(t, c)];
             if (t < len) dg[((size_t)(t0 + t) * H + h) * D + c] = acc;
         }
-    } else if (ok && tid >= 128 && tid - 128 < len) {
-        dbeta[(size_t)(t0 + tid - 128) * H + h] = dbs[tid - 128];
+        if (tid < len) dbeta[(size_t)(t0 + tid) * H + h] = dbs[tid];
     }
     if (!ok && tid == 0) {
         if (!bad) set_device_error(err, kErrWaitTimeout);
@@ -624,6 +653,7 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         mbar_wait(bar_ld, 0, 1u << 20);
         mbar_wait(bar_in2, 0, 1u << 20);
         if (in3_issued) mbar_wait(bar_in3, 0, 1u << 20);
+        if (fin_issued) mbar_wait(bar_fin, 0, 1u << 20);
     }
     tc_fence_before();
     __syncthreads();

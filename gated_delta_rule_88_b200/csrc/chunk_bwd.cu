@@ -20,8 +20,8 @@
 // TMEM columns (512, one CTA per SM):
 //   0-127   D_Q (+0)     D_W (+16)
 //   128-255 D_Kt (+0)    D_Kinv (+16)
-//   256-319 D_P (+0)     D_T (+16)     (first: MMA-AP, M = 128)
-//   320-383 X (+0)       Y (+16)
+//   256-319 MMA-AP (M = 128; A on lanes 0-63)
+//   320-383 D_P (+0), then X     D_T (+16), then Y
 //   384-511 D_bV (+0)    D_bKg (+16)
 #include "chunk_ws.h"
 #include "common.cuh"
@@ -228,7 +228,7 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     const uint32_t sb = smem_u32(sm);
     const uint32_t L16 = 16u << 16;                     // +16 lane tile
 
-    // ---- MMA-AP: [bKg ; Qg] Kinv^T -> cols 256-319 (A on lanes 0-63) ----
+    // ---- MMA-AP: [bKg ; Qg] Kinv^T -> cols 256-319 (A on lanes 0-63); then D_P, D_T ----
     if (tid == 0 && ok) {
         tc_fence_after();
         constexpr uint32_t ID = idesc_g(128, 64, false, false);
@@ -238,6 +238,23 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         for (int kk = 0; kk < 8; ++kk)
             umma_bf16_p(tmem + 256, a.lo + kmaj(kk, 16384), a.hi, b.lo + kmaj(kk, 8192), b.hi, ID, kk > 0);
         umma_commit(bar_mma);
+        // the two phase-2 products that need neither S nor dS' run while the
+        // CUDA cores form T: D_P = dO V_new^T (cols 320-383, +0) and
+        // D_T = dV_new (bV)^T (cols 320-383, +16); the phase-2a commit covers them
+        ok = mbar_wait(bar_in2, 0);
+        if (ok) {
+            constexpr uint32_t ID64 = idesc_g(64, 64, false, false);
+            const DescParts a_do = smem_desc_parts(sb + bl::DO, 16, 1024, 2);
+            const DescParts a_dvn = smem_desc_parts(sb + bl::DVN, 16, 1024, 2);
+            const DescParts b_vn = smem_desc_parts(sb + bl::VN, 16, 1024, 2);
+            const DescParts b_bv = smem_desc_parts(sb + bl::V, 16, 1024, 2);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                umma_bf16_p(tmem + 320, a_do.lo + kmaj(kk, 8192), a_do.hi, b_vn.lo + kmaj(kk, 8192), b_vn.hi, ID64, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                umma_bf16_p(tmem + 320 + L16, a_dvn.lo + kmaj(kk, 8192), a_dvn.hi, b_bv.lo + kmaj(kk, 8192), b_bv.hi, ID64, kk > 0);
+        }
     }
     ok = mma_done(ok);
 
@@ -303,14 +320,12 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     // ---- phase 2a products ----
     if (tid == 0 && ok) {
         tc_fence_after();
-        constexpr uint32_t ID128 = idesc_g(64, 128, false, false), ID64 = idesc_g(64, 64, false, false);
+        constexpr uint32_t ID128 = idesc_g(64, 128, false, false);
         const DescParts a_do = smem_desc_parts(sb + bl::DO, 16, 1024, 2);
         const DescParts a_dvn = smem_desc_parts(sb + bl::DVN, 16, 1024, 2);
         const DescParts a_vn = smem_desc_parts(sb + bl::VN, 16, 1024, 2);
         const DescParts b_s = smem_desc_parts(sb + bl::S, 16, 1024, 2);
         const DescParts b_ds = smem_desc_parts(sb + bl::DS, 16, 1024, 2);
-        const DescParts b_vn = smem_desc_parts(sb + bl::VN, 16, 1024, 2);
-        const DescParts b_bv = smem_desc_parts(sb + bl::V, 16, 1024, 2);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)      // D_Q = dO S^T
             umma_bf16_p(tmem + 0, a_do.lo + kmaj(kk, 8192), a_do.hi, b_s.lo + kmaj(kk, 16384), b_s.hi, ID128, kk > 0);
@@ -320,13 +335,7 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)      // D_Kt = V_new dS'^T
             umma_bf16_p(tmem + 128, a_vn.lo + kmaj(kk, 8192), a_vn.hi, b_ds.lo + kmaj(kk, 16384), b_ds.hi, ID128, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)      // D_P = dO V_new^T
-            umma_bf16_p(tmem + 256, a_do.lo + kmaj(kk, 8192), a_do.hi, b_vn.lo + kmaj(kk, 8192), b_vn.hi, ID64, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)      // D_T = dV_new (bV)^T
-            umma_bf16_p(tmem + 256 + L16, a_dvn.lo + kmaj(kk, 8192), a_dvn.hi, b_bv.lo + kmaj(kk, 8192), b_bv.hi, ID64, kk > 0);
-        umma_commit(bar_mma);
+        umma_commit(bar_mma);               // also covers D_P and D_T
     }
     // de^{G_C} = rowsum(S o dS') from the bf16 images (two threads per channel row)
     if (ok) {
@@ -383,7 +392,7 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 #pragma unroll
             for (int c2 = 0; c2 < 2; ++c2) {
                 float x[32];
-                tmem_ld32(tmem + lane_base + 256 + 32 * c2, x);
+                tmem_ld32(tmem + lane_base + 320 + 32 * c2, x);
                 tmem_wait_ld();
                 if (!hi) {
 #pragma unroll
@@ -410,7 +419,7 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         const DescParts b_qg = smem_desc_parts(sb + bl::KQ + 8192, 16384, 1024, 2);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-            umma_bf16_p(tmem + 256 + L16, a_dw.lo + kmaj(kk, 8192), a_dw.hi, b_bkg.lo + kmaj(kk, 16384), b_bkg.hi,
+            umma_bf16_p(tmem + 320 + L16, a_dw.lo + kmaj(kk, 8192), a_dw.hi, b_bkg.lo + kmaj(kk, 16384), b_bkg.hi,
                         idesc_g(64, 64, false, false), 1);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
@@ -424,12 +433,12 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     }
     ok = mma_done(ok);
 
-    // ---- dT (lanes +16, cols 256-319) -> DT image ----
+    // ---- dT (lanes +16, cols 320-383) -> DT image ----
     if (ok && warp >= 4) {
 #pragma unroll
         for (int c2 = 0; c2 < 2; ++c2) {
             float x[32];
-            tmem_ld32(tmem + lane_base + 256 + 32 * c2, x);
+            tmem_ld32(tmem + lane_base + 320 + 32 * c2, x);
             tmem_wait_ld();
             if (hi) {
 #pragma unroll
@@ -543,86 +552,75 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         const bool live = i < len;
         const float br = bet[i];
         float dbp = 0.f;
-        // steps in pairs (the same 32 channels, halves of 16): both steps'
-        // TMEM rows are read before either is worked on
 #pragma unroll 1
-        for (int sp = 0; sp < 2; ++sp) {
-            float a2[2][16], b2[2][16], c2[2][16];
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int ch0 = 32 * (2 * sp + csel) + 16 * hh;
-                tmem_ld16(tmem + lane_base + ch0, a2[hh]);            // D_Q | (dead D_W)
-                tmem_ld16(tmem + lane_base + 128 + ch0, b2[hh]);      // D_Kt | D_Kinv
-                tmem_ld16(tmem + lane_base + 384 + ch0, c2[hh]);      // D_bV | D_bKg
-            }
+        for (int step = 0; step < 4; ++step) {
+            const int cc = 2 * (step >> 1) + csel;
+            const int ch0 = 32 * cc + 16 * (step & 1);      // this step's 16 channels
+            const int cm = ch0 + 8 * hi;                     // this lane's 8
+            float a[16], b[16], c[16];
+            tmem_ld16(tmem + lane_base + ch0, a);            // D_Q | (dead D_W)
+            tmem_ld16(tmem + lane_base + 128 + ch0, b);      // D_Kt | D_Kinv
+            tmem_ld16(tmem + lane_base + 384 + ch0, c);      // D_bV | D_bKg
             tmem_wait_ld();
+            float dQg[8], dKt[8], dbV[8], dKinv[8], dbKg[8];
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int ch0 = 32 * (2 * sp + csel) + 16 * hh;      // this step's 16 channels
-                const int cm = ch0 + 8 * hi;                         // this lane's 8
-                const float (&a)[16] = a2[hh];
-                const float (&b)[16] = b2[hh];
-                const float (&c)[16] = c2[hh];
-                float dQg[8], dKt[8], dbV[8], dKinv[8], dbKg[8];
+            for (int jj = 0; jj < 8; ++jj) {
+                const float s1 = __shfl_xor_sync(0xffffffffu, hi ? b[jj] : a[8 + jj], 16);
+                const float s2 = __shfl_xor_sync(0xffffffffu, hi ? c[jj] : b[8 + jj], 16);
+                const float s3 = __shfl_xor_sync(0xffffffffu, c[8 + jj], 16);
+                dQg[jj] = hi ? s1 : a[jj];
+                dKt[jj] = hi ? s2 : b[jj];
+                dbV[jj] = hi ? s3 : c[jj];
+                dKinv[jj] = hi ? b[8 + jj] : s1;
+                dbKg[jj] = hi ? c[8 + jj] : s2;
+            }
+            const uint32_t so = (cm >> 6) * 8192 + sw(i, cm & 63);
+            const uint4 qx = *reinterpret_cast<const uint4 *>(sm + bl::DO + so);
+            const uint4 kx = *reinterpret_cast<const uint4 *>(sm + bl::VN + so);
+            const uint4 vx = *reinterpret_cast<const uint4 *>(sm + bl::V + so);
+            const uint32_t qw[4] = {qx.x, qx.y, qx.z, qx.w}, kw[4] = {kx.x, kx.y, kx.z, kx.w},
+                           vw[4] = {vx.x, vx.y, vx.z, vx.w};
+            float oq[8], ok_[8], ov[8], ktv[8];
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    const float s1 = __shfl_xor_sync(0xffffffffu, hi ? b[jj] : a[8 + jj], 16);
-                    const float s2 = __shfl_xor_sync(0xffffffffu, hi ? c[jj] : b[8 + jj], 16);
-                    const float s3 = __shfl_xor_sync(0xffffffffu, c[8 + jj], 16);
-                    dQg[jj] = hi ? s1 : a[jj];
-                    dKt[jj] = hi ? s2 : b[jj];
-                    dbV[jj] = hi ? s3 : c[jj];
-                    dKinv[jj] = hi ? b[8 + jj] : s1;
-                    dbKg[jj] = hi ? c[8 + jj] : s2;
+            for (int u = 0; u < 4; ++u) {
+                const float2 qf = bf16x2_to_float2(qw[u]), kf = bf16x2_to_float2(kw[u]),
+                             vf = bf16x2_to_float2(vw[u]);
+                const float qs[2] = {qf.x, qf.y}, ks[2] = {kf.x, kf.y}, vs[2] = {vf.x, vf.y};
+#pragma unroll
+                for (int w2 = 0; w2 < 2; ++w2) {
+                    const int jj = 2 * u + w2, ch = cm + jj;
+                    const float g2 = G2[gsw(i, ch)], gc2 = G2[gsw(63, ch)];
+                    const float eg = ex2_approx(g2), em = ex2_approx(-g2), egc = ex2_approx(gc2);
+                    const float kt = ks[w2] * em * egc;
+                    oq[jj] = dQg[jj] * eg;
+                    ok_[jj] = dbKg[jj] * br * eg + (dKinv[jj] + dKt[jj] * egc) * em;
+                    ov[jj] = dbV[jj] * br;
+                    if (live) dbp = fmaf(dbKg[jj] * ks[w2], eg, fmaf(dbV[jj], vs[w2], dbp));
+                    dG[gsw(i, ch)] = live ? dQg[jj] * qs[w2] * eg + dbKg[jj] * br * ks[w2] * eg -
+                                                dKinv[jj] * ks[w2] * em - dKt[jj] * kt
+                                          : 0.f;
+                    ktv[jj] = live ? dKt[jj] * kt : 0.f;
                 }
-                const uint32_t so = (cm >> 6) * 8192 + sw(i, cm & 63);
-                const uint4 qx = *reinterpret_cast<const uint4 *>(sm + bl::DO + so);
-                const uint4 kx = *reinterpret_cast<const uint4 *>(sm + bl::VN + so);
-                const uint4 vx = *reinterpret_cast<const uint4 *>(sm + bl::V + so);
-                const uint32_t qw[4] = {qx.x, qx.y, qx.z, qx.w}, kw[4] = {kx.x, kx.y, kx.z, kx.w},
-                               vw[4] = {vx.x, vx.y, vx.z, vx.w};
-                float oq[8], ok_[8], ov[8], ktv[8];
+            }
+            if (live) {
+                const size_t grow = ((size_t)(t0 + i) * H + h) * D + cm;
+                float4 *pq = reinterpret_cast<float4 *>(dq + grow);
+                float4 *pk = reinterpret_cast<float4 *>(dk + grow);
+                float4 *pv = reinterpret_cast<float4 *>(dv + grow);
+                pq[0] = make_float4(oq[0], oq[1], oq[2], oq[3]); pq[1] = make_float4(oq[4], oq[5], oq[6], oq[7]);
+                pk[0] = make_float4(ok_[0], ok_[1], ok_[2], ok_[3]); pk[1] = make_float4(ok_[4], ok_[5], ok_[6], ok_[7]);
+                pv[0] = make_float4(ov[0], ov[1], ov[2], ov[3]); pv[1] = make_float4(ov[4], ov[5], ov[6], ov[7]);
+            }
+            // column sums over the half's 16 token rows (xor steps stay inside
+            // each half), one shared atomic per channel and half
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float2 qf = bf16x2_to_float2(qw[u]), kf = bf16x2_to_float2(kw[u]),
-                                 vf = bf16x2_to_float2(vw[u]);
-                    const float qs[2] = {qf.x, qf.y}, ks[2] = {kf.x, kf.y}, vs[2] = {vf.x, vf.y};
-#pragma unroll
-                    for (int w2 = 0; w2 < 2; ++w2) {
-                        const int jj = 2 * u + w2, ch = cm + jj;
-                        const float g2 = G2[gsw(i, ch)], gc2 = G2[gsw(63, ch)];
-                        const float eg = ex2_approx(g2), em = ex2_approx(-g2), egc = ex2_approx(gc2);
-                        const float kt = ks[w2] * em * egc;
-                        oq[jj] = dQg[jj] * eg;
-                        ok_[jj] = dbKg[jj] * br * eg + (dKinv[jj] + dKt[jj] * egc) * em;
-                        ov[jj] = dbV[jj] * br;
-                        if (live) dbp = fmaf(dbKg[jj] * ks[w2], eg, fmaf(dbV[jj], vs[w2], dbp));
-                        dG[gsw(i, ch)] = live ? dQg[jj] * qs[w2] * eg + dbKg[jj] * br * ks[w2] * eg -
-                                                    dKinv[jj] * ks[w2] * em - dKt[jj] * kt
-                                              : 0.f;
-                        ktv[jj] = live ? dKt[jj] * kt : 0.f;
-                    }
-                }
-                if (live) {
-                    const size_t grow = ((size_t)(t0 + i) * H + h) * D + cm;
-                    float4 *pq = reinterpret_cast<float4 *>(dq + grow);
-                    float4 *pk = reinterpret_cast<float4 *>(dk + grow);
-                    float4 *pv = reinterpret_cast<float4 *>(dv + grow);
-                    pq[0] = make_float4(oq[0], oq[1], oq[2], oq[3]); pq[1] = make_float4(oq[4], oq[5], oq[6], oq[7]);
-                    pk[0] = make_float4(ok_[0], ok_[1], ok_[2], ok_[3]); pk[1] = make_float4(ok_[4], ok_[5], ok_[6], ok_[7]);
-                    pv[0] = make_float4(ov[0], ov[1], ov[2], ov[3]); pv[1] = make_float4(ov[4], ov[5], ov[6], ov[7]);
-                }
-                // column sums over the half's 16 token rows (xor steps stay inside
-                // each half), one shared atomic per channel and half
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    float t = ktv[jj];
-                    t += __shfl_xor_sync(0xffffffffu, t, 1);
-                    t += __shfl_xor_sync(0xffffffffu, t, 2);
-                    t += __shfl_xor_sync(0xffffffffu, t, 4);
-                    t += __shfl_xor_sync(0xffffffffu, t, 8);
-                    if (l16 == 0) atomicAdd(kts + cm + jj, t);
-                }
+            for (int jj = 0; jj < 8; ++jj) {
+                float t = ktv[jj];
+                t += __shfl_xor_sync(0xffffffffu, t, 1);
+                t += __shfl_xor_sync(0xffffffffu, t, 2);
+                t += __shfl_xor_sync(0xffffffffu, t, 4);
+                t += __shfl_xor_sync(0xffffffffu, t, 8);
+                if (l16 == 0) atomicAdd(kts + cm + jj, t);
             }
         }
         // dbeta of the row: both halves' channels, both channel groups (csel)

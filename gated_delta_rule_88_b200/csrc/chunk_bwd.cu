@@ -20,8 +20,8 @@
 // TMEM columns (512, one CTA per SM):
 //   0-127   D_Q (+0)     D_W (+16)
 //   128-255 D_Kt (+0)    D_Kinv (+16)
-//   256-319 MMA-AP (M = 128; A on lanes 0-63)
-//   320-383 D_P (+0), then X     D_T (+16), then Y
+//   256-319 D_P (+0)     D_T (+16)     (first: MMA-AP, M = 128)
+//   320-383 X (+0)       Y (+16)
 //   384-511 D_bV (+0)    D_bKg (+16)
 #include "chunk_ws.h"
 #include "common.cuh"
@@ -55,9 +55,9 @@ constexpr int S = WA, DS = WA + 32768;                                        //
 constexpr int DW = WA, DP = WA + 16384, DT = WA + 24576, XI = WA + 32768, DA = WA + 40960;
 constexpr int BETA = WA + 65536;                 // 64 floats
 constexpr int DEGC = BETA + 256;                 // 128 floats: rowsum(S o dS')
-constexpr int KTS = DEGC + 512;                  // 128 floats: sum_i dKt o Kt
-constexpr int DB = KTS + 512;                    // 64 floats: dbeta
-constexpr int BAR = DB + 256;                    // 6 mbarriers
+constexpr int KTS = DEGC + 512;                  // [4][128] floats: sum_i dKt o Kt per row group
+constexpr int DB = KTS + 2048;                   // [2][64] floats: dbeta per channel half
+constexpr int BAR = DB + 512;                    // 6 mbarriers
 constexpr int TSLOT = BAR + 48;
 constexpr int BYTES = TSLOT + 16;
 constexpr uint32_t TX_QKV = 6 * 8192, TX_G = 64 * 128 * 4, TX_IN2 = 2 * 8192 + 2 * 16384, TX_IN3 = 2 * 32768;
@@ -138,8 +138,6 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         bulk_g2s(sm + bl::DVN, dvn_img + slot * 16384, 16384, bar_in2);
     }
     if (tid < C) bet[tid] = tid < len ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
-    if (tid < 128) { kts[tid] = 0.f; }
-    if (tid < 64) dbs[tid] = 0.f;
     if (warp == 0) { tmem_alloc(tslot, 512); tmem_relinquish(); }
     bool ok = true;
     if (tid == 0) ok = mbar_wait(bar_g, 0);
@@ -228,7 +226,7 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     const uint32_t sb = smem_u32(sm);
     const uint32_t L16 = 16u << 16;                     // +16 lane tile
 
-    // ---- MMA-AP: [bKg ; Qg] Kinv^T -> cols 256-319 (A on lanes 0-63); then D_P, D_T ----
+    // ---- MMA-AP: [bKg ; Qg] Kinv^T -> cols 256-319 (A on lanes 0-63) ----
     if (tid == 0 && ok) {
         tc_fence_after();
         constexpr uint32_t ID = idesc_g(128, 64, false, false);
@@ -238,23 +236,6 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         for (int kk = 0; kk < 8; ++kk)
             umma_bf16_p(tmem + 256, a.lo + kmaj(kk, 16384), a.hi, b.lo + kmaj(kk, 8192), b.hi, ID, kk > 0);
         umma_commit(bar_mma);
-        // the two phase-2 products that need neither S nor dS' run while the
-        // CUDA cores form T: D_P = dO V_new^T (cols 320-383, +0) and
-        // D_T = dV_new (bV)^T (cols 320-383, +16); the phase-2a commit covers them
-        ok = mbar_wait(bar_in2, 0);
-        if (ok) {
-            constexpr uint32_t ID64 = idesc_g(64, 64, false, false);
-            const DescParts a_do = smem_desc_parts(sb + bl::DO, 16, 1024, 2);
-            const DescParts a_dvn = smem_desc_parts(sb + bl::DVN, 16, 1024, 2);
-            const DescParts b_vn = smem_desc_parts(sb + bl::VN, 16, 1024, 2);
-            const DescParts b_bv = smem_desc_parts(sb + bl::V, 16, 1024, 2);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                umma_bf16_p(tmem + 320, a_do.lo + kmaj(kk, 8192), a_do.hi, b_vn.lo + kmaj(kk, 8192), b_vn.hi, ID64, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                umma_bf16_p(tmem + 320 + L16, a_dvn.lo + kmaj(kk, 8192), a_dvn.hi, b_bv.lo + kmaj(kk, 8192), b_bv.hi, ID64, kk > 0);
-        }
     }
     ok = mma_done(ok);
 
@@ -320,12 +301,14 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     // ---- phase 2a products ----
     if (tid == 0 && ok) {
         tc_fence_after();
-        constexpr uint32_t ID128 = idesc_g(64, 128, false, false);
+        constexpr uint32_t ID128 = idesc_g(64, 128, false, false), ID64 = idesc_g(64, 64, false, false);
         const DescParts a_do = smem_desc_parts(sb + bl::DO, 16, 1024, 2);
         const DescParts a_dvn = smem_desc_parts(sb + bl::DVN, 16, 1024, 2);
         const DescParts a_vn = smem_desc_parts(sb + bl::VN, 16, 1024, 2);
         const DescParts b_s = smem_desc_parts(sb + bl::S, 16, 1024, 2);
         const DescParts b_ds = smem_desc_parts(sb + bl::DS, 16, 1024, 2);
+        const DescParts b_vn = smem_desc_parts(sb + bl::VN, 16, 1024, 2);
+        const DescParts b_bv = smem_desc_parts(sb + bl::V, 16, 1024, 2);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)      // D_Q = dO S^T
             umma_bf16_p(tmem + 0, a_do.lo + kmaj(kk, 8192), a_do.hi, b_s.lo + kmaj(kk, 16384), b_s.hi, ID128, kk > 0);
@@ -335,7 +318,13 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)      // D_Kt = V_new dS'^T
             umma_bf16_p(tmem + 128, a_vn.lo + kmaj(kk, 8192), a_vn.hi, b_ds.lo + kmaj(kk, 16384), b_ds.hi, ID128, kk > 0);
-        umma_commit(bar_mma);               // also covers D_P and D_T
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)      // D_P = dO V_new^T
+            umma_bf16_p(tmem + 256, a_do.lo + kmaj(kk, 8192), a_do.hi, b_vn.lo + kmaj(kk, 8192), b_vn.hi, ID64, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)      // D_T = dV_new (bV)^T
+            umma_bf16_p(tmem + 256 + L16, a_dvn.lo + kmaj(kk, 8192), a_dvn.hi, b_bv.lo + kmaj(kk, 8192), b_bv.hi, ID64, kk > 0);
+        umma_commit(bar_mma);
     }
     // de^{G_C} = rowsum(S o dS') from the bf16 images (two threads per channel row)
     if (ok) {
@@ -392,7 +381,7 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 #pragma unroll
             for (int c2 = 0; c2 < 2; ++c2) {
                 float x[32];
-                tmem_ld32(tmem + lane_base + 320 + 32 * c2, x);
+                tmem_ld32(tmem + lane_base + 256 + 32 * c2, x);
                 tmem_wait_ld();
                 if (!hi) {
 #pragma unroll
@@ -419,7 +408,7 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         const DescParts b_qg = smem_desc_parts(sb + bl::KQ + 8192, 16384, 1024, 2);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-            umma_bf16_p(tmem + 320 + L16, a_dw.lo + kmaj(kk, 8192), a_dw.hi, b_bkg.lo + kmaj(kk, 16384), b_bkg.hi,
+            umma_bf16_p(tmem + 256 + L16, a_dw.lo + kmaj(kk, 8192), a_dw.hi, b_bkg.lo + kmaj(kk, 16384), b_bkg.hi,
                         idesc_g(64, 64, false, false), 1);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
@@ -433,12 +422,12 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     }
     ok = mma_done(ok);
 
-    // ---- dT (lanes +16, cols 320-383) -> DT image ----
+    // ---- dT (lanes +16, cols 256-319) -> DT image ----
     if (ok && warp >= 4) {
 #pragma unroll
         for (int c2 = 0; c2 < 2; ++c2) {
             float x[32];
-            tmem_ld32(tmem + lane_base + 320 + 32 * c2, x);
+            tmem_ld32(tmem + lane_base + 256 + 32 * c2, x);
             tmem_wait_ld();
             if (hi) {
 #pragma unroll
@@ -612,7 +601,7 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 pv[0] = make_float4(ov[0], ov[1], ov[2], ov[3]); pv[1] = make_float4(ov[4], ov[5], ov[6], ov[7]);
             }
             // column sums over the half's 16 token rows (xor steps stay inside
-            // each half), one shared atomic per channel and half
+            // each half), one slot per channel and row group (no atomics)
 #pragma unroll
             for (int jj = 0; jj < 8; ++jj) {
                 float t = ktv[jj];
@@ -620,12 +609,12 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 t += __shfl_xor_sync(0xffffffffu, t, 2);
                 t += __shfl_xor_sync(0xffffffffu, t, 4);
                 t += __shfl_xor_sync(0xffffffffu, t, 8);
-                if (l16 == 0) atomicAdd(kts + cm + jj, t);
+                if (l16 == 0) kts[(warp & 3) * 128 + cm + jj] = t;
             }
         }
         // dbeta of the row: both halves' channels, both channel groups (csel)
         dbp += __shfl_xor_sync(0xffffffffu, dbp, 16);
-        if (hi == 0 && live) atomicAdd(dbs + i, dbp);
+        if (hi == 0 && live) dbs[csel * 64 + i] = dbp;
     }
     __syncthreads();
     // dg = reverse cumsum of dG inside the chunk, the G_C terms on the last
@@ -633,7 +622,8 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     // meeting once through shared memory (the upper half's total)
     if (ok) {
         const int c = tid & 127, hf = tid >> 7;
-        const float base_c = kts[c] + degc[c] * ex2_approx(G2[gsw(63, c)]);
+        const float base_c = (kts[c] + kts[128 + c]) + (kts[256 + c] + kts[384 + c]) +
+                             degc[c] * ex2_approx(G2[gsw(63, c)]);
         float up = base_c;
         if (hf) {
 #pragma unroll 8
@@ -649,7 +639,7 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             acc += dG[gsw(t, c)];
             if (t < len) dg[((size_t)(t0 + t) * H + h) * D + c] = acc;
         }
-        if (tid < len) dbeta[(size_t)(t0 + tid) * H + h] = dbs[tid];
+        if (tid < len) dbeta[(size_t)(t0 + tid) * H + h] = dbs[tid] + dbs[64 + tid];
     }
     if (!ok && tid == 0) {
         if (!bad) set_device_error(err, kErrWaitTimeout);

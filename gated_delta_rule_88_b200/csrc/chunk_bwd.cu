@@ -619,26 +619,25 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     __syncthreads();
     // dg = reverse cumsum of dG inside the chunk, the G_C terms on the last
     // row: two threads per channel, rows 32-63 (hf = 1) and 0-31 (hf = 0),
-    // meeting once through shared memory (the upper half's total)
+    // each scanning its 32 rows in registers; the lower half then adds the
+    // upper half's total, passed through shared memory
     if (ok) {
         const int c = tid & 127, hf = tid >> 7;
-        const float base_c = (kts[c] + kts[128 + c]) + (kts[256 + c] + kts[384 + c]) +
-                             degc[c] * ex2_approx(G2[gsw(63, c)]);
-        float up = base_c;
-        if (hf) {
-#pragma unroll 8
-            for (int t = 32; t < 64; ++t) up += dG[gsw(t, c)];
-        }
-        __syncthreads();                         // kts read by every thread
-        if (hf) kts[c] = up;
+        const int r0 = 32 * hf;
+        float x[32];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) x[t] = dG[gsw(r0 + t, c)];
+        if (hf) x[31] += (kts[c] + kts[128 + c]) + (kts[256 + c] + kts[384 + c]) +
+                         degc[c] * ex2_approx(G2[gsw(63, c)]);
+#pragma unroll
+        for (int t = 30; t >= 0; --t) x[t] += x[t + 1];
+        __syncthreads();                         // every thread has read kts
+        if (hf) kts[c] = x[0];
         __syncthreads();
-        float acc = hf ? base_c : kts[c];
-        const int t_hi = hf ? 63 : 31;
-#pragma unroll 8
-        for (int t = t_hi; t > t_hi - 32; --t) {
-            acc += dG[gsw(t, c)];
-            if (t < len) dg[((size_t)(t0 + t) * H + h) * D + c] = acc;
-        }
+        const float up = hf ? 0.f : kts[c];
+#pragma unroll
+        for (int t = 0; t < 32; ++t)
+            if (r0 + t < len) dg[((size_t)(t0 + r0 + t) * H + h) * D + c] = x[t] + up;
         if (tid < len) dbeta[(size_t)(t0 + tid) * H + h] = dbs[tid] + dbs[64 + tid];
     }
     if (!ok && tid == 0) {

@@ -92,9 +92,16 @@ _SRC = os.path.join(ROOT, "gated_delta_rule_88_b200", "csrc")
 PREFILL_SRC = ["chunk_prep.cu", "prep_common.cuh", "chunk_chain_tc.cu", "chunk_ws.h", "sm100.cuh",
                "common.cuh"]
 TRAFFIC = {
-    "prefill_t8192_h32_d128": {"files": PREFILL_SRC, "sha": "", "bytes": 0.0},
-    "prefill_t65536_h32_d128": {"files": PREFILL_SRC, "sha": "", "bytes": 0.0},
-    "varlen8_h32_d128_resume": {"files": PREFILL_SRC, "sha": "", "bytes": 0.0},
+    # prep read + write, chain read + write (ncu, one capture each)
+    "prefill_t8192_h32_d128": {"files": PREFILL_SRC, "sha": "928b340bc66bee09",
+                               "bytes": 336794368 + 255760384 + 304157440 + 49562880},
+    "prefill_t65536_h32_d128": {"files": PREFILL_SRC, "sha": "928b340bc66bee09",
+                                "bytes": 2693117952 + 2384294912 + 2483440640 + 521259008},
+    "varlen8_h32_d128_resume": {"files": PREFILL_SRC, "sha": "928b340bc66bee09",
+                                "bytes": 6035604992 + 5411583488 + 5477717504 + 1200050176},
+    # per call: prep, forward chain with images, reverse chain, per-chunk pass
+    "backward_chunk": {"files": PREFILL_SRC + ["chunk_chain_bwd.cu", "chunk_bwd.cu"], "sha": "56b917d26a13785c",
+                       "bytes": 2823976170},
     "decode": {"files": ["decode.cu", "common.cuh"], "sha": "4ceac309c0c18d2f",
                "bytes": (547.408128 + 480.674560) * 1e6},
     "decode_steps": {"files": ["decode_pipe.cu", "common.cuh", "sm100.cuh"], "sha": "d9cf376f965488af",
@@ -330,10 +337,20 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
 
-    if args.only_backward:
-        # profiling: just the chunked backward on its workload
-        bwd_inp = W.named_prefill(BWD_WORKLOAD).to(dev)
-        res = backward_leg(kda, bwd_inp, dev, dist, world, args, chunked=True)
+    if args.only_backward or args.only_decode:
+        # profiling: just the chunked backward (then the recurrent one), or
+        # just the three decode legs
+        if args.only_backward:
+            bwd_inp = W.named_prefill(BWD_WORKLOAD).to(dev)
+            res = {"backward_chunk": backward_leg(kda, bwd_inp, dev, dist, world, args, chunked=True),
+                   "backward": backward_leg(kda, bwd_inp, dev, dist, world, args)}
+        else:
+            res = {"decode": decode_leg(kda, W, dev, dist, world, args),
+                   "decode_steps": decode_steps_leg(kda, W, dev, dist, world, args),
+                   "decode_chunk": decode_steps_leg(kda, W, dev, dist, world, args, L=CHUNK_L,
+                                                    flags=kda.KDA_STEPS_CHUNK,
+                                                    kernel="decode_chunk_kernel",
+                                                    traffic_key="decode_chunk", ring=1)}
         if rank == 0:
             print(json.dumps(res), flush=True)
         if dist is not None:
@@ -662,7 +679,9 @@ def main():
                     help="sequences in the decode legs (a smaller case for profiling)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--only-backward", action="store_true",
-                    help="profiling: time only kda_chunk_bwd on the 8192-token workload")
+                    help="profiling: time only the backward legs (chunked, then recurrent)")
+    ap.add_argument("--only-decode", action="store_true",
+                    help="profiling: time only the three decode legs")
     ap.add_argument("--only-prefill", metavar="WORKLOAD", default=None,
                     help="profiling: time only kda_chunk_fwd on this named workload "
                          "(e.g. varlen8_h32_d128_resume) and print its line")

@@ -343,6 +343,8 @@ def run_ours(args):
         if args.only_backward:
             bwd_inp = W.named_prefill(BWD_WORKLOAD).to(dev)
             res = {"backward_chunk": backward_leg(kda, bwd_inp, dev, dist, world, args, chunked=True),
+                   "backward_chunk_saved": backward_leg(kda, bwd_inp, dev, dist, world, args,
+                                                        saved=True),
                    "backward": backward_leg(kda, bwd_inp, dev, dist, world, args)}
         else:
             res = {"decode": decode_leg(kda, W, dev, dist, world, args),
@@ -430,6 +432,7 @@ def run_ours(args):
         bwd_inp = W.named_prefill(BWD_WORKLOAD).to(dev)
         bwd = backward_leg(kda, bwd_inp, dev, dist, world, args)
         bwd_chunk = backward_leg(kda, bwd_inp, dev, dist, world, args, chunked=True)
+        bwd_saved = backward_leg(kda, bwd_inp, dev, dist, world, args, saved=True)
         del bwd_inp
     clk.samples += clk_dec.samples
     clk.reasons |= clk_dec.reasons
@@ -458,6 +461,7 @@ def run_ours(args):
         "decode_chunk": dec_chunk,
         "backward": bwd,
         "backward_chunk": bwd_chunk,
+        "backward_chunk_saved": bwd_saved,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(inp_cpu)
@@ -565,27 +569,42 @@ BWD_T = 8192
 BWD_BYTES = BWD_T * H * (4 * D * 2 + D * 4 + 4 + 4 * D * 4 + 4)
 
 
-def backward_leg(kda, inp, dev, dist, world, args, chunked=False):
+def backward_leg(kda, inp, dev, dist, world, args, chunked=False, saved=False):
     """Training backward on the 8192-token workload with a seeded output
     gradient; no initial or final state.  chunked: kda_chunk_bwd (tensor
-    cores), else kda_recurrent_bwd."""
+    cores), else kda_recurrent_bwd; saved: kda_chunk_bwd from the
+    intermediates of one kda_chunk_fwd_save (whose time is reported too)."""
     gen = torch.Generator().manual_seed(41)
     do = torch.randn(1, BWD_T, H, D, generator=gen).to(torch.bfloat16).to(dev)
-    fn = kda.kda_chunk_bwd if chunked else kda.kda_recurrent_bwd
-    run = lambda: fn(inp.q, inp.k, inp.v, inp.g, inp.beta, do, want_initial_state_grad=False)
-    calls = 3 if not chunked else 10
-    ms = time_calls(run, calls, max(1, min(args.warmup, 3)), torch.cuda.current_stream(dev), dist)
+    stream = torch.cuda.current_stream(dev)
+    extra = {}
+    if saved:
+        out, _, sv = kda.kda_chunk_fwd_save(inp.q, inp.k, inp.v, inp.g, inp.beta,
+                                            output_final_state=False)
+        fwd = lambda: kda.kda_chunk_fwd_save(inp.q, inp.k, inp.v, inp.g, inp.beta, out=out,
+                                             output_final_state=False, saved=sv)
+        extra["forward_save_ms"] = time_calls(fwd, 10, 2, stream, dist)
+        run = lambda: kda.kda_chunk_bwd(inp.q, inp.k, inp.v, inp.g, inp.beta, do,
+                                        want_initial_state_grad=False, saved=sv)
+    else:
+        fn = kda.kda_chunk_bwd if chunked else kda.kda_recurrent_bwd
+        run = lambda: fn(inp.q, inp.k, inp.v, inp.g, inp.beta, do, want_initial_state_grad=False)
+    calls = 3 if not (chunked or saved) else 10
+    ms = time_calls(run, calls, max(1, min(args.warmup, 3)), stream, dist)
     assert kda.kda_get_device_error() == 0
     peak, kind = measured_peak_hbm()
     ach = BWD_BYTES / (ms * 1e-3) / 1e9
-    if chunked:
+    if saved:
+        bound, kernel = "hbm", "kda_chunk_bwd from saved intermediates (reverse chain, per-chunk pass)"
+        traffic = None
+    elif chunked:
         bound, kernel = "hbm", "kda_chunk_bwd (prep, chain, reverse chain, per-chunk pass)"
         traffic = measured_traffic("backward_chunk")
     else:
         bound, kernel = "latency (sequential per token)", "recurrent_bwd_kernel"
         traffic = measured_traffic("backward")
     return {"workload": BWD_WORKLOAD + "_backward", "value": job_value(BWD_T, world, ms),
-            "unit": UNIT, "ms_per_call": ms, "calls": calls,
+            "unit": UNIT, "ms_per_call": ms, "calls": calls, **extra,
             "roofline": {"bound": bound, "kernel": kernel,
                          "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                          "peak_source": kind, "algorithmic_bytes_per_launch": BWD_BYTES,

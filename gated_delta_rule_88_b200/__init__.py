@@ -24,7 +24,10 @@ Entry points (same names as the C ABI):
     kda_gated_rmsnorm(x, gate, weight, eps=1e-5, out=None) -> out
     kda_recurrent_bwd(q, k, v, g, beta, do, initial_state=None, dsT=None)
         -> (dq, dk, dv, dg, dbeta, ds0)
-    kda_chunk_bwd(..., cu_seqlens=None): the same gradients by the chunked form
+    kda_chunk_fwd_save(q, k, v, g, beta, initial_state=None, cu_seqlens=None, ...)
+        -> (out, final_state, saved): kda_chunk_fwd that also keeps the
+        intermediates for the backward (a uint8 CUDA tensor)
+    kda_chunk_bwd(..., cu_seqlens=None, saved=None): the same gradients by the chunked form
                      (bf16, dk = dv = 128; tensor cores)
     kda_state_affine(M, B, S_in, out=None) -> S_out
     kda_get_device_error(stream=None) -> int
@@ -42,7 +45,8 @@ import torch
 __all__ = ["kda_chunk_fwd", "kda_chunk_fwd_ex", "kda_chunk_fwd_host", "kda_chunk_fwd_noalloc",
            "kda_recurrent_step",
            "kda_recurrent_step_ex", "kda_recurrent_steps", "kda_gated_rmsnorm", "kda_state_affine",
-           "kda_recurrent_bwd", "kda_chunk_bwd",
+           "kda_recurrent_bwd", "kda_chunk_bwd", "kda_chunk_fwd_save", "kda_chunk_saved_bytes",
+           "kda_chunk_bwd_saved",
            "kda_get_device_error", "kda_selftest_bounded_wait",
            "KDAError",
            "KDA_QK_L2NORM", "KDA_BETA_SIGMOID", "KDA_STEPS_CHUNK",
@@ -100,6 +104,13 @@ def load_library():
         lib.kda_recurrent_bwd.restype = i
         lib.kda_chunk_bwd.argtypes = [vp] * 15 + [i] * 7 + [vp]
         lib.kda_chunk_bwd.restype = i
+        ll = ctypes.c_longlong
+        lib.kda_chunk_bwd_saved.argtypes = [vp] * 15 + [i] * 7 + [vp, ll, vp]
+        lib.kda_chunk_bwd_saved.restype = i
+        lib.kda_chunk_fwd_save.argtypes = [vp] * 9 + [i] * 7 + [vp, ll, vp]
+        lib.kda_chunk_fwd_save.restype = i
+        lib.kda_chunk_saved_bytes.argtypes = [i] * 5
+        lib.kda_chunk_saved_bytes.restype = ll
         lib.kda_state_affine.restype = i
         lib.kda_get_device_error.argtypes = [vp, ctypes.POINTER(i)]
         lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp]
@@ -400,11 +411,60 @@ def kda_recurrent_bwd(q, k, v, g, beta, do, initial_state=None, dsT=None,
     return dq, dk_, dv_, dg, db, ds0
 
 
+def kda_chunk_saved_bytes(B: int, T: int, H: int, num_seqs: int = 0, varlen: bool = False) -> int:
+    """Bytes of the forward intermediates kda_chunk_fwd_save keeps."""
+    n = load_library().kda_chunk_saved_bytes(int(B), int(T), int(H), int(num_seqs), int(bool(varlen)))
+    if n < 0:
+        raise ValueError("kda_chunk_saved_bytes: bad sizes")
+    return int(n)
+
+
+def kda_chunk_fwd_save(q, k, v, g, beta, initial_state=None, cu_seqlens=None, out=None,
+                       final_state=None, output_final_state: bool = True, saved=None):
+    """kda_chunk_fwd (bf16, dk = dv = 128) that also writes the intermediates
+    the chunked backward needs into ``saved`` (allocated here if None).
+    Returns (out, final_state, saved); pass ``saved`` to kda_chunk_bwd."""
+    lib = load_library()
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("kda_chunk_fwd_save needs CUDA tensors (no CPU path)")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, name in ((k, "k"), (v, "v")):
+        _need(t, name, dev, q.dtype)
+    _need(q, "q", dev)
+    _need(g, "g", dev, torch.float32)
+    _need(beta, "beta", dev, torch.float32)
+    N = B
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", dev, torch.int32)
+        N = cu_seqlens.numel() - 1
+    if initial_state is not None:
+        _need(initial_state, "initial_state", dev, torch.float32)
+    nbytes = kda_chunk_saved_bytes(B, T, H, N, cu_seqlens is not None)
+    if saved is None:
+        saved = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    else:
+        _need(saved, "saved", dev, torch.uint8)
+    if out is None:
+        out = torch.empty(B, T, H, dv, dtype=q.dtype, device=dev)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib.kda_chunk_fwd_save(_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta),
+                                    _dptr(initial_state), _dptr(cu_seqlens), _dptr(out),
+                                    _dptr(final_state), B, T, H, dk, dv, N, _dtype_code(q),
+                                    _dptr(saved), saved.numel(), _stream_handle(dev))
+    _check(rc)
+    return out, final_state, saved
+
+
 def kda_chunk_bwd(q, k, v, g, beta, do, initial_state=None, dsT=None, cu_seqlens=None,
-                  want_initial_state_grad: bool = True):
+                  want_initial_state_grad: bool = True, saved=None):
     """Gradients by the chunked form on the tensor cores (bf16, dk = dv = 128):
     arguments and results as kda_recurrent_bwd, plus cu_seqlens (varlen, B == 1;
-    states then [N,H,dk,dv])."""
+    states then [N,H,dk,dv]) and ``saved`` (from kda_chunk_fwd_save on the same
+    inputs: the forward is then not recomputed)."""
     lib = load_library()
     dev = q.device
     if dev.type != "cuda":
@@ -424,18 +484,30 @@ def kda_chunk_bwd(q, k, v, g, beta, do, initial_state=None, dsT=None, cu_seqlens
     for t, name in ((initial_state, "initial_state"), (dsT, "dsT")):
         if t is not None:
             _need(t, name, dev, torch.float32)
+    if saved is not None:
+        _need(saved, "saved", dev, torch.uint8)
     f32 = dict(dtype=torch.float32, device=dev)
     dq, dk_, dg = (torch.empty(B, T, H, dk, **f32) for _ in range(3))
     dv_ = torch.empty(B, T, H, dv, **f32)
     db = torch.empty(B, T, H, **f32)
     ds0 = torch.empty(N, H, dk, dv, **f32) if want_initial_state_grad else None
+    args = (_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta), _dptr(initial_state),
+            _dptr(cu_seqlens), _dptr(do), _dptr(dsT), _dptr(dq), _dptr(dk_), _dptr(dv_), _dptr(dg),
+            _dptr(db), _dptr(ds0), B, T, H, dk, dv, N, dt)
     with torch.cuda.device(dev):
-        rc = lib.kda_chunk_bwd(_dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta),
-                               _dptr(initial_state), _dptr(cu_seqlens), _dptr(do), _dptr(dsT),
-                               _dptr(dq), _dptr(dk_), _dptr(dv_), _dptr(dg), _dptr(db), _dptr(ds0),
-                               B, T, H, dk, dv, N, dt, _stream_handle(dev))
+        if saved is None:
+            rc = lib.kda_chunk_bwd(*args, _stream_handle(dev))
+        else:
+            rc = lib.kda_chunk_bwd_saved(*args, _dptr(saved), saved.numel(), _stream_handle(dev))
     _check(rc)
     return dq, dk_, dv_, dg, db, ds0
+
+
+def kda_chunk_bwd_saved(q, k, v, g, beta, do, saved, initial_state=None, dsT=None,
+                        cu_seqlens=None, want_initial_state_grad: bool = True):
+    """kda_chunk_bwd given the intermediates of kda_chunk_fwd_save."""
+    return kda_chunk_bwd(q, k, v, g, beta, do, initial_state, dsT, cu_seqlens,
+                         want_initial_state_grad, saved=saved)
 
 
 def kda_state_affine(M, B, S_in, out=None):

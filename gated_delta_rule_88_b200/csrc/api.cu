@@ -435,44 +435,77 @@ extern "C" kda_status kda_gated_rmsnorm(const void *x, const void *gate, const f
     return KDA_OK;
 }
 
-extern "C" kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const float *g,
-                                    const float *beta, const float *initial_state,
-                                    const int32_t *cu_seqlens, const void *dout,
-                                    const float *dfinal_state, float *dq, float *dk, float *dv,
-                                    float *dg, float *dbeta, float *dinitial_state, int B, int T,
-                                    int H, int dk_, int dv_, int num_seqs, kda_dtype dtype,
-                                    void *stream) {
-    t_msg[0] = 0;
+// Saved forward intermediates for the chunked backward (kda_chunk_fwd_save):
+// the plan (chunk offsets and sequence order), then per (chunk slot, head)
+// the record (74,240 B), then the bf16 images of the state entering each
+// chunk (32 KiB) and of V_new (16 KiB).
+namespace {
+struct SavedLayout {
+    long long max_chunks = 0;
+    size_t plan = 0, records = 0, s_img = 0, v_img = 0, total = 0;
+};
+SavedLayout saved_layout(int N, int B, int T, int H, bool varlen) {
+    SavedLayout L;
+    const long long total_T = (long long)B * T;
+    L.max_chunks = varlen ? (total_T + 63) / 64 + N : (long long)B * ((T + 63) / 64);
+    const size_t slots = (size_t)L.max_chunks * H;
+    L.plan = 0;
+    L.records = (((size_t)2 * N + 1) * sizeof(int32_t) + 255) & ~(size_t)255;
+    L.s_img = L.records + slots * kda::ws::RECORD;
+    L.v_img = L.s_img + slots * 32768;
+    L.total = L.v_img + slots * 16384;
+    return L;
+}
+
+// Argument rules shared by kda_chunk_bwd and kda_chunk_bwd_saved.
+kda_status check_chunk_bwd_args(const char *fn, const void *q, const void *k, const void *v,
+                                const float *g, const float *beta, const float *initial_state,
+                                const int32_t *cu_seqlens, const void *dout,
+                                const float *dfinal_state, const float *dq, const float *dk,
+                                const float *dv, const float *dg, const float *dbeta,
+                                const float *dinitial_state, int B, int T, int H, int dk_,
+                                int dv_, int num_seqs, kda_dtype dtype, int *N_out) {
     if (!q || !k || !v || !g || !beta || !dout || !dq || !dk || !dv || !dg || !dbeta)
-        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: null pointer argument");
+        return fail(KDA_ERR_INVALID_ARG, "%s: null pointer argument", fn);
     if (B <= 0 || T < 0 || H <= 0 || dk_ <= 0 || dv_ <= 0 || B > 65535 || H > 65535)
-        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: bad sizes B=%d T=%d H=%d dk=%d dv=%d", B,
-                    T, H, dk_, dv_);
+        return fail(KDA_ERR_INVALID_ARG, "%s: bad sizes B=%d T=%d H=%d dk=%d dv=%d", fn, B, T, H,
+                    dk_, dv_);
     if (dtype != KDA_F32 && dtype != KDA_BF16)
-        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: unknown dtype %d", (int)dtype);
+        return fail(KDA_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, (int)dtype);
     if (dtype != KDA_BF16 || dk_ != 128 || dv_ != 128)
         return fail(KDA_ERR_UNSUPPORTED,
-                    "kda_chunk_bwd: dtype=%d dk=%d dv=%d (supported: bf16 with dk = dv = 128)",
+                    "%s: dtype=%d dk=%d dv=%d (supported: bf16 with dk = dv = 128)", fn,
                     (int)dtype, dk_, dv_);
     int N = B;
     if (cu_seqlens) {
         if (B != 1)
-            return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: varlen mode requires B == 1 (got %d)", B);
+            return fail(KDA_ERR_INVALID_ARG, "%s: varlen mode requires B == 1 (got %d)", fn, B);
         if (num_seqs <= 0 || num_seqs > 65535)
-            return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: num_seqs=%d out of [1, 65535]", num_seqs);
+            return fail(KDA_ERR_INVALID_ARG, "%s: num_seqs=%d out of [1, 65535]", fn, num_seqs);
         N = num_seqs;
     }
     const void *ptrs[] = {q, k, v, g, dout, dq, dk, dv, dg, initial_state, dfinal_state, dinitial_state};
     for (const void *p : ptrs)
         if (p && !aligned16(p))
-            return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: pointers must be 16-byte aligned");
+            return fail(KDA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", fn);
     if (((uintptr_t)beta & 3u) || ((uintptr_t)dbeta & 3u) || ((uintptr_t)cu_seqlens & 3u))
-        return fail(KDA_ERR_INVALID_ARG,
-                    "kda_chunk_bwd: beta, dbeta and cu_seqlens must be 4-byte aligned");
+        return fail(KDA_ERR_INVALID_ARG, "%s: beta, dbeta and cu_seqlens must be 4-byte aligned", fn);
     const long long total_T = (long long)B * T;
     if (total_T > 0x7fffffffLL || total_T * H > (1LL << 34))
-        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: problem too large (B*T=%lld)", total_T);
-    cudaStream_t st = (cudaStream_t)stream;
+        return fail(KDA_ERR_INVALID_ARG, "%s: problem too large (B*T=%lld)", fn, total_T);
+    *N_out = N;
+    return KDA_OK;
+}
+
+// The backward's launches; saved (nullable) holds the forward's plan,
+// records and images (kda_chunk_fwd_save), else they are recomputed.
+kda_status chunk_bwd_run(const char *fn, const void *q, const void *k, const void *v,
+                         const float *g, const float *beta, const float *initial_state,
+                         const int32_t *cu_seqlens, const void *dout, const float *dfinal_state,
+                         float *dq, float *dk, float *dv, float *dg, float *dbeta,
+                         float *dinitial_state, int B, int T, int H, int N,
+                         const unsigned char *saved, cudaStream_t st) {
+    const long long total_T = (long long)B * T;
     const size_t sbytes = (size_t)N * H * 128 * 128 * sizeof(float);
     if (total_T == 0) {
         // no tokens: the initial state's gradient is the final state's
@@ -481,50 +514,154 @@ extern "C" kda_status kda_chunk_bwd(const void *q, const void *k, const void *v,
             e = dfinal_state ? cudaMemcpyAsync(dinitial_state, dfinal_state, sbytes,
                                                cudaMemcpyDeviceToDevice, st)
                              : cudaMemsetAsync(dinitial_state, 0, sbytes, st);
-        return e == cudaSuccess ? KDA_OK : cuda_fail(e, "kda_chunk_bwd empty input");
+        return e == cudaSuccess ? KDA_OK : cuda_fail(e, fn);
     }
-    const long long max_chunks = cu_seqlens ? (total_T + 63) / 64 + N : (long long)B * ((T + 63) / 64);
-    const size_t slots = (size_t)max_chunks * H;
-    const size_t coff_bytes = (((size_t)N + 1) * sizeof(int32_t) + 255) & ~(size_t)255;
-    const size_t bytes = coff_bytes + slots * (kda::ws::RECORD + 2 * 32768 + 2 * 16384);
+    const SavedLayout L = saved_layout(N, B, T, H, cu_seqlens != nullptr);
+    const size_t slots = (size_t)L.max_chunks * H;
+    // scratch: the gradient images, and (recompute) a copy of the saved layout
+    const size_t bytes = slots * (32768 + 16384) + (saved ? 0 : L.total);
     cudaMemPool_t pool;
     int sms = 148;
     cudaError_t e = get_pool(&pool, &sms);
-    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_bwd memory pool");
+    if (e != cudaSuccess) return cuda_fail(e, fn);
     void *scratch = nullptr;
     e = cudaMallocFromPoolAsync(&scratch, bytes, pool, st);
-    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_bwd scratch allocation");
-    int32_t *coff = (int32_t *)scratch;
-    unsigned char *records = (unsigned char *)scratch + coff_bytes;
-    unsigned char *s_img = records + slots * kda::ws::RECORD;
-    unsigned char *dsp_img = s_img + slots * 32768;
-    unsigned char *v_img = dsp_img + slots * 32768;
-    unsigned char *dvn_img = v_img + slots * 16384;
-    kda::Prologue pro{0, 1.f};
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    unsigned char *dsp_img = (unsigned char *)scratch;
+    unsigned char *dvn_img = dsp_img + slots * 32768;
+    unsigned char *fwd = saved ? nullptr : dvn_img + slots * 16384;
+    const unsigned char *base = saved ? saved : fwd;
+    const int32_t *coff = (const int32_t *)(base + L.plan);
+    const unsigned char *records = base + L.records;
+    const unsigned char *s_img = base + L.s_img, *v_img = base + L.v_img;
     int *err = kda::error_word();
-    if (cu_seqlens) e = kda::launch_chunk_plan(cu_seqlens, N, (int)total_T, coff, st);
-    // forward recompute: records, then the chain storing S and V_new per chunk
-    if (e == cudaSuccess)
-        e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, cu_seqlens ? coff : nullptr, N, T,
-                                   (int)total_T, H, (int)max_chunks, records, pro, err, st);
-    if (e == cudaSuccess)
-        e = kda::launch_chunk_chain(records, cu_seqlens, cu_seqlens ? coff : nullptr, initial_state,
-                                    nullptr, nullptr, N, T, (int)total_T, H, 32, (int)max_chunks, err,
-                                    st, s_img, v_img);
+    if (!saved) {
+        // forward recompute: plan, records, then the chain storing S and V_new per chunk
+        kda::Prologue pro{0, 1.f};
+        if (cu_seqlens) e = kda::launch_chunk_plan(cu_seqlens, N, (int)total_T, (int32_t *)coff, st);
+        if (e == cudaSuccess)
+            e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, cu_seqlens ? coff : nullptr, N,
+                                       T, (int)total_T, H, (int)L.max_chunks,
+                                       fwd + L.records, pro, err, st);
+        if (e == cudaSuccess)
+            e = kda::launch_chunk_chain(records, cu_seqlens, cu_seqlens ? coff : nullptr,
+                                        initial_state, nullptr, nullptr, N, T, (int)total_T, H, 32,
+                                        (int)L.max_chunks, err, st, fwd + L.s_img, fwd + L.v_img);
+    }
     // reverse chain, then the per-(chunk, head) gradients
     if (e == cudaSuccess)
         e = kda::launch_chunk_chain_bwd(dout, records, cu_seqlens, cu_seqlens ? coff : nullptr,
                                         dfinal_state, dinitial_state, dsp_img, dvn_img, N, T,
-                                        (int)total_T, H, (int)max_chunks, err, st);
+                                        (int)total_T, H, (int)L.max_chunks, err, st);
     if (e == cudaSuccess)
         e = kda::launch_chunk_bwd_local(q, k, v, g, beta, dout, cu_seqlens,
                                         cu_seqlens ? coff : nullptr, N, T, (int)total_T, H,
-                                        (int)max_chunks, s_img, v_img, dsp_img, dvn_img, dq, dk, dv,
-                                        dg, dbeta, err, st);
+                                        (int)L.max_chunks, s_img, v_img, dsp_img, dvn_img, dq, dk,
+                                        dv, dg, dbeta, err, st);
     cudaError_t e2 = cudaFreeAsync(scratch, st);
-    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_bwd launch");
-    if (e2 != cudaSuccess) return cuda_fail(e2, "kda_chunk_bwd scratch release");
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    if (e2 != cudaSuccess) return cuda_fail(e2, fn);
     return KDA_OK;
+}
+}  // namespace
+
+extern "C" kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const float *g,
+                                    const float *beta, const float *initial_state,
+                                    const int32_t *cu_seqlens, const void *dout,
+                                    const float *dfinal_state, float *dq, float *dk, float *dv,
+                                    float *dg, float *dbeta, float *dinitial_state, int B, int T,
+                                    int H, int dk_, int dv_, int num_seqs, kda_dtype dtype,
+                                    void *stream) {
+    t_msg[0] = 0;
+    int N = 0;
+    kda_status s = check_chunk_bwd_args("kda_chunk_bwd", q, k, v, g, beta, initial_state, cu_seqlens,
+                                        dout, dfinal_state, dq, dk, dv, dg, dbeta, dinitial_state, B,
+                                        T, H, dk_, dv_, num_seqs, dtype, &N);
+    if (s != KDA_OK) return s;
+    return chunk_bwd_run("kda_chunk_bwd", q, k, v, g, beta, initial_state, cu_seqlens, dout,
+                         dfinal_state, dq, dk, dv, dg, dbeta, dinitial_state, B, T, H, N, nullptr,
+                         (cudaStream_t)stream);
+}
+
+extern "C" long long kda_chunk_saved_bytes(int B, int T, int H, int num_seqs, int varlen) {
+    if (B <= 0 || T < 0 || H <= 0 || B > 65535 || H > 65535 || (varlen && (B != 1 || num_seqs <= 0 ||
+                                                                              num_seqs > 65535)))
+        return -1;
+    if ((long long)B * T > 0x7fffffffLL) return -1;
+    return (long long)saved_layout(varlen ? num_seqs : B, B, T, H, varlen != 0).total;
+}
+
+extern "C" kda_status kda_chunk_fwd_save(const void *q, const void *k, const void *v,
+                                         const float *g, const float *beta,
+                                         const float *initial_state, const int32_t *cu_seqlens,
+                                         void *out, float *final_state, int B, int T, int H,
+                                         int dk, int dv, int num_seqs, kda_dtype dtype, void *saved,
+                                         long long saved_bytes, void *stream) {
+    t_msg[0] = 0;
+    int N = 0;
+    kda_status s = kda::check_chunk_fwd_args("kda_chunk_fwd_save", q, k, v, g, beta, initial_state,
+                                             cu_seqlens, out, final_state, B, T, H, dk, dv,
+                                             num_seqs, dtype, &N);
+    if (s != KDA_OK) return s;
+    if (dtype != KDA_BF16 || dk != 128 || dv != 128)
+        return fail(KDA_ERR_UNSUPPORTED,
+                    "kda_chunk_fwd_save: only bf16 with dk = dv = 128 (got dtype %d, %d, %d)",
+                    (int)dtype, dk, dv);
+    const SavedLayout L = saved_layout(N, B, T, H, cu_seqlens != nullptr);
+    if (!saved || ((uintptr_t)saved & 255u))
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_save: saved must be 256-byte aligned");
+    if (saved_bytes < (long long)L.total)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_save: saved holds %lld bytes, needs %zu",
+                    saved_bytes, L.total);
+    cudaStream_t st = (cudaStream_t)stream;
+    const long long total_T = (long long)B * T;
+    if (total_T == 0) {
+        cudaError_t e = kda::bf16_prefill_no_tokens(initial_state, final_state, N, H, st);
+        return e == cudaSuccess ? KDA_OK : cuda_fail(e, "kda_chunk_fwd_save empty input");
+    }
+    unsigned char *base = (unsigned char *)saved;
+    int32_t *coff = (int32_t *)(base + L.plan);
+    int32_t *order = cu_seqlens ? coff + N + 1 : nullptr;
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int dvt = kda::bf16_prefill_dvt((long long)N * H, sms);
+    int *err = kda::error_word();
+    cudaError_t e = cudaSuccess;
+    if (cu_seqlens) e = kda::launch_chunk_plan(cu_seqlens, N, (int)total_T, coff, st, order);
+    if (e == cudaSuccess)
+        e = kda::launch_chunk_prep(q, k, v, g, beta, cu_seqlens, coff, N, T, (int)total_T, H,
+                                   (int)L.max_chunks, base + L.records, kda::Prologue{0, 1.f}, err, st);
+    if (e == cudaSuccess)
+        e = kda::launch_chunk_chain(base + L.records, cu_seqlens, coff, initial_state, final_state,
+                                    out, N, T, (int)total_T, H, dvt, (int)L.max_chunks, err, st,
+                                    base + L.s_img, base + L.v_img, order);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_save launch");
+    return KDA_OK;
+}
+
+extern "C" kda_status kda_chunk_bwd_saved(const void *q, const void *k, const void *v,
+                                          const float *g, const float *beta,
+                                          const float *initial_state, const int32_t *cu_seqlens,
+                                          const void *dout, const float *dfinal_state, float *dq,
+                                          float *dk, float *dv, float *dg, float *dbeta,
+                                          float *dinitial_state, int B, int T, int H, int dk_,
+                                          int dv_, int num_seqs, kda_dtype dtype,
+                                          const void *saved, long long saved_bytes, void *stream) {
+    t_msg[0] = 0;
+    int N = 0;
+    kda_status s = check_chunk_bwd_args("kda_chunk_bwd_saved", q, k, v, g, beta, initial_state,
+                                        cu_seqlens, dout, dfinal_state, dq, dk, dv, dg, dbeta,
+                                        dinitial_state, B, T, H, dk_, dv_, num_seqs, dtype, &N);
+    if (s != KDA_OK) return s;
+    const SavedLayout L = saved_layout(N, B, T, H, cu_seqlens != nullptr);
+    if (!saved || ((uintptr_t)saved & 255u))
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd_saved: saved must be 256-byte aligned");
+    if (saved_bytes < (long long)L.total)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd_saved: saved holds %lld bytes, needs %zu",
+                    saved_bytes, L.total);
+    return chunk_bwd_run("kda_chunk_bwd_saved", q, k, v, g, beta, initial_state, cu_seqlens, dout,
+                         dfinal_state, dq, dk, dv, dg, dbeta, dinitial_state, B, T, H, N,
+                         (const unsigned char *)saved, (cudaStream_t)stream);
 }
 
 extern "C" kda_status kda_recurrent_bwd(const void *q, const void *k, const void *v,

@@ -351,6 +351,48 @@ kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const floa
                          int num_seqs, kda_dtype dtype, void *stream);
 
 /*
+ * kda_chunk_fwd_save, kda_chunk_bwd_saved -- a training step that keeps the
+ * forward's intermediates for the backward instead of recomputing them.
+ *
+ * Source: Kimi Linear paper notes (paper-notes-site), section 3: the chunked
+ * forward used in training saves its intermediates (the decay cumsum, the
+ * A/P blocks, w, u, the decayed q and k, v_new and the chunk states) so
+ * that the backward can use them; the same role here is played by the
+ * per-(chunk, head) records, the bf16 state entering each chunk and V_new.
+ *
+ * kda_chunk_saved_bytes: bytes of the intermediates for a call of these
+ *   sizes (varlen = 0: dense [B, T]; varlen = 1: B == 1 and num_seqs
+ *   sequences); -1 for bad sizes.  About 122 KB per (64-token chunk, head):
+ *   500 MB for T = 8192, H = 32.
+ * kda_chunk_fwd_save: kda_chunk_fwd (same arguments, layouts, results;
+ *   KDA_BF16 with dk = dv = 128 only) that also writes the intermediates into
+ *   `saved` (device memory, 256-byte aligned, at least saved_bytes >=
+ *   kda_chunk_saved_bytes; the caller owns it).  It allocates nothing.
+ * kda_chunk_bwd_saved: kda_chunk_bwd (same arguments and results) given the
+ *   `saved` buffer of a kda_chunk_fwd_save call on the SAME inputs,
+ *   initial_state and cu_seqlens (nothing checks this; other contents give
+ *   wrong gradients); it skips recomputing the forward.  The gradients are
+ *   bitwise equal to kda_chunk_bwd's.  Scratch for the reverse chain's
+ *   images (48 KB per (chunk, head)) comes from the library pool.
+ * Errors: as kda_chunk_fwd / kda_chunk_bwd, plus KDA_ERR_INVALID_ARG for a
+ *   null, misaligned or too small `saved`.
+ */
+long long kda_chunk_saved_bytes(int B, int T, int H, int num_seqs, int varlen);
+kda_status kda_chunk_fwd_save(const void *q, const void *k, const void *v,
+                              const float *g, const float *beta,
+                              const float *initial_state, const int32_t *cu_seqlens,
+                              void *out, float *final_state,
+                              int B, int T, int H, int dk, int dv, int num_seqs,
+                              kda_dtype dtype, void *saved, long long saved_bytes, void *stream);
+kda_status kda_chunk_bwd_saved(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, const float *initial_state,
+                               const int32_t *cu_seqlens, const void *dout,
+                               const float *dfinal_state, float *dq, float *dk, float *dv,
+                               float *dg, float *dbeta, float *dinitial_state, int B, int T,
+                               int H, int dk_, int dv_, int num_seqs, kda_dtype dtype,
+                               const void *saved, long long saved_bytes, void *stream);
+
+/*
  * kda_state_affine -- S_out = M S_in + B for `count` independent blocks.
  *
  * Source: the recurrence of the paper notes (section 2) is affine in the

@@ -291,3 +291,27 @@ def test_chunk_bwd_bad_arguments_rejected(lib, kw):
 @pytest.mark.parametrize("kw", [dict(d_k=64), dict(d_v=64), dict(dtype=0)])
 def test_chunk_bwd_unsupported_rejected(lib, kw):
     assert cbwd(lib, **kw) == 2
+
+
+def test_saved_bytes_rule(lib):
+    lib.kda_chunk_saved_bytes.restype = ctypes.c_longlong
+    per = 74240 + 32768 + 16384
+    # dense: B * ceil(T / 64) chunk slots per head, plus the 256-byte plan
+    assert lib.kda_chunk_saved_bytes(2, 130, 3, 0, 0) == 256 + 2 * 3 * 3 * per
+    # varlen: ceil(T / 64) + num_seqs slots
+    assert lib.kda_chunk_saved_bytes(1, 300, 2, 4, 1) == 256 + (5 + 4) * 2 * per
+    for bad in ((0, 64, 1, 0, 0), (1, -1, 1, 0, 0), (2, 64, 1, 3, 1), (1, 64, 1, 0, 1)):
+        assert lib.kda_chunk_saved_bytes(*bad) == -1
+
+
+def save_fwd(lib, *, saved=FAKE, nbytes=1 << 30, T=64, dtype=1, dk=128):
+    P = ctypes.c_void_p
+    lib.kda_chunk_fwd_save.argtypes = [P] * 9 + [ctypes.c_int] * 7 + [P, ctypes.c_longlong, P]
+    return lib.kda_chunk_fwd_save(P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), None, None, P(FAKE),
+                                  None, 1, T, 1, dk, 128, 1, dtype, P(saved), nbytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [(dict(saved=0), 1), (dict(saved=FAKE + 16), 1),
+                                     (dict(nbytes=1000), 1), (dict(dtype=0), 2), (dict(dk=64), 2)])
+def test_save_fwd_bad_arguments_rejected(lib, kw, code):
+    assert save_fwd(lib, **kw) == code

@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import oracle
-from gated_delta_rule_88_b200 import kda_chunk_bwd, kda_recurrent_bwd
+from gated_delta_rule_88_b200 import kda_chunk_bwd, kda_get_device_error, kda_recurrent_bwd
 from gated_delta_rule_88_b200 import workloads as W
 from helpers import rel_inf
 
@@ -70,3 +70,35 @@ def test_chunk_bwd_matches_recurrent_bwd_full_size_sampled():
                               inp.initial_state[:, h:h + 1].contiguous(), dsT[:, h:h + 1].contiguous())
         for name, x, r in zip(("dq", "dk", "dv", "dg", "dbeta"), a, ref):
             assert rel_inf(x[:, :, h:h + 1].cpu(), r) <= TOL, (name, h)
+
+
+@pytest.mark.parametrize("case", ["dense_6_units", "dense_32_units", "dense_64_units", "varlen_256_units"])
+def test_saved_intermediates_bitwise(case):
+    """kda_chunk_fwd_save gives kda_chunk_fwd's outputs bitwise, and the
+    backward from its saved intermediates gives kda_chunk_bwd's gradients
+    bitwise (the saved state images are the same whatever state-tile width
+    the forward chain ran with: 16, 32, 64 or 128 columns here)."""
+    from gated_delta_rule_88_b200 import kda_chunk_fwd, kda_chunk_fwd_save
+    if case == "varlen_256_units":
+        inp = W.prefill(1, 0, 32, 128, 128, torch.bfloat16, seed=320, initial_state_std=0.05,
+                        seq_lens=[70, 0, 130, 64, 1, 200, 65, 90, 33])
+    else:
+        B, T, H = {"dense_6_units": (2, 150, 3), "dense_32_units": (1, 200, 32),
+                   "dense_64_units": (2, 100, 32)}[case]
+        inp = W.prefill(B, T, H, 128, 128, torch.bfloat16, seed=321, initial_state_std=0.05)
+    d = inp.to(DEV)
+    B, T, H, _ = d.q.shape
+    gen = torch.Generator().manual_seed(322)
+    do = torch.randn(B, T, H, 128, generator=gen).to(torch.bfloat16).to(DEV)
+    N = inp.num_seqs
+    dsT = (torch.randn(N, H, 128, 128, generator=gen) * 0.1).to(DEV)
+    o1, s1 = kda_chunk_fwd(d.q, d.k, d.v, d.g, d.beta, d.initial_state, d.cu_seqlens)
+    o2, s2, saved = kda_chunk_fwd_save(d.q, d.k, d.v, d.g, d.beta, d.initial_state, d.cu_seqlens)
+    g1 = kda_chunk_bwd(d.q, d.k, d.v, d.g, d.beta, do, d.initial_state, dsT, d.cu_seqlens)
+    g2 = kda_chunk_bwd(d.q, d.k, d.v, d.g, d.beta, do, d.initial_state, dsT, d.cu_seqlens,
+                       saved=saved)
+    torch.cuda.synchronize()
+    assert kda_get_device_error() == 0
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+    for name, x, y in zip(("dq", "dk", "dv", "dg", "dbeta", "ds0"), g1, g2):
+        assert torch.equal(x, y), name

@@ -102,14 +102,15 @@ TRAFFIC = {
     # per call: prep, forward chain with images, reverse chain, per-chunk pass
     "backward_chunk": {"files": PREFILL_SRC + ["chunk_chain_bwd.cu", "chunk_bwd.cu"], "sha": "56b917d26a13785c",
                        "bytes": 2823976170},
-    "decode": {"files": ["decode.cu", "common.cuh"], "sha": "4ceac309c0c18d2f",
-               "bytes": (547.408128 + 480.674560) * 1e6},
-    "decode_steps": {"files": ["decode_pipe.cu", "common.cuh", "sm100.cuh"], "sha": "d9cf376f965488af",
-                     "bytes": (621.110016 + 492.918016) * 1e6},
-    "backward": {"files": ["recurrent_bwd.cu", "common.cuh"], "sha": "ba9d9318f1b1cd87",
-                 "bytes": (2902.812672 + 3861.861120) * 1e6},
-    "decode_chunk": {"files": ["decode_chunk.cu", "common.cuh"], "sha": "23a550bc05b00c2b",
-                     "bytes": (1210.240000 + 623.093504) * 1e6},
+    # one launch each at full size, -k <kernel> -c 1 (decode legs: --decode-steps 64)
+    "decode": {"files": ["decode.cu", "common.cuh"], "sha": "05d923d8fde4c25f",
+               "bytes": 547407616 + 479790080},
+    "decode_steps": {"files": ["decode_pipe.cu", "common.cuh", "sm100.cuh"],
+                     "sha": "68dca8336a4f6cbf", "bytes": 621144832 + 496053248},
+    "backward": {"files": ["recurrent_bwd.cu", "common.cuh"], "sha": "0c58bb721f4cdeeb",
+                 "bytes": 2902945280 + 3862875392 + 1614867456 + 385818880},
+    "decode_chunk": {"files": ["decode_chunk.cu", "common.cuh"], "sha": "a0fa479bec9da035",
+                     "bytes": 1210701056 + 622548224},
 }
 
 

@@ -29,6 +29,8 @@
 // forms) are bf16, as in the prefill.
 #include "common.cuh"
 #include "kernels.h"
+#include "prep_common.cuh"
+#include "sm100.cuh"
 
 namespace kda {
 namespace {
@@ -64,9 +66,11 @@ constexpr int OFF_GAM = OFF_TM + 1024;       // e^{G_last} per channel, fp32 [12
 constexpr int OFF_KD = OFF_GAM + 512;        // k e^{-G} (factorised A and P)
 constexpr int OFF_SN = OFF_KD + 4096;        // next item's state, fp32 [128][128], fsw layout
 constexpr int OFF_SO = OFF_SN + D * D * 4;   // finished item's state on its way out, fsw layout
-constexpr int SMEM = OFF_SO + D * D * 4;
+constexpr int OFF_BAR = OFF_SO + D * D * 4;  // mbarrier of the raw rows
+constexpr int SMEM = OFF_BAR + 16;
+constexpr uint32_t TX_RAW = 3 * 4096 + 8192;   // q, k, v, g rows of one block
 static_assert(OFF_QG % 16 == 0 && OFF_SB % 16 == 0 && OFF_KD % 16 == 0 && OFF_SN % 16 == 0 &&
-              SMEM <= 227 * 1024, "layout");
+              OFF_BAR % 8 == 0 && SMEM <= 227 * 1024, "layout");
 
 // 2^x by the hardware approximation (PTX ex2.approx.ftz: relative error about
 // 2^-22, results below 2^-126 flush to zero); the operands of the products it
@@ -86,10 +90,6 @@ __device__ __forceinline__ void cp_async4_zfill(void *smem_dst, const void *gmem
 __device__ __forceinline__ int fsw(int r, int c) {
     return r * 512 + ((((c >> 2) ^ (2 * (r & 3)))) << 4) + ((c & 3) << 2);
 }
-__device__ __forceinline__ void cp_async16_zfill(void *smem_dst, const void *gmem_src, bool ok) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem_dst)),
-                 "l"(gmem_src), "r"(ok ? 16 : 0));
-}
 
 // A fragment (rows gid / gid + 8, k pairs) of a 16 x 16 fp32 matrix in shared memory
 __device__ __forceinline__ void frag16(uint32_t (&a)[4], const float *M, int gid, int tig) {
@@ -106,8 +106,8 @@ __device__ __forceinline__ void frag16(uint32_t (&a)[4], const float *M, int gid
 }  // namespace
 
 __global__ void __launch_bounds__(NT, 1)
-decode_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                    const __nv_bfloat16 *__restrict__ v, const float *__restrict__ g,
+decode_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                     const float *__restrict__ beta, float *__restrict__ pool,
                     const int32_t *__restrict__ slots, int num_slots,
                     __nv_bfloat16 *__restrict__ out, int N, int H, int L, int *__restrict__ err)
@@ -145,26 +145,27 @@ decode_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         return (size_t)nn * L * H + hh;
     };
 
-    // raw rows of block b of item `it` (zero past the last token), one cp.async group
+    // raw rows of block b of item `it`: q, k, v and g by TMA (16 token rows
+    // of one head; rows past the item's last token hold whatever follows and
+    // are masked where they are read), beta by cp.async (zero past the last
+    // token), one cp.async group
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     auto issue_raw = [&](int it, int b) {
         const int l0 = b * BT, nt = min(BT, L - l0);
-        const size_t base = row0(it);
-        for (int c = tid; c < BT * 80; c += NT) {
-            const int i = c / 80, r = c - i * 80;
-            const bool ok = i < nt;
-            const size_t row = base + (size_t)(ok ? l0 + i : l0) * H;
-            if (r < 48) {
-                const int vec = r >> 4, j = r & 15;
-                const __nv_bfloat16 *src = (vec == 0 ? q : vec == 1 ? k : v) + row * D + j * 8;
-                cp_async16_zfill(sm + OFF_RQ + vec * 4096 + i * 256 + j * 16, src, ok);
-            } else {
-                const int j = r - 48;
-                cp_async16_zfill(sm + OFF_G + i * 512 + j * 16, g + row * D + j * 4, ok);
-            }
+        const int nn = it / H, hh = it - nn * H;
+        if (tid == 0) {
+            const int row = nn * L + l0;
+            sm100::mbar_arrive_expect_tx(bar, TX_RAW);
+            prep::tma_load_3d(sm + OFF_RQ, &tm_q, 0, hh, row, bar);
+            prep::tma_load_3d(sm + OFF_RK, &tm_k, 0, hh, row, bar);
+            prep::tma_load_3d(sm + OFF_RV, &tm_v, 0, hh, row, bar);
+            prep::tma_load_3d(sm + OFF_G, &tm_g, 0, hh, row, bar);
         }
+        const size_t base = row0(it);
         if (tid < BT) cp_async4_zfill(bs + tid, beta + base + (size_t)(tid < nt ? l0 + tid : l0) * H, tid < nt);
         cp_async_commit();
     };
+    uint32_t raw_phase = 0;    // parity of the raw-row barrier's next completion
 
     // the state, fp32, in the accumulator layout: s[j] = rows (16w + gid,
     // 16w + gid + 8) x columns (8j + 2tig, + 1).  Element pair (j, half) of
@@ -189,6 +190,11 @@ decode_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         }
     };
 
+    if (tid == 0) {
+        sm100::mbar_init(bar, 1);
+        sm100::fence_mbar_init();
+    }
+    __syncthreads();
     int cur = next_valid(blockIdx.x);
     if (cur < 0) return;
     issue_state(cur);
@@ -199,7 +205,18 @@ decode_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     for (int b = 0; b < nblk; ++b) {
         const int l0 = b * BT, nt = min(BT, L - l0);
         cp_async_wait<0>();
-        __syncthreads();                       // raw rows of block b (and at b = 0 the state) landed
+        bool ok = true;
+        if (tid == 0) ok = sm100::mbar_wait(bar, raw_phase);
+        raw_phase ^= 1u;
+        if (!__syncthreads_and(ok)) {
+            // the raw rows never arrived: report, give the copy a bounded
+            // second wait, and stop before shared memory is released
+            if (tid == 0) {
+                set_device_error(err, kErrWaitTimeout);
+                sm100::mbar_wait(bar, raw_phase ^ 1u);
+            }
+            return;
+        }                                      // raw rows of block b (and at b = 0 the state) landed
         if (b == 0) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -217,7 +234,7 @@ decode_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
             float acc = 0.f;
 #pragma unroll
             for (int i = 0; i < BT; ++i) {
-                const float gv = Gs[i * D + tid];
+                const float gv = i < nt ? Gs[i * D + tid] : 0.f;
                 in_range = in_range && gv >= -5.f;
                 acc = fmaf(gv, LOG2E, acc);
                 Gs[i * D + tid] = acc;
@@ -236,9 +253,11 @@ decode_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
             const float2 gl = *reinterpret_cast<const float2 *>(Gs + (BT - 1) * D + c);
             const float ex = ex2(gi.x), ey = ex2(gi.y);
             const float tx = ex2(gl.x - gi.x), ty = ex2(gl.y - gi.y);
-            const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(sm + OFF_RQ + i * 256 + 2 * c);
-            const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(sm + OFF_RK + i * 256 + 2 * c);
-            const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162 *>(sm + OFF_RV + i * 256 + 2 * c);
+            const bool row_ok = i < nt;
+            const __nv_bfloat162 zero2 = __floats2bfloat162_rn(0.f, 0.f);
+            const __nv_bfloat162 q2 = row_ok ? *reinterpret_cast<const __nv_bfloat162 *>(sm + OFF_RQ + i * 256 + 2 * c) : zero2;
+            const __nv_bfloat162 k2 = row_ok ? *reinterpret_cast<const __nv_bfloat162 *>(sm + OFF_RK + i * 256 + 2 * c) : zero2;
+            const __nv_bfloat162 v2 = row_ok ? *reinterpret_cast<const __nv_bfloat162 *>(sm + OFF_RV + i * 256 + 2 * c) : zero2;
             const float b_ = bs[i];
             const float qx = __low2float(q2), qy = __high2float(q2);
             const float kx = __low2float(k2), ky = __high2float(k2);
@@ -296,6 +315,8 @@ decode_chunk_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
                 }
             }
         }
+        // the in-place cumsum wrote g rows that the next TMA overwrites
+        sm100::fence_proxy_async_smem();
         __syncthreads();
         if (fact) {
             // A = (beta k e^G)(k e^{-G})^T, P = (q e^G)(k e^{-G})^T: warps
@@ -496,9 +517,20 @@ cudaError_t launch_decode_chunk(const void *q, const void *k, const void *v, con
     }
     const int items = N * H;
     const int grid = items < grid_for[dev] ? items : grid_for[dev];
-    decode_chunk_kernel<<<grid, NT, SMEM, st>>>(
-        (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, g, beta, pool,
-        slots, num_slots, (__nv_bfloat16 *)out, N, H, L, err);
+    // [N * L token rows, H, 128] views, boxes of one head's 16 token rows
+    if ((long long)N * L > 0x7fffffffLL) return cudaErrorInvalidValue;
+    CUtensorMap mq, mk, mv, mg;
+    const int rows = N * L;
+    e = prep::make_token_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, rows, D, CU_TENSOR_MAP_SWIZZLE_NONE, BT);
+    if (e == cudaSuccess)
+        e = prep::make_token_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, rows, D, CU_TENSOR_MAP_SWIZZLE_NONE, BT);
+    if (e == cudaSuccess)
+        e = prep::make_token_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, rows, D, CU_TENSOR_MAP_SWIZZLE_NONE, BT);
+    if (e == cudaSuccess)
+        e = prep::make_token_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, rows, D, CU_TENSOR_MAP_SWIZZLE_NONE, BT);
+    if (e != cudaSuccess) return e;
+    decode_chunk_kernel<<<grid, NT, SMEM, st>>>(mq, mk, mv, mg, beta, pool, slots, num_slots,
+                                                (__nv_bfloat16 *)out, N, H, L, err);
     return cudaGetLastError();
 }
 

@@ -103,6 +103,22 @@ __device__ __forceinline__ void frag16(uint32_t (&a)[4], const float *M, int gid
     a[3] = pack_bf16(x3.x, x3.y);
 }
 
+// Tensor map over a [rows, H, 128] token tensor of `elem`-byte elements,
+// boxes of one head's 16 token rows (no swizzle: plain 128-element rows)
+cudaError_t make_block_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem, int H,
+                           int rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = prep::tensor_map_encoder();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * elem, (cuuint64_t)D * elem * H};
+    const cuuint32_t box[3] = {(cuuint32_t)D, 1, (cuuint32_t)BT};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(NT, 1)
@@ -521,13 +537,10 @@ cudaError_t launch_decode_chunk(const void *q, const void *k, const void *v, con
     if ((long long)N * L > 0x7fffffffLL) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv, mg;
     const int rows = N * L;
-    e = prep::make_token_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, rows, D, CU_TENSOR_MAP_SWIZZLE_NONE, BT);
-    if (e == cudaSuccess)
-        e = prep::make_token_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, rows, D, CU_TENSOR_MAP_SWIZZLE_NONE, BT);
-    if (e == cudaSuccess)
-        e = prep::make_token_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, rows, D, CU_TENSOR_MAP_SWIZZLE_NONE, BT);
-    if (e == cudaSuccess)
-        e = prep::make_token_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, rows, D, CU_TENSOR_MAP_SWIZZLE_NONE, BT);
+    e = make_block_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, rows);
+    if (e == cudaSuccess) e = make_block_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, rows);
+    if (e == cudaSuccess) e = make_block_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, rows);
+    if (e == cudaSuccess) e = make_block_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, rows);
     if (e != cudaSuccess) return e;
     decode_chunk_kernel<<<grid, NT, SMEM, st>>>(mq, mk, mv, mg, beta, pool, slots, num_slots,
                                                 (__nv_bfloat16 *)out, N, H, L, err);

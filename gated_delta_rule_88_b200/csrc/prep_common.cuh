@@ -168,14 +168,14 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // Tensor map over a [total_T, H, 128] tensor of `elem`-byte elements, boxes
-// of {box_c channels, 1 head, box_t tokens}.
+// of {box_c channels, 1 head, 64 tokens}.
 static cudaError_t make_token_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem,
-                                  int H, int total_T, int box_c, CUtensorMapSwizzle swz, int box_t = C) {
+                                  int H, int total_T, int box_c, CUtensorMapSwizzle swz) {
     PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
     if (!fn) return cudaErrorNotSupported;
     const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)total_T};
     const cuuint64_t strides[2] = {(cuuint64_t)D * elem, (cuuint64_t)D * elem * H};
-    const cuuint32_t box[3] = {(cuuint32_t)box_c, 1, (cuuint32_t)box_t};
+    const cuuint32_t box[3] = {(cuuint32_t)box_c, 1, (cuuint32_t)C};
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUresult r = fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

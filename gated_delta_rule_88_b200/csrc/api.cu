@@ -16,6 +16,13 @@
 #include "../../include/kda.h"
 #include "common.cuh"
 #include "kernels.h"
+
+// Chunk-form serving decode: from this many tokens per call on, 64-token
+// chunks on tcgen05 (decode_chunk_tc.cu); below it, 16-token blocks
+// (decode_chunk.cu).
+#ifndef KDA_TC_CHUNK_MIN_L
+#define KDA_TC_CHUNK_MIN_L 33
+#endif
 #include "chunk_ws.h"
 #include "api_internal.h"
 
@@ -235,11 +242,30 @@ kda_status kda_recurrent_steps(const void *q, const void *k, const void *v, cons
     if (NH == 0) return KDA_OK;
     const bool tc = chunk && L >= 2 && dtype == KDA_BF16 && dk == 128 && dv == 128 &&
                     pro.flags == 0 && pro.q_scale == 1.f;
+    cudaStream_t st = (cudaStream_t)stream;
+    // (the 64-token path moves the state and the output in 32-byte pieces)
+    if (tc && L >= KDA_TC_CHUNK_MIN_L && !((uintptr_t)state_pool & 31u) && !((uintptr_t)out & 31u)) {
+        // 64-token chunks on tcgen05, with a scratch of per-CTA slots and
+        // the list of out-of-range items
+        cudaMemPool_t mp;
+        int sms = 148;
+        cudaError_t e = get_pool(&mp, &sms);
+        if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_steps memory pool");
+        void *scratch = nullptr;
+        e = cudaMallocFromPoolAsync(&scratch, kda::decode_chunk_tc_scratch_bytes(N, H, sms), mp, st);
+        if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_steps scratch allocation");
+        e = kda::launch_decode_chunk_tc(q, k, v, g, beta, state_pool, slots, num_slots, out, N, H, L, sms,
+                                        scratch, kda::error_word(), st);
+        cudaError_t e2 = cudaFreeAsync(scratch, st);
+        if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_steps launch");
+        if (e2 != cudaSuccess) return cuda_fail(e2, "kda_recurrent_steps scratch release");
+        return KDA_OK;
+    }
     cudaError_t e = tc ? kda::launch_decode_chunk(q, k, v, g, beta, state_pool, slots, num_slots,
-                                                  out, N, H, L, kda::error_word(), (cudaStream_t)stream)
+                                                  out, N, H, L, kda::error_word(), st)
                        : kda::launch_decode_pipe(q, k, v, g, beta, state_pool, slots, num_slots, out,
                                                  N, H, L, dk, dv, dtype == KDA_BF16,
-                                                 kda::error_word(), pro, (cudaStream_t)stream);
+                                                 kda::error_word(), pro, st);
     if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_steps launch");
     return KDA_OK;
 }

@@ -126,7 +126,8 @@ decode_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                     const float *__restrict__ beta, float *__restrict__ pool,
                     const int32_t *__restrict__ slots, int num_slots,
-                    __nv_bfloat16 *__restrict__ out, int N, int H, int L, int *__restrict__ err)
+                    __nv_bfloat16 *__restrict__ out, int N, int H, int L,
+                    const int2 *__restrict__ list, const int *__restrict__ list_count, int *__restrict__ err)
 {
     extern __shared__ __align__(128) unsigned char sm[];
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
@@ -141,7 +142,13 @@ decode_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int nblk = (L + BT - 1) / BT;
     // the next item at or after `it` (grid stride) with a valid slot; -1 if
     // none.  Every thread walks the same items, so the answer is uniform.
+    // With a list, the walk is over list entries (item, first token, a
+    // multiple of 64) instead of items; listed items have valid slots.
+    const int n_list = list ? *list_count : 0;
+    auto item_of = [&](int ix) -> int { return list ? list[ix].x : ix; };
+    auto first_blk = [&](int ix) -> int { return list ? list[ix].y / BT : 0; };
     auto next_valid = [&](int it) -> int {
+        if (list) return it < n_list ? it : -1;
         for (; it < items; it += gridDim.x) {
             const int nn = it / H;
             const int sl = slots ? slots[nn] : nn;
@@ -213,12 +220,13 @@ decode_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncthreads();
     int cur = next_valid(blockIdx.x);
     if (cur < 0) return;
-    issue_state(cur);
-    issue_raw(cur, 0);
+    issue_state(item_of(cur));
+    issue_raw(item_of(cur), first_blk(cur));
     while (cur >= 0) {
     const int nxt = next_valid(cur + gridDim.x);
-    const size_t orow = row0(cur);
-    for (int b = 0; b < nblk; ++b) {
+    const int cit = item_of(cur), b_first = first_blk(cur);
+    const size_t orow = row0(cit);
+    for (int b = b_first; b < nblk; ++b) {
         const int l0 = b * BT, nt = min(BT, L - l0);
         cp_async_wait<0>();
         bool ok = true;
@@ -233,7 +241,7 @@ decode_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             return;
         }                                      // raw rows of block b (and at b = 0 the state) landed
-        if (b == 0) {
+        if (b == b_first) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const float2 x = *reinterpret_cast<const float2 *>(sm + OFF_SN + fsw(r0, 8 * j + 2 * tig));
@@ -368,8 +376,8 @@ decode_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         // the raw rows are dead: the next block's (or the next item's first
         // block's) arrive while this one runs
-        if (b + 1 < nblk) issue_raw(cur, b + 1);
-        else if (nxt >= 0) issue_raw(nxt, 0);
+        if (b + 1 < nblk) issue_raw(cit, b + 1);
+        else if (nxt >= 0) issue_raw(item_of(nxt), first_blk(nxt));
 
         // 3. T = (I + A)^-1 by forward substitution, one column per thread
         if (tid < BT) {
@@ -398,8 +406,8 @@ decode_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         __syncthreads();
         // every thread's reads of its state slots are long complete (several
         // barriers): the next item's state may now land there
-        if (b == 0 && nxt >= 0) {
-            issue_state(nxt);
+        if (b == b_first && nxt >= 0) {
+            issue_state(item_of(nxt));
             cp_async_commit();
         }
 
@@ -499,7 +507,7 @@ decode_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             *reinterpret_cast<float2 *>(sm + OFF_SO + fsw(r1, 8 * j + 2 * tig)) = make_float2(s[j][2], s[j][3]);
         }
         __syncthreads();
-        float *Sg = state_of(cur);
+        float *Sg = state_of(cit);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
             const int idx = e * NT + tid, r = idx >> 5, c = 4 * (idx & 31);
@@ -511,10 +519,10 @@ decode_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
 }
 
-cudaError_t launch_decode_chunk(const void *q, const void *k, const void *v, const float *g,
-                                const float *beta, float *pool, const int32_t *slots,
-                                int num_slots, void *out, int N, int H, int L, int *err,
-                                cudaStream_t st)
+namespace {
+cudaError_t launch_walk(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                        float *pool, const int32_t *slots, int num_slots, void *out, int N, int H, int L,
+                        const int2 *list, const int *list_count, int *err, cudaStream_t st)
 {
     if (N == 0 || L == 0) return cudaSuccess;
     static int grid_for[64] = {0};
@@ -543,8 +551,25 @@ cudaError_t launch_decode_chunk(const void *q, const void *k, const void *v, con
     if (e == cudaSuccess) e = make_block_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, rows);
     if (e != cudaSuccess) return e;
     decode_chunk_kernel<<<grid, NT, SMEM, st>>>(mq, mk, mv, mg, beta, pool, slots, num_slots,
-                                                (__nv_bfloat16 *)out, N, H, L, err);
+                                                (__nv_bfloat16 *)out, N, H, L, list, list_count, err);
     return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_decode_chunk(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, float *pool, const int32_t *slots,
+                                int num_slots, void *out, int N, int H, int L, int *err,
+                                cudaStream_t st)
+{
+    return launch_walk(q, k, v, g, beta, pool, slots, num_slots, out, N, H, L, nullptr, nullptr, err, st);
+}
+
+cudaError_t launch_decode_chunk_list(const void *q, const void *k, const void *v, const float *g,
+                                     const float *beta, float *pool, const int32_t *slots, int num_slots,
+                                     void *out, int N, int H, int L, const int2 *list, const int *list_count,
+                                     int *err, cudaStream_t st)
+{
+    return launch_walk(q, k, v, g, beta, pool, slots, num_slots, out, N, H, L, list, list_count, err, st);
 }
 
 }  // namespace kda

@@ -47,6 +47,20 @@ cudaError_t launch_decode_chunk(const void *q, const void *k, const void *v, con
                                 const float *beta, float *pool, const int32_t *slots,
                                 int num_slots, void *out, int N, int H, int L, int *err,
                                 cudaStream_t st);
+// The same, for listed (item, first token) pairs only; the count is read on
+// the device.
+cudaError_t launch_decode_chunk_list(const void *q, const void *k, const void *v, const float *g,
+                                     const float *beta, float *pool, const int32_t *slots, int num_slots,
+                                     void *out, int N, int H, int L, const int2 *list, const int *list_count,
+                                     int *err, cudaStream_t st);
+// The chunk-form decode on 64-token chunks on tcgen05 (decode_chunk_tc.cu),
+// then the listed out-of-range items on the 16-token kernel.  `scratch`:
+// decode_chunk_tc_scratch_bytes(N, H, sms) bytes, 256-byte aligned.
+size_t decode_chunk_tc_scratch_bytes(int N, int H, int sms);
+cudaError_t launch_decode_chunk_tc(const void *q, const void *k, const void *v, const float *g,
+                                   const float *beta, float *pool, const int32_t *slots, int num_slots,
+                                   void *out, int N, int H, int L, int sms, void *scratch, int *err,
+                                   cudaStream_t st);
 
 // Gradients of the recurrence (recurrent_bwd.cu): one warp per (sequence,
 // head, 16-column state tile), workspace of recurrent_bwd_workspace bytes.

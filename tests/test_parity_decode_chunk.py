@@ -140,3 +140,51 @@ def test_chunk_steps_bad_slot_reported_and_skipped_long():
     assert_close(pool[[2, 5]], s_ref, BF, "their pool entries")
     keep = [0, 1, 3, 4]
     assert torch.equal(pool.cpu()[keep], pool0[keep])
+
+
+def test_chunk_steps_out_of_range_from_a_later_chunk():
+    """From 33 tokens on the chunk form takes 64-token chunks on tcgen05; a
+    chunk whose decay leaves the chunk-start range sends its item, from that
+    chunk's first token on, to the 16-token blocks.  Sequence 1 head 0 leaves
+    the range in its second chunk only, sequence 2 head 1 in its first, the
+    rest stays in range: all of it against the oracle."""
+    N, L, H, d = 4, 100, 2, 128
+    q, k, v, g, b = _tokens(N, L, H, d, seed=61)
+    g[1, 64:, 0] = -20.0
+    g[2, :, 1] = -20.0
+    pool0 = W.decode_initial_state(N, H, d, d, seed=61, std=0.02)
+    pool = pool0.to(DEV)
+    out = kda_recurrent_steps(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), b.to(DEV), pool,
+                              flags=KDA_STEPS_CHUNK)
+    torch.cuda.synchronize()
+    assert kda_get_device_error() == 0
+    assert torch.isfinite(out.float()).all() and torch.isfinite(pool).all()
+    o_ref, s_ref = oracle.forward(q, k, v, g, b, initial_state=pool0.double())
+    assert_close(out, o_ref, BF, "o")
+    for n in range(N):
+        assert_close(pool[n], s_ref[n], BF, f"state {n}")
+
+
+def test_chunk_steps_decode_workload_64_tokens():
+    """256 sequences x 32 heads, 64 tokens each, pool of 512 (the serving
+    decode's chunk-form workload): every output finite and within the bf16
+    bound of the recurrent kernel; 16 sampled sequences against the oracle."""
+    N, H, d, L, S = W.DECODE_N, W.DECODE_H, W.DECODE_D, 64, 2 * W.DECODE_N
+    pool0 = W.decode_initial_state(S, H, d, d)
+    gen = torch.Generator().manual_seed(33)
+    slots = torch.randperm(S, generator=gen)[:N].to(torch.int32).to(DEV)
+    q, k, v, g, b = [t.to(DEV) for t in _tokens(N, L, H, d, seed=W.DECODE_SEED)]
+    pool_c, pool_r = pool0.to(DEV), pool0.to(DEV)
+    out_c = kda_recurrent_steps(q, k, v, g, b, pool_c, slots, flags=KDA_STEPS_CHUNK)
+    out_r = kda_recurrent_steps(q, k, v, g, b, pool_r, slots)
+    torch.cuda.synchronize()
+    assert kda_get_device_error() == 0
+    assert torch.isfinite(out_c.float()).all() and torch.isfinite(pool_c).all()
+    assert rel_inf(out_c, out_r) <= 2e-2
+    assert rel_inf(pool_c, pool_r) <= 2e-2
+    ns = torch.randperm(N, generator=gen)[:16]
+    sl = slots.cpu()[ns].long()
+    o_ref, s_ref = oracle.forward(q.cpu()[ns], k.cpu()[ns], v.cpu()[ns], g.cpu()[ns], b.cpu()[ns],
+                                  initial_state=pool0[sl].double())
+    assert_close(out_c[ns.to(DEV)], o_ref, BF, "sampled o")
+    assert_close(pool_c[sl.to(DEV)], s_ref, BF, "sampled states")

@@ -136,6 +136,7 @@ decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                        const float *__restrict__ beta, float *__restrict__ pool,
                        const int32_t *__restrict__ slots, int num_slots, __nv_bfloat16 *__restrict__ out,
+                       const __grid_constant__ CUtensorMap tm_kt,
                        int N, int H, int L, unsigned char *__restrict__ kt_scratch,
                        int2 *__restrict__ fb_list, int *__restrict__ fb_count, int *__restrict__ err)
 {
@@ -243,14 +244,13 @@ decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     while (cur.it >= 0) {
     const int h = cur.it % H, len = len_of(cur), t0 = row0(cur);
     float *S = state_of(cur.it);
-    // the unit after this one, and its state if it starts an item (thread 0;
-    // the slot lookups overlap the waits below)
+    // the unit after this one, and its state if it starts an item (thread 0):
+    // the next item's slot is loaded now and used while MMA-W/U runs
     Unit nx{-1, -1};
     const float *nxS = nullptr;
-    if (tid == 0) {
-        nx = next_unit(cur, false);
-        if (nx.it >= 0 && nx.c == 0) nxS = state_of(nx.it);
-    }
+    const int nit = cur.it + gridDim.x;
+    int nslot = -1;
+    if (tid == 0 && cur.c + 1 >= nch && nit < items) nslot = slots ? slots[nit / H] : nit / H;
     if (tid < C) bet[tid] = bt_cur;
     if (tid == 0) ok = wait_bar(dtc::B_G);
     ok = __syncthreads_and(ok);
@@ -345,13 +345,15 @@ decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 kt_prev = kt2;
             }
         }
+        // plain rows of 64 tokens (128 bytes): tokens 16 I .. 16 I + 15 of
+        // channels c0, c0 + 1 are one 32-byte piece each
 #pragma unroll
         for (int e = 0; e < 2; ++e)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-                *reinterpret_cast<uint4 *>(kts + ws::sw128(c0 + e, 16 * I + 8 * hh)) =
-                    make_uint4(kt[e][4 * hh], kt[e][4 * hh + 1], kt[e][4 * hh + 2], kt[e][4 * hh + 3]);
-        // the slot is read back by a bulk copy (async proxy)
+            asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"l"(kts + (c0 + e) * 128 + 32 * I),
+                         "r"(kt[e][0]), "r"(kt[e][1]), "r"(kt[e][2]), "r"(kt[e][3]), "r"(kt[e][4]), "r"(kt[e][5]),
+                         "r"(kt[e][6]), "r"(kt[e][7])
+                         : "memory");
+        // the slot returns by TMA (async proxy), swizzled for MMA-upd
         asm volatile("fence.proxy.async.global;\n" ::: "memory");
     }
     fence_proxy_async_smem();
@@ -466,8 +468,17 @@ decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         arm(dtc::B_MMA);
         // K e^{G_C - G} back from the slot over T (fp32), read above
         mbar_arrive_expect_tx(bars + dtc::B_KT, dtc::KT_BYTES);
-        bulk_g2s(sm + dtc::OFF_TM, kts, dtc::KT_BYTES, bars + dtc::B_KT);
+        tma_load_3d(sm + dtc::OFF_TM, &tm_kt, 0, 0, blockIdx.x, bars + dtc::B_KT);
         arm(dtc::B_KT);
+        if (cur.c + 1 < nch) {
+            nx = Unit{cur.it, cur.c + 1};
+        } else if (nslot >= 0 && nslot < num_slots) {
+            nx = Unit{nit, 0};
+            nxS = pool + ((size_t)nslot * H + nit % H) * (size_t)(D * D);
+        } else {
+            nx = next_unit(cur, false);
+            if (nx.it >= 0) nxS = state_of(nx.it);
+        }
         ok = wait_bar(dtc::B_MMA);
     }
     ok = __syncthreads_and(ok);
@@ -520,7 +531,7 @@ decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             }
 #pragma unroll
             for (int j = 0; j < 32; ++j) so[j] *= gc;
-            tmem_st32(tmem + lanes + 128u + 64u * hf + 32u * half, so);
+            tmem_st32(tmem + lanes + 128u + 64u * hf + 32u * half, *reinterpret_cast<const float (*)[32]>(so));
         }
         tmem_wait_st();
     }
@@ -691,12 +702,27 @@ cudaError_t launch_decode_chunk_tc(const void *q, const void *k, const void *v, 
     if (e == cudaSuccess)
         e = make_token_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, rows, D, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (e != cudaSuccess) return e;
+    // the K e^{G_C - G} slots: [grid][128 channel rows][64 tokens] bf16, one
+    // box per slot, 128-byte swizzle on arrival
+    CUtensorMap mkt;
+    {
+        PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+        if (!fn) return cudaErrorNotSupported;
+        const cuuint64_t dims[3] = {64, 128, (cuuint64_t)grid};
+        const cuuint64_t strides[2] = {128, dtc::KT_BYTES};
+        const cuuint32_t box[3] = {64, 128, 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (fn(&mkt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, kt_scratch, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
     const size_t smem = dtc::BYTES + 1024;
     e = cudaFuncSetAttribute(decode_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     decode_chunk_tc_kernel<<<grid, NT, smem, st>>>(mq, mk, mv, mg, beta, pool, slots, num_slots,
-                                                   (__nv_bfloat16 *)out, N, H, L, kt_scratch, list, count,
-                                                   err);
+                                                   (__nv_bfloat16 *)out, mkt, N, H, L, kt_scratch, list,
+                                                   count, err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     // the listed items, from their first out-of-range chunk on

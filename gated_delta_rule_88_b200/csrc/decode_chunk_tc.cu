@@ -240,8 +240,26 @@ decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     Unit cur = *uslot;
     if (tid < C && cur.it >= 0) bt_cur = load_beta(cur);
     bool ok = true;
+    const int qd = warp & 3, hf = warp >> 2;            // TMEM lane quarter, 64-column half
+    const uint32_t lanes = (uint32_t)(qd * 32) << 16;
+    // The new state of a unit stays in TMEM columns 128-255 until the top of
+    // the next unit, where it goes to the pool while that unit's inputs land
+    // (its state pass writes those columns again).  Row c = TMEM lane.
+    float *S_out = nullptr;
+    auto store_state = [&](float *Sg) {
+        float *srow = Sg + (qd * 32 + lane) * D + 64 * hf;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float x[32];
+            tmem_ld32(tmem + lanes + 128u + 64u * hf + 32u * half, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 4; ++j) st_v8(srow + 32 * half + 8 * j, x + 8 * j);
+        }
+    };
 
     while (cur.it >= 0) {
+    if (S_out) { store_state(S_out); S_out = nullptr; }
     const int h = cur.it % H, len = len_of(cur), t0 = row0(cur);
     float *S = state_of(cur.it);
     // the unit after this one, and its state if it starts an item (thread 0):
@@ -485,8 +503,6 @@ decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     tc_fence_after();
     if (!ok) break;
 
-    const int qd = warp & 3, hf = warp >> 2;            // TMEM lane quarter, 64-column half
-    const uint32_t lanes = (uint32_t)(qd * 32) << 16;
     {
         // -W (rows 16 qd + l, l < 16, of the +0 tile) as bf16 over the dead k
         // rows: the A operand that turns U into V_new = U - W S in place
@@ -624,7 +640,8 @@ decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     // V_new, P and K e^{G_C - G} are read: the next unit's v goes over V_new
     if (tid == 0 && nx.it >= 0) load_v(nx);
 
-    // ---- epilogue: O (rows of the +0 tile, l < 16) and the new state ----
+    // ---- epilogue: O (rows of the +0 tile, l < 16); the new state leaves at
+    // the top of the next unit ----
     {
         const int r = 16 * qd + lane;
 #pragma unroll
@@ -638,17 +655,8 @@ decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 st_v8_bf16(dst + 16, x + 16);
             }
         }
-        const int c = qd * 32 + lane;
-        float *srow = S + c * D + 64 * hf;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float x[32];
-            tmem_ld32(tmem + lanes + 128u + 64u * hf + 32u * half, x);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 4; ++j) st_v8(srow + 32 * half + 8 * j, x + 8 * j);
-        }
     }
+    S_out = S;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -656,6 +664,7 @@ decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     bt_cur = bt_next;
     }   // units
 
+    if (ok && S_out) store_state(S_out);
     if (!ok && tid == 0) {
         // a bounded wait ran out: report it, and let what this CTA has in
         // flight (loads, copies, MMAs) finish, with bounded waits again,

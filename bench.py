@@ -109,8 +109,8 @@ TRAFFIC = {
                      "sha": "68dca8336a4f6cbf", "bytes": 621144832 + 496053248},
     "backward": {"files": ["recurrent_bwd.cu", "common.cuh"], "sha": "0c58bb721f4cdeeb",
                  "bytes": 2902945280 + 3862875392 + 1614867456 + 385818880},
-    "decode_chunk": {"files": ["decode_chunk.cu", "common.cuh"], "sha": "a0fa479bec9da035",
-                     "bytes": 1210701056 + 622548224},
+    "decode_chunk": {"files": ["decode_chunk_tc.cu", "decode_chunk.cu", "prep_common.cuh", "common.cuh",
+                               "sm100.cuh"], "sha": "277e01a9145f9723", "bytes": 1284074240 + 648703488},
 }
 
 
@@ -352,7 +352,7 @@ def run_ours(args):
                    "decode_steps": decode_steps_leg(kda, W, dev, dist, world, args),
                    "decode_chunk": decode_steps_leg(kda, W, dev, dist, world, args, L=CHUNK_L,
                                                     flags=kda.KDA_STEPS_CHUNK,
-                                                    kernel="decode_chunk_kernel",
+                                                    kernel="decode_chunk_tc_kernel",
                                                     traffic_key="decode_chunk", ring=1)}
         if rank == 0:
             print(json.dumps(res), flush=True)
@@ -428,7 +428,7 @@ def run_ours(args):
         dec = decode_leg(kda, W, dev, dist, world, args)
         dec_steps = decode_steps_leg(kda, W, dev, dist, world, args)
         dec_chunk = decode_steps_leg(kda, W, dev, dist, world, args, L=CHUNK_L,
-                                     flags=kda.KDA_STEPS_CHUNK, kernel="decode_chunk_kernel",
+                                     flags=kda.KDA_STEPS_CHUNK, kernel="decode_chunk_tc_kernel",
                                      traffic_key="decode_chunk", ring=1)
         bwd_inp = W.named_prefill(BWD_WORKLOAD).to(dev)
         bwd = backward_leg(kda, bwd_inp, dev, dist, world, args)

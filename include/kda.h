@@ -244,12 +244,18 @@ kda_status kda_recurrent_step_ex(const void *q, const void *k, const void *v,
  * KDA_STEPS_CHUNK in flags selects, for dtype KDA_BF16 with dk = dv = 128,
  * L >= 2 and no prologue flags (q_scale = 1), the chunk form of the same L
  * steps (section 3 of the notes: a WY-like representation of the block's
- * writes, then one product with the state) in blocks of 16 tokens on tensor
- * cores: the operands of the state products (state, V_new, T, P and the
- * decayed k, q) are rounded to bf16 as in kda_chunk_fwd, the state stays
- * fp32.  Any finite g <= 0, and g <= 5 for positive gates.  Other
- * combinations run the recurrent kernel, which is bitwise equal to L calls
- * of kda_recurrent_step.
+ * writes, then one product with the state) on tensor cores: blocks of 16
+ * tokens up to L = 32; from L = 33 on, 64-token chunks on tcgen05 with the
+ * intra-chunk work and the state product fused per (sequence, head) (when
+ * state_pool and out are 32-byte aligned; else the 16-token blocks).  The
+ * operands of the state products (state, V_new, T, P and the decayed k, q)
+ * are rounded to bf16 as in kda_chunk_fwd, the state stays fp32.  Any
+ * finite g <= 0, and g <= 5 for positive gates (a 64-token chunk whose decay
+ * leaves e^{+-80} is finished in 16-token blocks).  The 64-token path takes
+ * a scratch of 32 KB per SM plus 8 bytes per (sequence, head) from the
+ * library's stream-ordered memory pool, released on the stream before the
+ * call returns.  Other combinations run the recurrent kernel, which is
+ * bitwise equal to L calls of kda_recurrent_step.
  */
 kda_status kda_recurrent_steps(const void *q, const void *k, const void *v,
                                const float *g, const float *beta,

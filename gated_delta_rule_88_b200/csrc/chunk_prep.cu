@@ -768,14 +768,21 @@ chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             }
         }
         // K e^{G_C - G} transposed (channel rows, 64 tokens, 128-byte swizzle)
-        // straight into the record: each 16-byte piece is half a sector, the
-        // other half follows from the same thread
+        // straight into the record: tokens 16 I .. 16 I + 15 of a row are the
+        // 16-byte chunks 2I and 2I + 1, which the swizzle (XOR with row & 7)
+        // keeps in one aligned 32-byte pair, swapped when row & 7 is odd: one
+        // 256-bit store per row
 #pragma unroll
-        for (int e = 0; e < 2; ++e)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-                *reinterpret_cast<uint4 *>(rec + ws::OFF_KTT + ws::sw128(c0 + e, 16 * I + 8 * hh)) =
-                    make_uint4(kt[e][4 * hh], kt[e][4 * hh + 1], kt[e][4 * hh + 2], kt[e][4 * hh + 3]);
+        for (int e = 0; e < 2; ++e) {
+            const int r = c0 + e, x = r & 7;
+            unsigned char *dst = rec + ws::OFF_KTT + r * 128 + ((((2 * I) ^ x) & ~1) << 4);
+            const bool sw = x & 1;
+            asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"l"(dst),
+                         "r"(sw ? kt[e][4] : kt[e][0]), "r"(sw ? kt[e][5] : kt[e][1]), "r"(sw ? kt[e][6] : kt[e][2]),
+                         "r"(sw ? kt[e][7] : kt[e][3]), "r"(sw ? kt[e][0] : kt[e][4]), "r"(sw ? kt[e][1] : kt[e][5]),
+                         "r"(sw ? kt[e][2] : kt[e][6]), "r"(sw ? kt[e][3] : kt[e][7])
+                         : "memory");
+        }
     }
     fence_proxy_async_smem();
     tc_fence_before();

@@ -128,6 +128,24 @@ __device__ __forceinline__ void st_v8_bf16(void *p, const float *v) {
                  : "memory");
 }
 
+// 16 lanes x 32 columns, twice: threads 0-15 read lanes base .. base + 15 at
+// columns [c, c + 32), threads 16-31 the same lanes at [c + 32, c + 64)
+__device__ __forceinline__ void tmem_ld16x2(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 32;\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // one chunk of one item: item it = n * H + h, chunk index c (-1 = none)
 struct Unit { int it, c; };
 
@@ -506,22 +524,19 @@ decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     {
         // -W (rows 16 qd + l, l < 16, of the +0 tile) as bf16 over the dead k
         // rows: the A operand that turns U into V_new = U - W S in place
-        const int r = 16 * qd + (lane & 15);
+        const int r = 16 * qd + (lane & 15), half = lane >> 4;
         unsigned char *dst = sm + dtc::OFF_KQ + hf * 16384 + r * 128;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        {
             float x[32];
-            tmem_ld32(tmem + lanes + 64u * hf + 32u * half, x);
+            tmem_ld16x2(tmem + lanes + 64u * hf, x);
             tmem_wait_ld();
-            if (lane < 16) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int jc = 4 * half + j;
-                    const float *w = x + 8 * j;
-                    *reinterpret_cast<uint4 *>(dst + ((jc ^ (r & 7)) << 4)) =
-                        make_uint4(pack_bf16(-w[0], -w[1]), pack_bf16(-w[2], -w[3]),
-                                   pack_bf16(-w[4], -w[5]), pack_bf16(-w[6], -w[7]));
-                }
+            for (int j = 0; j < 4; ++j) {
+                const int jc = 4 * half + j;
+                const float *w = x + 8 * j;
+                *reinterpret_cast<uint4 *>(dst + ((jc ^ (r & 7)) << 4)) =
+                    make_uint4(pack_bf16(-w[0], -w[1]), pack_bf16(-w[2], -w[3]),
+                               pack_bf16(-w[4], -w[5]), pack_bf16(-w[6], -w[7]));
             }
         }
         // S row c = TMEM lane, values 64 hf .. + 63: bf16 into the MN-major B
@@ -585,22 +600,19 @@ decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     // ---- V_new (rows 16 qd + l - 16, l >= 16, of the +16 tile) -> bf16 over
     // beta v, as the MN-major B operand of MMA-O and MMA-upd ----
     {
-        const int r = 16 * qd + (lane & 15);
+        const int r = 16 * qd + (lane & 15), half = lane >> 4;
         unsigned char *dst = sm + dtc::OFF_V + hf * 8192 + r * 128;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        {
             float x[32];
-            tmem_ld32(tmem + lanes + 64u * hf + 32u * half, x);
+            tmem_ld16x2(tmem + lanes + L16 + 64u * hf, x);
             tmem_wait_ld();
-            if (lane >= 16) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int jc = 4 * half + j;
-                    const float *a = x + 8 * j;
-                    *reinterpret_cast<uint4 *>(dst + ((jc ^ (r & 7)) << 4)) =
-                        make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]),
-                                   pack_bf16(a[6], a[7]));
-                }
+            for (int j = 0; j < 4; ++j) {
+                const int jc = 4 * half + j;
+                const float *a = x + 8 * j;
+                *reinterpret_cast<uint4 *>(dst + ((jc ^ (r & 7)) << 4)) =
+                    make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]),
+                               pack_bf16(a[6], a[7]));
             }
         }
     }
@@ -643,13 +655,12 @@ decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     // ---- epilogue: O (rows of the +0 tile, l < 16); the new state leaves at
     // the top of the next unit ----
     {
-        const int r = 16 * qd + lane;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        const int r = 16 * qd + (lane & 15), half = lane >> 4;
+        {
             float x[32];
-            tmem_ld32(tmem + lanes + 64u * hf + 32u * half, x);
+            tmem_ld16x2(tmem + lanes + 64u * hf, x);
             tmem_wait_ld();
-            if (lane < 16 && r < len) {
+            if (r < len) {
                 __nv_bfloat16 *dst = out + ((size_t)(t0 + r) * H + h) * D + 64 * hf + 32 * half;
                 st_v8_bf16(dst, x);
                 st_v8_bf16(dst + 16, x + 16);

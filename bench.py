@@ -93,15 +93,18 @@ PREFILL_SRC = ["chunk_prep.cu", "prep_common.cuh", "chunk_chain_tc.cu", "chunk_w
                "common.cuh"]
 TRAFFIC = {
     # prep read + write, chain read + write (ncu, one capture each)
-    "prefill_t8192_h32_d128": {"files": PREFILL_SRC, "sha": "928b340bc66bee09",
-                               "bytes": 336794368 + 255760384 + 304157440 + 49562880},
-    "prefill_t65536_h32_d128": {"files": PREFILL_SRC, "sha": "928b340bc66bee09",
-                                "bytes": 2693117952 + 2384294912 + 2483440640 + 521259008},
-    "varlen8_h32_d128_resume": {"files": PREFILL_SRC, "sha": "928b340bc66bee09",
-                                "bytes": 6035604992 + 5411583488 + 5477717504 + 1200050176},
+    "prefill_t8192_h32_d128": {"files": PREFILL_SRC, "sha": "acf294f7253cc47e",
+                               "bytes": 336671232 + 257490176 + 304156672 + 49854720},
+    "prefill_t65536_h32_d128": {"files": PREFILL_SRC, "sha": "acf294f7253cc47e",
+                                "bytes": 2692927744 + 2386122496 + 2469848576 + 520827904},
+    "varlen8_h32_d128_resume": {"files": PREFILL_SRC, "sha": "acf294f7253cc47e",
+                                "bytes": 6035194880 + 5412791296 + 5479799296 + 1200356864},
     # per call: prep, forward chain with images, reverse chain, per-chunk pass
-    "backward_chunk": {"files": PREFILL_SRC + ["chunk_chain_bwd.cu", "chunk_bwd.cu"], "sha": "56b917d26a13785c",
-                       "bytes": 2823976170},
+    "backward_chunk": {"files": PREFILL_SRC + ["chunk_chain_bwd.cu", "chunk_bwd.cu"], "sha": "72a300444f116fde",
+                       "bytes": 2828195072},
+    # per call from saved intermediates: reverse chain, per-chunk pass
+    "backward_chunk_saved": {"files": ['chunk_chain_bwd.cu', 'chunk_bwd.cu', 'prep_common.cuh', 'chunk_ws.h', 'sm100.cuh', 'common.cuh'], "sha": "69aeaa582a77757f",
+                             "bytes": 304194816 + 162793984 + 811781120 + 493754368},
     # one launch each at full size, -k <kernel> -c 1 (decode legs: --decode-steps 64)
     "decode": {"files": ["decode.cu", "common.cuh"], "sha": "05d923d8fde4c25f",
                "bytes": 547407616 + 479790080},
@@ -110,7 +113,7 @@ TRAFFIC = {
     "backward": {"files": ["recurrent_bwd.cu", "common.cuh"], "sha": "0c58bb721f4cdeeb",
                  "bytes": 2902945280 + 3862875392 + 1614867456 + 385818880},
     "decode_chunk": {"files": ["decode_chunk_tc.cu", "decode_chunk.cu", "prep_common.cuh", "common.cuh",
-                               "sm100.cuh"], "sha": "277e01a9145f9723", "bytes": 1284074240 + 648703488},
+                               "sm100.cuh"], "sha": "3c0993f15efe7d03", "bytes": 1271683072 + 648224512},
 }
 
 
@@ -597,7 +600,7 @@ def backward_leg(kda, inp, dev, dist, world, args, chunked=False, saved=False):
     ach = BWD_BYTES / (ms * 1e-3) / 1e9
     if saved:
         bound, kernel = "hbm", "kda_chunk_bwd from saved intermediates (reverse chain, per-chunk pass)"
-        traffic = None
+        traffic = measured_traffic("backward_chunk_saved")
     elif chunked:
         bound, kernel = "hbm", "kda_chunk_bwd (prep, chain, reverse chain, per-chunk pass)"
         traffic = measured_traffic("backward_chunk")

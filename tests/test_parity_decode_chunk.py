@@ -188,3 +188,26 @@ def test_chunk_steps_decode_workload_64_tokens():
                                   initial_state=pool0[sl].double())
     assert_close(out_c[ns.to(DEV)], o_ref, BF, "sampled o")
     assert_close(pool_c[sl.to(DEV)], s_ref, BF, "sampled states")
+
+
+def test_chunk_steps_16_byte_aligned_buffers():
+    """The 64-token path moves the state and the output in 32-byte pieces; a
+    pool and an output that are only 16-byte aligned (the entry point's
+    contract) take the 16-token blocks instead, and match the oracle."""
+    N, L, H, d = 3, 64, 2, 128
+    q, k, v, g, b = _tokens(N, L, H, d, seed=63)
+    pool0 = W.decode_initial_state(N, H, d, d, seed=63, std=0.02)
+    pool_buf = torch.zeros(pool0.numel() + 4, dtype=torch.float32, device=DEV)
+    pool = pool_buf[4:].view(pool0.shape)                 # 16 bytes past a 256-byte boundary
+    pool.copy_(pool0.to(DEV))
+    out_buf = torch.zeros(N * L * H * d + 8, dtype=BF, device=DEV)
+    out = out_buf[8:].view(N, L, H, d)                    # likewise
+    assert pool.data_ptr() % 32 == 16 and out.data_ptr() % 32 == 16
+    kda_recurrent_steps(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), b.to(DEV), pool, out=out,
+                        flags=KDA_STEPS_CHUNK)
+    torch.cuda.synchronize()
+    assert kda_get_device_error() == 0
+    o_ref, s_ref = oracle.forward(q, k, v, g, b, initial_state=pool0.double())
+    assert_close(out, o_ref, BF, "o")
+    for n in range(N):
+        assert_close(pool[n], s_ref[n], BF, f"state {n}")

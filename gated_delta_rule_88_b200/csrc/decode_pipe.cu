@@ -284,25 +284,28 @@ decode_pipe_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                         pq1 = __ffma2_rn(q2, s1[i + ii], pq1);
                     }
                 }
-                float pk[4] = {pk0.x, pk0.y, pk1.x, pk1.y}, pq[4] = {pq0.x, pq0.y, pq1.x, pq1.y};
-                // across the warp's row groups: a balanced tree in row-group order
+                // across the warp's row groups: a balanced tree in row-group
+                // order (column pairs added as fp32x2, each half rounding like
+                // the scalar add)
 #pragma unroll
                 for (int o = C::C4W; o < 32; o <<= 1) {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        pk[c] += __shfl_xor_sync(0xffffffffu, pk[c], o);
-                        pq[c] += __shfl_xor_sync(0xffffffffu, pq[c], o);
-                    }
+                    pk0 = __fadd2_rn(pk0, make_float2(__shfl_xor_sync(0xffffffffu, pk0.x, o),
+                                                      __shfl_xor_sync(0xffffffffu, pk0.y, o)));
+                    pk1 = __fadd2_rn(pk1, make_float2(__shfl_xor_sync(0xffffffffu, pk1.x, o),
+                                                      __shfl_xor_sync(0xffffffffu, pk1.y, o)));
+                    pq0 = __fadd2_rn(pq0, make_float2(__shfl_xor_sync(0xffffffffu, pq0.x, o),
+                                                      __shfl_xor_sync(0xffffffffu, pq0.y, o)));
+                    pq1 = __fadd2_rn(pq1, make_float2(__shfl_xor_sync(0xffffffffu, pq1.x, o),
+                                                      __shfl_xor_sync(0xffffffffu, pq1.y, o)));
                 }
-                float u[4], ov[4];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    u[c] = b * (vv[c] - pk[c]);
-                    ov[c] = __fmaf_rn(qk, u[c], pq[c]);
-                }
+                // u = beta (v - k^T S'), o = q^T S' + (q.k) u, per column pair
+                const float2 b2 = make_float2(b, b), qk2 = make_float2(qk, qk);
+                const float2 u01 = __fmul2_rn(b2, __fadd2_rn(make_float2(vv[0], vv[1]), make_float2(-pk0.x, -pk0.y)));
+                const float2 u23 = __fmul2_rn(b2, __fadd2_rn(make_float2(vv[2], vv[3]), make_float2(-pk1.x, -pk1.y)));
+                const float2 o01 = __ffma2_rn(qk2, u01, pq0), o23 = __ffma2_rn(qk2, u23, pq1);
+                float ov[4] = {o01.x, o01.y, o23.x, o23.y};
                 if (rgl == 0) store4(out + token_row(cur, tb * C::TB + t) * DV + col0, ov);
                 // S = S' + k u^T
-                const float2 u01 = make_float2(u[0], u[1]), u23 = make_float2(u[2], u[3]);
 #pragma unroll
                 for (int i = 0; i < C::RPT; i += 4) {
                     const float4 K = *reinterpret_cast<const float4 *>(sv + rgl * C::RS + i);

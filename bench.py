@@ -109,7 +109,7 @@ TRAFFIC = {
     "decode": {"files": ["decode.cu", "common.cuh"], "sha": "05d923d8fde4c25f",
                "bytes": 547407616 + 479790080},
     "decode_steps": {"files": ["decode_pipe.cu", "common.cuh", "sm100.cuh"],
-                     "sha": "68dca8336a4f6cbf", "bytes": 621144832 + 496053248},
+                     "sha": "4c819c7229465848", "bytes": 621124352 + 497842176},
     "backward": {"files": ["recurrent_bwd.cu", "common.cuh"], "sha": "0c58bb721f4cdeeb",
                  "bytes": 2902945280 + 3862875392 + 1614867456 + 385818880},
     "decode_chunk": {"files": ["decode_chunk_tc.cu", "decode_chunk.cu", "prep_common.cuh", "common.cuh",

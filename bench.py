@@ -113,7 +113,7 @@ TRAFFIC = {
     "backward": {"files": ["recurrent_bwd.cu", "common.cuh"], "sha": "0c58bb721f4cdeeb",
                  "bytes": 2902945280 + 3862875392 + 1614867456 + 385818880},
     "decode_chunk": {"files": ["decode_chunk_tc.cu", "decode_chunk.cu", "prep_common.cuh", "common.cuh",
-                               "sm100.cuh"], "sha": "3c0993f15efe7d03", "bytes": 1271683072 + 648224512},
+                               "sm100.cuh"], "sha": "4a6e5d9712a95aac", "bytes": 1271683072 + 648224512},
 }
 
 

@@ -15,24 +15,26 @@
 // The prefill's algebra (chunk_prep.cu, chunk_chain_tc.cu) with the state read
 // from and written back to the pool inside the same CTA, so nothing but the
 // inputs, the outputs and the state crosses HBM.  One CTA per (sequence,
-// head) item at a time, persistent (two per SM), each chunk:
+// head) item at a time, persistent (two per SM), each 64-token chunk:
 //
-//   forms, MMA-AP  [beta K e^G ; Q e^G] (K e^{-G})^T          -> A, P
+//   forms, MMA-AP  [beta K e^G ; Q e^G] (K e^{-G})^T (M = 128)  -> A, P
 //   T (fp32, diagonal substitution and tf32 block levels), bf16
-//   MMA-W / MMA-U  [T ; *] (beta K e^G), [T ; *] (beta V)      -> W, U
-//   MMA-S          [W ; Q e^G] S      (S bf16, MN-major)        -> W S, Q e^G S
-//   V_new = U - W S (bf16)
-//   MMA-O          [* ; P] V_new accumulated onto Q e^G S       -> O
-//   MMA-upd        (K e^{G_C - G})^T V_new                       -> S' - Diag(e^{G_C}) S
-//   epilogue       O (bf16) and S' = e^{G_C} S + (...) (fp32) to global memory
+//   MMA-W / MMA-U  T (beta K e^G) -> W, T (beta V) -> U           (M = 64 each)
+//   state pass     -W (bf16); S (bf16, MN-major B operand);
+//                  e^{G_C} S (fp32) into TMEM by tcgen05.st
+//   MMA-S          U + (-W) S -> V_new in place, (Q e^G) S          (M = 64 each)
+//   MMA-O          P V_new accumulated onto (Q e^G) S -> O          (M = 64)
+//   MMA-upd        (K e^{G_C - G})^T V_new accumulated onto e^{G_C} S -> S'   (M = 128)
+//   epilogue       O (bf16); S' leaves TMEM at the top of the next unit
 //
-// Rows marked * are whatever lies next to T or P in shared memory; their
-// products land in tensor-memory lanes that are never read.  K e^{G_C - G}
-// leaves the forms pass from registers into a per-CTA slot of global scratch
-// (it stays in L2) and returns by a bulk copy when shared memory is free
-// again.  The next chunk's inputs are staged by TMA into regions of the
-// current chunk that are dead: g, q and k once MMA-S has read W and S, v once
-// MMA-O and MMA-upd have read V_new.
+// TMEM (256 columns): columns 0-127 hold two M = 64 accumulators, one on
+// lanes 0-15 of each 32-lane sub-partition (+0: W, then (Q e^G) S and O),
+// one on lanes 16-31 (+16: U, then V_new); columns 128-255 hold the state
+// (e^{G_C} S, then S').  K e^{G_C - G} leaves the forms pass from registers
+// into a per-CTA slot of global scratch (it stays in L2) and returns by TMA
+// when shared memory is free again.  The next chunk's inputs are staged by
+// TMA into regions of the current chunk that are dead: g, q and k once MMA-S
+// has read -W, Q e^G and S, v once MMA-O and MMA-upd have read V_new.
 //
 // A chunk whose decay leaves the chunk-start exponent range (every e^{+-G}
 // and e^{G_C - G} within e^{+-80}) is not computed here: its (item, first

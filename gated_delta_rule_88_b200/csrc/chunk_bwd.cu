@@ -39,6 +39,12 @@ __device__ __forceinline__ int sw(int r, int c) {
     return r * 128 + ((((c >> 3) ^ (r & 7))) << 4) + ((c & 7) << 1);
 }
 constexpr float RANGE2 = 80.f * 1.4426950408889634f;   // e^{+-80}, in log2 units
+// 256-bit global store (32-byte aligned address)
+__device__ __forceinline__ void st_v8(float *p, const float *v) {
+    asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"l"(p), "f"(v[0]), "f"(v[1]), "f"(v[2]),
+                 "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
+                 : "memory");
+}
 
 namespace bl {
 constexpr int KQ = 0;            // [k -> bKg : 64 rows][q -> Qg : 64 rows] per 64-ch block (16 KB); finale: dG fp32
@@ -95,7 +101,7 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                        const unsigned char *__restrict__ s_img, const unsigned char *__restrict__ v_img,
                        const unsigned char *__restrict__ dsp_img, const unsigned char *__restrict__ dvn_img,
                        float *__restrict__ dq, float *__restrict__ dk, float *__restrict__ dv,
-                       float *__restrict__ dg, float *__restrict__ dbeta, int *__restrict__ err)
+                       float *__restrict__ dg, float *__restrict__ dbeta, int v8, int *__restrict__ err)
 {
     using namespace sm100;
     extern __shared__ unsigned char smem_raw[];
@@ -593,12 +599,19 @@ chunk_bwd_local_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             }
             if (live) {
                 const size_t grow = ((size_t)(t0 + i) * H + h) * D + cm;
-                float4 *pq = reinterpret_cast<float4 *>(dq + grow);
-                float4 *pk = reinterpret_cast<float4 *>(dk + grow);
-                float4 *pv = reinterpret_cast<float4 *>(dv + grow);
-                pq[0] = make_float4(oq[0], oq[1], oq[2], oq[3]); pq[1] = make_float4(oq[4], oq[5], oq[6], oq[7]);
-                pk[0] = make_float4(ok_[0], ok_[1], ok_[2], ok_[3]); pk[1] = make_float4(ok_[4], ok_[5], ok_[6], ok_[7]);
-                pv[0] = make_float4(ov[0], ov[1], ov[2], ov[3]); pv[1] = make_float4(ov[4], ov[5], ov[6], ov[7]);
+                if (v8) {
+                    // 8 channels = one 32-byte sector per gradient and row
+                    st_v8(dq + grow, oq);
+                    st_v8(dk + grow, ok_);
+                    st_v8(dv + grow, ov);
+                } else {
+                    float4 *pq = reinterpret_cast<float4 *>(dq + grow);
+                    float4 *pk = reinterpret_cast<float4 *>(dk + grow);
+                    float4 *pv = reinterpret_cast<float4 *>(dv + grow);
+                    pq[0] = make_float4(oq[0], oq[1], oq[2], oq[3]); pq[1] = make_float4(oq[4], oq[5], oq[6], oq[7]);
+                    pk[0] = make_float4(ok_[0], ok_[1], ok_[2], ok_[3]); pk[1] = make_float4(ok_[4], ok_[5], ok_[6], ok_[7]);
+                    pv[0] = make_float4(ov[0], ov[1], ov[2], ov[3]); pv[1] = make_float4(ov[4], ov[5], ov[6], ov[7]);
+                }
             }
             // column sums over the half's 16 token rows (xor steps stay inside
             // each half), one slot per channel and row group (no atomics)
@@ -677,7 +690,8 @@ cudaError_t launch_chunk_bwd_local(const void *q, const void *k, const void *v, 
     dim3 grid(max_chunks, H);
     chunk_bwd_local_kernel<<<grid, NT, smem, st>>>(
         mq, mk, mv, mg, mdo, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, beta,
-        cu, coff, N, T, total_T, H, (T + C - 1) / C, s_img, v_img, dsp_img, dvn_img, dq, dk, dv, dg, dbeta, err);
+        cu, coff, N, T, total_T, H, (T + C - 1) / C, s_img, v_img, dsp_img, dvn_img, dq, dk, dv, dg, dbeta,
+        (((uintptr_t)dq | (uintptr_t)dk | (uintptr_t)dv) & 31u) == 0, err);
     return cudaGetLastError();
 }
 

@@ -100,11 +100,11 @@ TRAFFIC = {
     "varlen8_h32_d128_resume": {"files": PREFILL_SRC, "sha": "acf294f7253cc47e",
                                 "bytes": 6035194880 + 5412791296 + 5479799296 + 1200356864},
     # per call: prep, forward chain with images, reverse chain, per-chunk pass
-    "backward_chunk": {"files": PREFILL_SRC + ["chunk_chain_bwd.cu", "chunk_bwd.cu"], "sha": "72a300444f116fde",
-                       "bytes": 2828195072},
+    "backward_chunk": {"files": PREFILL_SRC + ["chunk_chain_bwd.cu", "chunk_bwd.cu"], "sha": "cdf3da396b022dcd",
+                       "bytes": 2832467200},
     # per call from saved intermediates: reverse chain, per-chunk pass
-    "backward_chunk_saved": {"files": ['chunk_chain_bwd.cu', 'chunk_bwd.cu', 'prep_common.cuh', 'chunk_ws.h', 'sm100.cuh', 'common.cuh'], "sha": "69aeaa582a77757f",
-                             "bytes": 304194816 + 162793984 + 811781120 + 493754368},
+    "backward_chunk_saved": {"files": ['chunk_chain_bwd.cu', 'chunk_bwd.cu', 'prep_common.cuh', 'chunk_ws.h', 'sm100.cuh', 'common.cuh'], "sha": "17f685e0cda4b450",
+                             "bytes": 304158720 + 163587072 + 811437312 + 497039360},
     # one launch each at full size, -k <kernel> -c 1 (decode legs: --decode-steps 64)
     "decode": {"files": ["decode.cu", "common.cuh"], "sha": "05d923d8fde4c25f",
                "bytes": 547407616 + 479790080},

@@ -89,7 +89,7 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
                       float *__restrict__ sT, __nv_bfloat16 *__restrict__ out, int T, int total_T,
                       int H, int cps, int max_chunks, int *__restrict__ err,
                       unsigned char *__restrict__ s_img, unsigned char *__restrict__ v_img,
-                      const int32_t *__restrict__ order)
+                      const int32_t *__restrict__ order, int out_v8)
 {
     using L = TcLayout<DVT, NS>;
     extern __shared__ unsigned char smem_raw[];
@@ -311,11 +311,25 @@ chunk_chain_tc_kernel(const unsigned char *__restrict__ wsp, const int32_t *__re
             float o[CPT];
             tmem_row((ci & 1) * DVT, o);
             if (out && tok < eos) {        // out == nullptr: the backward's recompute pass
-                uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)tok * H + h) * D + n0 + cb);
+                __nv_bfloat16 *row = out + ((size_t)tok * H + h) * D + n0 + cb;
+                if (out_v8) {
+                    // 16 columns = one 32-byte sector per store
 #pragma unroll
-                for (int e = 0; e < CPT / 8; ++e)
-                    dst[e] = make_uint4(pack_bf16(o[8 * e], o[8 * e + 1]), pack_bf16(o[8 * e + 2], o[8 * e + 3]),
-                                        pack_bf16(o[8 * e + 4], o[8 * e + 5]), pack_bf16(o[8 * e + 6], o[8 * e + 7]));
+                    for (int e = 0; e < CPT / 16; ++e) {
+                        const float *x = o + 16 * e;
+                        asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"l"(row + 16 * e),
+                                     "r"(pack_bf16(x[0], x[1])), "r"(pack_bf16(x[2], x[3])), "r"(pack_bf16(x[4], x[5])),
+                                     "r"(pack_bf16(x[6], x[7])), "r"(pack_bf16(x[8], x[9])), "r"(pack_bf16(x[10], x[11])),
+                                     "r"(pack_bf16(x[12], x[13])), "r"(pack_bf16(x[14], x[15]))
+                                     : "memory");
+                    }
+                } else {
+                    uint4 *dst = reinterpret_cast<uint4 *>(row);
+#pragma unroll
+                    for (int e = 0; e < CPT / 8; ++e)
+                        dst[e] = make_uint4(pack_bf16(o[8 * e], o[8 * e + 1]), pack_bf16(o[8 * e + 2], o[8 * e + 3]),
+                                            pack_bf16(o[8 * e + 4], o[8 * e + 5]), pack_bf16(o[8 * e + 6], o[8 * e + 7]));
+                }
             }
             return true;
         };
@@ -418,7 +432,7 @@ cudaError_t launch_tc(const unsigned char *wsp, const int32_t *cu, const int32_t
     dim3 grid(D / DVT, H, N);
     chunk_chain_tc_kernel<DVT, NS><<<grid, L::NTHREADS, smem, st>>>(
         wsp, cu, coff, s0, sT, (__nv_bfloat16 *)out, T, total_T, H, (T + C - 1) / C, max_chunks, err,
-        s_img, v_img, order);
+        s_img, v_img, order, ((uintptr_t)out & 31u) == 0);
     return cudaGetLastError();
 }
 

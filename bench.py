@@ -93,15 +93,15 @@ PREFILL_SRC = ["chunk_prep.cu", "prep_common.cuh", "chunk_chain_tc.cu", "chunk_w
                "common.cuh"]
 TRAFFIC = {
     # prep read + write, chain read + write (ncu, one capture each)
-    "prefill_t8192_h32_d128": {"files": PREFILL_SRC, "sha": "acf294f7253cc47e",
-                               "bytes": 336671232 + 257490176 + 304156672 + 49854720},
-    "prefill_t65536_h32_d128": {"files": PREFILL_SRC, "sha": "acf294f7253cc47e",
-                                "bytes": 2692927744 + 2386122496 + 2469848576 + 520827904},
-    "varlen8_h32_d128_resume": {"files": PREFILL_SRC, "sha": "acf294f7253cc47e",
-                                "bytes": 6035194880 + 5412791296 + 5479799296 + 1200356864},
+    "prefill_t8192_h32_d128": {"files": PREFILL_SRC, "sha": "36d0ac55854a3ca5",
+                               "bytes": 336789760 + 257384192 + 304157696 + 50902784},
+    "prefill_t65536_h32_d128": {"files": PREFILL_SRC, "sha": "36d0ac55854a3ca5",
+                                "bytes": 2692875264 + 2386116096 + 2452307712 + 521305856},
+    "varlen8_h32_d128_resume": {"files": PREFILL_SRC, "sha": "36d0ac55854a3ca5",
+                                "bytes": 6036765184 + 5413019136 + 5480518400 + 1200050432},
     # per call: prep, forward chain with images, reverse chain, per-chunk pass
-    "backward_chunk": {"files": PREFILL_SRC + ["chunk_chain_bwd.cu", "chunk_bwd.cu"], "sha": "cdf3da396b022dcd",
-                       "bytes": 2832467200},
+    "backward_chunk": {"files": PREFILL_SRC + ["chunk_chain_bwd.cu", "chunk_bwd.cu"], "sha": "4f22c08865933e43",
+                       "bytes": 2832923904},
     # per call from saved intermediates: reverse chain, per-chunk pass
     "backward_chunk_saved": {"files": ['chunk_chain_bwd.cu', 'chunk_bwd.cu', 'prep_common.cuh', 'chunk_ws.h', 'sm100.cuh', 'common.cuh'], "sha": "17f685e0cda4b450",
                              "bytes": 304158720 + 163587072 + 811437312 + 497039360},
